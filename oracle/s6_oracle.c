@@ -1,0 +1,182 @@
+/*
+ * s6_oracle.c -- plain, sequential fp64 CPU oracle for the selective scan (S6).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
+ * this file; only the tests, the smoke check and the bench's CPU-baseline leg do.
+ * It shares no code, header, table or helper with the CUDA library.
+ *
+ * What it computes (Mamba: Linear-Time Sequence Modeling with Selective State
+ * Spaces, page "xyznot.com/ar/paper/2312.00752", sections "Method" and
+ * "Selection mechanism (S6)"; plus the serial "MambaMini" scan and the Q&A on
+ * page "yongjin360.com/news/29389"):
+ *
+ *   for every independent (batch, channel) lane, with h[0..N) = h0 (0 if absent):
+ *     for t = 0 .. L-1:
+ *       x      = delta_raw[t] + delta_bias                 (bias added before tau)
+ *       Delta  = softplus(x)  if softplus else x           (tau_Delta = softplus)
+ *       for n:  Abar_n = exp(Delta * A[n])                 (ZOH: Abar = exp(Delta A))
+ *               h[n]   = Abar_n * h[n] + Delta * B[n,t] * u[t]
+ *                                                          (Bbar = Delta * B, the
+ *                                                           element-wise product the
+ *                                                           page-2 Q&A describes)
+ *       y[t]  = (sum_n C[n,t] * h[n] + D * u[t]) * silu(z[t])
+ *     last_state = h
+ *
+ * The output at step t reads the state AFTER the update at step t (h_t = Abar h_{t-1}
+ * + Bbar x_t, y_t = C h_t, page 4 "Method").  Absent D / z / delta_bias act as
+ * 0 / no gate / 0.  Arithmetic is IEEE double with libm exp/log1p, no fast-math,
+ * strictly sequential in t; OpenMP only spreads independent lanes over cores.
+ *
+ * Every function here is pinned by tests that do not reuse its code: hand-worked
+ * examples, the LTI convolution form, the associative-combine prefix, closed
+ * forms and limiting cases (see tests/test_oracle_pins.py).
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#define S6O_OK 0
+#define S6O_ERR_ARG (-1)
+#define S6O_MAX_N 256 /* largest state width the scan accepts */
+
+/* softplus(x) = log(1 + e^x), written so neither branch overflows.
+ * Page 4, "Selection mechanism": Delta = tau_Delta(Parameter + s_Delta(x)) with
+ * tau_Delta = softplus. */
+double s6o_softplus(double x) {
+    if (x > 0.0) return x + log1p(exp(-x));
+    return log1p(exp(x));
+}
+
+/* Step size for one (lane, t): bias first, then the optional softplus. */
+static double step_size(double delta_raw, double bias, int softplus) {
+    double x = delta_raw + bias;
+    return softplus ? s6o_softplus(x) : x;
+}
+
+/* SiLU gate: z * sigmoid(z) = z / (1 + e^{-z}) (page 2 Q&A on the gate). */
+static double silu(double z) {
+    if (z >= 0.0) return z / (1.0 + exp(-z));
+    double e = exp(z);
+    return z * e / (1.0 + e);
+}
+
+/*
+ * Discretisation only: Delta[lane, t] and Abar[lane, t, n] = exp(Delta * A[lane, n]).
+ * Page 4 "Method" (ZOH: Abar = exp(Delta A)); Delta as in the selection mechanism.
+ * Shapes: delta_raw (nlanes, L); A (nlanes, N); delta_bias (nlanes) or NULL.
+ */
+int s6o_discretize(long nlanes, long N, long L, const double* delta_raw,
+                   const double* A, const double* delta_bias, int softplus,
+                   double* delta_out, double* abar_out) {
+    if (nlanes < 0 || N < 1 || L < 0 || !delta_raw || !A) return S6O_ERR_ARG;
+    for (long i = 0; i < nlanes; ++i) {
+        double bias = delta_bias ? delta_bias[i] : 0.0;
+        for (long t = 0; t < L; ++t) {
+            double dt = step_size(delta_raw[i * L + t], bias, softplus);
+            if (delta_out) delta_out[i * L + t] = dt;
+            if (abar_out)
+                for (long n = 0; n < N; ++n)
+                    abar_out[(i * L + t) * N + n] = exp(dt * A[i * N + n]);
+        }
+    }
+    return S6O_OK;
+}
+
+/*
+ * The sequential selective scan over independent lanes.
+ *
+ *   u, delta_raw, z : (nlanes, L)          z may be NULL (no gate)
+ *   A               : (nlanes, N)
+ *   D, delta_bias   : (nlanes) or NULL
+ *   Bm, Cm          : (nbatch, N, L); lane i reads batch lane_batch[i]
+ *   h0              : (nlanes, N) or NULL (zero initial state, h_{-1} = 0)
+ *   y               : (nlanes, L)          required
+ *   h_last          : (nlanes, N) or NULL
+ *   h_all           : (nlanes, L, N) or NULL  every state h_t (small inputs only)
+ */
+int s6o_scan(long nlanes, long N, long L, long nbatch,
+             const double* u, const double* delta_raw, const double* z,
+             const double* A, const double* D, const double* delta_bias,
+             const double* Bm, const double* Cm, const long* lane_batch,
+             int softplus, const double* h0,
+             double* y, double* h_last, double* h_all) {
+    if (nlanes < 0 || N < 1 || N > S6O_MAX_N || L < 0 || nbatch < 1) return S6O_ERR_ARG;
+    if (!u || !delta_raw || !A || !Bm || !Cm || !lane_batch || !y) return S6O_ERR_ARG;
+    for (long i = 0; i < nlanes; ++i)
+        if (lane_batch[i] < 0 || lane_batch[i] >= nbatch) return S6O_ERR_ARG;
+
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long i = 0; i < nlanes; ++i) {
+        double hv[S6O_MAX_N];
+        for (long n = 0; n < N; ++n) hv[n] = h0 ? h0[i * N + n] : 0.0;
+        const double* Bb = Bm + lane_batch[i] * N * L;
+        const double* Cb = Cm + lane_batch[i] * N * L;
+        double bias = delta_bias ? delta_bias[i] : 0.0;
+        double dskip = D ? D[i] : 0.0;
+        for (long t = 0; t < L; ++t) {
+            double ut = u[i * L + t];
+            double dt = step_size(delta_raw[i * L + t], bias, softplus);
+            double acc = 0.0;
+            for (long n = 0; n < N; ++n) {
+                double abar = exp(dt * A[i * N + n]);
+                hv[n] = abar * hv[n] + dt * Bb[n * L + t] * ut;
+                acc += Cb[n * L + t] * hv[n];
+                if (h_all) h_all[(i * L + t) * N + n] = hv[n];
+            }
+            acc += dskip * ut;
+            if (z) acc *= silu(z[i * L + t]);
+            y[i * L + t] = acc;
+        }
+        if (h_last)
+            for (long n = 0; n < N; ++n) h_last[i * N + n] = hv[n];
+    }
+    return S6O_OK;
+}
+
+/*
+ * One decode step (selective_state_update): the scan body for a single token,
+ * applied in place to the carried state (page 4 FAQ: generation keeps only a
+ * fixed D x N state per layer and costs O(1) per token).
+ *
+ *   state : (nlanes, N) in/out;   u, delta_raw, z : (nlanes)   z may be NULL
+ *   A     : (nlanes, N);          D, delta_bias   : (nlanes) or NULL
+ *   Bv, Cv: (nbatch, N); lane i reads row lane_batch[i]
+ *   y     : (nlanes)
+ */
+int s6o_state_update(long nlanes, long N, long nbatch, double* state,
+                     const double* u, const double* delta_raw, const double* z,
+                     const double* A, const double* D, const double* delta_bias,
+                     const double* Bv, const double* Cv, const long* lane_batch,
+                     int softplus, double* y) {
+    if (nlanes < 0 || N < 1 || nbatch < 1) return S6O_ERR_ARG;
+    if (!state || !u || !delta_raw || !A || !Bv || !Cv || !lane_batch || !y)
+        return S6O_ERR_ARG;
+    for (long i = 0; i < nlanes; ++i)
+        if (lane_batch[i] < 0 || lane_batch[i] >= nbatch) return S6O_ERR_ARG;
+
+#pragma omp parallel for schedule(static)
+    for (long i = 0; i < nlanes; ++i) {
+        const double* Bb = Bv + lane_batch[i] * N;
+        const double* Cb = Cv + lane_batch[i] * N;
+        double dt = step_size(delta_raw[i], delta_bias ? delta_bias[i] : 0.0, softplus);
+        double acc = 0.0;
+        for (long n = 0; n < N; ++n) {
+            double abar = exp(dt * A[i * N + n]);
+            double hn = abar * state[i * N + n] + dt * Bb[n] * u[i];
+            state[i * N + n] = hn;
+            acc += Cb[n] * hn;
+        }
+        acc += (D ? D[i] : 0.0) * u[i];
+        if (z) acc *= silu(z[i]);
+        y[i] = acc;
+    }
+    return S6O_OK;
+}
+
+/* Threads the OpenMP runtime would use for the parallel loops above. */
+#ifdef _OPENMP
+#include <omp.h>
+int s6o_num_threads(void) { return omp_get_max_threads(); }
+#else
+int s6o_num_threads(void) { return 1; }
+#endif
