@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""Benchmark of the selective scan (S6) hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one fused selective-scan forward over the Mamba-2.8B-shaped layer
+(batch 4, dim 5120, N 16, L 4096, bf16 u/delta/z/B/C/y, fp32 state) through the
+C ABI.  Its inputs (671 MB) exceed the 126 MB L2, so no flush is needed between
+steps.  Timing: W untimed warm-up steps, then K steps between CUDA events on the
+launching stream, bracketed by a barrier and a device synchronize; with N > 1
+ranks (one process per GPU under torchrun) every rank scans its own independent
+batch (weak scaling, no data-path collective) and the max time over ranks is
+used.  The same run measures the decode workload (selective_state_update,
+batch 256, dim 5120, N 16, 1000 fresh tokens, L2 flushed before each token),
+the end-to-end path from pinned host buffers, the SM clocks during the timed
+region, and (rank 0, N = 1) the fp64 CPU oracle on a bounded sample.
+
+``--impl reference`` times the CPU oracle itself as the reference arm.
+Rank 0 prints exactly one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = ("selective-scan fwd (b·d·L) elems/s & % of roofline; "
+          "decode state-updates/s")
+WORKLOAD = "m2p8b"
+SM_COUNT_B200 = 148
+SFU_OPS_PER_CLK_PER_SM = 16  # ex2/lg2/rcp results per clock per SM
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ----------------------------------------------------------------------------- ranks
+
+def dist_setup():
+    """Rank, world size and local rank from torchrun's environment (1 process per GPU)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120),
+                                **({"device_id": torch.device("cuda", local)}
+                                   if backend == "nccl" else {}))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    """Host-side reduction of one timing scalar (not a data-path collective)."""
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank scans an independent batch: same recipe, its own seed."""
+    return base + 1000 * rank
+
+
+def dist_teardown(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clk_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        busy = [r for r in rows if r["power"] > 250.0] or rows
+        reasons = set()
+        for r in busy:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in busy),
+                "sm_max_mhz": max(r["smax"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(busy), "power_w_median": statistics.median(r["power"] for r in busy)}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+def profile_traffic(name: str, source: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    digest = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()[:16]
+    if vals.get("source_sha256_16") != digest:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def scan_bytes(b, d, n, L, in_size=2, out_size=2):
+    """Algorithmic bytes of one scan: u, delta, z, B, C read once, y written once, plus
+    A, D, bias and last_state (the expanded state is never materialised)."""
+    return (3 * b * d * L * in_size + 2 * b * n * L * in_size + b * d * L * out_size +
+            d * n * 4 + 2 * d * 4 + b * d * n * 4)
+
+
+def decode_bytes(b, d, n, io_size=2):
+    """Algorithmic bytes of one decode token: the state read and written, u/delta/z and
+    y per lane, B/C per batch row, A/D/bias per channel."""
+    return 2 * b * d * n * 4 + 4 * b * d * io_size + 2 * b * n * io_size + d * n * 4 + 2 * d * 4
+
+
+def flush_l2(buf):
+    buf.add_(1)  # reads and writes 2x L2 worth of bytes
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local):
+    from selective_state_space_56_b200 import inputs, ops
+    import selective_state_space_56_b200.build as s6build
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200)")
+    s6build.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = inputs.SCAN_WORKLOADS[WORKLOAD]
+    b, d, n, L = w.batch, w.dim, w.dstate, w.seqlen
+    host = inputs.scan_inputs(b, d, n, L, w.in_dtype, rank_seed(w.seed, rank))
+    host = {k: (v.pin_memory() if v is not None else None) for k, v in host.items()}
+    g = {k: v.to(dev) for k, v in host.items()}
+    y = torch.empty((b, d, L), dtype=w.out_dtype, device=dev)
+    last = torch.empty((b, d, n), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ops.selective_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                               delta_bias=g["delta_bias"], y=y, last_state=last)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    # Per-launch durations for the roofline: events around each launch on the launching
+    # stream, inside the same timed loop.
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        t0.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    ms_total = t0.elapsed_time(t1)
+    ms_kernel = statistics.fmean(a.elapsed_time(bb) for a, bb in ev)
+    ms_total = max_over_ranks(ms_total, world)
+    ms_step = ms_total / args.steps
+    elems = b * d * L
+    value = world * elems * args.steps / (ms_total * 1e-3)
+    clocks = clk.summary()
+
+    peaks, peak_kind = measured_peaks()
+    fmax_mhz = peaks.get("sm_max_mhz", 1965.0)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    sfu_peak = sms * SFU_OPS_PER_CLK_PER_SM * fmax_mhz * 1e6       # ops/s
+    exps = elems * (n + 2)                                          # Abar x N, softplus, SiLU
+    achieved = exps / (ms_kernel * 1e-3)
+    byts = scan_bytes(b, d, n, L)
+    roofline = {
+        "bound": "alu", "unit": "Gexp/s",
+        "achieved": achieved / 1e9, "peak": sfu_peak / 1e9, "frac": achieved / sfu_peak,
+        "traffic": profile_traffic("scan_fwd_m2p8b.txt", "selective_state_space_56_b200/csrc/scan_fwd.cu"),
+        "algorithmic_bytes": byts,
+        "hbm_GBps": byts / (ms_kernel * 1e-3) / 1e9,
+        "hbm_frac": byts / (ms_kernel * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "peak_note": "SFU: %d SMs x %d ops/clk x %.0f MHz (derived); HBM peak %s %.0f GB/s" % (
+            sms, SFU_OPS_PER_CLK_PER_SM, fmax_mhz, peak_kind, peaks["hbm_gbs"]),
+        "kernel_ms": ms_kernel,
+    }
+
+    # End to end through the C ABI from pinned host buffers: copies inside the timed region.
+    e2e_steps = max(1, min(args.steps, 5))
+    h2d = sum(host[k].numel() * host[k].element_size() for k in ("u", "delta", "z", "B", "C"))
+    d2h = y.numel() * y.element_size()
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for k in ("u", "delta", "z", "B", "C"):
+            g[k].copy_(host[k], non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    e2e = {"value": world * elems / (e2e_ms * 1e-3), "unit": "elems/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    decode = run_decode(dev, stream, world)
+    del g, y, last
+    torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, budget_s=args.cpu_seconds)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "elems/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "io_dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "Mamba-2.8B-shaped layer scan (m2p8b): batch 4, dim 5120, N 16, "
+                               "L 4096, bf16 I/O, fp32 state",
+                   "batch": b, "dim": d, "dstate": n, "seqlen": L,
+                   "l2": "no flush: each step reads %.0f MB of inputs (> %d MB L2)" % (
+                       (h2d) / 1e6, L2_BYTES >> 20),
+                   "parallelism": "replicas x%d (independent batches per GPU)" % world},
+        "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
+        "clocks": clocks, "decode": decode, "cpu_baseline": cpu, "impl": "ours",
+    }
+    return line
+
+
+def run_decode(dev, stream, world, steps=1000):
+    """Decode workload: 1000 tokens with fresh seeded inputs; each token timed alone with
+    events after an L2 flush (the 84 MB state would otherwise stay in the 126 MB L2)."""
+    from selective_state_space_56_b200 import inputs, ops
+    w = inputs.DECODE_WORKLOAD
+    prm = {k: v.to(dev) for k, v in inputs.decode_params(w).items()}
+    state = prm["state0"].clone()
+    toks = [inputs.decode_step_inputs(s, w, device=dev) for s in range(steps)]
+    y = torch.empty((w.batch, w.dim), dtype=w.io_dtype, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def tok(x):
+        ops.selective_state_update(state, x["u"], x["delta"], prm["A"], x["B"], x["C"],
+                                   D=prm["D"], z=x["z"], delta_bias=prm["delta_bias"], y=y)
+
+    for x in toks[:5]:
+        tok(x)
+    torch.cuda.synchronize(dev)
+    evs = []
+    for x in toks:
+        flush_l2(flush)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        tok(x)
+        b_.record(stream)
+        evs.append((a, b_))
+    torch.cuda.synchronize(dev)
+    ms_cold = statistics.fmean(a.elapsed_time(b_) for a, b_ in evs)
+    # back to back (state L2-resident between tokens), for context
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for x in toks:
+        tok(x)
+    b_.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_warm = a.elapsed_time(b_) / steps
+    ms_cold = max_over_ranks(ms_cold, world)
+    peaks, kind = measured_peaks()
+    byts = decode_bytes(w.batch, w.dim, w.dstate)
+    lanes = w.batch * w.dim
+    del toks, flush
+    return {
+        "metric": "decode state-updates/s", "unit": "(b,d) lane updates/s",
+        "value": world * lanes / (ms_cold * 1e-3), "steps_per_s": 1e3 / ms_cold,
+        "ms_per_token_l2_flushed": ms_cold, "ms_per_token_back_to_back": ms_warm,
+        "workload": "decode: batch 256, dim 5120, N 16, bf16 I/O, fp32 state, 1000 fresh tokens",
+        "roofline": {"bound": "hbm", "unit": "GB/s", "achieved": byts / (ms_cold * 1e-3) / 1e9,
+                     "peak": peaks["hbm_gbs"], "frac": byts / (ms_cold * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "algorithmic_bytes": byts, "peak_kind": kind,
+                     "traffic": profile_traffic("state_update_decode.txt",
+                                                "selective_state_space_56_b200/csrc/state_update.cu")},
+        "gpu_launches": 2 * steps,
+    }
+
+
+# ----------------------------------------------------------------------------- oracle arm
+
+def cpu_baseline(w, budget_s=10.0):
+    """The fp64 oracle as it stands, on a bounded channel sample of the same workload."""
+    import numpy as np
+    import oracle
+    from selective_state_space_56_b200 import inputs
+
+    p = inputs.workload_inputs(w) if w.name != "million" else None
+    rng = np.random.default_rng(0)
+
+    def run(nl):
+        bi = rng.integers(0, w.batch, nl)
+        di = rng.integers(0, w.dim, nl)
+        t = time.perf_counter()
+        oracle.scan_lanes(p["u"][bi, di], p["delta"][bi, di], p["A"][di], p["B"], p["C"], bi,
+                          D=p["D"][di], z=p["z"][bi, di], delta_bias=p["delta_bias"][di])
+        return time.perf_counter() - t
+
+    cores = oracle.num_threads()
+    probe = max(cores, 8)
+    t = run(probe)
+    nl = int(min(w.batch * w.dim, max(probe, probe * budget_s / max(t, 1e-3))))
+    t = run(nl)
+    return {"value": nl * w.seqlen / t, "unit": "elems/s", "cores": cores, "kind": "oracle",
+            "sample": "%d of %d channels x full L=%d (fp64, sequential per channel, %d OpenMP "
+                      "threads), %.1f s" % (nl, w.batch * w.dim, w.seqlen, cores, t)}
+
+
+def run_reference(args, rank, world):
+    from selective_state_space_56_b200 import inputs
+    w = inputs.SCAN_WORKLOADS[WORKLOAD]
+    if rank != 0:
+        return None
+    per_step = max(1.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(w, budget_s=per_step / 4)
+    vals = [cpu_baseline(w, budget_s=per_step) for _ in range(args.steps)]
+    v = statistics.fmean(x["value"] for x in vals)
+    cpu = dict(vals[-1])
+    cpu["value"] = v
+    return {"metric": METRIC, "value": v, "unit": "elems/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": w.batch * w.dim * w.seqlen / v * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": "Mamba-2.8B-shaped layer scan (m2p8b): batch 4, dim 5120, "
+                                   "N 16, L 4096; each step a bounded channel sample",
+                       "batch": w.batch, "dim": w.dim, "dstate": w.dstate, "seqlen": w.seqlen},
+            "cpu_baseline": cpu,
+            "e2e": {"value": v, "unit": "elems/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[1])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        # The oracle arm runs on rank 0's host cores only; other ranks have no work and
+        # take part in no collective.
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    rank, world, local = dist_setup()
+    try:
+        line = run_ours(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        dist_teardown(world)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,135 @@
+/*
+ * mamba_s6.h -- C ABI of the B200 (sm_100a) selective-scan library.
+ *
+ * Two operations, each a hand-written CUDA kernel sequence launched on the
+ * caller's stream:
+ *
+ *   mamba_selective_scan_fwd      the fused S6 forward scan over a whole sequence
+ *   mamba_selective_state_update  one decode token, updating a carried state in place
+ *
+ * Definitions (Mamba: Linear-Time Sequence Modeling with Selective State Spaces,
+ * page "xyznot.com/ar/paper/2312.00752", sections "Method", "Selection mechanism
+ * (S6)" and "Hardware-aware state expansion"; page "yongjin360.com/news/29389",
+ * serial scan, parallel-scan derivation steps 1-4 and the Q&A):
+ *
+ *   Delta_t  = softplus(delta[t] + delta_bias)   (or delta[t] + delta_bias when
+ *                                                 delta_softplus == 0)
+ *   Abar_t,n = exp(Delta_t * A[n])                ZOH discretisation of a diagonal A
+ *   h_t,n    = Abar_t,n * h_{t-1},n + Delta_t * B[n,t] * u[t]     (h_{-1} = 0)
+ *   y[t]     = (sum_n C[n,t] * h_t,n + D * u[t]) * silu(z[t]),  silu(x) = x / (1 + e^-x)
+ *
+ * per independent (batch, channel) lane.  B and C are per token and shared by
+ * all channels of a batch; A, D and delta_bias are per channel.  The expanded
+ * (batch, L, dim, N) state never reaches device memory: it lives in registers.
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers owned by the caller, contiguous in
+ *     the layouts stated below (last dimension fastest), 16-byte aligned.  The
+ *     library keeps no pointer after a call returns and allocates nothing.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *     asynchronous: they enqueue kernels and return without synchronising.
+ *   - Argument errors are detected on the host before anything is launched and
+ *     return a negative mamba_status; nothing is written in that case.
+ *   - A launch failure reported by the CUDA runtime returns MAMBA_ERR_CUDA.
+ *   - Outputs must not alias inputs (except `state`, which is updated in place).
+ */
+#ifndef MAMBA_S6_H
+#define MAMBA_S6_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { MAMBA_F32 = 0, MAMBA_BF16 = 1 } mamba_dtype;
+
+typedef enum {
+    MAMBA_OK = 0,
+    MAMBA_ERR_NULL = -1,      /* a required pointer is NULL                         */
+    MAMBA_ERR_DIMS = -2,      /* a size is negative, too large, or dstate not 1..16 */
+    MAMBA_ERR_ALIGN = -3,     /* a pointer is not 16-byte aligned                   */
+    MAMBA_ERR_DTYPE = -4,     /* an unknown dtype enum                              */
+    MAMBA_ERR_WORKSPACE = -5, /* workspace missing or smaller than required          */
+    MAMBA_ERR_CUDA = -6,      /* the CUDA runtime reported an error                 */
+    MAMBA_ERR_TIMEOUT = -7    /* a bounded device-side wait gave up                 */
+} mamba_status;
+
+/* Problem sizes: batch >= 1, dim >= 1, 1 <= dstate <= 16, seqlen >= 0. */
+typedef struct {
+    int64_t batch;
+    int64_t dim;    /* d_inner: channels */
+    int64_t dstate; /* N: state width per channel */
+    int64_t seqlen; /* L */
+} mamba_scan_dims;
+
+/*
+ * Bytes of device workspace mamba_selective_scan_fwd needs for `dims`.
+ *
+ * Zero unless the sequence is split into segments (few channels, long L: the
+ * "million-length" regime).  Then the scan runs as three launches -- per-segment
+ * aggregates (the segment's state from h = 0 and its summed step), the exclusive
+ * prefix of the associative combine (Abar_j Abar_i, Abar_j b_i + b_j) across
+ * segments (parallel-scan derivation, steps 2-4), and a final pass from each
+ * segment's true initial state -- and the workspace holds the aggregates.
+ * Depends on `dims` only.  Returns 0 for invalid dims.
+ */
+size_t mamba_selective_scan_workspace_size(mamba_scan_dims dims);
+
+/*
+ * Fused selective-scan forward.
+ *
+ *   u, delta, z : (batch, dim, seqlen)  in_dtype       z may be NULL (no gate)
+ *   A           : (dim, dstate)         float32        any real values (Mamba uses A < 0)
+ *   B, C        : (batch, dstate, seqlen) in_dtype
+ *   D           : (dim) float32 or NULL (no skip term)
+ *   delta_bias  : (dim) float32 or NULL (no bias)
+ *   delta_softplus : nonzero applies softplus to delta + delta_bias
+ *   y           : (batch, dim, seqlen)  out_dtype      written
+ *   last_state  : (batch, dim, dstate)  float32 or NULL; receives h_{L-1} (zeros when L = 0)
+ *   (when seqlen == 0, u, delta, z, B, C and y hold no elements and may be NULL)
+ *   workspace   : device buffer of at least mamba_selective_scan_workspace_size(dims)
+ *                 bytes, or NULL when that size is 0; its contents on entry do not matter
+ *
+ * Accumulation and state are float32; exp/log run on the SFU (ex2/lg2/rcp).
+ * Errors: NULL (required pointer), DIMS, ALIGN, DTYPE, WORKSPACE, CUDA.
+ */
+int mamba_selective_scan_fwd(const void* u, const void* delta, const float* A, const void* B,
+                             const void* C, const float* D, const void* z,
+                             const float* delta_bias, int delta_softplus, void* y,
+                             float* last_state, mamba_scan_dims dims, mamba_dtype in_dtype,
+                             mamba_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/*
+ * One decode token (selective_state_update): the recurrence above for a single
+ * t, applied in place to a carried state (the generation mode keeps only a
+ * fixed dim x dstate state per layer and costs O(1) per token).
+ *
+ *   state       : (batch, dim, dstate) float32, read and overwritten in place
+ *   u, delta, z : (batch, dim)   io_dtype       z may be NULL
+ *   A           : (dim, dstate)  float32
+ *   B, C        : (batch, dstate) io_dtype
+ *   D, delta_bias : (dim) float32 or NULL
+ *   y           : (batch, dim)   io_dtype       written
+ *
+ * Errors: NULL, DIMS (batch, dim >= 1; 1 <= dstate <= 16), ALIGN, DTYPE, CUDA.
+ */
+int mamba_selective_state_update(float* state, const void* u, const void* delta, const float* A,
+                                 const void* B, const void* C, const float* D, const void* z,
+                                 const float* delta_bias, int delta_softplus, void* y,
+                                 int64_t batch, int64_t dim, int64_t dstate,
+                                 mamba_dtype io_dtype, void* stream);
+
+/* A static, human-readable name for a status code. */
+const char* mamba_status_string(int status);
+
+/* ABI version of this library (major * 100 + minor). */
+int mamba_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAMBA_S6_H */

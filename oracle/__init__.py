@@ -200,3 +200,26 @@ def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, soft
     if rc != 0:
         raise ValueError("s6o_state_update rejected its arguments")
     return st, y.reshape(b, d)
+
+
+def state_update_lanes(state, u, delta_raw, A, B, C, lane_batch, D=None, z=None, delta_bias=None,
+                       softplus=True):
+    """One decode token on independent lanes: returns (new_state (nlanes, N), y (nlanes)).
+
+    state, A: (nlanes, N); u, delta_raw, z, D, delta_bias: (nlanes);
+    B, C: (nbatch, N); lane i reads row lane_batch[i].  ``state`` is not modified.
+    """
+    st = _f64(state).copy()
+    nl, N = st.shape
+    uu, dd, zz = _f64(u).reshape(nl), _f64(delta_raw).reshape(nl), _f64(z)
+    Aa, Dd, bb = _f64(A), _f64(D), _f64(delta_bias)
+    Bv, Cv = _f64(B), _f64(C)
+    assert Aa.shape == (nl, N) and Bv.shape[1] == N and Cv.shape == Bv.shape
+    lb = np.ascontiguousarray(np.asarray(lane_batch, dtype=np.int64).reshape(nl))
+    y = np.empty(nl)
+    rc = _load().s6o_state_update(
+        nl, N, Bv.shape[0], _ptr(st), _ptr(uu), _ptr(dd), _ptr(zz), _ptr(Aa), _ptr(Dd), _ptr(bb),
+        _ptr(Bv), _ptr(Cv), lb.ctypes.data_as(_lp), int(bool(softplus)), _ptr(y))
+    if rc != 0:
+        raise ValueError("s6o_state_update rejected its arguments")
+    return st, y

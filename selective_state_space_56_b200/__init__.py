@@ -1,0 +1,15 @@
+"""B200-native selective scan (S6): fused forward scan and single-token state update.
+
+The compute lives in hand-written sm_100a CUDA kernels behind a C ABI
+(``include/mamba_s6.h``, built into ``libmamba_s6.so`` in this package by
+``python -m selective_state_space_56_b200.build``).  The Python functions here
+only marshal torch tensors into that ABI.
+"""
+from .ops import (  # noqa: F401
+    MambaError,
+    load_library,
+    selective_scan_fwd,
+    selective_scan_workspace_size,
+    selective_state_update,
+    status_string,
+)

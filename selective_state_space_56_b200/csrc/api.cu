@@ -1,0 +1,153 @@
+// api.cu -- the extern "C" boundary declared in include/mamba_s6.h.
+//
+// Host-side only: validates every argument before anything is enqueued, turns
+// the plain pointers and sizes into launch arguments and forwards to the kernel
+// launchers.  No allocation, no synchronisation, no state kept between calls.
+#include <stdint.h>
+
+#include "../../include/mamba_s6.h"
+#include "s6_launch.h"
+
+namespace {
+
+constexpr int64_t kMaxDstate = 16;
+constexpr int64_t kMaxGridYZ = 65535;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool dtype_ok(int dt) { return dt == MAMBA_F32 || dt == MAMBA_BF16; }
+
+s6::DType to_dtype(int dt) { return dt == MAMBA_BF16 ? s6::DType::BF16 : s6::DType::F32; }
+
+bool mul_ok(int64_t a, int64_t b) { return a == 0 || b <= INT64_MAX / a; }
+
+// Shared size checks: positive batch/dim, dstate in [1, 16], L >= 0, and every
+// element count representable.
+bool dims_ok(int64_t batch, int64_t dim, int64_t dstate, int64_t L) {
+    if (batch < 1 || dim < 1 || dstate < 1 || dstate > kMaxDstate || L < 0) return false;
+    if (batch > kMaxGridYZ) return false;
+    if (!mul_ok(batch, dim)) return false;
+    const int64_t bd = batch * dim;
+    if (!mul_ok(bd, L) || !mul_ok(bd, dstate) || !mul_ok(bd * dstate, 8)) return false;
+    if (!mul_ok(batch * dstate, L) || !mul_ok(bd * (L > 0 ? L : 1), 8)) return false;
+    return (bd + 31) / 32 <= (int64_t)0x7fffffff;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t mamba_selective_scan_workspace_size(mamba_scan_dims dims) {
+    if (!dims_ok(dims.batch, dims.dim, dims.dstate, dims.seqlen)) return 0;
+    int64_t nseg = 1, seg_len = 0;
+    s6::plan_segments(dims.batch, dims.dim, dims.seqlen, &nseg, &seg_len);
+    if (nseg <= 1) return 0;
+    const int64_t rows = nseg * dims.batch * dims.dim;
+    // seg_h (rows x N) then seg_sum (rows), fp32; the tail rounded to 256 bytes
+    const int64_t bytes = rows * (dims.dstate + 1) * 4;
+    return (size_t)((bytes + 255) / 256 * 256);
+}
+
+int mamba_selective_scan_fwd(const void* u, const void* delta, const float* A, const void* B,
+                             const void* C, const float* D, const void* z,
+                             const float* delta_bias, int delta_softplus, void* y,
+                             float* last_state, mamba_scan_dims dims, mamba_dtype in_dtype,
+                             mamba_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+    // With seqlen == 0 the (batch, dim, 0) and (batch, dstate, 0) arrays are empty and
+    // may be NULL; only last_state (zeros) is written.
+    const bool empty = dims.seqlen == 0;
+    if (!A || (!empty && (!u || !delta || !B || !C || !y))) return MAMBA_ERR_NULL;
+    if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return MAMBA_ERR_DTYPE;
+    if (!dims_ok(dims.batch, dims.dim, dims.dstate, dims.seqlen)) return MAMBA_ERR_DIMS;
+    const void* ptrs[] = {u, delta, A, B, C, D, z, delta_bias, y, last_state};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MAMBA_ERR_ALIGN;
+
+    int64_t nseg = 1, seg_len = 0;
+    s6::plan_segments(dims.batch, dims.dim, dims.seqlen, &nseg, &seg_len);
+    if (nseg > kMaxGridYZ) return MAMBA_ERR_DIMS;
+    const size_t need = mamba_selective_scan_workspace_size(dims);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need) return MAMBA_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return MAMBA_ERR_ALIGN;
+    }
+
+    s6::ScanArgs a;
+    a.u = u;
+    a.delta = delta;
+    a.z = z;
+    a.A = A;
+    a.B = B;
+    a.C = C;
+    a.D = D;
+    a.delta_bias = delta_bias;
+    a.y = y;
+    a.last_state = last_state;
+    a.batch = dims.batch;
+    a.dim = dims.dim;
+    a.N = dims.dstate;
+    a.L = dims.seqlen;
+    a.softplus = delta_softplus;
+    a.in_dtype = to_dtype(in_dtype);
+    a.out_dtype = to_dtype(out_dtype);
+    a.nseg = nseg;
+    a.seg_len = seg_len;
+    a.seg_h = nullptr;
+    a.seg_sum = nullptr;
+    if (nseg > 1) {
+        a.seg_h = static_cast<float*>(workspace);
+        a.seg_sum = a.seg_h + nseg * dims.batch * dims.dim * dims.dstate;
+    }
+    return cuda_status(s6::launch_scan(a, static_cast<cudaStream_t>(stream)));
+}
+
+int mamba_selective_state_update(float* state, const void* u, const void* delta, const float* A,
+                                 const void* B, const void* C, const float* D, const void* z,
+                                 const float* delta_bias, int delta_softplus, void* y,
+                                 int64_t batch, int64_t dim, int64_t dstate,
+                                 mamba_dtype io_dtype, void* stream) {
+    if (!state || !u || !delta || !A || !B || !C || !y) return MAMBA_ERR_NULL;
+    if (!dtype_ok(io_dtype)) return MAMBA_ERR_DTYPE;
+    if (!dims_ok(batch, dim, dstate, 1)) return MAMBA_ERR_DIMS;
+    const void* ptrs[] = {state, u, delta, A, B, C, D, z, delta_bias, y};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MAMBA_ERR_ALIGN;
+    s6::StateUpdateArgs a;
+    a.state = state;
+    a.u = u;
+    a.delta = delta;
+    a.z = z;
+    a.A = A;
+    a.B = B;
+    a.C = C;
+    a.D = D;
+    a.delta_bias = delta_bias;
+    a.y = y;
+    a.batch = batch;
+    a.dim = dim;
+    a.N = dstate;
+    a.softplus = delta_softplus;
+    a.io_dtype = to_dtype(io_dtype);
+    return cuda_status(s6::launch_state_update(a, static_cast<cudaStream_t>(stream)));
+}
+
+const char* mamba_status_string(int status) {
+    switch (status) {
+        case MAMBA_OK: return "ok";
+        case MAMBA_ERR_NULL: return "a required pointer is NULL";
+        case MAMBA_ERR_DIMS: return "invalid sizes (batch, dim >= 1; 1 <= dstate <= 16; seqlen >= 0)";
+        case MAMBA_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+        case MAMBA_ERR_DTYPE: return "unknown dtype";
+        case MAMBA_ERR_WORKSPACE: return "workspace missing or too small";
+        case MAMBA_ERR_CUDA: return "CUDA runtime error";
+        case MAMBA_ERR_TIMEOUT: return "a bounded device wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int mamba_abi_version(void) { return 100; }
+
+}  // extern "C"

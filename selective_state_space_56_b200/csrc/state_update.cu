@@ -1,0 +1,142 @@
+// state_update.cu -- single-token selective_state_update for sm_100a.
+//
+// Decode keeps only the (batch, dim, N) fp32 state per layer and advances it by one
+// token (Mamba FAQ on generation: a fixed-size state, constant cost per token).
+// The step is a pure stream over the state: each element is read once and
+// written once in place, so the kernel is laid out for HBM: G = NMAX / 4 adjacent
+// threads share one (batch, channel) lane and each moves 16 contiguous bytes of
+// state, so a warp touches 512 consecutive bytes per access.  The per-lane
+// readout sum_n C_n h_n is finished with log2(G) xor-shuffles.
+#include "s6_device.cuh"
+#include "s6_launch.h"
+
+namespace s6 {
+namespace {
+
+struct UParams {
+    float* state;
+    const void* u;
+    const void* delta;
+    const void* z;
+    const float* A;
+    const void* B;
+    const void* C;
+    const float* D;
+    const float* delta_bias;
+    void* y;
+    int64_t batch, dim, lanes;
+    int N;
+    int softplus;
+    int vec;  // N % 4 == 0: 16-byte state / A accesses
+};
+
+template <int NMAX, typename Tio>
+__global__ void __launch_bounds__(256) state_update_kernel(const UParams p) {
+    constexpr int G = NMAX / 4;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t lane_id = gid / G;
+    const int j = (int)(gid % G);
+    const bool active = lane_id < p.lanes;
+    const int64_t li = active ? lane_id : 0;
+    const int64_t bb = li / p.dim, d = li % p.dim;
+
+    const float uu = io<Tio>::load(static_cast<const Tio*>(p.u) + li);
+    const float x = io<Tio>::load(static_cast<const Tio*>(p.delta) + li) +
+                    (p.delta_bias ? p.delta_bias[d] : 0.f);
+    const float dt = p.softplus ? softplus(x) : x;
+    const float du = dt * uu;
+
+    float st[4], a[4], bv[4], cv[4];
+    const int n0 = 4 * j;
+    float* sp = p.state + li * p.N + n0;
+    const float* ap = p.A + d * p.N + n0;
+    const Tio* bp = static_cast<const Tio*>(p.B) + bb * p.N + n0;
+    const Tio* cp = static_cast<const Tio*>(p.C) + bb * p.N + n0;
+    const bool jok = n0 < p.N;  // with N % 4 == 0, all four states exist or none
+    if (p.vec) {
+        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 s4 = (active && jok) ? *reinterpret_cast<const float4*>(sp) : z4;
+        const float4 a4 = jok ? *reinterpret_cast<const float4*>(ap) : z4;
+        st[0] = s4.x, st[1] = s4.y, st[2] = s4.z, st[3] = s4.w;
+        a[0] = a4.x, a[1] = a4.y, a[2] = a4.z, a[3] = a4.w;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            bv[k] = jok ? io<Tio>::load(bp + k) : 0.f;
+            cv[k] = jok ? io<Tio>::load(cp + k) : 0.f;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const bool ok = active && n0 + k < p.N;
+            st[k] = ok ? sp[k] : 0.f;
+            a[k] = ok ? ap[k] : 0.f;
+            bv[k] = ok ? io<Tio>::load(bp + k) : 0.f;
+            cv[k] = ok ? io<Tio>::load(cp + k) : 0.f;
+        }
+    }
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float abar = ex2(dt * (a[k] * kLog2e));
+        st[k] = fmaf(abar, st[k], du * bv[k]);
+        acc = fmaf(cv[k], st[k], acc);
+    }
+    if (active && jok) {
+        if (p.vec) {
+            *reinterpret_cast<float4*>(sp) = make_float4(st[0], st[1], st[2], st[3]);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (n0 + k < p.N) sp[k] = st[k];
+        }
+    }
+#pragma unroll
+    for (int m = G / 2; m >= 1; m /= 2) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (active && j == 0) {
+        float yv = acc + (p.D ? p.D[d] : 0.f) * uu;
+        if (p.z) yv *= silu(io<Tio>::load(static_cast<const Tio*>(p.z) + li));
+        static_cast<Tio*>(p.y)[li] = io<Tio>::from_f(yv);
+    }
+}
+
+template <int NMAX, typename Tio>
+cudaError_t launch_u(const UParams& p, cudaStream_t s) {
+    constexpr int G = NMAX / 4;
+    const int64_t threads = p.lanes * G;
+    const unsigned blocks = (unsigned)((threads + 255) / 256);
+    state_update_kernel<NMAX, Tio><<<blocks, 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename Tio>
+cudaError_t launch_u_typed(const UParams& p, cudaStream_t s) {
+    if (p.N <= 4) return launch_u<4, Tio>(p, s);
+    if (p.N <= 8) return launch_u<8, Tio>(p, s);
+    return launch_u<16, Tio>(p, s);
+}
+
+}  // namespace
+
+cudaError_t launch_state_update(const StateUpdateArgs& a, cudaStream_t stream) {
+    UParams p;
+    p.state = a.state;
+    p.u = a.u;
+    p.delta = a.delta;
+    p.z = a.z;
+    p.A = a.A;
+    p.B = a.B;
+    p.C = a.C;
+    p.D = a.D;
+    p.delta_bias = a.delta_bias;
+    p.y = a.y;
+    p.batch = a.batch;
+    p.dim = a.dim;
+    p.lanes = a.batch * a.dim;
+    p.N = (int)a.N;
+    p.softplus = a.softplus ? 1 : 0;
+    p.vec = (a.N % 4 == 0) ? 1 : 0;
+    if (a.io_dtype == DType::BF16) return launch_u_typed<__nv_bfloat16>(p, stream);
+    return launch_u_typed<float>(p, stream);
+}
+
+}  // namespace s6

@@ -1,0 +1,185 @@
+"""Thin ctypes binding over the C ABI in include/mamba_s6.h (argument marshalling only).
+
+Every function here checks that its tensors sit on one CUDA device with the
+layouts the ABI expects, allocates any output the caller did not pass (with
+torch), and forwards raw device pointers plus the current torch stream to
+``libmamba_s6.so``.  All arithmetic runs in the library's CUDA kernels; there is
+no fallback: if the library is missing or the ABI rejects the call, a
+``MambaError`` is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmamba_s6.so")
+
+MAMBA_F32, MAMBA_BF16 = 0, 1
+_DTYPES = {torch.float32: MAMBA_F32, torch.bfloat16: MAMBA_BF16}
+
+
+class MambaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s failed: %s (status %d)" % (where, status_string(status), status))
+
+
+class ScanDims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("dim", ctypes.c_int64), ("dstate", ctypes.c_int64),
+                ("seqlen", ctypes.c_int64)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load_library():
+    """Load libmamba_s6.so (build it first with ``python -m selective_state_space_56_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError("libmamba_s6.so is not built (run: python -m "
+                                  "selective_state_space_56_b200.build)")
+            lib = ctypes.CDLL(LIB_PATH)
+            vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+            lib.mamba_selective_scan_workspace_size.restype = ctypes.c_size_t
+            lib.mamba_selective_scan_workspace_size.argtypes = [ScanDims]
+            lib.mamba_selective_scan_fwd.restype = i32
+            lib.mamba_selective_scan_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp,
+                                                     ScanDims, i32, i32, vp, ctypes.c_size_t, vp]
+            lib.mamba_selective_state_update.restype = i32
+            lib.mamba_selective_state_update.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
+                                                         vp, i64, i64, i64, i32, vp]
+            lib.mamba_status_string.restype = ctypes.c_char_p
+            lib.mamba_status_string.argtypes = [i32]
+            lib.mamba_abi_version.restype = i32
+            lib.mamba_abi_version.argtypes = []
+            _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return load_library().mamba_status_string(int(status)).decode()
+    except ImportError:
+        return "status %d" % status
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(t, name, device, shape=None, dtypes=None):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.device != device:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError("%s has dtype %s, expected one of %s" % (name, t.dtype, dtypes))
+
+
+def selective_scan_workspace_size(batch: int, dim: int, dstate: int, seqlen: int) -> int:
+    """Bytes of workspace ``mamba_selective_scan_fwd`` needs for these sizes (0 if none)."""
+    return int(load_library().mamba_selective_scan_workspace_size(
+        ScanDims(batch, dim, dstate, seqlen)))
+
+
+def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+                       out_dtype=None, y=None, last_state=None, return_last_state=False,
+                       workspace=None):
+    """Fused selective scan.  u, delta, z: (batch, dim, L); A: (dim, N) fp32;
+    B, C: (batch, N, L); D, delta_bias: (dim) fp32.  Returns y (batch, dim, L)
+    [and last_state (batch, dim, N) fp32]."""
+    if not isinstance(u, torch.Tensor) or u.dim() != 3:
+        raise ValueError("u must be a (batch, dim, L) tensor")
+    dev = u.device
+    if dev.type != "cuda":
+        raise ValueError("selective_scan_fwd runs on CUDA tensors only")
+    b, d, L = u.shape
+    N = A.shape[1] if A.dim() == 2 else -1
+    in_dt = u.dtype
+    if in_dt not in _DTYPES:
+        raise ValueError("unsupported input dtype %s" % in_dt)
+    out_dt = in_dt if out_dtype is None else out_dtype
+    if out_dt not in _DTYPES:
+        raise ValueError("unsupported output dtype %s" % out_dt)
+    _check(u, "u", dev, (b, d, L), (in_dt,))
+    _check(delta, "delta", dev, (b, d, L), (in_dt,))
+    _check(z, "z", dev, (b, d, L), (in_dt,))
+    _check(A, "A", dev, (d, N), (torch.float32,))
+    _check(B, "B", dev, (b, N, L), (in_dt,))
+    _check(C, "C", dev, (b, N, L), (in_dt,))
+    _check(D, "D", dev, (d,), (torch.float32,))
+    _check(delta_bias, "delta_bias", dev, (d,), (torch.float32,))
+    if y is None:
+        y = torch.empty((b, d, L), dtype=out_dt, device=dev)
+    _check(y, "y", dev, (b, d, L), (out_dt,))
+    if last_state is None and return_last_state:
+        last_state = torch.empty((b, d, N), dtype=torch.float32, device=dev)
+    _check(last_state, "last_state", dev, (b, d, N), (torch.float32,))
+    lib = load_library()
+    dims = ScanDims(b, d, N, L)
+    need = int(lib.mamba_selective_scan_workspace_size(dims))
+    if need > 0 and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        rc = lib.mamba_selective_scan_fwd(
+            _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+            int(bool(delta_softplus)), _ptr(y), _ptr(last_state), dims, _DTYPES[in_dt],
+            _DTYPES[out_dt], _ptr(workspace), ws_bytes, _stream_handle(dev))
+    if rc != 0:
+        raise MambaError(rc, "mamba_selective_scan_fwd")
+    if return_last_state:
+        return y, last_state
+    return y
+
+
+def selective_state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                           delta_softplus=True, y=None):
+    """One decode token, in place on ``state`` (batch, dim, N) fp32.
+    u, delta, z: (batch, dim); B, C: (batch, N); A: (dim, N).  Returns y (batch, dim)."""
+    if not isinstance(state, torch.Tensor) or state.dim() != 3:
+        raise ValueError("state must be a (batch, dim, N) tensor")
+    dev = state.device
+    if dev.type != "cuda":
+        raise ValueError("selective_state_update runs on CUDA tensors only")
+    b, d, N = state.shape
+    io_dt = u.dtype
+    if io_dt not in _DTYPES:
+        raise ValueError("unsupported dtype %s" % io_dt)
+    _check(state, "state", dev, (b, d, N), (torch.float32,))
+    _check(u, "u", dev, (b, d), (io_dt,))
+    _check(delta, "delta", dev, (b, d), (io_dt,))
+    _check(z, "z", dev, (b, d), (io_dt,))
+    _check(A, "A", dev, (d, N), (torch.float32,))
+    _check(B, "B", dev, (b, N), (io_dt,))
+    _check(C, "C", dev, (b, N), (io_dt,))
+    _check(D, "D", dev, (d,), (torch.float32,))
+    _check(delta_bias, "delta_bias", dev, (d,), (torch.float32,))
+    if y is None:
+        y = torch.empty((b, d), dtype=io_dt, device=dev)
+    _check(y, "y", dev, (b, d), (io_dt,))
+    with torch.cuda.device(dev):
+        rc = load_library().mamba_selective_state_update(
+            _ptr(state), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+            _ptr(delta_bias), int(bool(delta_softplus)), _ptr(y), b, d, N, _DTYPES[io_dt],
+            _stream_handle(dev))
+    if rc != 0:
+        raise MambaError(rc, "mamba_selective_state_update")
+    return y

@@ -1,0 +1,143 @@
+"""CPU-side checks of the C ABI: the library loads, exports every declared symbol,
+and rejects bad arguments on the host before anything is launched.
+
+No compute call is made here (there is no GPU): every call below fails
+validation, which runs before the library touches the CUDA runtime.  Fake
+pointers are small integers that are never dereferenced.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from selective_state_space_56_b200 import build as s6build
+from selective_state_space_56_b200 import ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+OK, ERR_NULL, ERR_DIMS, ERR_ALIGN, ERR_DTYPE, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
+
+
+@pytest.fixture(scope="module")
+def lib():
+    s6build.build()
+    return ops.load_library()
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(mamba_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert {"mamba_selective_scan_fwd", "mamba_selective_state_update",
+            "mamba_selective_scan_workspace_size", "mamba_status_string"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), "symbol %s declared in include/ but not exported" % n
+
+
+def test_built_for_sm100a_only():
+    assert "arch=compute_100a,code=sm_100a" in " ".join(s6build.ARCH)
+
+
+def test_status_strings(lib):
+    for code in range(-7, 1):
+        assert ops.status_string(code) and ops.status_string(code) != "unknown status"
+    assert ops.status_string(-99) == "unknown status"
+    assert lib.mamba_abi_version() >= 100
+
+
+def _dims(b=2, d=64, n=16, L=128):
+    return ops.ScanDims(b, d, n, L)
+
+
+A16 = 16 * 1024  # a fake, 16-byte aligned, never dereferenced address
+
+
+def _scan(lib, **kw):
+    args = dict(u=A16, delta=A16, A=A16, B=A16, C=A16, D=None, z=None, bias=None, sp=1, y=A16,
+                last=None, dims=_dims(), i=0, o=0, ws=None, wsb=0)
+    args.update(kw)
+    vp = lambda v: None if v is None else ctypes.c_void_p(v)  # noqa: E731
+    return lib.mamba_selective_scan_fwd(
+        vp(args["u"]), vp(args["delta"]), vp(args["A"]), vp(args["B"]), vp(args["C"]),
+        vp(args["D"]), vp(args["z"]), vp(args["bias"]), args["sp"], vp(args["y"]),
+        vp(args["last"]), args["dims"], args["i"], args["o"], vp(args["ws"]), args["wsb"], None)
+
+
+@pytest.mark.parametrize("field", ["u", "delta", "A", "B", "C", "y"])
+def test_scan_null_required_pointer(lib, field):
+    assert _scan(lib, **{field: None}) == ERR_NULL
+
+
+@pytest.mark.parametrize("dims", [(0, 64, 16, 8), (2, 0, 16, 8), (2, 64, 0, 8), (2, 64, 17, 8),
+                                  (2, 64, 16, -1), (70000, 4, 16, 8), (1 << 40, 1 << 40, 16, 8)])
+def test_scan_bad_dims(lib, dims):
+    assert _scan(lib, dims=_dims(*dims)) == ERR_DIMS
+
+
+@pytest.mark.parametrize("i,o", [(2, 0), (0, 7), (-1, 1)])
+def test_scan_bad_dtype(lib, i, o):
+    assert _scan(lib, i=i, o=o) == ERR_DTYPE
+
+
+@pytest.mark.parametrize("field", ["u", "delta", "A", "B", "C", "D", "z", "bias", "y", "last"])
+def test_scan_misaligned_pointer(lib, field):
+    assert _scan(lib, **{field: A16 + 4}) == ERR_ALIGN
+
+
+def test_scan_workspace_checks(lib):
+    long_dims = _dims(1, 64, 16, 1 << 16)  # few channels, long L: the split plan needs scratch
+    need = lib.mamba_selective_scan_workspace_size(long_dims)
+    assert need > 0 and need % 256 == 0
+    assert _scan(lib, dims=long_dims) == ERR_WORKSPACE
+    assert _scan(lib, dims=long_dims, ws=A16, wsb=need - 1) == ERR_WORKSPACE
+    assert _scan(lib, dims=long_dims, ws=A16 + 8, wsb=need) == ERR_ALIGN
+
+
+def test_workspace_plan(lib):
+    ws = lambda *d: lib.mamba_selective_scan_workspace_size(_dims(*d))  # noqa: E731
+    assert ws(4, 5120, 16, 4096) == 0          # enough channels: one pass
+    assert ws(8, 1536, 16, 2048) == 0
+    assert ws(1, 2048, 16, 1 << 20) > 0        # million-length: split
+    assert ws(1, 2048, 16, 1 << 20) < 64 << 20
+    assert ws(0, 2048, 16, 1 << 20) == 0       # invalid dims report 0
+
+
+def _upd(lib, **kw):
+    args = dict(state=A16, u=A16, delta=A16, A=A16, B=A16, C=A16, D=None, z=None, bias=None,
+                sp=1, y=A16, b=4, d=64, n=16, io=1)
+    args.update(kw)
+    vp = lambda v: None if v is None else ctypes.c_void_p(v)  # noqa: E731
+    return lib.mamba_selective_state_update(
+        vp(args["state"]), vp(args["u"]), vp(args["delta"]), vp(args["A"]), vp(args["B"]),
+        vp(args["C"]), vp(args["D"]), vp(args["z"]), vp(args["bias"]), args["sp"], vp(args["y"]),
+        args["b"], args["d"], args["n"], args["io"], None)
+
+
+@pytest.mark.parametrize("field", ["state", "u", "delta", "A", "B", "C", "y"])
+def test_update_null(lib, field):
+    assert _upd(lib, **{field: None}) == ERR_NULL
+
+
+def test_update_dims_dtype_align(lib):
+    assert _upd(lib, b=0) == ERR_DIMS
+    assert _upd(lib, n=17) == ERR_DIMS
+    assert _upd(lib, d=-3) == ERR_DIMS
+    assert _upd(lib, io=5) == ERR_DTYPE
+    for f in ("state", "u", "delta", "A", "B", "C", "D", "z", "bias", "y"):
+        assert _upd(lib, **{f: A16 + 2}) == ERR_ALIGN, f
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    u = torch.zeros(1, 2, 8)
+    with pytest.raises(ValueError):
+        ops.selective_scan_fwd(u, u, torch.zeros(2, 4), torch.zeros(1, 4, 8), torch.zeros(1, 4, 8))

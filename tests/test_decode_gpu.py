@@ -1,0 +1,117 @@
+"""Parity of the CUDA selective_state_update (decode) with the fp64 oracle (needs a B200).
+
+The decode workload (batch 256, dim 5120, N 16, bf16 I/O, fp32 state) runs 1000
+steps with fresh seeded inputs each step, as the bench does.  The oracle
+checks the full tensors after step 1 and a fixed sample of (batch, channel)
+lanes, carried in fp64 through all 1000 steps, after steps 10 and 1000.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from selective_state_space_56_b200 import inputs, ops
+from tests.s6_compare import check_bf16_out, check_fp32, check_rms, rms, to64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def test_decode_workload_1000_steps(cuda_ok):
+    w = inputs.DECODE_WORKLOAD
+    prm = inputs.decode_params(w)
+    A, D, bias = prm["A"], prm["D"], prm["delta_bias"]
+    state = prm["state0"].to(DEV)
+    Ag, Dg, bg = A.to(DEV), D.to(DEV), bias.to(DEV)
+    rng = np.random.default_rng(56005)
+    nl = 512
+    lb = rng.integers(0, w.batch, nl)
+    ld = rng.integers(0, w.dim, nl)
+    ref_state = to64(prm["state0"])[lb, ld]          # (nl, N) fp64 carried by the oracle
+    A64, D64, b64 = to64(A)[ld], to64(D)[ld], to64(bias)[ld]
+    for step in range(w.steps):
+        x = inputs.decode_step_inputs(step, w)
+        if step == 0:
+            full_prev = to64(state.cpu())
+        g = {k: v.to(DEV) for k, v in x.items()}
+        y = ops.selective_state_update(state, g["u"], g["delta"], Ag, g["B"], g["C"], D=Dg,
+                                       z=g["z"], delta_bias=bg)
+        st_new, y_ref = oracle.state_update_lanes(
+            ref_state, to64(x["u"])[lb, ld], to64(x["delta"])[lb, ld], A64, x["B"], x["C"], lb,
+            D=D64, z=to64(x["z"])[lb, ld], delta_bias=b64)
+        ref_state = st_new
+        if step == 0:
+            full_state, full_y = oracle.state_update(full_prev, x["u"], x["delta"], A, x["B"],
+                                                     x["C"], D=D, z=x["z"], delta_bias=bias)
+            torch.cuda.synchronize()
+            check_bf16_out(y.cpu(), full_y, "y step 1 (full)")
+            check_rms(state.cpu(), full_state, "state step 1 (full)")
+        if step + 1 in (10, w.steps):
+            torch.cuda.synchronize()
+            got_y = to64(y.cpu())[lb, ld]
+            got_s = to64(state.cpu())[lb, ld]
+            check_bf16_out(got_y, y_ref, "y step %d (sampled)" % (step + 1))
+            check_rms(got_s, ref_state, "state step %d (sampled)" % (step + 1))
+    assert rms(ref_state) > 0
+
+
+@pytest.mark.parametrize("N", [1, 4, 6, 8, 12, 16])
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+def test_decode_shapes(cuda_ok, N, io):
+    b, d = 3, 37
+    g = torch.Generator().manual_seed(100 + N)
+    st0 = 0.1 * torch.randn(b, d, N, generator=g)
+    x = {k: torch.randn(*s, generator=g).to(io) for k, s in
+         dict(u=(b, d), delta=(b, d), z=(b, d), B=(b, N), C=(b, N)).items()}
+    A = -torch.arange(1, N + 1, dtype=torch.float32).expand(d, N).contiguous()
+    D = torch.randn(d, generator=g)
+    bias = torch.log(torch.expm1(0.001 + 0.099 * torch.rand(d, generator=g, dtype=torch.float64))).float()
+    state = st0.to(DEV)
+    y = ops.selective_state_update(state, *(x[k].to(DEV) for k in ("u", "delta")), A.to(DEV),
+                                   x["B"].to(DEV), x["C"].to(DEV), D=D.to(DEV), z=x["z"].to(DEV),
+                                   delta_bias=bias.to(DEV))
+    s_ref, y_ref = oracle.state_update(st0, x["u"], x["delta"], A, x["B"], x["C"], D=D, z=x["z"],
+                                       delta_bias=bias)
+    torch.cuda.synchronize()
+    if io == torch.float32:
+        check_fp32(y.cpu(), y_ref, "y")
+        check_fp32(state.cpu(), s_ref, "state")
+    else:
+        check_bf16_out(y.cpu(), y_ref, "y")
+        check_rms(state.cpu(), s_ref, "state")
+
+
+def test_decode_without_optional_inputs(cuda_ok):
+    b, d, N = 2, 50, 16
+    g = torch.Generator().manual_seed(5)
+    st0 = torch.randn(b, d, N, generator=g)
+    u, dl = torch.randn(b, d, generator=g), torch.rand(b, d, generator=g) * 0.5
+    B, C = torch.randn(b, N, generator=g), torch.randn(b, N, generator=g)
+    A = -torch.rand(d, N, generator=g) - 0.1
+    state = st0.to(DEV)
+    y = ops.selective_state_update(state, u.to(DEV), dl.to(DEV), A.to(DEV), B.to(DEV), C.to(DEV),
+                                   delta_softplus=False)
+    s_ref, y_ref = oracle.state_update(st0, u, dl, A, B, C, softplus=False)
+    torch.cuda.synchronize()
+    check_fp32(y.cpu(), y_ref, "y")
+    check_fp32(state.cpu(), s_ref, "state")
+
+
+def test_decode_steps_reproduce_the_scan(cuda_ok):
+    """L decode steps from a zero state give the scan's y_t and last_state (GPU vs GPU)."""
+    b, d, N, L = 2, 40, 16, 48
+    p = inputs.scan_inputs(b, d, N, L, in_dtype=torch.float32, seed=77)
+    g = {k: (None if v is None else v.to(DEV)) for k, v in p.items()}
+    y_scan, st_scan = ops.selective_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"],
+                                             z=g["z"], delta_bias=g["delta_bias"],
+                                             return_last_state=True)
+    state = torch.zeros(b, d, N, device=DEV)
+    ys = []
+    for t in range(L):
+        ys.append(ops.selective_state_update(
+            state, g["u"][..., t].contiguous(), g["delta"][..., t].contiguous(), g["A"],
+            g["B"][..., t].contiguous(), g["C"][..., t].contiguous(), D=g["D"],
+            z=g["z"][..., t].contiguous(), delta_bias=g["delta_bias"]))
+    torch.cuda.synchronize()
+    check_fp32(torch.stack(ys, -1).cpu(), y_scan.cpu(), "decode y vs scan y")
+    check_fp32(state.cpu(), st_scan.cpu(), "decode state vs scan last_state")
