@@ -122,6 +122,26 @@ int mamba_selective_state_update(float* state, const void* u, const void* delta,
                                  int64_t batch, int64_t dim, int64_t dstate,
                                  mamba_dtype io_dtype, void* stream);
 
+/*
+ * Reads the library's device error word on `stream`, synchronising that stream.
+ * Every device-side wait in the kernels (on the completion barrier of an
+ * asynchronous tile copy) is bounded to about a second; a wait that gives up sets
+ * the word and its CTA stops instead of hanging the GPU.  With `clear` nonzero the
+ * word is reset.  Returns MAMBA_OK, MAMBA_ERR_TIMEOUT if a wait gave up since the
+ * last clear (outputs of that call are then undefined), or MAMBA_ERR_CUDA.
+ */
+int mamba_check_device_error(int clear, void* stream);
+
+/*
+ * Diagnostic: evaluates 2^x for n floats three ways on the device -- the FMA-pipe
+ * polynomial the scan uses for part of its Abar factors (out_fma), the SFU
+ * ex2.approx instruction (out_sfu) and CUDA's exp2f (out_lib) -- so tests can bound
+ * the polynomial's error.  All pointers are device arrays of n floats.
+ * Errors: NULL, DIMS (n < 0), CUDA.
+ */
+int mamba_diag_exp2(const float* x, float* out_fma, float* out_sfu, float* out_lib, int64_t n,
+                    void* stream);
+
 /* A static, human-readable name for a status code. */
 const char* mamba_status_string(int status);
 

@@ -7,6 +7,7 @@ only marshal torch tensors into that ABI.
 """
 from .ops import (  # noqa: F401
     MambaError,
+    check_device_error,
     load_library,
     selective_scan_fwd,
     selective_scan_workspace_size,

@@ -134,6 +134,13 @@ int mamba_selective_state_update(float* state, const void* u, const void* delta,
     return cuda_status(s6::launch_state_update(a, static_cast<cudaStream_t>(stream)));
 }
 
+int mamba_check_device_error(int clear, void* stream) {
+    unsigned word = 0;
+    if (s6::read_device_error(&word, clear != 0, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return MAMBA_ERR_CUDA;
+    return word ? MAMBA_ERR_TIMEOUT : MAMBA_OK;
+}
+
 const char* mamba_status_string(int status) {
     switch (status) {
         case MAMBA_OK: return "ok";

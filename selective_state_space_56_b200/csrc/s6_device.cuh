@@ -34,18 +34,23 @@ __device__ __forceinline__ float rcp(float x) {
     return y;
 }
 
-// softplus(x) = log(1 + e^x) from one ex2 and one lg2.
-//  * x > 15: log(1 + e^x) - x < e^-15, below half an fp32 ulp of x; return x.
-//  * x < -5: e = e^x < 6.8e-3 and log1p(e) = e - e^2/2 + e^3/3 - ...; three terms
-//    leave a relative error under 1e-7, where forming 1 + e in fp32 would lose
-//    up to 1e-5 of the result.
-//  * otherwise log2(1 + e) * ln 2, with 1 + e >= 1.0067 so its rounding is benign.
+// log1p(e) / e on [0, 1] as a degree-7 polynomial (Remez fit for relative error made
+// for this library: 1.9e-7 in exact arithmetic, 3.3e-7 with fp32 Horner steps).
+__device__ __forceinline__ float log1p_over_x(float e) {
+    float q = fmaf(-8.5392082e-3f, e, 4.4089634e-2f);
+    q = fmaf(q, e, -1.0768171e-1f);
+    q = fmaf(q, e, 1.7745242e-1f);
+    q = fmaf(q, e, -2.4495463e-1f);
+    q = fmaf(q, e, 3.3275479e-1f);
+    q = fmaf(q, e, -4.9997404e-1f);
+    return fmaf(q, e, 9.9999982e-1f);
+}
+
+// softplus(x) = log(1 + e^x) = max(x, 0) + log1p(e^-|x|): one SFU exponential and a
+// polynomial, no cancellation for either sign of x (e^-|x| lies in (0, 1]).
 __device__ __forceinline__ float softplus(float x) {
-    float e = ex2(x * kLog2e);
-    float small = e * (1.f - e * (0.5f - e * (1.f / 3.f)));
-    float mid = lg2(1.f + e) * kLn2;
-    float r = x < -5.f ? small : mid;
-    return x > 15.f ? x : r;
+    const float e = ex2(-fabsf(x) * kLog2e);
+    return fmaxf(x, 0.f) + e * log1p_over_x(e);
 }
 
 // z * sigmoid(z) = z / (1 + e^-z); e^-z = +inf for very negative z gives z * 0.
@@ -76,6 +81,189 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+}  // namespace s6
+
+namespace s6 {
+
+// Two fp32 lanes in one 64-bit register pair, for the packed sm_100 FP32 instructions
+// (add/mul/fma .f32x2: one issue slot for two operations).
+struct f2 {
+    unsigned long long v;
+};
+
+__device__ __forceinline__ f2 pack2(float lo, float hi) {
+    f2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack2(f2 x, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x.v));
+}
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+    f2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d.v) : "l"(a.v), "l"(b.v), "l"(c.v));
+    return d;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+    f2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
+    return d;
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+    f2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
+    return d;
+}
+__device__ __forceinline__ f2 sub2(f2 a, f2 b) {
+    f2 d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
+    return d;
+}
+
+// 2^x on both halves using only the FMA and integer pipes, so part of the exponentials
+// can bypass the SFU.  Cody-Waite style split in base 2: x is clamped to [-126, 127],
+// j = rint(x) is obtained by adding and subtracting 1.5 * 2^23 (which also leaves j in
+// the low mantissa bits of the sum), f = x - j lies in [-1/2, 1/2], 2^f comes from a
+// degree-5 polynomial fitted here by the Remez exchange for minimum relative error on
+// [-1/2, 1/2] (max 7.5e-8 in exact arithmetic, 2.1e-7 with fp32 Horner steps, about
+// the SFU's ex2.approx bound), and 2^j is added into the exponent field as j << 23.
+__device__ __forceinline__ f2 exp2_fma2(f2 x) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    float x0, x1;
+    unpack2(x, x0, x1);
+    x0 = fminf(fmaxf(x0, -126.f), 127.f);
+    x1 = fminf(fmaxf(x1, -126.f), 127.f);
+    const f2 xc = pack2(x0, x1);
+    const f2 t = add2(xc, pack2(kRound, kRound));
+    const f2 f = sub2(xc, sub2(t, pack2(kRound, kRound)));
+    f2 p = fma2(pack2(1.3276472e-3f, 1.3276472e-3f), f, pack2(9.6755410e-3f, 9.6755410e-3f));
+    p = fma2(p, f, pack2(5.5507131e-2f, 5.5507131e-2f));
+    p = fma2(p, f, pack2(2.4022120e-1f, 2.4022120e-1f));
+    p = fma2(p, f, pack2(6.9314694e-1f, 6.9314694e-1f));
+    p = fma2(p, f, pack2(1.0000001f, 1.0000001f));
+    float t0, t1, p0, p1;
+    unpack2(t, t0, t1);
+    unpack2(p, p0, p1);
+    return pack2(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+
+// A bf16 pair (element 0 in the low half of the word) widened exactly to an fp32 pair.
+__device__ __forceinline__ f2 bf16pair(uint32_t w) {
+    return pack2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+// 2^x on both halves (two SFU operations).
+__device__ __forceinline__ f2 ex2x2(f2 x) {
+    float lo, hi;
+    unpack2(x, lo, hi);
+    return pack2(ex2(lo), ex2(hi));
+}
+
+// Four consecutive input elements of type T as one aligned vector load.
+template <typename T> struct vec4;
+template <> struct vec4<float> {
+    using type = float4;
+    __device__ __forceinline__ static void to_f(const type& v, float (&o)[4]) {
+        o[0] = v.x, o[1] = v.y, o[2] = v.z, o[3] = v.w;
+    }
+};
+template <> struct vec4<__nv_bfloat16> {
+    using type = uint2;  // 4 x bf16
+    __device__ __forceinline__ static void to_f(const type& v, float (&o)[4]) {
+        o[0] = __uint_as_float(v.x << 16);
+        o[1] = __uint_as_float(v.x & 0xffff0000u);
+        o[2] = __uint_as_float(v.y << 16);
+        o[3] = __uint_as_float(v.y & 0xffff0000u);
+    }
+};
+
+}  // namespace s6
+
+// ---- Tensor-memory-accelerator (TMA) bulk copies and mbarriers (sm_90+ PTX) ----
+namespace s6 {
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+// Make barrier initialisation visible to the async (TMA) proxy.
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Order this thread's earlier generic-proxy shared-memory accesses before later
+// async-proxy (TMA) accesses of the same memory.
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Bounded wait for phase `parity` of `bar`: gives up after `limit_cycles` SM clocks
+// (about a second) and returns false, so a lost transfer cannot hang the GPU.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  long long limit_cycles) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long start = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - start > limit_cycles) return false;
+    }
+    return true;
+}
+
+// 3-D tiled bulk tensor load global -> shared, completing on `bar` (transaction bytes).
+// c0 is the innermost coordinate; out-of-range elements are filled with zeros.
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// 3-D tiled bulk tensor store shared -> global; elements outside the tensor are skipped.
+__device__ __forceinline__ void tma_store_3d(const void* tmap, const void* src, int c0, int c1,
+                                             int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(tmap)),
+        "r"(smem_addr(src)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+__device__ __forceinline__ void tma_store_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until at most N committed store groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void tma_store_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until every committed store group has completed.
+__device__ __forceinline__ void tma_store_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 }  // namespace s6

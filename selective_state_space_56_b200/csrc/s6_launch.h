@@ -45,8 +45,9 @@ struct StateUpdateArgs {
     DType io_dtype;
 };
 
-// Time steps one CTA stages per chunk; a split sequence's segments are multiples of it.
-constexpr int kChunk = 64;
+// A split sequence's segments are multiples of this many steps (a multiple of every
+// chunk length a scan kernel stages at once).
+constexpr int kChunk = 128;
 
 // Split plan for a problem: number of segments and their length (a multiple of kChunk).
 void plan_segments(int64_t batch, int64_t dim, int64_t L, int64_t* nseg, int64_t* seg_len);
@@ -54,5 +55,9 @@ void plan_segments(int64_t batch, int64_t dim, int64_t L, int64_t* nseg, int64_t
 // Each returns a cudaError_t from the launches (cudaSuccess when all were enqueued).
 cudaError_t launch_scan(const ScanArgs& a, cudaStream_t stream);
 cudaError_t launch_state_update(const StateUpdateArgs& a, cudaStream_t stream);
+
+// Reads (and optionally clears) the device error word on `stream`, synchronising it.
+// Bit 0: a bounded device-side wait gave up.
+cudaError_t read_device_error(unsigned* out, bool clear, cudaStream_t stream);
 
 }  // namespace s6

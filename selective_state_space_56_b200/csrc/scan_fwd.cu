@@ -1,19 +1,24 @@
 // scan_fwd.cu -- fused selective-scan (S6) forward for sm_100a.
 //
-// One CTA owns 32 channels of one batch row (and, for a split sequence, one
-// segment of L) and walks L in chunks of kChunk steps:
+// One CTA owns a tile of CH channels of one batch row (and, for a split sequence,
+// one segment of L) and walks L in chunks of T steps:
 //
-//   stage     u, delta, z rows and the batch's B, C rows of the chunk are copied
-//             global -> shared with 16-byte async copies (double-buffered, the next
-//             chunk streams in while this one computes);
-//   phase A   per (channel, t): Delta = softplus(delta + bias), Delta*u  (one warp
-//             per 32/P channels; lanes walk t, so every access is conflict-free);
+//   stage     one thread issues 3-D TMA bulk-tensor loads of the chunk's u, delta, z
+//             rows and the batch's B, C rows into shared memory (double-buffered,
+//             completion on an mbarrier; the tensor edges are zero-filled by the
+//             copy engine).  Rows whose length is not a multiple of 16 bytes cannot
+//             be described to TMA and are staged element-wise instead;
+//   convert   B, C of the chunk -> fp32, time-major, through 4x4 register blocks;
+//   phase A   per (channel, t): Delta = softplus(delta + bias), Delta*u  (each warp
+//             on its own channels, four steps per lane);
 //   phase B   the recurrence.  P lanes share a channel, each holding NS = N/P states
 //             in registers: Abar = 2^(Delta * A log2 e) on the SFU,
-//             h = Abar h + (Delta u) B, partial y = sum C h.  The P partial sums of
-//             each t are combined by a transpose-reduce over lanes (P - 1 shuffles
-//             per P steps), leaving one lane with the complete C.h for one t;
-//   phase C   y = (C.h + D u) * silu(z), rounded to the output type and stored.
+//             h = Abar h + (Delta u) B, partial y = sum C h, two states per packed
+//             fp32x2 instruction.  The P partial sums of each t are combined by a
+//             transpose-reduce over lanes (P - 1 shuffles per P steps), leaving one
+//             lane with the complete C.h for one t;
+//   phase C   y = (C.h + D u) * silu(z), rounded to the output type into a shared
+//             tile that one thread writes back with a TMA bulk-tensor store.
 //
 // The expanded state (batch, L, dim, N) exists only in registers (Mamba,
 // "Hardware-aware state expansion": load Delta, A, B, C to on-chip memory,
@@ -27,13 +32,27 @@
 // exp(A * sum Delta_s) * start_s + end_s (the pair (prod Abar, h_end) of segment s
 // combined with the prefix before it); (3) every segment rescans from its true
 // start state and writes y.
+//
+// Every wait on an mbarrier is bounded (about a second of SM clocks); a wait that
+// gives up sets bit 0 of the device error word and the CTA leaves its loop.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
+#include <mutex>
+#include <cstring>
 
 #include "s6_device.cuh"
 #include "s6_launch.h"
 
 namespace s6 {
+
+// Bit 0: a bounded device wait gave up (read and cleared through read_device_error).
+__device__ unsigned int g_device_error = 0;
+
 namespace {
+
+constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at the SM clock
 
 struct KParams {
     const void* u;
@@ -52,34 +71,91 @@ struct KParams {
     int N;
     int nseg;
     int softplus;
-    int aligned;
+    int y_vec;  // L % 4 == 0: four outputs per vector store
+    int y_tma;  // output rows are 16-byte multiples: tiles go back by TMA store
 };
+
+// TMA descriptors of the operands (unused when rows are not 16-byte multiples).
+struct TMaps {
+    CUtensorMap u, dr, z, B, C, y;
+};
+
+// Four outputs as one 8-byte (bf16) or 16-byte (fp32) store.
+__device__ __forceinline__ void store4(float* dst, const float (&o)[4]) {
+    *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+}
+__device__ __forceinline__ void store4(__nv_bfloat16* dst, const float (&o)[4]) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(o[0], o[1]);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(o[2], o[3]);
+    uint2 v;
+    v.x = *reinterpret_cast<uint32_t*>(&lo);
+    v.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(dst) = v;
+}
 
 enum Mode : int { kFull = 0, kAggregate = 1 };
 
+// Tuning of the N = 16 instantiation: lanes per channel, warps per CTA, chunk length.
+#ifndef S6_P16
+#define S6_P16 4
+#endif
+#ifndef S6_WARPS16
+#define S6_WARPS16 3
+#endif
+#ifndef S6_CHUNK
+#define S6_CHUNK 32
+#endif
+// bf16 inputs keep B, C as bf16 pairs in shared memory (half the bytes per lane-step).
+#ifndef S6_PACKBC
+#define S6_PACKBC 1
+#endif
+// Abar pairs evaluated on the FMA pipe (exp2_fma2) instead of the SFU: 0 = none,
+// 1 = the second pair of every other step (a quarter of them), 2 = the second pair of
+// every step (half).
+#ifndef S6_POLY
+#define S6_POLY 0
+#endif
+
+constexpr size_t align128(size_t x) { return (x + 127) / 128 * 128; }
+
 // Shared-memory carve-up for one instantiation.
-template <int NMAX, int P, typename Tin>
+template <int NMAX, int P, int WARPS_, int T_, typename Tin, typename Tout>
 struct Layout {
-    static constexpr int T = kChunk;
+    static constexpr int T = T_;
     static constexpr int NS = NMAX / P;        // states per lane
-    static constexpr int CW = 32 / P;          // channels per warp
-    static constexpr int WARPS = P;            // 32 channels per CTA
-    static constexpr int CH = WARPS * CW;
+    static constexpr int G = 32 / P;           // channels per warp
+    static constexpr int WARPS = WARPS_;
+    static constexpr int CH = WARPS * G;       // channels per CTA
     static constexpr int THREADS = WARPS * 32;
     static constexpr int RS = T + 4;           // fp32 row stride: rows land 16 B apart in banks
-    static constexpr int PADB = 16 / (int)sizeof(Tin);
-    static constexpr int RB = T + PADB;        // raw B/C row stride (elements)
-    static constexpr size_t stage_elems = (size_t)3 * CH * T + (size_t)2 * NMAX * RB;
-    static constexpr size_t stage_bytes = stage_elems * sizeof(Tin);
-    static constexpr size_t off_bt = 2 * stage_bytes;            // float [T][NMAX]
-    static constexpr size_t off_ct = off_bt + (size_t)T * NMAX * 4;
-    static constexpr size_t off_del = off_ct + (size_t)T * NMAX * 4;  // float [CH][RS]
+    static constexpr size_t rows_bytes = (size_t)CH * T * sizeof(Tin);    // one of u, delta, z
+    static constexpr size_t coef_bytes = (size_t)NMAX * T * sizeof(Tin);  // one of B, C
+    static constexpr size_t off_dr = align128(rows_bytes);
+    static constexpr size_t off_z = 2 * off_dr;
+    static constexpr size_t off_B = 3 * off_dr;
+    static constexpr size_t off_C = off_B + align128(coef_bytes);
+    static constexpr size_t stage_bytes = off_C + align128(coef_bytes);
+    // Per-step coefficients for the recurrence.  bf16 inputs: one 16-byte group per
+    // (step, 4 states) holding B[4] and C[4] as bf16 pairs; fp32 inputs: B and C as
+    // fp32 [T][NMAX] each.
+    static constexpr bool kPackedBC = sizeof(Tin) == 2 && S6_PACKBC;
+    // Two buffers (chunk parity), so a chunk's coefficients can be written while the
+    // previous chunk's are still being read.
+    static constexpr size_t coef_fp32_bytes = (size_t)T * NMAX * 4;
+    static constexpr size_t coef_bytes_all = (kPackedBC ? 1 : 2) * coef_fp32_bytes;
+    static constexpr size_t off_coef = 2 * stage_bytes;
+    static constexpr size_t off_del = off_coef + 2 * coef_bytes_all;   // float [CH][RS]
     static constexpr size_t off_du = off_del + (size_t)CH * RS * 4;
     static constexpr size_t off_y = off_du + (size_t)CH * RS * 4;
-    static constexpr size_t off_par = off_y + (size_t)CH * RS * 4;   // bias[CH], D[CH]
-    static constexpr size_t bytes = off_par + (size_t)2 * CH * 4;
+    static constexpr size_t off_out = align128(off_y + (size_t)CH * RS * 4);  // Tout [CH][T]
+    static constexpr size_t out_bytes = align128((size_t)CH * T * sizeof(Tout));
+    static constexpr size_t off_par = off_out + out_bytes;               // bias[CH], D[CH]
+    static constexpr size_t off_bar = align128(off_par + (size_t)2 * CH * 4);  // 2 mbarriers
+    static constexpr size_t bytes = off_bar + 16;
     static_assert(NS % 4 == 0, "states per lane must be a multiple of 4");
-    static_assert(stage_bytes % 16 == 0, "stages must stay 16-byte aligned");
+    static_assert(T % 4 == 0 && kChunk % T == 0, "chunks of whole 4-step groups");
+    static_assert(T * sizeof(Tin) % 16 == 0 && T * sizeof(Tout) % 16 == 0, "TMA rows");
+    static_assert(T <= 256 && CH <= 256, "TMA box extents");
 };
 
 // Transpose-reduce of P partial sums over the P lanes of a channel: afterwards
@@ -103,21 +179,20 @@ __device__ __forceinline__ float transpose_reduce(const float* v, int pp) {
     }
 }
 
-template <int NMAX, int P, typename Tin, typename Tout, int MODE>
-__global__ void __launch_bounds__(Layout<NMAX, P, Tin>::THREADS)
-scan_kernel(const KParams p) {
-    using Lo = Layout<NMAX, P, Tin>;
-    constexpr int T = Lo::T, NS = Lo::NS, CW = Lo::CW, CH = Lo::CH, RS = Lo::RS, RB = Lo::RB;
-    extern __shared__ __align__(16) unsigned char smem[];
-    Tin* stage0 = reinterpret_cast<Tin*>(smem);
-    Tin* stage1 = reinterpret_cast<Tin*>(smem + Lo::stage_bytes);
-    float* sBt = reinterpret_cast<float*>(smem + Lo::off_bt);
-    float* sCt = reinterpret_cast<float*>(smem + Lo::off_ct);
+template <int NMAX, int P, int WARPS, int T_, typename Tin, typename Tout, int MODE, bool TMA>
+__global__ void __launch_bounds__(WARPS * 32)
+scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
+    using Lo = Layout<NMAX, P, WARPS, T_, Tin, Tout>;
+    using V4 = vec4<Tin>;
+    using VT = typename V4::type;
+    constexpr int T = Lo::T, NS = Lo::NS, G = Lo::G, CH = Lo::CH, RS = Lo::RS;
+    extern __shared__ __align__(128) unsigned char smem[];
     float* sDel = reinterpret_cast<float*>(smem + Lo::off_del);
     float* sDu = reinterpret_cast<float*>(smem + Lo::off_du);
     float* sY = reinterpret_cast<float*>(smem + Lo::off_y);
     float* sBias = reinterpret_cast<float*>(smem + Lo::off_par);
     float* sDsk = sBias + CH;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Lo::off_bar);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t b = blockIdx.y;
@@ -127,6 +202,7 @@ scan_kernel(const KParams p) {
     const int64_t t_end = min(p.L, t_begin + p.seg_len);
     const int64_t nchunks = t_end > t_begin ? (t_end - t_begin + T - 1) / T : 0;
     const bool has_z = (MODE == kFull) && p.z != nullptr;
+    const bool out_tma = TMA && (MODE == kFull) && p.y_tma;
 
     for (int c = tid; c < CH; c += Lo::THREADS) {
         const int64_t d = d0 + c;
@@ -134,153 +210,228 @@ scan_kernel(const KParams p) {
         sBias[c] = (ok && p.delta_bias) ? p.delta_bias[d] : 0.f;
         sDsk[c] = (ok && p.D) ? p.D[d] : 0.f;
     }
+    if (TMA && tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_barrier_init();
+    }
 
     // This lane's channel and states.
     const int pp = lane % P;
-    const int cw = warp * CW + lane / P;
+    const int cw = warp * G + lane / P;
     const int64_t dch = d0 + cw;
-    const bool ch_ok = dch < p.dim;
-    float a2[NS], h[NS];
+    f2 a2p[NS / 2], hp[NS / 2];
 #pragma unroll
-    for (int n = 0; n < NS; ++n) {
-        const int nn = pp * NS + n;
-        const bool ok = ch_ok && nn < p.N;
-        a2[n] = ok ? p.A[dch * p.N + nn] * kLog2e : 0.f;  // padded states: Abar = 1, b = 0
-        h[n] = 0.f;
-        if (MODE == kFull && p.nseg > 1 && ok)
-            h[n] = p.seg_h[(((int64_t)seg * p.batch + b) * p.dim + dch) * p.N + nn];
+    for (int j = 0; j < NS; j += 2) {
+        float a[2], h[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int nn = pp * NS + j + q;
+            const bool ok = dch < p.dim && nn < p.N;
+            a[q] = ok ? p.A[dch * p.N + nn] * kLog2e : 0.f;  // padded states: Abar = 1, b = 0
+            h[q] = (MODE == kFull && p.nseg > 1 && ok)
+                       ? p.seg_h[(((int64_t)seg * p.batch + b) * p.dim + dch) * p.N + nn]
+                       : 0.f;
+        }
+        a2p[j / 2] = pack2(a[0], a[1]);
+        hp[j / 2] = pack2(h[0], h[1]);
     }
     float dsum = 0.f;
+    __syncthreads();
 
-    const Tin* gu = static_cast<const Tin*>(p.u);
-    const Tin* gdr = static_cast<const Tin*>(p.delta);
-    const Tin* gz = static_cast<const Tin*>(p.z);
-    const Tin* gB = static_cast<const Tin*>(p.B);
-    const Tin* gC = static_cast<const Tin*>(p.C);
-    const int nrows_x = has_z ? 3 * CH : 2 * CH;
-
-    // Stage chunk k of this CTA's segment into `st`; rows past dim / N and steps
-    // past L are zero-filled.
-    auto load_chunk = [&](int64_t k, Tin* st) {
+    // Stage chunk k of this CTA's segment into stage buffer k & 1.
+    auto stage_ptr = [&](int64_t k) -> Tin* {
+        return reinterpret_cast<Tin*>(smem + (k & 1) * Lo::stage_bytes);
+    };
+    auto issue_chunk = [&](int64_t k) {  // TMA: called by one thread
+        unsigned char* st = smem + (k & 1) * Lo::stage_bytes;
+        const int tt = (int)(t_begin + k * T);
+        const uint32_t bytes = (uint32_t)((has_z ? 3 : 2) * Lo::rows_bytes + 2 * Lo::coef_bytes);
+        uint64_t* bk = &bar[k & 1];
+        mbar_arrive_expect_tx(bk, bytes);
+        tma_load_3d(st, &tm.u, tt, (int)d0, (int)b, bk);
+        tma_load_3d(st + Lo::off_dr, &tm.dr, tt, (int)d0, (int)b, bk);
+        if (has_z) tma_load_3d(st + Lo::off_z, &tm.z, tt, (int)d0, (int)b, bk);
+        tma_load_3d(st + Lo::off_B, &tm.B, tt, 0, (int)b, bk);
+        tma_load_3d(st + Lo::off_C, &tm.C, tt, 0, (int)b, bk);
+    };
+    auto load_chunk_elementwise = [&](int64_t k) {  // rows not 16-byte multiples
+        unsigned char* st = smem + (k & 1) * Lo::stage_bytes;
         const int64_t t0 = t_begin + k * T;
-        if (p.aligned) {
-            constexpr int EPP = 16 / (int)sizeof(Tin);
-            constexpr int PPR = T / EPP;
-            const int total = (nrows_x + 2 * NMAX) * PPR;
-            for (int i = tid; i < total; i += Lo::THREADS) {
-                const int r = i / PPR, j = i % PPR;
-                const int64_t tt = t0 + j * EPP;
-                const Tin* src;
-                Tin* dst;
-                bool ok;
-                if (r < nrows_x) {
-                    const int which = r / CH, c = r % CH;
-                    const int64_t d = d0 + c;
-                    ok = d < p.dim && tt < p.L;
-                    const Tin* base = which == 0 ? gu : (which == 1 ? gdr : gz);
-                    src = base + ((b * p.dim + (ok ? d : 0)) * p.L + (ok ? tt : 0));
-                    dst = st + (size_t)which * CH * T + c * T + j * EPP;
-                } else {
-                    const int r2 = r - nrows_x, which = r2 / NMAX, n = r2 % NMAX;
-                    ok = n < p.N && tt < p.L;
-                    const Tin* base = which == 0 ? gB : gC;
-                    src = base + ((b * p.N + (ok ? n : 0)) * p.L + (ok ? tt : 0));
-                    dst = st + (size_t)3 * CH * T + (size_t)which * NMAX * RB + n * RB + j * EPP;
-                }
-                cp_async16(dst, src, ok ? 16 : 0);
+        const Tin* gsrc[5] = {static_cast<const Tin*>(p.u), static_cast<const Tin*>(p.delta),
+                              static_cast<const Tin*>(p.z), static_cast<const Tin*>(p.B),
+                              static_cast<const Tin*>(p.C)};
+        const size_t off[5] = {0, Lo::off_dr, Lo::off_z, Lo::off_B, Lo::off_C};
+        const int nx = has_z ? 3 : 2;
+        for (int i = tid; i < (nx * CH + 2 * NMAX) * T; i += Lo::THREADS) {
+            const int r = i / T, j = i % T;
+            const int64_t t = t0 + j;
+            int which, row;
+            int64_t grow;
+            bool ok;
+            if (r < nx * CH) {
+                which = r / CH, row = r % CH;
+                ok = d0 + row < p.dim && t < p.L;
+                grow = b * p.dim + d0 + row;
+            } else {
+                which = 3 + (r - nx * CH) / NMAX, row = (r - nx * CH) % NMAX;
+                ok = row < p.N && t < p.L;
+                grow = b * p.N + row;
             }
-        } else {
-            const int total = (nrows_x + 2 * NMAX) * T;
-            for (int i = tid; i < total; i += Lo::THREADS) {
-                const int r = i / T, j = i % T;
-                const int64_t tt = t0 + j;
-                if (r < nrows_x) {
-                    const int which = r / CH, c = r % CH;
-                    const int64_t d = d0 + c;
-                    const Tin* base = which == 0 ? gu : (which == 1 ? gdr : gz);
-                    Tin v = Tin(0.f);
-                    if (d < p.dim && tt < p.L) v = base[(b * p.dim + d) * p.L + tt];
-                    st[(size_t)which * CH * T + c * T + j] = v;
-                } else {
-                    const int r2 = r - nrows_x, which = r2 / NMAX, n = r2 % NMAX;
-                    const Tin* base = which == 0 ? gB : gC;
-                    Tin v = Tin(0.f);
-                    if (n < p.N && tt < p.L) v = base[(b * p.N + n) * p.L + tt];
-                    st[(size_t)3 * CH * T + (size_t)which * NMAX * RB + n * RB + j] = v;
-                }
-            }
+            reinterpret_cast<Tin*>(st + off[which])[row * T + j] =
+                ok ? gsrc[which][grow * p.L + t] : Tin(0.f);
         }
     };
 
-    if (nchunks > 0) load_chunk(0, stage0);
-    cp_async_commit();
+    if constexpr (TMA) {
+        if (tid == 0 && nchunks > 0) issue_chunk(0);
+    }
+    bool aborted = false;
     for (int64_t k = 0; k < nchunks; ++k) {
-        if (k + 1 < nchunks) load_chunk(k + 1, ((k + 1) & 1) ? stage1 : stage0);
-        cp_async_commit();
-        cp_async_wait<1>();
-        __syncthreads();
+        bool ok = true;
+        if constexpr (TMA) {
+            ok = mbar_wait_bounded(&bar[k & 1], (uint32_t)((k >> 1) & 1), kWaitLimitCycles);
+        } else {
+            load_chunk_elementwise(k);
+            __syncthreads();
+        }
 
-        const Tin* st = (k & 1) ? stage1 : stage0;
+        const Tin* st = stage_ptr(k);
+        const unsigned char* stb = reinterpret_cast<const unsigned char*>(st);
         const Tin* rU = st;
-        const Tin* rDr = st + CH * T;
-        const Tin* rZ = st + 2 * CH * T;
-        const Tin* rB = st + 3 * CH * T;
-        const Tin* rC = rB + NMAX * RB;
+        const Tin* rDr = reinterpret_cast<const Tin*>(stb + Lo::off_dr);
+        const Tin* rZ = reinterpret_cast<const Tin*>(stb + Lo::off_z);
+        const Tin* rB = reinterpret_cast<const Tin*>(stb + Lo::off_B);
+        const Tin* rC = reinterpret_cast<const Tin*>(stb + Lo::off_C);
         const int64_t t0 = t_begin + k * T;
         const int valid = (int)min((int64_t)T, t_end - t0);
+        float* sBt = reinterpret_cast<float*>(smem + Lo::off_coef + (k & 1) * Lo::coef_bytes_all);
+        float* sCt = sBt + T * NMAX;  // fp32 inputs only
 
-        // B, C of the chunk to fp32, time-major: every lane then reads its states'
-        // coefficients for step t as one 16-byte vector.
-        for (int i = tid; i < NMAX * T; i += Lo::THREADS) {
-            const int t = i / NMAX, n = i % NMAX;
-            sBt[i] = io<Tin>::to_f(rB[n * RB + t]);
-            sCt[i] = io<Tin>::to_f(rC[n * RB + t]);
+        // B, C of the chunk, time-major, through 4x4 register blocks: every lane then reads
+        // the coefficients of its four states for step t with one 16-byte load.
+        for (int i = tid; i < (NMAX / 4) * (T / 4); i += Lo::THREADS) {
+            const int n4 = i % (NMAX / 4), t4 = i / (NMAX / 4);
+            if constexpr (Lo::kPackedBC) {
+                uint2 bw[4], cwd[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    bw[r] = *reinterpret_cast<const uint2*>(rB + (4 * n4 + r) * T + 4 * t4);
+                    cwd[r] = *reinterpret_cast<const uint2*>(rC + (4 * n4 + r) * T + 4 * t4);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    // step q sits in word q/2, half q%2, of each row; pair rows (0,1), (2,3)
+                    const unsigned sel = (q & 1) ? 0x7632u : 0x5410u;
+                    auto word = [&](const uint2& v) { return (q >> 1) ? v.y : v.x; };
+                    uint4 g;
+                    g.x = __byte_perm(word(bw[0]), word(bw[1]), sel);
+                    g.y = __byte_perm(word(bw[2]), word(bw[3]), sel);
+                    g.z = __byte_perm(word(cwd[0]), word(cwd[1]), sel);
+                    g.w = __byte_perm(word(cwd[2]), word(cwd[3]), sel);
+                    reinterpret_cast<uint4*>(sBt)[(4 * t4 + q) * (NMAX / 4) + n4] = g;
+                }
+            } else {
+                float bv[4][4], cv[4][4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    V4::to_f(*reinterpret_cast<const VT*>(rB + (4 * n4 + r) * T + 4 * t4), bv[r]);
+                    V4::to_f(*reinterpret_cast<const VT*>(rC + (4 * n4 + r) * T + 4 * t4), cv[r]);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    *reinterpret_cast<float4*>(sBt + (4 * t4 + q) * NMAX + 4 * n4) =
+                        make_float4(bv[0][q], bv[1][q], bv[2][q], bv[3][q]);
+                    *reinterpret_cast<float4*>(sCt + (4 * t4 + q) * NMAX + 4 * n4) =
+                        make_float4(cv[0][q], cv[1][q], cv[2][q], cv[3][q]);
+                }
+            }
         }
-        __syncthreads();
+        // The one CTA-wide barrier of a chunk: coefficients visible to every warp, and
+        // every warp done with chunk k-1, so its stage can take chunk k+1.
+        if (__syncthreads_or(!ok)) {  // every thread agrees to stop if any wait gave up
+            if (tid == 0) atomicOr(&g_device_error, 1u);
+            aborted = true;
+            break;
+        }
+        if constexpr (TMA) {
+            if (tid == 0 && k + 1 < nchunks) {
+                fence_proxy_async();  // stage (k+1)&1 was last read through the generic proxy
+                issue_chunk(k + 1);
+            }
+        }
 
-        // Phase A: step sizes of this warp's channels.  Steps past the end of the
-        // segment get Delta = 0 (Abar = 1, no input): the state passes through.
-        for (int i = lane; i < CW * T; i += 32) {
-            const int c = warp * CW + i / T, t = i % T;
-            const float x = io<Tin>::to_f(rDr[c * T + t]) + sBias[c];
-            float dt = p.softplus ? softplus(x) : x;
-            dt = t < valid ? dt : 0.f;
-            sDel[c * RS + t] = dt;
-            sDu[c * RS + t] = dt * io<Tin>::to_f(rU[c * T + t]);
+        // Phase A: step sizes of this warp's channels, four steps per lane.  Steps past
+        // the end of the segment get Delta = 0 (Abar = 1, no input): the state passes.
+        for (int i = lane; i < G * (T / 4); i += 32) {
+            const int c = warp * G + i / (T / 4), tb = 4 * (i % (T / 4));
+            float x[4], uu[4];
+            V4::to_f(*reinterpret_cast<const VT*>(rDr + c * T + tb), x);
+            V4::to_f(*reinterpret_cast<const VT*>(rU + c * T + tb), uu);
+            const float bias = sBias[c];
+            float dt[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float xb = x[q] + bias;
+                dt[q] = p.softplus ? softplus(xb) : xb;
+            }
+            if (valid < T) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) dt[q] = tb + q < valid ? dt[q] : 0.f;
+            }
+            const float q0 = dt[0] * uu[0], q1 = dt[1] * uu[1], q2 = dt[2] * uu[2], q3 = dt[3] * uu[3];
+            *reinterpret_cast<float4*>(sDel + c * RS + tb) = make_float4(dt[0], dt[1], dt[2], dt[3]);
+            *reinterpret_cast<float4*>(sDu + c * RS + tb) = make_float4(q0, q1, q2, q3);
         }
         __syncwarp();
 
-        // Phase B: the recurrence, four steps per iteration.
+        // Phase B: the recurrence, four steps per iteration, states in packed pairs.
+#pragma unroll
         for (int t = 0; t < T; t += 4) {
             const float4 d4 = *reinterpret_cast<const float4*>(sDel + cw * RS + t);
             const float4 q4 = *reinterpret_cast<const float4*>(sDu + cw * RS + t);
-            const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-            const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+            const f2 dd4[4] = {pack2(d4.x, d4.x), pack2(d4.y, d4.y), pack2(d4.z, d4.z),
+                               pack2(d4.w, d4.w)};
+            const f2 qq4[4] = {pack2(q4.x, q4.x), pack2(q4.y, q4.y), pack2(q4.z, q4.z),
+                               pack2(q4.w, q4.w)};
             float yp[4];
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                const float* bt = sBt + (t + kk) * NMAX + pp * NS;
-                const float* ct = sCt + (t + kk) * NMAX + pp * NS;
-                float acc0 = 0.f, acc1 = 0.f;
+                const f2 dd = dd4[kk];
+                const f2 qq = qq4[kk];
+                f2 acc = pack2(0.f, 0.f);
 #pragma unroll
-                for (int n = 0; n < NS; n += 4) {
-                    const float4 bb = *reinterpret_cast<const float4*>(bt + n);
-                    const float4 cc = *reinterpret_cast<const float4*>(ct + n);
-                    const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
-                    const float cv[4] = {cc.x, cc.y, cc.z, cc.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float abar = ex2(dv[kk] * a2[n + j]);
-                        h[n + j] = fmaf(abar, h[n + j], qv[kk] * bv[j]);
-                        if (j & 1)
-                            acc1 = fmaf(cv[j], h[n + j], acc1);
-                        else
-                            acc0 = fmaf(cv[j], h[n + j], acc0);
+                for (int j = 0; j < NS / 4; ++j) {
+                    f2 b01, b23, c01, c23;
+                    if constexpr (Lo::kPackedBC) {
+                        const uint4 g = reinterpret_cast<const uint4*>(sBt)[(t + kk) * (NMAX / 4) +
+                                                                            pp * (NS / 4) + j];
+                        b01 = bf16pair(g.x), b23 = bf16pair(g.y);
+                        c01 = bf16pair(g.z), c23 = bf16pair(g.w);
+                    } else {
+                        const ulonglong2 bb = reinterpret_cast<const ulonglong2*>(
+                            sBt + (t + kk) * NMAX + pp * NS)[j];
+                        const ulonglong2 cc = reinterpret_cast<const ulonglong2*>(
+                            sCt + (t + kk) * NMAX + pp * NS)[j];
+                        b01 = f2{bb.x}, b23 = f2{bb.y}, c01 = f2{cc.x}, c23 = f2{cc.y};
                     }
+                    const f2 e0 = ex2x2(mul2(dd, a2p[2 * j]));
+                    const bool on_fma = S6_POLY == 2 || (S6_POLY == 1 && (kk & 1));
+                    const f2 e1 = on_fma ? exp2_fma2(mul2(dd, a2p[2 * j + 1]))
+                                         : ex2x2(mul2(dd, a2p[2 * j + 1]));
+                    hp[2 * j] = fma2(e0, hp[2 * j], mul2(qq, b01));
+                    hp[2 * j + 1] = fma2(e1, hp[2 * j + 1], mul2(qq, b23));
+                    acc = fma2(c01, hp[2 * j], acc);
+                    acc = fma2(c23, hp[2 * j + 1], acc);
                 }
-                yp[kk] = acc0 + acc1;
+                float lo, hi;
+                unpack2(acc, lo, hi);
+                yp[kk] = lo + hi;
             }
             if (MODE == kAggregate) {
+                float dv[4], dup;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) unpack2(dd4[kk], dv[kk], dup);
                 dsum += (dv[0] + dv[1]) + (dv[2] + dv[3]);
             } else if constexpr (P == 1) {
                 *reinterpret_cast<float4*>(sY + cw * RS + t) = make_float4(yp[0], yp[1], yp[2], yp[3]);
@@ -291,38 +442,86 @@ scan_kernel(const KParams p) {
         }
 
         if (MODE == kFull) {
+            // Phase C: skip term, gate; four steps per lane into this warp's rows of the
+            // output tile, which its lane 0 then stores with TMA (or straight to global
+            // memory when rows cannot be described to TMA).  The warp's previous store
+            // has long finished reading the tile; lane 0 confirms before it is rewritten.
+            if (out_tma && lane == 0) tma_store_wait_read<0>();
             __syncwarp();
-            // Phase C: skip term, gate, store (lanes walk t: coalesced rows).
+            Tout* sOut = reinterpret_cast<Tout*>(smem + Lo::off_out);
             Tout* gy = static_cast<Tout*>(p.y);
-            for (int i = lane; i < CW * T; i += 32) {
-                const int c = warp * CW + i / T, t = i % T;
-                const int64_t d = d0 + c;
-                if (t < valid && d < p.dim) {
-                    float yv = sY[c * RS + t] + sDsk[c] * io<Tin>::to_f(rU[c * T + t]);
-                    if (has_z) yv *= silu(io<Tin>::to_f(rZ[c * T + t]));
-                    gy[(b * p.dim + d) * p.L + t0 + t] = io<Tout>::from_f(yv);
+            for (int i = lane; i < G * (T / 4); i += 32) {
+                const int c = warp * G + i / (T / 4), tb = 4 * (i % (T / 4));
+                const float4 y4 = *reinterpret_cast<const float4*>(sY + c * RS + tb);
+                float uu[4], zz[4];
+                V4::to_f(*reinterpret_cast<const VT*>(rU + c * T + tb), uu);
+                if (has_z) V4::to_f(*reinterpret_cast<const VT*>(rZ + c * T + tb), zz);
+                const float yv[4] = {y4.x, y4.y, y4.z, y4.w};
+                const float dsk = sDsk[c];
+                float o[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    o[q] = fmaf(dsk, uu[q], yv[q]);
+                    if (has_z) o[q] *= silu(zz[q]);
+                }
+                if (out_tma) {
+                    store4(sOut + c * T + tb, o);
+                } else {
+                    const int64_t d = d0 + c;
+                    if (d >= p.dim || tb >= valid) continue;
+                    Tout* dst = gy + (b * p.dim + d) * p.L + t0 + tb;
+                    if (p.y_vec && tb + 4 <= valid) {
+                        store4(dst, o);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            if (tb + q < valid) dst[q] = io<Tout>::from_f(o[q]);
+                    }
+                }
+            }
+            if (out_tma) {
+                fence_proxy_async();  // this lane's tile writes, before the async-proxy read
+                __syncwarp();
+                if (lane == 0 && d0 + warp * G < p.dim) {  // rows past dim are clipped
+                    tma_store_3d(&tm.y, sOut + warp * G * T, (int)t0, (int)(d0 + warp * G), (int)b);
+                    tma_store_commit();
                 }
             }
         }
-        __syncthreads();
     }
 
-    if (MODE == kFull) {
-        if (p.last_state && seg == (int)gridDim.z - 1 && ch_ok) {
+    if constexpr (TMA) {
+        if (tid == 0) {
+            if (aborted) {  // let copies still in flight land before the CTA exits
+                mbar_wait_bounded(&bar[0], 0, kWaitLimitCycles);
+                mbar_wait_bounded(&bar[1], 0, kWaitLimitCycles);
+            }
+        }
+    }
+    if (out_tma && lane == 0) tma_store_wait_all();
+    if (aborted) return;
+
+    if (dch < p.dim) {
+        float h[NS];
+#pragma unroll
+        for (int j = 0; j < NS / 2; ++j) unpack2(hp[j], h[2 * j], h[2 * j + 1]);
+        if (MODE == kFull) {
+            if (p.last_state && seg == (int)gridDim.z - 1) {
+#pragma unroll
+                for (int n = 0; n < NS; ++n) {
+                    const int nn = pp * NS + n;
+                    if (nn < p.N) p.last_state[(b * p.dim + dch) * p.N + nn] = h[n];
+                }
+            }
+        } else {
+            const int64_t row = ((int64_t)seg * p.batch + b) * p.dim + dch;
 #pragma unroll
             for (int n = 0; n < NS; ++n) {
                 const int nn = pp * NS + n;
-                if (nn < p.N) p.last_state[(b * p.dim + dch) * p.N + nn] = h[n];
+                if (nn < p.N) p.seg_h[row * p.N + nn] = h[n];
             }
+            if (pp == 0) p.seg_sum[row] = dsum;
         }
-    } else if (ch_ok) {
-        const int64_t row = ((int64_t)seg * p.batch + b) * p.dim + dch;
-#pragma unroll
-        for (int n = 0; n < NS; ++n) {
-            const int nn = pp * NS + n;
-            if (nn < p.N) p.seg_h[row * p.N + nn] = h[n];
-        }
-        if (pp == 0) p.seg_sum[row] = dsum;
     }
 }
 
@@ -348,25 +547,69 @@ __global__ void carry_kernel(float* seg_h, const float* seg_sum, const float* A,
     seg_h[((int64_t)(nseg - 1) * batch * dim + bd) * N + n] = H;
 }
 
-template <int NMAX, int P, typename Tin, typename Tout, int MODE>
-cudaError_t launch_one(const KParams& kp, dim3 grid, cudaStream_t s) {
-    using Lo = Layout<NMAX, P, Tin>;
-    auto kern = scan_kernel<NMAX, P, Tin, Tout, MODE>;
+// ---- host side ---------------------------------------------------------------------------
+
+using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+EncodeFn tensor_map_encoder() {
+    static EncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeFn>(ptr);
+    });
+    return fn;
+}
+
+// Describe a row-major (outer, mid, inner) tensor with a (box_inner, box_mid, 1) box.
+template <typename T>
+bool encode_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+               uint32_t box_inner, uint32_t box_mid) {
+    EncodeFn enc = tensor_map_encoder();
+    if (!enc) return false;
+    const CUtensorMapDataType dt = sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                  : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    cuuint64_t dims[3] = {inner, mid, outer};
+    cuuint64_t strides[2] = {inner * sizeof(T), inner * mid * sizeof(T)};
+    cuuint32_t box[3] = {box_inner, box_mid, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NMAX, int P, int WARPS, int T, typename Tin, typename Tout, int MODE, bool TMA>
+cudaError_t launch_one(const KParams& kp, const TMaps& tm, dim3 grid, cudaStream_t s) {
+    using Lo = Layout<NMAX, P, WARPS, T, Tin, Tout>;
+    auto kern = scan_kernel<NMAX, P, WARPS, T, Tin, Tout, MODE, TMA>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Lo::bytes);
     if (e != cudaSuccess) return e;
-    kern<<<grid, Lo::THREADS, Lo::bytes, s>>>(kp);
+    kern<<<grid, Lo::THREADS, Lo::bytes, s>>>(kp, tm);
     return cudaGetLastError();
 }
 
-template <int NMAX, typename Tin, typename Tout>
-cudaError_t launch_typed(const ScanArgs& a, KParams kp, cudaStream_t s) {
-    constexpr int P = NMAX / 4;
-    using Lo = Layout<NMAX, P, Tin>;
+// Instantiation per state width: N = 16 uses the tuned tile; narrower states keep four
+// states per lane.
+template <int NMAX>
+struct Tile {
+    static constexpr int P = NMAX == 16 ? S6_P16 : NMAX / 4;
+    static constexpr int WARPS = NMAX == 16 ? S6_WARPS16 : (NMAX == 8 ? 2 : 1);
+    static constexpr int T = NMAX == 16 ? S6_CHUNK : 64;
+};
+
+template <int NMAX, typename Tin, typename Tout, bool TMA>
+cudaError_t launch_typed(const ScanArgs& a, const KParams& kp, const TMaps& tm, cudaStream_t s) {
+    using TL = Tile<NMAX>;
+    using Lo = Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout>;
     const unsigned gx = (unsigned)((a.dim + Lo::CH - 1) / Lo::CH);
     if (a.nseg > 1) {
-        cudaError_t e = launch_one<NMAX, P, Tin, Tout, kAggregate>(
-            kp, dim3(gx, (unsigned)a.batch, (unsigned)(a.nseg - 1)), s);
+        cudaError_t e = launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kAggregate, TMA>(
+            kp, tm, dim3(gx, (unsigned)a.batch, (unsigned)(a.nseg - 1)), s);
         if (e != cudaSuccess) return e;
         const int64_t lanes = a.batch * a.dim * a.N;
         carry_kernel<<<(unsigned)((lanes + 255) / 256), 256, 0, s>>>(
@@ -374,20 +617,60 @@ cudaError_t launch_typed(const ScanArgs& a, KParams kp, cudaStream_t s) {
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    return launch_one<NMAX, P, Tin, Tout, kFull>(kp, dim3(gx, (unsigned)a.batch, (unsigned)a.nseg),
-                                                 s);
+    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA>(
+        kp, tm, dim3(gx, (unsigned)a.batch, (unsigned)a.nseg), s);
+}
+
+template <int NMAX, typename Tin, typename Tout>
+cudaError_t launch_io(const ScanArgs& a, KParams kp, cudaStream_t s) {
+    using TL = Tile<NMAX>;
+    using Lo = Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout>;
+    TMaps tm;
+    memset(&tm, 0, sizeof(tm));
+    const bool rows16 = (a.L * (int64_t)sizeof(Tin)) % 16 == 0 && a.L > 0;
+    const bool out16 = (a.L * (int64_t)sizeof(Tout)) % 16 == 0 && a.L > 0;
+    // TMA coordinates are 32-bit signed integers.
+    const bool fits = a.L < (1LL << 31) && a.dim < (1LL << 31) && a.batch < (1LL << 31);
+    if (!(rows16 && fits)) {
+        kp.y_tma = 0;
+        return launch_typed<NMAX, Tin, Tout, false>(a, kp, tm, s);
+    }
+    bool ok = encode_3d<Tin>(&tm.u, a.u, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
+              encode_3d<Tin>(&tm.dr, a.delta, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
+              encode_3d<Tin>(&tm.B, a.B, a.L, a.N, a.batch, Lo::T, NMAX) &&
+              encode_3d<Tin>(&tm.C, a.C, a.L, a.N, a.batch, Lo::T, NMAX);
+    if (ok && a.z) ok = encode_3d<Tin>(&tm.z, a.z, a.L, a.dim, a.batch, Lo::T, Lo::CH);
+    kp.y_tma = out16 ? 1 : 0;
+    if (ok && out16) ok = encode_3d<Tout>(&tm.y, a.y, a.L, a.dim, a.batch, Lo::T, Lo::G);
+    if (!ok) return cudaErrorInvalidValue;
+    return launch_typed<NMAX, Tin, Tout, true>(a, kp, tm, s);
 }
 
 template <int NMAX>
 cudaError_t launch_nmax(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
     const bool ib = a.in_dtype == DType::BF16, ob = a.out_dtype == DType::BF16;
-    if (ib && ob) return launch_typed<NMAX, __nv_bfloat16, __nv_bfloat16>(a, kp, s);
-    if (ib && !ob) return launch_typed<NMAX, __nv_bfloat16, float>(a, kp, s);
-    if (!ib && ob) return launch_typed<NMAX, float, __nv_bfloat16>(a, kp, s);
-    return launch_typed<NMAX, float, float>(a, kp, s);
+    if (ib && ob) return launch_io<NMAX, __nv_bfloat16, __nv_bfloat16>(a, kp, s);
+    if (ib && !ob) return launch_io<NMAX, __nv_bfloat16, float>(a, kp, s);
+    if (!ib && ob) return launch_io<NMAX, float, __nv_bfloat16>(a, kp, s);
+    return launch_io<NMAX, float, float>(a, kp, s);
 }
 
 }  // namespace
+
+cudaError_t read_device_error(unsigned* out, bool clear, cudaStream_t stream) {
+    unsigned v = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_device_error, sizeof(v), 0,
+                                              cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess && clear && v) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(zero), 0,
+                                    cudaMemcpyHostToDevice, stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    }
+    *out = v;
+    return e;
+}
 
 void plan_segments(int64_t batch, int64_t dim, int64_t L, int64_t* nseg, int64_t* seg_len) {
     // Split only when the channels alone cannot fill the GPU (fewer than 4096 lanes
@@ -429,8 +712,8 @@ cudaError_t launch_scan(const ScanArgs& a, cudaStream_t stream) {
     kp.N = (int)a.N;
     kp.nseg = (int)a.nseg;
     kp.softplus = a.softplus ? 1 : 0;
-    const int64_t esize = a.in_dtype == DType::BF16 ? 2 : 4;
-    kp.aligned = (a.L * esize) % 16 == 0 ? 1 : 0;  // base pointers are checked by the ABI
+    kp.y_vec = a.L % 4 == 0 ? 1 : 0;
+    kp.y_tma = 0;
     if (a.N <= 4) return launch_nmax<4>(a, kp, stream);
     if (a.N <= 8) return launch_nmax<8>(a, kp, stream);
     return launch_nmax<16>(a, kp, stream);

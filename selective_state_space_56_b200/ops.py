@@ -57,6 +57,10 @@ def load_library():
                                                          vp, i64, i64, i64, i32, vp]
             lib.mamba_status_string.restype = ctypes.c_char_p
             lib.mamba_status_string.argtypes = [i32]
+            lib.mamba_check_device_error.restype = i32
+            lib.mamba_check_device_error.argtypes = [i32, vp]
+            lib.mamba_diag_exp2.restype = i32
+            lib.mamba_diag_exp2.argtypes = [vp, vp, vp, vp, i64, vp]
             lib.mamba_abi_version.restype = i32
             lib.mamba_abi_version.argtypes = []
             _lib = lib
@@ -91,6 +95,28 @@ def _check(t, name, device, shape=None, dtypes=None):
         raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
     if dtypes is not None and t.dtype not in dtypes:
         raise ValueError("%s has dtype %s, expected one of %s" % (name, t.dtype, dtypes))
+
+
+def check_device_error(clear: bool = True, device=None) -> None:
+    """Raise MambaError if a bounded device-side wait gave up since the last clear."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        rc = load_library().mamba_check_device_error(int(bool(clear)), _stream_handle(dev))
+    if rc != 0:
+        raise MambaError(rc, "mamba_check_device_error")
+
+
+def diag_exp2(x):
+    """2^x of a float32 CUDA tensor via (FMA-pipe polynomial, SFU ex2.approx, exp2f)."""
+    if x.dtype != torch.float32 or x.device.type != "cuda" or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 CUDA tensor")
+    outs = [torch.empty_like(x) for _ in range(3)]
+    with torch.cuda.device(x.device):
+        rc = load_library().mamba_diag_exp2(_ptr(x), _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]),
+                                            x.numel(), _stream_handle(x.device))
+    if rc != 0:
+        raise MambaError(rc, "mamba_diag_exp2")
+    return tuple(outs)
 
 
 def selective_scan_workspace_size(batch: int, dim: int, dstate: int, seqlen: int) -> int:

@@ -18,3 +18,16 @@ def cuda_ok():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return True
+
+
+@pytest.fixture(autouse=True)
+def _no_device_wait_timeouts(request):
+    """After every GPU test: no bounded device-side wait gave up during it."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    from selective_state_space_56_b200 import ops
+    ops.check_device_error(clear=True)
