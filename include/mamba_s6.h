@@ -123,6 +123,36 @@ int mamba_selective_state_update(float* state, const void* u, const void* delta,
                                  mamba_dtype io_dtype, void* stream);
 
 /*
+ * mamba_selective_scan_fwd for callers that cannot allocate device memory.  (This
+ * entry point has no counterpart in the method's description; it only changes where
+ * scratch memory comes from.)
+ *
+ * Some callers may not allocate: extension code inside a host framework that owns the
+ * whole device-memory budget, or latency-sensitive code that cannot afford cudaMalloc /
+ * cudaFree, which may synchronise the device.  mamba_selective_scan_fwd needs a
+ * caller-provided workspace whenever it splits a long sequence into segments; this
+ * variant instead uses a fixed 2.25 MiB scratch array compiled into the library and
+ * calls no allocator.  Arguments, layouts and results are those of
+ * mamba_selective_scan_fwd (without the workspace arguments).
+ *
+ *   - Limit: when the split plan needs more than 2.25 MiB (segments x batch x dim x
+ *     (dstate + 1) x 4 bytes) the call returns MAMBA_ERR_WORKSPACE and launches
+ *     nothing.  The million-length layer (1, 2048, 16, 2^20) needs 2.125 MiB.
+ *   - The array exists on every GPU that loads the library and stays allocated until
+ *     the process exits.  The first call on a device (with that device current) looks
+ *     up the array's device address; make that first call before any stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents; the scan
+ *     writes each entry before reading it, so nothing needs clearing.  Calls whose
+ *     kernels overlap on the GPU (e.g. on two streams at once) race on the array:
+ *     serialise them.
+ */
+int mamba_selective_scan_fwd_noalloc(const void* u, const void* delta, const float* A,
+                                     const void* B, const void* C, const float* D, const void* z,
+                                     const float* delta_bias, int delta_softplus, void* y,
+                                     float* last_state, mamba_scan_dims dims,
+                                     mamba_dtype in_dtype, mamba_dtype out_dtype, void* stream);
+
+/*
  * Reads the library's device error word on `stream`, synchronising that stream.
  * Every device-side wait in the kernels (on the completion barrier of an
  * asynchronous tile copy) is bounded to about a second; a wait that gives up sets
