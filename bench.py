@@ -293,7 +293,7 @@ def run_ours(args, rank, world, local):
     e2e = {"value": world * elems / (e2e_ms * 1e-3), "unit": "elems/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
-    decode = run_decode(dev, stream, world)
+    decode = run_decode(dev, stream, world, steps=args.decode_steps)
     del g, y, last
     torch.cuda.empty_cache()
 
@@ -325,7 +325,8 @@ def run_decode(dev, stream, world, steps=1000):
     w = inputs.DECODE_WORKLOAD
     prm = {k: v.to(dev) for k, v in inputs.decode_params(w).items()}
     state = prm["state0"].clone()
-    toks = [inputs.decode_step_inputs(s, w, device=dev) for s in range(steps)]
+    allt = inputs.decode_tokens_batched(steps, w, device=dev)
+    toks = [{k: v[s] for k, v in allt.items()} for s in range(steps)]
     y = torch.empty((w.batch, w.dim), dtype=w.io_dtype, device=dev)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
@@ -358,18 +359,18 @@ def run_decode(dev, stream, world, steps=1000):
     peaks, kind = measured_peaks()
     byts = decode_bytes(w.batch, w.dim, w.dstate)
     lanes = w.batch * w.dim
-    del toks, flush
+    del toks, allt, flush
     return {
         "metric": "decode state-updates/s", "unit": "(b,d) lane updates/s",
         "value": world * lanes / (ms_cold * 1e-3), "steps_per_s": 1e3 / ms_cold,
         "ms_per_token_l2_flushed": ms_cold, "ms_per_token_back_to_back": ms_warm,
-        "workload": "decode: batch 256, dim 5120, N 16, bf16 I/O, fp32 state, 1000 fresh tokens",
+        "workload": "decode: batch 256, dim 5120, N 16, bf16 I/O, fp32 state, %d fresh tokens" % steps,
         "roofline": {"bound": "hbm", "unit": "GB/s", "achieved": byts / (ms_cold * 1e-3) / 1e9,
                      "peak": peaks["hbm_gbs"], "frac": byts / (ms_cold * 1e-3) / 1e9 / peaks["hbm_gbs"],
                      "algorithmic_bytes": byts, "peak_kind": kind,
                      "traffic": profile_traffic("state_update_decode.txt",
                                                 "selective_state_space_56_b200/csrc/state_update.cu")},
-        "gpu_launches": 2 * steps,
+        "gpu_launches": 2 * steps + 5,
     }
 
 
@@ -427,6 +428,33 @@ def run_reference(args, rank, world):
             "gpu_launches": 0}
 
 
+def profile_target(which):
+    """Three launches of the scan (m2p8b) or eight decode tokens, for ncu captures."""
+    from selective_state_space_56_b200 import inputs, ops
+    import selective_state_space_56_b200.build as s6build
+    s6build.build()
+    dev = torch.device("cuda", 0)
+    if which == "scan":
+        w = inputs.SCAN_WORKLOADS[WORKLOAD]
+        p = inputs.scan_inputs(w.batch, w.dim, w.dstate, w.seqlen, w.in_dtype, w.seed, device=dev)
+        y = torch.empty((w.batch, w.dim, w.seqlen), dtype=w.out_dtype, device=dev)
+        for _ in range(3):
+            ops.selective_scan_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
+                                   delta_bias=p["delta_bias"], y=y)
+    else:
+        w = inputs.DECODE_WORKLOAD
+        prm = {k: v.to(dev) for k, v in inputs.decode_params(w).items()}
+        state = prm["state0"].clone()
+        toks = inputs.decode_tokens_batched(8, w, device=dev)
+        y = torch.empty((w.batch, w.dim), dtype=w.io_dtype, device=dev)
+        for s in range(8):
+            ops.selective_state_update(state, toks["u"][s], toks["delta"][s], prm["A"], toks["B"][s],
+                                       toks["C"][s], D=prm["D"], z=toks["z"][s],
+                                       delta_bias=prm["delta_bias"], y=y)
+    torch.cuda.synchronize(dev)
+    ops.check_device_error()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[1])
     ap.add_argument("--gpus", type=int, default=1)
@@ -435,9 +463,16 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--profile", choices=["scan", "decode"],
+                    help="run a few untimed launches of one workload (an ncu capture target) "
+                         "and exit")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.profile:
+        profile_target(args.profile)
+        return
     if args.impl == "reference":
         # The oracle arm runs on rank 0's host cores only; other ranks have no work and
         # take part in no collective.

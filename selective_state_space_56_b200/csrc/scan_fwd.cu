@@ -308,30 +308,30 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         float* sBt = reinterpret_cast<float*>(smem + Lo::off_coef + (k & 1) * Lo::coef_bytes_all);
         float* sCt = sBt + T * NMAX;  // fp32 inputs only
 
-        // B, C of the chunk, time-major, through 4x4 register blocks: every lane then reads
-        // the coefficients of its four states for step t with one 16-byte load.
-        for (int i = tid; i < (NMAX / 4) * (T / 4); i += Lo::THREADS) {
-            const int n4 = i % (NMAX / 4), t4 = i / (NMAX / 4);
-            if constexpr (Lo::kPackedBC) {
-                uint2 bw[4], cwd[4];
+        // B, C of the chunk, time-major: every lane then reads the coefficients of its four
+        // states for step t with one 16-byte load (bf16: B[4] and C[4] as pairs; fp32: a
+        // 16-byte vector from each of two tiles, transposed through 4x4 register blocks).
+        if constexpr (Lo::kPackedBC) {
+            // work item: (4-state group, step pair, B or C) -> two 8-byte half-groups
+            for (int i = tid; i < (NMAX / 4) * (T / 2) * 2; i += Lo::THREADS) {
+                const int which = i & 1, n4 = (i >> 1) % (NMAX / 4), t2 = (i >> 1) / (NMAX / 4);
+                const Tin* src = (which ? rC : rB) + (4 * n4) * T + 2 * t2;
+                uint32_t w[4];
 #pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    bw[r] = *reinterpret_cast<const uint2*>(rB + (4 * n4 + r) * T + 4 * t4);
-                    cwd[r] = *reinterpret_cast<const uint2*>(rC + (4 * n4 + r) * T + 4 * t4);
-                }
+                for (int r = 0; r < 4; ++r) w[r] = *reinterpret_cast<const uint32_t*>(src + r * T);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    // step q sits in word q/2, half q%2, of each row; pair rows (0,1), (2,3)
-                    const unsigned sel = (q & 1) ? 0x7632u : 0x5410u;
-                    auto word = [&](const uint2& v) { return (q >> 1) ? v.y : v.x; };
-                    uint4 g;
-                    g.x = __byte_perm(word(bw[0]), word(bw[1]), sel);
-                    g.y = __byte_perm(word(bw[2]), word(bw[3]), sel);
-                    g.z = __byte_perm(word(cwd[0]), word(cwd[1]), sel);
-                    g.w = __byte_perm(word(cwd[2]), word(cwd[3]), sel);
-                    reinterpret_cast<uint4*>(sBt)[(4 * t4 + q) * (NMAX / 4) + n4] = g;
+                for (int q = 0; q < 2; ++q) {
+                    // step 2*t2+q sits in half q of each row's word; pair rows (0,1), (2,3)
+                    const unsigned sel = q ? 0x7632u : 0x5410u;
+                    uint2 g;
+                    g.x = __byte_perm(w[0], w[1], sel);
+                    g.y = __byte_perm(w[2], w[3], sel);
+                    reinterpret_cast<uint2*>(sBt)[((2 * t2 + q) * (NMAX / 4) + n4) * 2 + which] = g;
                 }
-            } else {
+            }
+        } else {
+            for (int i = tid; i < (NMAX / 4) * (T / 4); i += Lo::THREADS) {
+                const int n4 = i % (NMAX / 4), t4 = i / (NMAX / 4);
                 float bv[4][4], cv[4][4];
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {

@@ -99,6 +99,100 @@ __global__ void __launch_bounds__(256) state_update_kernel(const UParams p) {
     }
 }
 
+// N = 16 fast path.  Two threads per (batch, channel) lane, each owning eight states:
+// thread h holds states 4h..4h+3 and 8+4h..8+4h+3, so for every 16-byte access the two
+// threads of a lane cover one whole 32-byte sector and a warp moves 16 contiguous lanes
+// (1 KiB of state) per instruction pair.  Each thread serves kItems lanes, one grid
+// stride apart, and issues every load of all of them before any arithmetic, keeping
+// 64 bytes of state per thread in flight.  Math runs on packed fp32 pairs.
+constexpr int kItems = 2;
+
+template <typename Tio>
+struct Lane16 {
+    float4 s0, s1, a0, a1;
+    typename vec4<Tio>::type b0, b1, c0, c1;
+    float u, x, z, dsk;
+};
+
+template <typename Tio>
+__global__ void __launch_bounds__(256) state_update16_kernel(const UParams p) {
+    using VT = typename vec4<Tio>::type;
+    const uint32_t pairs = (uint32_t)(gridDim.x * blockDim.x) / 2;  // lanes per item sweep
+    const uint32_t gid = blockIdx.x * blockDim.x + threadIdx.x;
+    const int h = gid & 1;
+    const uint32_t dim = (uint32_t)p.dim;
+    const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    Lane16<Tio> v[kItems];
+    uint32_t lid[kItems];
+    bool act[kItems];
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) {
+        const uint32_t lane_id = (gid >> 1) + it * pairs;
+        act[it] = lane_id < (uint32_t)p.lanes;
+        const uint32_t li = act[it] ? lane_id : 0;
+        lid[it] = li;
+        const uint32_t bb = li / dim, d = li - bb * dim;
+        const float* sp = p.state + (size_t)li * 16;
+        const float* ap = p.A + (size_t)d * 16;
+        const Tio* bp = static_cast<const Tio*>(p.B) + (size_t)bb * 16;
+        const Tio* cp = static_cast<const Tio*>(p.C) + (size_t)bb * 16;
+        v[it].s0 = act[it] ? *reinterpret_cast<const float4*>(sp + 4 * h) : z4;
+        v[it].s1 = act[it] ? *reinterpret_cast<const float4*>(sp + 8 + 4 * h) : z4;
+        v[it].a0 = __ldg(reinterpret_cast<const float4*>(ap + 4 * h));
+        v[it].a1 = __ldg(reinterpret_cast<const float4*>(ap + 8 + 4 * h));
+        v[it].b0 = *reinterpret_cast<const VT*>(bp + 4 * h);
+        v[it].b1 = *reinterpret_cast<const VT*>(bp + 8 + 4 * h);
+        v[it].c0 = *reinterpret_cast<const VT*>(cp + 4 * h);
+        v[it].c1 = *reinterpret_cast<const VT*>(cp + 8 + 4 * h);
+        v[it].u = io<Tio>::load(static_cast<const Tio*>(p.u) + li);
+        v[it].x = io<Tio>::load(static_cast<const Tio*>(p.delta) + li) +
+                  (p.delta_bias ? p.delta_bias[d] : 0.f);
+        v[it].z = p.z ? io<Tio>::load(static_cast<const Tio*>(p.z) + li) : 0.f;
+        v[it].dsk = p.D ? p.D[d] : 0.f;
+    }
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) {
+        const Lane16<Tio>& w = v[it];
+        float bv[8], cv[8], t[4];
+        vec4<Tio>::to_f(w.b0, t);
+        bv[0] = t[0], bv[1] = t[1], bv[2] = t[2], bv[3] = t[3];
+        vec4<Tio>::to_f(w.b1, t);
+        bv[4] = t[0], bv[5] = t[1], bv[6] = t[2], bv[7] = t[3];
+        vec4<Tio>::to_f(w.c0, t);
+        cv[0] = t[0], cv[1] = t[1], cv[2] = t[2], cv[3] = t[3];
+        vec4<Tio>::to_f(w.c1, t);
+        cv[4] = t[0], cv[5] = t[1], cv[6] = t[2], cv[7] = t[3];
+        const float dt = p.softplus ? softplus(w.x) : w.x;
+        const f2 dd = pack2(dt * kLog2e, dt * kLog2e);
+        const f2 qq = pack2(dt * w.u, dt * w.u);
+        const float sv[8] = {w.s0.x, w.s0.y, w.s0.z, w.s0.w, w.s1.x, w.s1.y, w.s1.z, w.s1.w};
+        const float av[8] = {w.a0.x, w.a0.y, w.a0.z, w.a0.w, w.a1.x, w.a1.y, w.a1.z, w.a1.w};
+        float out[8];
+        f2 acc = pack2(0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+            const f2 e = ex2x2(mul2(dd, pack2(av[j], av[j + 1])));
+            const f2 hn = fma2(e, pack2(sv[j], sv[j + 1]), mul2(qq, pack2(bv[j], bv[j + 1])));
+            acc = fma2(pack2(cv[j], cv[j + 1]), hn, acc);
+            unpack2(hn, out[j], out[j + 1]);
+        }
+        if (act[it]) {
+            float* wp = p.state + (size_t)lid[it] * 16;
+            *reinterpret_cast<float4*>(wp + 4 * h) = make_float4(out[0], out[1], out[2], out[3]);
+            *reinterpret_cast<float4*>(wp + 8 + 4 * h) = make_float4(out[4], out[5], out[6], out[7]);
+        }
+        float lo, hi;
+        unpack2(acc, lo, hi);
+        float yv = lo + hi;
+        yv += __shfl_xor_sync(0xffffffffu, yv, 1);
+        if (act[it] && h == 0) {
+            yv = fmaf(w.dsk, w.u, yv);
+            if (p.z) yv *= silu(w.z);
+            static_cast<Tio*>(p.y)[lid[it]] = io<Tio>::from_f(yv);
+        }
+    }
+}
+
 template <int NMAX, typename Tio>
 cudaError_t launch_u(const UParams& p, cudaStream_t s) {
     constexpr int G = NMAX / 4;
@@ -110,6 +204,11 @@ cudaError_t launch_u(const UParams& p, cudaStream_t s) {
 
 template <typename Tio>
 cudaError_t launch_u_typed(const UParams& p, cudaStream_t s) {
+    if (p.N == 16 && p.lanes < (1LL << 29)) {
+        const int64_t threads = 2 * ((p.lanes + kItems - 1) / kItems);
+        state_update16_kernel<Tio><<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(p);
+        return cudaGetLastError();
+    }
     if (p.N <= 4) return launch_u<4, Tio>(p, s);
     if (p.N <= 8) return launch_u<8, Tio>(p, s);
     return launch_u<16, Tio>(p, s);

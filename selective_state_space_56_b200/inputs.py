@@ -148,6 +148,21 @@ def decode_step_inputs(step: int, w: DecodeWorkload = DECODE_WORKLOAD, device="c
     return dict(u=u, delta=delta, z=z, B=B, C=C)
 
 
+def decode_tokens_batched(steps: int, w: DecodeWorkload = DECODE_WORKLOAD, device="cpu"):
+    """u, delta, z (steps, batch, dim) and B, C (steps, batch, N) for `steps` tokens at once,
+    drawn in that order from one generator seeded with the workload seed + 1_000_000
+    (used where per-token seeding is not needed and fewer, larger draws are wanted)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed + 1_000_000)
+
+    def normal(*shape):
+        return torch.randn(*shape, generator=g, dtype=torch.float32, device=device).to(w.io_dtype)
+
+    return dict(u=normal(steps, w.batch, w.dim), delta=normal(steps, w.batch, w.dim),
+                z=normal(steps, w.batch, w.dim), B=normal(steps, w.batch, w.dstate),
+                C=normal(steps, w.batch, w.dstate))
+
+
 def inverse_softplus_range():
     """The bias range the recipe produces: [log(expm1(0.001)), log(expm1(0.1))]."""
     return math.log(math.expm1(0.001)), math.log(math.expm1(0.1))

@@ -1,0 +1,62 @@
+"""The bench's multi-process host logic on CPU: two ranks over gloo.
+
+bench.py runs one process per GPU; every rank scans its own batch (weak scaling, no
+data-path collective) and the ranks only agree on timing through a max-reduction of
+one scalar.  Here two CPU processes run that plumbing over gloo on 127.0.0.1.
+"""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import bench
+    r, w, local = bench.dist_setup()
+    assert (r, w, local) == (rank, world, rank)
+    bench.barrier(w)
+    timed = 10.0 + rank          # each rank "measured" a different time
+    out[rank] = (bench.max_over_ranks(timed, w), bench.rank_seed(56003, r))
+    bench.barrier(w)
+    bench.dist_teardown(w)
+
+
+def test_two_ranks_agree_on_max_time_and_use_distinct_seeds():
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        procs = [ctx.Process(target=_rank_main, args=(r, world, port, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+            assert p.exitcode == 0
+        res = dict(out)
+    assert [res[r][0] for r in range(world)] == [11.0, 11.0]
+    assert len({res[r][1] for r in range(world)}) == world
+
+
+def test_single_rank_needs_no_process_group():
+    import bench
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+    bench.barrier(1)
+    bench.dist_teardown(1)
+
+
+@pytest.mark.parametrize("n", [1, 2, 4, 8])
+def test_weak_scaling_value_counts_every_rank(n):
+    # value = units all ranks processed / max time over ranks
+    elems = 4 * 5120 * 4096
+    ms_total, steps = 637.0, 1000
+    assert n * elems * steps / (ms_total * 1e-3) == pytest.approx(n * 1.3168e11, rel=1e-3)
