@@ -150,6 +150,26 @@ __device__ __forceinline__ f2 exp2_fma2(f2 x) {
                  __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
 }
 
+// softplus on four values at once, the polynomial on packed pairs.
+__device__ __forceinline__ void softplus4(const float (&x)[4], float (&out)[4]) {
+    float e[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) e[q] = ex2(-fabsf(x[q]) * kLog2e);
+#pragma unroll
+    for (int q = 0; q < 4; q += 2) {
+        const f2 ee = pack2(e[q], e[q + 1]);
+        f2 p = fma2(pack2(-8.5392082e-3f, -8.5392082e-3f), ee, pack2(4.4089634e-2f, 4.4089634e-2f));
+        p = fma2(p, ee, pack2(-1.0768171e-1f, -1.0768171e-1f));
+        p = fma2(p, ee, pack2(1.7745242e-1f, 1.7745242e-1f));
+        p = fma2(p, ee, pack2(-2.4495463e-1f, -2.4495463e-1f));
+        p = fma2(p, ee, pack2(3.3275479e-1f, 3.3275479e-1f));
+        p = fma2(p, ee, pack2(-4.9997404e-1f, -4.9997404e-1f));
+        p = fma2(p, ee, pack2(9.9999982e-1f, 9.9999982e-1f));
+        const f2 r = fma2(ee, p, pack2(fmaxf(x[q], 0.f), fmaxf(x[q + 1], 0.f)));
+        unpack2(r, out[q], out[q + 1]);
+    }
+}
+
 // A bf16 pair (element 0 in the low half of the word) widened exactly to an fp32 pair.
 __device__ __forceinline__ f2 bf16pair(uint32_t w) {
     return pack2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));

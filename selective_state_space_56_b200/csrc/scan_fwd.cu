@@ -105,9 +105,11 @@ enum Mode : int { kFull = 0, kAggregate = 1 };
 #ifndef S6_CHUNK
 #define S6_CHUNK 32
 #endif
-// bf16 inputs keep B, C as bf16 pairs in shared memory (half the bytes per lane-step).
-#ifndef S6_PACKBC
-#define S6_PACKBC 1
+// Coefficient tile format for bf16 inputs: 0 = B and C widened to fp32; 1 = B and C kept
+// as bf16 pairs (half the shared-memory bytes, widened in registers); 2 = B in fp32, C as
+// bf16 pairs.  fp32 inputs always use format 0.
+#ifndef S6_BC_MODE
+#define S6_BC_MODE 2
 #endif
 // Abar pairs evaluated on the FMA pipe (exp2_fma2) instead of the SFU: 0 = none,
 // 1 = the second pair of every other step (a quarter of them), 2 = the second pair of
@@ -135,14 +137,13 @@ struct Layout {
     static constexpr size_t off_B = 3 * off_dr;
     static constexpr size_t off_C = off_B + align128(coef_bytes);
     static constexpr size_t stage_bytes = off_C + align128(coef_bytes);
-    // Per-step coefficients for the recurrence.  bf16 inputs: one 16-byte group per
-    // (step, 4 states) holding B[4] and C[4] as bf16 pairs; fp32 inputs: B and C as
-    // fp32 [T][NMAX] each.
-    static constexpr bool kPackedBC = sizeof(Tin) == 2 && S6_PACKBC;
-    // Two buffers (chunk parity), so a chunk's coefficients can be written while the
-    // previous chunk's are still being read.
+    // Per-step coefficients for the recurrence (format S6_BC_MODE for bf16 inputs, 0 for
+    // fp32 inputs).  Two buffers (chunk parity), so a chunk's coefficients can be written
+    // while the previous chunk's are still being read.
+    static constexpr int kBC = sizeof(Tin) == 2 ? S6_BC_MODE : 0;
     static constexpr size_t coef_fp32_bytes = (size_t)T * NMAX * 4;
-    static constexpr size_t coef_bytes_all = (kPackedBC ? 1 : 2) * coef_fp32_bytes;
+    static constexpr size_t coef_bytes_all =
+        kBC == 0 ? 2 * coef_fp32_bytes : (kBC == 1 ? coef_fp32_bytes : coef_fp32_bytes * 3 / 2);
     static constexpr size_t off_coef = 2 * stage_bytes;
     static constexpr size_t off_del = off_coef + 2 * coef_bytes_all;   // float [CH][RS]
     static constexpr size_t off_du = off_del + (size_t)CH * RS * 4;
@@ -306,15 +307,20 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         const int64_t t0 = t_begin + k * T;
         const int valid = (int)min((int64_t)T, t_end - t0);
         float* sBt = reinterpret_cast<float*>(smem + Lo::off_coef + (k & 1) * Lo::coef_bytes_all);
-        float* sCt = sBt + T * NMAX;  // fp32 inputs only
+        float* sCt = sBt + T * NMAX;  // formats 0 and 2: what follows the fp32 B tile
 
         // B, C of the chunk, time-major: every lane then reads the coefficients of its four
         // states for step t with one 16-byte load (bf16: B[4] and C[4] as pairs; fp32: a
         // 16-byte vector from each of two tiles, transposed through 4x4 register blocks).
-        if constexpr (Lo::kPackedBC) {
-            // work item: (4-state group, step pair, B or C) -> two 8-byte half-groups
-            for (int i = tid; i < (NMAX / 4) * (T / 2) * 2; i += Lo::THREADS) {
-                const int which = i & 1, n4 = (i >> 1) % (NMAX / 4), t2 = (i >> 1) / (NMAX / 4);
+        if constexpr (Lo::kBC == 1 || Lo::kBC == 2) {
+            // bf16 pairs.  Format 1: per (step, 4-state group) [B0|B1][B2|B3][C0|C1][C2|C3];
+            // format 2: the C half only, [C0|C1][C2|C3] per (step, group), after the B tile.
+            // Work item: (4-state group, step pair, B or C) -> two 8-byte half-groups.
+            constexpr int kWhich = Lo::kBC == 1 ? 2 : 1;
+            for (int i = tid; i < (NMAX / 4) * (T / 2) * kWhich; i += Lo::THREADS) {
+                const int which = kWhich == 2 ? (i & 1) : 1;
+                const int i2 = kWhich == 2 ? (i >> 1) : i;
+                const int n4 = i2 % (NMAX / 4), t2 = i2 / (NMAX / 4);
                 const Tin* src = (which ? rC : rB) + (4 * n4) * T + 2 * t2;
                 uint32_t w[4];
 #pragma unroll
@@ -326,25 +332,31 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
                     uint2 g;
                     g.x = __byte_perm(w[0], w[1], sel);
                     g.y = __byte_perm(w[2], w[3], sel);
-                    reinterpret_cast<uint2*>(sBt)[((2 * t2 + q) * (NMAX / 4) + n4) * 2 + which] = g;
+                    const int grp = (2 * t2 + q) * (NMAX / 4) + n4;
+                    if (Lo::kBC == 1)
+                        reinterpret_cast<uint2*>(sBt)[grp * 2 + which] = g;
+                    else
+                        reinterpret_cast<uint2*>(sCt)[grp] = g;
                 }
             }
-        } else {
-            for (int i = tid; i < (NMAX / 4) * (T / 4); i += Lo::THREADS) {
-                const int n4 = i % (NMAX / 4), t4 = i / (NMAX / 4);
-                float bv[4][4], cv[4][4];
+        }
+        if constexpr (Lo::kBC == 0 || Lo::kBC == 2) {
+            // fp32 tiles [T][NMAX], transposed through 4x4 register blocks
+            constexpr int kTiles = Lo::kBC == 0 ? 2 : 1;
+            for (int i = tid; i < (NMAX / 4) * (T / 4) * kTiles; i += Lo::THREADS) {
+                const int which = kTiles == 2 ? (i & 1) : 0;
+                const int i2 = kTiles == 2 ? (i >> 1) : i;
+                const int n4 = i2 % (NMAX / 4), t4 = i2 / (NMAX / 4);
+                const Tin* src = which ? rC : rB;
+                float* dst = which ? sCt : sBt;
+                float v[4][4];
 #pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    V4::to_f(*reinterpret_cast<const VT*>(rB + (4 * n4 + r) * T + 4 * t4), bv[r]);
-                    V4::to_f(*reinterpret_cast<const VT*>(rC + (4 * n4 + r) * T + 4 * t4), cv[r]);
-                }
+                for (int r = 0; r < 4; ++r)
+                    V4::to_f(*reinterpret_cast<const VT*>(src + (4 * n4 + r) * T + 4 * t4), v[r]);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    *reinterpret_cast<float4*>(sBt + (4 * t4 + q) * NMAX + 4 * n4) =
-                        make_float4(bv[0][q], bv[1][q], bv[2][q], bv[3][q]);
-                    *reinterpret_cast<float4*>(sCt + (4 * t4 + q) * NMAX + 4 * n4) =
-                        make_float4(cv[0][q], cv[1][q], cv[2][q], cv[3][q]);
-                }
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<float4*>(dst + (4 * t4 + q) * NMAX + 4 * n4) =
+                        make_float4(v[0][q], v[1][q], v[2][q], v[3][q]);
             }
         }
         // The one CTA-wide barrier of a chunk: coefficients visible to every warp, and
@@ -369,11 +381,14 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
             V4::to_f(*reinterpret_cast<const VT*>(rDr + c * T + tb), x);
             V4::to_f(*reinterpret_cast<const VT*>(rU + c * T + tb), uu);
             const float bias = sBias[c];
-            float dt[4];
+            float dt[4], xb[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float xb = x[q] + bias;
-                dt[q] = p.softplus ? softplus(xb) : xb;
+            for (int q = 0; q < 4; ++q) xb[q] = x[q] + bias;
+            if (p.softplus) {
+                softplus4(xb, dt);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) dt[q] = xb[q];
             }
             if (valid < T) {
 #pragma unroll
@@ -403,11 +418,18 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
 #pragma unroll
                 for (int j = 0; j < NS / 4; ++j) {
                     f2 b01, b23, c01, c23;
-                    if constexpr (Lo::kPackedBC) {
+                    if constexpr (Lo::kBC == 1) {
                         const uint4 g = reinterpret_cast<const uint4*>(sBt)[(t + kk) * (NMAX / 4) +
                                                                             pp * (NS / 4) + j];
                         b01 = bf16pair(g.x), b23 = bf16pair(g.y);
                         c01 = bf16pair(g.z), c23 = bf16pair(g.w);
+                    } else if constexpr (Lo::kBC == 2) {
+                        const ulonglong2 bb = reinterpret_cast<const ulonglong2*>(
+                            sBt + (t + kk) * NMAX + pp * NS)[j];
+                        const uint2 g = reinterpret_cast<const uint2*>(sCt)[(t + kk) * (NMAX / 4) +
+                                                                          pp * (NS / 4) + j];
+                        b01 = f2{bb.x}, b23 = f2{bb.y};
+                        c01 = bf16pair(g.x), c23 = bf16pair(g.y);
                     } else {
                         const ulonglong2 bb = reinterpret_cast<const ulonglong2*>(
                             sBt + (t + kk) * NMAX + pp * NS)[j];

@@ -58,7 +58,21 @@ def test_decode_workload_1000_steps(cuda_ok):
 @pytest.mark.parametrize("N", [1, 4, 6, 8, 12, 16])
 @pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
 def test_decode_shapes(cuda_ok, N, io):
-    b, d = 3, 37
+    _decode_case(3, 37, N, io)
+
+
+# N = 16 shapes for the two-lanes-per-thread path: one tile, many tiles, several batch
+# rows, lane counts whose last warp is only partly used; each with and without z / D /
+# bias.
+@pytest.mark.parametrize("bd", [(1, 128), (2, 256), (3, 1024), (5, 640), (1, 136), (3, 40),
+                                (4, 1000), (7, 584)])
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+def test_decode_n16_shapes(cuda_ok, bd, io):
+    _decode_case(bd[0], bd[1], 16, io)
+    _decode_case(bd[0], bd[1], 16, io, with_optional=False)
+
+
+def _decode_case(b, d, N, io, with_optional=True):
     g = torch.Generator().manual_seed(100 + N)
     st0 = 0.1 * torch.randn(b, d, N, generator=g)
     x = {k: torch.randn(*s, generator=g).to(io) for k, s in
@@ -66,10 +80,14 @@ def test_decode_shapes(cuda_ok, N, io):
     A = -torch.arange(1, N + 1, dtype=torch.float32).expand(d, N).contiguous()
     D = torch.randn(d, generator=g)
     bias = torch.log(torch.expm1(0.001 + 0.099 * torch.rand(d, generator=g, dtype=torch.float64))).float()
+    if not with_optional:
+        D = bias = None
+        x["z"] = None
+    dev = lambda t: None if t is None else t.to(DEV)  # noqa: E731
     state = st0.to(DEV)
     y = ops.selective_state_update(state, *(x[k].to(DEV) for k in ("u", "delta")), A.to(DEV),
-                                   x["B"].to(DEV), x["C"].to(DEV), D=D.to(DEV), z=x["z"].to(DEV),
-                                   delta_bias=bias.to(DEV))
+                                   x["B"].to(DEV), x["C"].to(DEV), D=dev(D), z=dev(x["z"]),
+                                   delta_bias=dev(bias))
     s_ref, y_ref = oracle.state_update(st0, x["u"], x["delta"], A, x["B"], x["C"], D=D, z=x["z"],
                                        delta_bias=bias)
     torch.cuda.synchronize()
