@@ -69,6 +69,9 @@ def _load():
             lib.s6o_state_update.restype = ctypes.c_int
             lib.s6o_state_update.argtypes = ([ctypes.c_long] * 3 + [_dp] * 9 + [_lp, ctypes.c_int,
                                                                              _dp])
+            lib.s6o_scan_backward.restype = ctypes.c_int
+            lib.s6o_scan_backward.argtypes = ([ctypes.c_long] * 4 + [_dp] * 8 + [_lp, ctypes.c_int]
+                                              + [_dp] * 9)
             lib.s6o_num_threads.restype = ctypes.c_int
             lib.s6o_num_threads.argtypes = []
             _lib = lib
@@ -223,3 +226,48 @@ def state_update_lanes(state, u, delta_raw, A, B, C, lane_batch, D=None, z=None,
     if rc != 0:
         raise ValueError("s6o_state_update rejected its arguments")
     return st, y
+
+
+def scan_backward_lanes(u, delta_raw, A, B, C, lane_batch, dy, D=None, z=None, delta_bias=None,
+                        softplus=True):
+    """Gradients of sum(y * dy) for lanes: returns dict du, ddelta, dz (nlanes, L),
+    dA (nlanes, N), dD, dbias (nlanes), dB, dC (nbatch, N, L)."""
+    u, dr, z, dy = _f64(u), _f64(delta_raw), _f64(z), _f64(dy)
+    Aa, Dd, bb = _f64(A), _f64(D), _f64(delta_bias)
+    Bm, Cm = _f64(B), _f64(C)
+    nl, L = u.shape
+    N = Aa.shape[1]
+    nb = Bm.shape[0]
+    lb = np.ascontiguousarray(np.asarray(lane_batch, dtype=np.int64).reshape(nl))
+    out = dict(du=np.empty((nl, L)), ddelta=np.empty((nl, L)), dz=np.empty((nl, L)),
+               dA=np.empty((nl, N)), dD=np.empty(nl), dbias=np.empty(nl),
+               dB=np.empty((nb, N, L)), dC=np.empty((nb, N, L)))
+    rc = _load().s6o_scan_backward(
+        nl, N, L, nb, _ptr(u), _ptr(dr), _ptr(z), _ptr(Aa), _ptr(Dd), _ptr(bb), _ptr(Bm),
+        _ptr(Cm), lb.ctypes.data_as(_lp), int(bool(softplus)), _ptr(dy), _ptr(out["du"]),
+        _ptr(out["ddelta"]), _ptr(out["dz"]), _ptr(out["dA"]), _ptr(out["dD"]),
+        _ptr(out["dbias"]), _ptr(out["dB"]), _ptr(out["dC"]))
+    if rc != 0:
+        raise ValueError("s6o_scan_backward rejected its arguments")
+    return out
+
+
+def selective_scan_backward(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
+                            softplus=True):
+    """Backward in the library's layouts: u, delta, z, dy (b, d, L); A (d, N); B, C
+    (b, N, L); D, delta_bias (d).  Returns du, ddelta, dz (b, d, L), dA (d, N), dD, dbias (d),
+    dB, dC (b, N, L): the gradients of sum(y * dy)."""
+    u = _f64(u)
+    b, d, L = u.shape
+    Aa = _f64(A)
+    N = Aa.shape[1]
+    rep = lambda v: None if v is None else np.tile(_f64(v), b)  # noqa: E731
+    r = scan_backward_lanes(u.reshape(b * d, L), _f64(delta).reshape(b * d, L),
+                            np.tile(Aa, (b, 1)), B, C, np.repeat(np.arange(b), d),
+                            _f64(dy).reshape(b * d, L), D=rep(D),
+                            z=None if z is None else _f64(z).reshape(b * d, L),
+                            delta_bias=rep(delta_bias), softplus=softplus)
+    return dict(du=r["du"].reshape(b, d, L), ddelta=r["ddelta"].reshape(b, d, L),
+                dz=r["dz"].reshape(b, d, L), dA=r["dA"].reshape(b, d, N).sum(0),
+                dD=r["dD"].reshape(b, d).sum(0), dbias=r["dbias"].reshape(b, d).sum(0),
+                dB=r["dB"], dC=r["dC"])

@@ -34,6 +34,7 @@
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #define S6O_OK 0
 #define S6O_ERR_ARG (-1)
@@ -170,6 +171,106 @@ int s6o_state_update(long nlanes, long N, long nbatch, double* state,
         if (z) acc *= silu(z[i]);
         y[i] = acc;
     }
+    return S6O_OK;
+}
+
+/*
+ * Backward of the scan (gradients of a scalar loss through y), for lanes.
+ *
+ * Forward recap per lane: x_t = delta_raw_t + bias; Delta_t = softplus(x_t) (or x_t);
+ * Abar_tn = exp(Delta_t A_n); q_t = Delta_t u_t; h_tn = Abar_tn h_{t-1,n} + q_t B_tn
+ * (h_{-1} = 0); yt_t = sum_n C_tn h_tn + D u_t (pre-gate); y_t = yt_t silu(z_t).
+ *
+ * Reverse sweep (chain rule, adjoint state g_n = dL/dh_tn accumulated backwards):
+ *   dyt_t = dy_t silu(z_t);   dz_t = dy_t yt_t silu'(z_t)
+ *   g_n  += dyt_t C_tn                        (g also holds Abar_{t+1} g_{t+1})
+ *   dC_tn += dyt_t h_tn;  dB_tn += g_n q_t;   dq_t = sum_n g_n B_tn
+ *   dDelta_t = dq_t u_t + sum_n g_n h_{t-1,n} Abar_tn A_n
+ *   dA_n += g_n h_{t-1,n} Abar_tn Delta_t;    dD += dyt_t u_t
+ *   du_t = dyt_t D + dq_t Delta_t;  dx_t = dDelta_t softplus'(x_t) (= sigmoid(x_t))
+ *   dbias += dx_t;  then g_n *= Abar_tn  (carried to step t-1)
+ *
+ * Shapes as in s6o_scan; dy (nlanes, L); outputs du, ddelta, dz (nlanes, L);
+ * dA (nlanes, N); dD, dbias (nlanes); dB, dC (nbatch, N, L) accumulated over lanes
+ * (zeroed here first).  Any output pointer may be NULL except du and ddelta.
+ * Sequential over lanes (dB / dC are shared by the lanes of a batch).
+ */
+static double sigmoid(double x) {
+    if (x >= 0.0) return 1.0 / (1.0 + exp(-x));
+    double e = exp(x);
+    return e / (1.0 + e);
+}
+
+int s6o_scan_backward(long nlanes, long N, long L, long nbatch,
+                      const double* u, const double* delta_raw, const double* z,
+                      const double* A, const double* D, const double* delta_bias,
+                      const double* Bm, const double* Cm, const long* lane_batch,
+                      int softplus, const double* dy,
+                      double* du, double* ddelta, double* dz, double* dA, double* dD,
+                      double* dbias, double* dB, double* dC) {
+    if (nlanes < 0 || N < 1 || N > S6O_MAX_N || L < 0 || nbatch < 1) return S6O_ERR_ARG;
+    if (!u || !delta_raw || !A || !Bm || !Cm || !lane_batch || !dy || !du || !ddelta)
+        return S6O_ERR_ARG;
+    for (long i = 0; i < nlanes; ++i)
+        if (lane_batch[i] < 0 || lane_batch[i] >= nbatch) return S6O_ERR_ARG;
+    if (dB) for (long k = 0; k < nbatch * N * L; ++k) dB[k] = 0.0;
+    if (dC) for (long k = 0; k < nbatch * N * L; ++k) dC[k] = 0.0;
+    double* hs = (double*)malloc(sizeof(double) * (size_t)(L + 1) * (size_t)N);
+    if (!hs) return S6O_ERR_ARG;
+    for (long i = 0; i < nlanes; ++i) {
+        const double* Bb = Bm + lane_batch[i] * N * L;
+        const double* Cb = Cm + lane_batch[i] * N * L;
+        const double bias = delta_bias ? delta_bias[i] : 0.0;
+        const double dskip = D ? D[i] : 0.0;
+        /* forward, keeping every state: hs[(t+1)*N + n] = h_tn, hs[n] = h_{-1} = 0 */
+        for (long n = 0; n < N; ++n) hs[n] = 0.0;
+        for (long t = 0; t < L; ++t) {
+            const double dt = step_size(delta_raw[i * L + t], bias, softplus);
+            for (long n = 0; n < N; ++n)
+                hs[(t + 1) * N + n] = exp(dt * A[i * N + n]) * hs[t * N + n] +
+                                      dt * u[i * L + t] * Bb[n * L + t];
+        }
+        double g[S6O_MAX_N], dAn[S6O_MAX_N];
+        for (long n = 0; n < N; ++n) g[n] = 0.0, dAn[n] = 0.0;
+        double dDi = 0.0, dbi = 0.0;
+        for (long t = L - 1; t >= 0; --t) {
+            const double x = delta_raw[i * L + t] + bias;
+            const double dt = softplus ? s6o_softplus(x) : x;
+            const double ut = u[i * L + t];
+            double yt = dskip * ut;
+            for (long n = 0; n < N; ++n) yt += Cb[n * L + t] * hs[(t + 1) * N + n];
+            double dyt = dy[i * L + t];
+            if (z) {
+                const double zz = z[i * L + t], sg = sigmoid(zz);
+                if (dz) dz[i * L + t] = dy[i * L + t] * yt * sg * (1.0 + zz * (1.0 - sg));
+                dyt = dy[i * L + t] * zz * sg;
+            } else if (dz) {
+                dz[i * L + t] = 0.0;
+            }
+            double dq = 0.0, ddt = 0.0;
+            for (long n = 0; n < N; ++n) {
+                const double abar = exp(dt * A[i * N + n]);
+                g[n] += dyt * Cb[n * L + t];
+                if (dC) dC[(lane_batch[i] * N + n) * L + t] += dyt * hs[(t + 1) * N + n];
+                if (dB) dB[(lane_batch[i] * N + n) * L + t] += g[n] * dt * ut;
+                dq += g[n] * Bb[n * L + t];
+                const double gh = g[n] * hs[t * N + n] * abar;
+                ddt += gh * A[i * N + n];
+                dAn[n] += gh * dt;
+                g[n] *= abar;
+            }
+            ddt += dq * ut;
+            dDi += dyt * ut;
+            du[i * L + t] = dyt * dskip + dq * dt;
+            const double dx = softplus ? ddt * sigmoid(x) : ddt;
+            ddelta[i * L + t] = dx;
+            dbi += dx;
+        }
+        if (dA) for (long n = 0; n < N; ++n) dA[i * N + n] = dAn[n];
+        if (dD) dD[i] = dDi;
+        if (dbias) dbias[i] = dbi;
+    }
+    free(hs);
     return S6O_OK;
 }
 
