@@ -1,11 +1,12 @@
 /*
  * mamba_s6.h -- C ABI of the B200 (sm_100a) selective-scan library.
  *
- * Two operations, each a hand-written CUDA kernel sequence launched on the
+ * Three operations, each a hand-written CUDA kernel sequence launched on the
  * caller's stream:
  *
  *   mamba_selective_scan_fwd      the fused S6 forward scan over a whole sequence
  *   mamba_selective_state_update  one decode token, updating a carried state in place
+ *   mamba_selective_scan_bwd      gradients of the forward scan, states recomputed
  *
  * Definitions (Mamba: Linear-Time Sequence Modeling with Selective State Spaces,
  * page "xyznot.com/ar/paper/2312.00752", sections "Method", "Selection mechanism
@@ -151,6 +152,50 @@ int mamba_selective_scan_fwd_noalloc(const void* u, const void* delta, const flo
                                      const float* delta_bias, int delta_softplus, void* y,
                                      float* last_state, mamba_scan_dims dims,
                                      mamba_dtype in_dtype, mamba_dtype out_dtype, void* stream);
+
+/*
+ * Bytes of device workspace mamba_selective_scan_bwd needs for `dims`:
+ * batch x dim x ceil(seqlen / T) x dstate x 4, T = 32 steps for dstate > 8 and 64
+ * otherwise, rounded up to 256 bytes (0 when seqlen == 0).  Returns 0 for invalid dims.
+ */
+size_t mamba_selective_scan_bwd_workspace_size(mamba_scan_dims dims);
+
+/*
+ * Backward of mamba_selective_scan_fwd: given dy = dLoss/dy, writes the gradients of
+ * every input.  The intermediate states are not read from memory (the forward never
+ * stored them); as the method's hardware-aware algorithm prescribes, they are
+ * recomputed: a forward pass records the state entering every T-step chunk in the
+ * workspace, and a reverse sweep rebuilds each chunk's states from its record
+ * before propagating the adjoint state backwards through it (Mamba, section
+ * "Hardware-aware state expansion").
+ *
+ *   u, delta, A, B, C, D, z, delta_bias, delta_softplus, dims, in_dtype
+ *               : exactly the forward's inputs (same layouts and rules)
+ *   dy          : (batch, dim, seqlen)  in_dtype       gradient of y
+ *   du, ddelta  : (batch, dim, seqlen)  in_dtype       written; ddelta is the gradient
+ *                                                      of the raw delta (before the
+ *                                                      bias and softplus)
+ *   dz          : (batch, dim, seqlen)  in_dtype       written; NULL iff z is NULL
+ *   dA          : (dim, dstate)         float32        written (summed over batch, t)
+ *   dB, dC      : (batch, dstate, seqlen) float32      written (summed over channels)
+ *   dD          : (dim) float32                        written; NULL iff D is NULL
+ *   ddelta_bias : (dim) float32                        written; NULL iff delta_bias is NULL
+ *   workspace   : at least mamba_selective_scan_bwd_workspace_size(dims) bytes; its
+ *                 contents on entry do not matter
+ *
+ * dA, dB, dC, dD and ddelta_bias are sums over many CTAs, formed with float32
+ * atomics: their last bits may differ between runs.  With seqlen == 0 the
+ * per-token arrays may be NULL and dA, dD, ddelta_bias are set to zero.
+ * Errors: NULL (a required pointer, or a gradient whose presence does not match its
+ * input's), DIMS, ALIGN, DTYPE, WORKSPACE, CUDA.
+ */
+int mamba_selective_scan_bwd(const void* u, const void* delta, const float* A, const void* B,
+                             const void* C, const float* D, const void* z,
+                             const float* delta_bias, int delta_softplus, const void* dy,
+                             void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC,
+                             float* dD, float* ddelta_bias, mamba_scan_dims dims,
+                             mamba_dtype in_dtype, void* workspace, size_t workspace_bytes,
+                             void* stream);
 
 /*
  * Reads the library's device error word on `stream`, synchronising that stream.

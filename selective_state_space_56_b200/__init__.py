@@ -1,4 +1,5 @@
-"""B200-native selective scan (S6): fused forward scan and single-token state update.
+"""B200-native selective scan (S6): fused forward scan, its backward, and the
+single-token state update.
 
 The compute lives in hand-written sm_100a CUDA kernels behind a C ABI
 (``include/mamba_s6.h``, built into ``libmamba_s6.so`` in this package by
@@ -9,6 +10,8 @@ from .ops import (  # noqa: F401
     MambaError,
     check_device_error,
     load_library,
+    selective_scan_bwd,
+    selective_scan_bwd_workspace_size,
     selective_scan_fwd,
     selective_scan_workspace_size,
     selective_state_update,

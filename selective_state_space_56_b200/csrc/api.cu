@@ -134,6 +134,78 @@ int mamba_selective_state_update(float* state, const void* u, const void* delta,
     return cuda_status(s6::launch_state_update(a, static_cast<cudaStream_t>(stream)));
 }
 
+size_t mamba_selective_scan_bwd_workspace_size(mamba_scan_dims dims) {
+    if (!dims_ok(dims.batch, dims.dim, dims.dstate, dims.seqlen)) return 0;
+    const int64_t T = s6::scan_chunk_steps(dims.dstate);
+    const int64_t chunks = (dims.seqlen + T - 1) / T;
+    if (!mul_ok(dims.batch * dims.dim, chunks) || !mul_ok(dims.batch * dims.dim * chunks, dims.dstate * 4))
+        return 0;
+    const int64_t bytes = dims.batch * dims.dim * chunks * dims.dstate * 4;
+    return (size_t)((bytes + 255) / 256 * 256);
+}
+
+int mamba_selective_scan_bwd(const void* u, const void* delta, const float* A, const void* B,
+                             const void* C, const float* D, const void* z,
+                             const float* delta_bias, int delta_softplus, const void* dy,
+                             void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC,
+                             float* dD, float* ddelta_bias, mamba_scan_dims dims,
+                             mamba_dtype in_dtype, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+    const bool empty = dims.seqlen == 0;
+    if (!A || !dA) return MAMBA_ERR_NULL;
+    if (!empty && (!u || !delta || !B || !C || !dy || !du || !ddelta || !dB || !dC))
+        return MAMBA_ERR_NULL;
+    // a gradient is present exactly when its input is
+    if ((D == nullptr) != (dD == nullptr) || (delta_bias == nullptr) != (ddelta_bias == nullptr))
+        return MAMBA_ERR_NULL;
+    if (!empty && (z == nullptr) != (dz == nullptr)) return MAMBA_ERR_NULL;
+    if (!dtype_ok(in_dtype)) return MAMBA_ERR_DTYPE;
+    if (!dims_ok(dims.batch, dims.dim, dims.dstate, dims.seqlen)) return MAMBA_ERR_DIMS;
+    const void* ptrs[] = {u, delta, A, B, C, D, z, delta_bias, dy, du, ddelta, dz,
+                          dA, dB, dC, dD, ddelta_bias};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MAMBA_ERR_ALIGN;
+    const size_t need = mamba_selective_scan_bwd_workspace_size(dims);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need) return MAMBA_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return MAMBA_ERR_ALIGN;
+    }
+    s6::ScanArgs a;
+    a.u = u;
+    a.delta = delta;
+    a.z = z;
+    a.A = A;
+    a.B = B;
+    a.C = C;
+    a.D = D;
+    a.delta_bias = delta_bias;
+    a.y = nullptr;
+    a.last_state = nullptr;
+    a.batch = dims.batch;
+    a.dim = dims.dim;
+    a.N = dims.dstate;
+    a.L = dims.seqlen;
+    a.softplus = delta_softplus;
+    a.in_dtype = to_dtype(in_dtype);
+    a.out_dtype = a.in_dtype;
+    a.nseg = 1;
+    a.seg_len = dims.seqlen;
+    a.seg_h = nullptr;
+    a.seg_sum = nullptr;
+    s6::BackwardArgs g;
+    g.dy = dy;
+    g.du = du;
+    g.ddelta = ddelta;
+    g.dz = dz;
+    g.dA = dA;
+    g.dB = dB;
+    g.dC = dC;
+    g.dD = dD;
+    g.ddelta_bias = ddelta_bias;
+    return cuda_status(s6::launch_scan_backward(a, g, static_cast<float*>(workspace),
+                                                static_cast<cudaStream_t>(stream)));
+}
+
 int mamba_check_device_error(int clear, void* stream) {
     unsigned word = 0;
     if (s6::read_device_error(&word, clear != 0, static_cast<cudaStream_t>(stream)) != cudaSuccess)
@@ -155,6 +227,6 @@ const char* mamba_status_string(int status) {
     }
 }
 
-int mamba_abi_version(void) { return 100; }
+int mamba_abi_version(void) { return 101; }
 
 }  // extern "C"

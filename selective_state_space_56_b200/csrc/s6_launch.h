@@ -56,6 +56,35 @@ void plan_segments(int64_t batch, int64_t dim, int64_t L, int64_t* nseg, int64_t
 cudaError_t launch_scan(const ScanArgs& a, cudaStream_t stream);
 cudaError_t launch_state_update(const StateUpdateArgs& a, cudaStream_t stream);
 
+// Steps per chunk of the forward kernel for state width N (the backward recomputes
+// states chunk by chunk from checkpoints taken at these boundaries).
+int scan_chunk_steps(int64_t N);
+
+// Forward pass that writes the state entering every chunk to
+// ckpt[((b * dim + d) * chunks + k) * N + n], chunks = ceil(L / scan_chunk_steps(N)),
+// and no output.  Uses a.u, delta, A, B, C, delta_bias, softplus, dims and in_dtype.
+cudaError_t launch_scan_checkpoints(const ScanArgs& a, float* ckpt, cudaStream_t stream);
+
+// Gradients of the scan (outputs of the backward); dy is read, the rest written.
+struct BackwardArgs {
+    const void* dy;     // (batch, dim, L) in_dtype
+    void* du;           // (batch, dim, L) in_dtype
+    void* ddelta;       // (batch, dim, L) in_dtype, gradient of the raw delta
+    void* dz;           // (batch, dim, L) in_dtype, null when there is no gate
+    float* dA;          // (dim, N)
+    float* dB;          // (batch, N, L)
+    float* dC;          // (batch, N, L)
+    float* dD;          // (dim), null when there is no skip term
+    float* ddelta_bias; // (dim), null when there is no bias
+};
+
+// Backward of the scan described by `a` (its y, last_state and segment fields are
+// unused): zeroes the accumulated outputs, runs the checkpointing forward into
+// `ckpt` (batch * dim * ceil(L / scan_chunk_steps(N)) * N floats) and then the
+// reverse sweep.
+cudaError_t launch_scan_backward(const ScanArgs& a, const BackwardArgs& g, float* ckpt,
+                                 cudaStream_t stream);
+
 // Reads (and optionally clears) the device error word on `stream`, synchronising it.
 // Bit 0: a bounded device-side wait gave up.
 cudaError_t read_device_error(unsigned* out, bool clear, cudaStream_t stream);

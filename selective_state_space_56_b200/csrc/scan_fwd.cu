@@ -93,7 +93,10 @@ __device__ __forceinline__ void store4(__nv_bfloat16* dst, const float (&o)[4]) 
     *reinterpret_cast<uint2*>(dst) = v;
 }
 
-enum Mode : int { kFull = 0, kAggregate = 1 };
+// kFull: the scan itself; kAggregate: split-sequence pass 1 (end state and summed step
+// per segment, no output); kCheckpoint: the backward's forward pass (the state at the
+// start of every chunk, no output).
+enum Mode : int { kFull = 0, kAggregate = 1, kCheckpoint = 2 };
 
 // Tuning of the N = 16 instantiation: lanes per channel, warps per CTA, chunk length.
 #ifndef S6_P16
@@ -400,6 +403,19 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         }
         __syncwarp();
 
+        if (MODE == kCheckpoint && dch < p.dim) {
+            // state entering chunk k: ckpt[((b * dim + d) * chunks + k) * N + n]
+            const int64_t chunks = (p.L + T - 1) / T;
+            float* ck = p.seg_h + ((b * p.dim + dch) * chunks + k) * p.N;
+#pragma unroll
+            for (int j = 0; j < NS / 2; ++j) {
+                float h0, h1;
+                unpack2(hp[j], h0, h1);
+                if (pp * NS + 2 * j < p.N) ck[pp * NS + 2 * j] = h0;
+                if (pp * NS + 2 * j + 1 < p.N) ck[pp * NS + 2 * j + 1] = h1;
+            }
+        }
+
         // Phase B: the recurrence, four steps per iteration, states in packed pairs.
 #pragma unroll
         for (int t = 0; t < T; t += 4) {
@@ -450,7 +466,9 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
                 unpack2(acc, lo, hi);
                 yp[kk] = lo + hi;
             }
-            if (MODE == kAggregate) {
+            if (MODE == kCheckpoint) {
+                // states only
+            } else if (MODE == kAggregate) {
                 float dv[4], dup;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) unpack2(dd4[kk], dv[kk], dup);
@@ -535,7 +553,7 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
                     if (nn < p.N) p.last_state[(b * p.dim + dch) * p.N + nn] = h[n];
                 }
             }
-        } else {
+        } else if (MODE == kAggregate) {
             const int64_t row = ((int64_t)seg * p.batch + b) * p.dim + dch;
 #pragma unroll
             for (int n = 0; n < NS; ++n) {
@@ -668,6 +686,34 @@ cudaError_t launch_io(const ScanArgs& a, KParams kp, cudaStream_t s) {
     return launch_typed<NMAX, Tin, Tout, true>(a, kp, tm, s);
 }
 
+template <int NMAX, typename Tin, bool TMA>
+cudaError_t launch_ckpt_typed(const ScanArgs& a, const KParams& kp, const TMaps& tm,
+                              cudaStream_t s) {
+    using TL = Tile<NMAX>;
+    using Lo = Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin>;
+    const unsigned gx = (unsigned)((a.dim + Lo::CH - 1) / Lo::CH);
+    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kCheckpoint, TMA>(
+        kp, tm, dim3(gx, (unsigned)a.batch, 1), s);
+}
+
+template <int NMAX, typename Tin>
+cudaError_t launch_ckpt_io(const ScanArgs& a, KParams kp, cudaStream_t s) {
+    using TL = Tile<NMAX>;
+    using Lo = Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin>;
+    TMaps tm;
+    memset(&tm, 0, sizeof(tm));
+    kp.y_tma = 0;
+    const bool rows16 = (a.L * (int64_t)sizeof(Tin)) % 16 == 0 && a.L > 0;
+    const bool fits = a.L < (1LL << 31) && a.dim < (1LL << 31) && a.batch < (1LL << 31);
+    if (!(rows16 && fits)) return launch_ckpt_typed<NMAX, Tin, false>(a, kp, tm, s);
+    const bool ok = encode_3d<Tin>(&tm.u, a.u, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
+                    encode_3d<Tin>(&tm.dr, a.delta, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
+                    encode_3d<Tin>(&tm.B, a.B, a.L, a.N, a.batch, Lo::T, NMAX) &&
+                    encode_3d<Tin>(&tm.C, a.C, a.L, a.N, a.batch, Lo::T, NMAX);
+    if (!ok) return cudaErrorInvalidValue;
+    return launch_ckpt_typed<NMAX, Tin, true>(a, kp, tm, s);
+}
+
 template <int NMAX>
 cudaError_t launch_nmax(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
     const bool ib = a.in_dtype == DType::BF16, ob = a.out_dtype == DType::BF16;
@@ -678,6 +724,35 @@ cudaError_t launch_nmax(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
 }
 
 }  // namespace
+
+int scan_chunk_steps(int64_t N) {
+    if (N <= 4) return Tile<4>::T;
+    if (N <= 8) return Tile<8>::T;
+    return Tile<16>::T;
+}
+
+cudaError_t launch_scan_checkpoints(const ScanArgs& a, float* ckpt, cudaStream_t stream) {
+    KParams kp;
+    memset(&kp, 0, sizeof(kp));
+    kp.u = a.u;
+    kp.delta = a.delta;
+    kp.A = a.A;
+    kp.B = a.B;
+    kp.C = a.C;
+    kp.delta_bias = a.delta_bias;
+    kp.seg_h = ckpt;
+    kp.batch = a.batch;
+    kp.dim = a.dim;
+    kp.L = a.L;
+    kp.seg_len = a.L;
+    kp.N = (int)a.N;
+    kp.nseg = 1;
+    kp.softplus = a.softplus ? 1 : 0;
+    const bool ib = a.in_dtype == DType::BF16;
+    if (a.N <= 4) return ib ? launch_ckpt_io<4, __nv_bfloat16>(a, kp, stream) : launch_ckpt_io<4, float>(a, kp, stream);
+    if (a.N <= 8) return ib ? launch_ckpt_io<8, __nv_bfloat16>(a, kp, stream) : launch_ckpt_io<8, float>(a, kp, stream);
+    return ib ? launch_ckpt_io<16, __nv_bfloat16>(a, kp, stream) : launch_ckpt_io<16, float>(a, kp, stream);
+}
 
 cudaError_t read_device_error(unsigned* out, bool clear, cudaStream_t stream) {
     unsigned v = 0;

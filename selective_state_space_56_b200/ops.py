@@ -52,6 +52,11 @@ def load_library():
             lib.mamba_selective_scan_fwd.restype = i32
             lib.mamba_selective_scan_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp,
                                                      ScanDims, i32, i32, vp, ctypes.c_size_t, vp]
+            lib.mamba_selective_scan_bwd_workspace_size.restype = ctypes.c_size_t
+            lib.mamba_selective_scan_bwd_workspace_size.argtypes = [ScanDims]
+            lib.mamba_selective_scan_bwd.restype = i32
+            lib.mamba_selective_scan_bwd.argtypes = [vp] * 8 + [i32] + [vp] * 9 + [
+                ScanDims, i32, vp, ctypes.c_size_t, vp]
             lib.mamba_selective_state_update.restype = i32
             lib.mamba_selective_state_update.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
                                                          vp, i64, i64, i64, i32, vp]
@@ -174,6 +179,60 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
     if return_last_state:
         return y, last_state
     return y
+
+
+def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
+                       delta_softplus=True, workspace=None):
+    """Gradients of ``selective_scan_fwd`` for the upstream gradient dy (batch, dim, L),
+    in the inputs' dtype.  Returns a dict with du, ddelta, dz (input dtype, dz None
+    without a gate), dA (dim, N), dB, dC (batch, N, L), dD, ddelta_bias (dim) in fp32
+    (None where the input is None)."""
+    if not isinstance(u, torch.Tensor) or u.dim() != 3:
+        raise ValueError("u must be a (batch, dim, L) tensor")
+    dev = u.device
+    if dev.type != "cuda":
+        raise ValueError("selective_scan_bwd runs on CUDA tensors only")
+    b, d, L = u.shape
+    N = A.shape[1] if A.dim() == 2 else -1
+    dt = u.dtype
+    if dt not in _DTYPES:
+        raise ValueError("unsupported input dtype %s" % dt)
+    for t, name, shape, dts in ((u, "u", (b, d, L), (dt,)), (delta, "delta", (b, d, L), (dt,)),
+                                (z, "z", (b, d, L), (dt,)), (dy, "dy", (b, d, L), (dt,)),
+                                (A, "A", (d, N), (torch.float32,)), (B, "B", (b, N, L), (dt,)),
+                                (C, "C", (b, N, L), (dt,)), (D, "D", (d,), (torch.float32,)),
+                                (delta_bias, "delta_bias", (d,), (torch.float32,))):
+        _check(t, name, dev, shape, dts)
+    f32 = torch.float32
+    g = dict(du=torch.empty((b, d, L), dtype=dt, device=dev),
+             ddelta=torch.empty((b, d, L), dtype=dt, device=dev),
+             dz=None if z is None else torch.empty((b, d, L), dtype=dt, device=dev),
+             dA=torch.empty((d, N), dtype=f32, device=dev),
+             dB=torch.empty((b, N, L), dtype=f32, device=dev),
+             dC=torch.empty((b, N, L), dtype=f32, device=dev),
+             dD=None if D is None else torch.empty(d, dtype=f32, device=dev),
+             ddelta_bias=None if delta_bias is None else torch.empty(d, dtype=f32, device=dev))
+    lib = load_library()
+    dims = ScanDims(b, d, N, L)
+    need = int(lib.mamba_selective_scan_bwd_workspace_size(dims))
+    if need > 0 and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        rc = lib.mamba_selective_scan_bwd(
+            _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+            int(bool(delta_softplus)), _ptr(dy), _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dz"]),
+            _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]), _ptr(g["ddelta_bias"]),
+            dims, _DTYPES[dt], _ptr(workspace), ws_bytes, _stream_handle(dev))
+    if rc != 0:
+        raise MambaError(rc, "mamba_selective_scan_bwd")
+    return g
+
+
+def selective_scan_bwd_workspace_size(batch: int, dim: int, dstate: int, seqlen: int) -> int:
+    """Bytes of workspace ``mamba_selective_scan_bwd`` needs (the chunk checkpoints)."""
+    return int(load_library().mamba_selective_scan_bwd_workspace_size(
+        ScanDims(batch, dim, dstate, seqlen)))
 
 
 def selective_state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,

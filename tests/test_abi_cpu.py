@@ -141,3 +141,50 @@ def test_binding_rejects_cpu_tensors():
     u = torch.zeros(1, 2, 8)
     with pytest.raises(ValueError):
         ops.selective_scan_fwd(u, u, torch.zeros(2, 4), torch.zeros(1, 4, 8), torch.zeros(1, 4, 8))
+
+
+def _bwd(lib, **kw):
+    args = dict(u=A16, delta=A16, A=A16, B=A16, C=A16, D=None, z=None, bias=None, sp=1, dy=A16,
+                du=A16, ddelta=A16, dz=None, dA=A16, dB=A16, dC=A16, dD=None, dbias=None,
+                dims=_dims(), i=1, ws=A16, wsb=1 << 30)
+    args.update(kw)
+    vp = lambda v: None if v is None else ctypes.c_void_p(v)  # noqa: E731
+    names = ("u", "delta", "A", "B", "C", "D", "z", "bias")
+    grads = ("dy", "du", "ddelta", "dz", "dA", "dB", "dC", "dD", "dbias")
+    return lib.mamba_selective_scan_bwd(*[vp(args[n]) for n in names], args["sp"],
+                                        *[vp(args[n]) for n in grads], args["dims"], args["i"],
+                                        vp(args["ws"]), args["wsb"], None)
+
+
+@pytest.mark.parametrize("field", ["u", "delta", "A", "B", "C", "dy", "du", "ddelta", "dA",
+                                   "dB", "dC"])
+def test_bwd_null_required_pointer(lib, field):
+    assert _bwd(lib, **{field: None}) == ERR_NULL
+
+
+@pytest.mark.parametrize("inp,grad", [("D", "dD"), ("z", "dz"), ("bias", "dbias")])
+def test_bwd_gradient_present_iff_input_present(lib, inp, grad):
+    assert _bwd(lib, **{inp: A16}) == ERR_NULL       # input without its gradient
+    assert _bwd(lib, **{grad: A16}) == ERR_NULL      # gradient without its input
+
+
+def test_bwd_dims_dtype_align_workspace(lib):
+    assert _bwd(lib, dims=_dims(2, 64, 17, 8)) == ERR_DIMS
+    assert _bwd(lib, i=3) == ERR_DTYPE
+    for f in ("u", "delta", "A", "B", "C", "dy", "du", "ddelta", "dA", "dB", "dC"):
+        assert _bwd(lib, **{f: A16 + 4}) == ERR_ALIGN, f
+    need = lib.mamba_selective_scan_bwd_workspace_size(_dims())
+    assert _bwd(lib, ws=None, wsb=0) == ERR_WORKSPACE
+    assert _bwd(lib, wsb=need - 1) == ERR_WORKSPACE
+    assert _bwd(lib, ws=A16 + 8, wsb=need) == ERR_ALIGN
+
+
+def test_bwd_workspace_is_one_checkpoint_per_chunk(lib):
+    ws = lambda *d: lib.mamba_selective_scan_bwd_workspace_size(_dims(*d))  # noqa: E731
+    # 32-step chunks for dstate > 8, 64-step chunks otherwise; fp32 states
+    assert ws(4, 5120, 16, 4096) == 4 * 5120 * 128 * 16 * 4
+    assert ws(2, 64, 16, 33) == 2 * 64 * 2 * 16 * 4
+    assert ws(2, 64, 8, 64) == 2 * 64 * 1 * 8 * 4
+    assert ws(1, 3, 5, 65) == (1 * 3 * 2 * 5 * 4 + 255) // 256 * 256
+    assert ws(2, 64, 16, 0) == 0
+    assert ws(2, 64, 17, 8) == 0
