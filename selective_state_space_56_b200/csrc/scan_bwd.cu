@@ -1,27 +1,35 @@
 // scan_bwd.cu -- backward of the selective scan (S6) with recomputation, sm_100a.
 //
 // Mamba ("Hardware-aware state expansion"): the intermediate states are not stored for
-// the backward pass; they are recomputed on chip.  Here the forward kernel first records
-// only the state entering every chunk (checkpoints, one N-vector per 32 steps per
-// channel).  This kernel then walks the chunks of a channel tile in reverse:
+// the backward pass; they are recomputed on chip.  The forward kernel first records
+// only the state entering every chunk (checkpoints, one N-vector per chunk of T steps
+// per channel).  This kernel then walks the chunks of a channel tile in reverse:
 //
-//   stage     u, delta, z, dy rows and the batch's B, C for the chunk -> shared memory;
-//   phase A   per (channel, t): Delta, softplus'(x), Delta*u, silu(z), silu'(z);
-//   forward   the chunk's states h_t recomputed from the checkpoint into shared memory
-//             (4 states per lane, 4 lanes per channel), and the pre-gate output
-//             yt_t = C.h + D u (lane transpose-reduce) for dz;
-//   reverse   the adjoint state g (registers) swept from the chunk's last step to its
-//             first: g += dyt C;  dC += dyt h;  dB += g Delta u;  dq = g.B;
-//             dDelta = dq u + sum g h_{t-1} Abar A;  dA += g h_{t-1} Abar Delta;
-//             g *= Abar.  dq and the state part of dDelta are summed over a channel's
-//             lanes every four steps (transpose-reduce); dB and dC, shared by all
-//             channels of a batch, are summed over the warp's channels per step
-//             (8-lane transpose-reduce), over the CTA in shared memory, and added to
-//             global memory with one atomic per (t, n) and CTA;
-//   store     du, dDelta_raw (= dDelta * softplus'(x)), dz; dA, dD, dbias by atomics.
+//   stage     u, delta, z, dy rows and the batch's B, C for the chunk -> shared memory
+//             (16-byte cp.async copies into rows padded against bank conflicts);
+//   phase A   per (channel, t): Delta = softplus(delta + bias);
+//   forward   from the checkpoint, the chunk's states are recomputed; the state
+//             entering every group of 4 steps is kept in shared memory, and the
+//             pre-gate output yt_t = C_t . h_t + D u_t (4-lane transpose-reduce) gives
+//             dz_t = dy_t yt_t silu'(z_t) and the gated gradient dyt_t = dy_t silu(z_t);
+//   reverse   per group of 4 steps, last group first: the group's states and Abar are
+//             recomputed into registers from the group's entry state; then the adjoint
+//             state g (registers) is swept from the group's last step to its first:
+//               g += dyt C;  dC += dyt h;  dB += g Delta u;  dq = g . B;
+//               dDelta = dq u + sum_n g h_{t-1} Abar A;  dA += g h_{t-1} Abar Delta;
+//               g *= Abar.
+//             dq and the state part of dDelta are summed over a channel's 4 lanes once
+//             per group.  dB and dC, shared by all channels of a batch, go through a
+//             per-warp exchange buffer: every channel stores its 32 values of a step,
+//             and after each pair of steps the warp's lanes sum them over the warp's 8
+//             channels (16-byte loads), add the sums into the CTA's chunk accumulator
+//             (shared atomics), which is added to global memory once per (t, n) and CTA;
+//   store     du, dDelta_raw (= dDelta softplus'(x)), dz rows; dA, dD, dbias by atomics.
 //
-// Gradients flowing through softplus use softplus'(x) = sigmoid(x); through the gate
-// silu'(z) = sigmoid(z) (1 + z (1 - sigmoid(z))).
+// State arithmetic runs on packed fp32 pairs (two states per instruction).  Gradients
+// through softplus use softplus'(x) = sigmoid(x); through the gate
+// silu'(z) = sigmoid(z) (1 + z (1 - sigmoid(z))).  Per state and step the kernel
+// evaluates Abar twice (forward and group recompute), the checkpoint pass once.
 #include <cstring>
 
 #include "s6_device.cuh"
@@ -53,54 +61,49 @@ struct BParams {
     int N;
     int softplus;
     int chunks;
+    int vec;  // rows start on 16-byte boundaries: stage them with 16-byte copies
 };
 
-constexpr int kBW = 2;           // warps per CTA
-constexpr int kBP = 4;           // lanes per channel
-constexpr int kBG = 32 / kBP;    // channels per warp
-constexpr int kBCH = kBW * kBG;  // channels per CTA
+#ifndef S6_BWD_WARPS
+#define S6_BWD_WARPS 4
+#endif
+constexpr int kBW = S6_BWD_WARPS;  // warps per CTA
+constexpr int kBP = 4;             // lanes per channel, 4 states each
+constexpr int kBG = 32 / kBP;      // channels per warp
+constexpr int kBCH = kBW * kBG;    // channels per CTA
 
 constexpr size_t a16(size_t x) { return (x + 15) / 16 * 16; }
 
 template <int T, typename Tin>
 struct BLayout {
-    static constexpr int RS = T + 4;
-    static constexpr size_t raw = a16((size_t)kBCH * T * sizeof(Tin));  // one [CH][T] row set
-    static constexpr size_t off_u = 0;
-    static constexpr size_t off_dr = off_u + raw;
-    static constexpr size_t off_z = off_dr + raw;
-    static constexpr size_t off_dy = off_z + raw;
-    static constexpr size_t off_B = off_dy + raw;                 // fp32 [T][16]
+    static constexpr int RR = T + 16 / (int)sizeof(Tin);  // raw row stride: 16 B of padding
+    static constexpr int RS = T + 4;                      // fp32 row stride
+    static constexpr size_t rows = (size_t)kBCH * RR * sizeof(Tin);  // one [CH][RR] set
+    static constexpr size_t coef = (size_t)16 * RR * sizeof(Tin);    // one [16][RR] set
+    // raw (input-dtype) staging: u, delta, z, dy rows, then B, C.  After use the delta,
+    // z and dy rows hold the ddelta, dz and du outputs of the chunk.
+    static constexpr size_t off_stage = 0;
+    static constexpr size_t stage = 4 * rows + 2 * coef;
+    static constexpr size_t off_B = a16(off_stage + stage);      // fp32 [T][16]
     static constexpr size_t off_C = off_B + (size_t)T * 16 * 4;
     static constexpr size_t f = (size_t)kBCH * RS * 4;           // one fp32 [CH][RS]
     static constexpr size_t off_del = off_C + (size_t)T * 16 * 4;
-    static constexpr size_t off_q = off_del + f;
-    static constexpr size_t off_sg = off_q + f;                  // softplus'(x)
-    static constexpr size_t off_gz = off_sg + f;                 // silu(z), then dy*silu(z)
-    static constexpr size_t off_ds = off_gz + f;                 // silu'(z)
-    static constexpr size_t off_yt = off_ds + f;                 // pre-gate output
-    static constexpr size_t off_odu = off_yt + f;                // Tin [CH][T] outputs
-    static constexpr size_t off_odd = off_odu + raw;
-    static constexpr size_t off_odz = off_odd + raw;
-    static constexpr size_t off_h = a16(off_odz + raw);          // fp32 [T][CH][16]
-    static constexpr size_t off_acc = off_h + (size_t)T * kBCH * 16 * 4;  // fp32 [T][32]
-    static constexpr size_t bytes = off_acc + (size_t)T * 32 * 4;
+    static constexpr size_t off_dyt = off_del + f;               // dy * silu(z)
+    static constexpr size_t off_h = off_dyt + f;                 // fp32 [T/4][CH][16]
+    static constexpr size_t off_acc = off_h + (size_t)(T / 4) * kBCH * 16 * 4;  // fp32 [T][32]
+    static constexpr size_t off_red = off_acc + (size_t)T * 32 * 4;  // per warp fp32 [2][8][32]
+    static constexpr size_t bytes = off_red + (size_t)kBW * 2 * 8 * 32 * 4;
+    static_assert(T % 8 == 0, "chunk length");
+    static_assert((RR * sizeof(Tin)) % 16 == 0, "raw rows must stay 16-byte aligned");
 };
 
-__device__ __forceinline__ float sigmoidf_fast(float x) { return rcp(1.f + ex2(-x * kLog2e)); }
-
-// Sum of v[0..7] over the 8 lanes that share lane % 4 (lane bits 2..4): afterwards the
-// lane with channel index cl = lane / 4 holds the total of entry cl.
-__device__ __forceinline__ float transpose_reduce8(const float (&v)[8], int lane) {
-    const bool b1 = lane & 16, b2 = lane & 8, b3 = lane & 4;
-    float w[4], x[2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        w[i] = (b1 ? v[i + 4] : v[i]) + __shfl_xor_sync(0xffffffffu, b1 ? v[i] : v[i + 4], 16);
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-        x[i] = (b2 ? w[i + 2] : w[i]) + __shfl_xor_sync(0xffffffffu, b2 ? w[i] : w[i + 2], 8);
-    return (b3 ? x[1] : x[0]) + __shfl_xor_sync(0xffffffffu, b3 ? x[0] : x[1], 4);
+// softplus(x) and sigmoid(x) from one exponential e = e^-|x|:
+// softplus = max(x, 0) + log1p(e), sigmoid = 1 / (1 + e) for x >= 0, e / (1 + e) otherwise.
+__device__ __forceinline__ void softplus_sigmoid(float x, float& sp, float& sg) {
+    const float e = ex2(-fabsf(x) * kLog2e);
+    sp = fmaxf(x, 0.f) + e * log1p_over_x(e);
+    const float r = rcp(1.f + e);
+    sg = x >= 0.f ? r : e * r;
 }
 
 // Four partial sums (entries 0..3) over the 4 lanes of a channel: lane pp gets entry pp.
@@ -112,180 +115,297 @@ __device__ __forceinline__ float transpose_reduce4(const float (&v)[4], int pp) 
     return (hi1 ? w1 : w0) + __shfl_xor_sync(0xffffffffu, hi1 ? w0 : w1, 1);
 }
 
+__device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ f2 lo2(const float4& v) { return pack2(v.x, v.y); }
+__device__ __forceinline__ f2 hi2(const float4& v) { return pack2(v.z, v.w); }
+__device__ __forceinline__ float hsum(f2 v) {
+    float a, b;
+    unpack2(v, a, b);
+    return a + b;
+}
+
+// dB / dC exchange rows: channel ch of a warp stores its 32 values (8 quads: dB states
+// 0-15, then dC states 0-15) with the quad index XOR-ed by 4 for half of the channels,
+// so that both the per-channel 16-byte stores and the per-quad 16-byte loads of the
+// reduction hit distinct banks.
+__device__ __forceinline__ int red_quad(int q, int ch) { return q ^ (((ch ^ (ch >> 2)) & 1) << 2); }
+// Accumulator slot of (t, slot): rotated by t mod 4 so that the reduction's atomic adds,
+// 4 steps x 8 quads at a time, fall in distinct banks.
+__device__ __forceinline__ int acc_idx(int t, int slot) { return t * 32 + ((slot + (t & 3)) & 31); }
+
+// Stage chunk k's rows into the raw buffer.  Rows past dim, steps past L and a missing z
+// become zeros.  16-byte cp.async copies when rows are 16-byte aligned (then every
+// 16-byte piece is either wholly inside the sequence or wholly past it); plain loads
+// otherwise.
+template <int T, typename Tin>
+__device__ __forceinline__ void stage_chunk(const BParams& p, unsigned char* st, int64_t b,
+                                            int64_t d0, int k, int tid) {
+    using Lo = BLayout<T, Tin>;
+    constexpr int RR = Lo::RR;
+    const int64_t t0 = (int64_t)k * T;
+    const int valid = (int)min((int64_t)T, p.L - t0);
+    if (p.vec) {
+        constexpr int E = 16 / sizeof(Tin);  // elements per copy
+        constexpr int VPR = T / E;           // copies per row
+        constexpr int NROW = 4 * kBCH + 32;  // 4 row sets, then 16 rows each of B and C
+        for (int i = tid; i < NROW * VPR; i += kBW * 32) {
+            const int row = i / VPR, col = (i % VPR) * E;
+            const Tin* src;
+            Tin* dst;
+            bool ok;
+            if (row < 4 * kBCH) {
+                const int which = row / kBCH, r = row % kBCH;
+                src = static_cast<const Tin*>(which == 0 ? p.u : which == 1 ? p.delta
+                                              : which == 2 ? p.z : p.dy);
+                ok = src != nullptr && d0 + r < p.dim && col < valid;
+                if (ok) src += (b * p.dim + d0 + r) * p.L + t0 + col;
+                dst = reinterpret_cast<Tin*>(st + which * Lo::rows) + r * RR + col;
+            } else {
+                const int which = (row - 4 * kBCH) / 16, n = (row - 4 * kBCH) % 16;
+                src = static_cast<const Tin*>(which ? p.C : p.B);
+                ok = n < p.N && col < valid;
+                if (ok) src += (b * p.N + n) * p.L + t0 + col;
+                dst = reinterpret_cast<Tin*>(st + 4 * Lo::rows + which * Lo::coef) + n * RR + col;
+            }
+            cp_async16(dst, ok ? static_cast<const void*>(src) : p.A, ok ? 16 : 0);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+    } else {
+        for (int i = tid; i < 4 * kBCH * T; i += kBW * 32) {
+            const int which = i / (kBCH * T), r = (i / T) % kBCH, t = i % T;
+            const Tin* src = static_cast<const Tin*>(which == 0 ? p.u : which == 1 ? p.delta
+                                                     : which == 2 ? p.z : p.dy);
+            Tin v = Tin(0.f);
+            if (src && d0 + r < p.dim && t < valid) v = src[(b * p.dim + d0 + r) * p.L + t0 + t];
+            reinterpret_cast<Tin*>(st + which * Lo::rows)[r * RR + t] = v;
+        }
+        for (int i = tid; i < 32 * T; i += kBW * 32) {
+            const int which = i / (16 * T), n = (i / T) % 16, t = i % T;
+            const Tin* src = static_cast<const Tin*>(which ? p.C : p.B);
+            Tin v = Tin(0.f);
+            if (n < p.N && t < valid) v = src[(b * p.N + n) * p.L + t0 + t];
+            reinterpret_cast<Tin*>(st + 4 * Lo::rows + which * Lo::coef)[n * RR + t] = v;
+        }
+    }
+}
+
 template <int T, typename Tin>
 __global__ void __launch_bounds__(kBW * 32) scan_bwd_kernel(const BParams p) {
     using Lo = BLayout<T, Tin>;
-    constexpr int RS = Lo::RS;
+    constexpr int RS = Lo::RS, RR = Lo::RR;
+    using V4 = vec4<Tin>;
+    using VT = typename V4::type;
     extern __shared__ __align__(16) unsigned char smem[];
-    Tin* rU = reinterpret_cast<Tin*>(smem + Lo::off_u);
-    Tin* rDr = reinterpret_cast<Tin*>(smem + Lo::off_dr);
-    Tin* rZ = reinterpret_cast<Tin*>(smem + Lo::off_z);
-    Tin* rDy = reinterpret_cast<Tin*>(smem + Lo::off_dy);
+    unsigned char* st = smem + Lo::off_stage;
+    Tin* rU = reinterpret_cast<Tin*>(st);
+    Tin* rDr = reinterpret_cast<Tin*>(st + Lo::rows);      // later: ddelta
+    Tin* rZ = reinterpret_cast<Tin*>(st + 2 * Lo::rows);   // later: dz
+    Tin* rDy = reinterpret_cast<Tin*>(st + 3 * Lo::rows);  // later: du
+    const Tin* rB = reinterpret_cast<const Tin*>(st + 4 * Lo::rows);
+    const Tin* rC = reinterpret_cast<const Tin*>(st + 4 * Lo::rows + Lo::coef);
     float* sB = reinterpret_cast<float*>(smem + Lo::off_B);
     float* sC = reinterpret_cast<float*>(smem + Lo::off_C);
     float* sDel = reinterpret_cast<float*>(smem + Lo::off_del);
-    float* sQ = reinterpret_cast<float*>(smem + Lo::off_q);
-    float* sSg = reinterpret_cast<float*>(smem + Lo::off_sg);
-    float* sGz = reinterpret_cast<float*>(smem + Lo::off_gz);
-    float* sDs = reinterpret_cast<float*>(smem + Lo::off_ds);
-    float* sYt = reinterpret_cast<float*>(smem + Lo::off_yt);
-    Tin* oDu = reinterpret_cast<Tin*>(smem + Lo::off_odu);
-    Tin* oDd = reinterpret_cast<Tin*>(smem + Lo::off_odd);
-    Tin* oDz = reinterpret_cast<Tin*>(smem + Lo::off_odz);
+    float* sDyt = reinterpret_cast<float*>(smem + Lo::off_dyt);
     float* sH = reinterpret_cast<float*>(smem + Lo::off_h);
     float* sAcc = reinterpret_cast<float*>(smem + Lo::off_acc);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int pp = lane & 3, cl = lane >> 2;
     const int cw = warp * kBG + cl;
+    float* sRed = reinterpret_cast<float*>(smem + Lo::off_red) + warp * (2 * 8 * 32);
     const int64_t b = blockIdx.y, d0 = (int64_t)blockIdx.x * kBCH, dch = d0 + cw;
     const bool chok = dch < p.dim;
     const bool has_z = p.z != nullptr;
 
-    float a2[4], an[4], g[4], dAacc[4];
+    float a2[4], an[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int n = pp * 4 + j;
         an[j] = (chok && n < p.N) ? p.A[dch * p.N + n] : 0.f;  // padded states stay zero
         a2[j] = an[j] * kLog2e;
-        g[j] = 0.f;
-        dAacc[j] = 0.f;
     }
+    const f2 a2p[2] = {pack2(a2[0], a2[1]), pack2(a2[2], a2[3])};
+    const f2 anp[2] = {pack2(an[0], an[1]), pack2(an[2], an[3])};
+    const f2 zero2 = pack2(0.f, 0.f);
+    f2 gp[2] = {zero2, zero2}, dAp[2] = {zero2, zero2};
     const float Dd = (chok && p.D) ? p.D[dch] : 0.f;
+    const float bias = (chok && p.delta_bias) ? p.delta_bias[dch] : 0.f;
     float dDacc = 0.f, dbacc = 0.f;
+    // reduction lane roles: step ss of a step pair, quad q of the 32 slots, channel half
+    const int rss = lane >> 4, rq = (lane >> 1) & 7, rhalf = lane & 1;
 
     for (int k = p.chunks - 1; k >= 0; --k) {
         const int64_t t0 = (int64_t)k * T;
         const int valid = (int)min((int64_t)T, p.L - t0);
-        __syncthreads();  // the previous (later) chunk is done with shared memory
+        __syncthreads();  // the previous chunk's outputs have left the staging rows
+        stage_chunk<T, Tin>(p, st, b, d0, k, tid);
+        __syncthreads();  // chunk k staged
 
-        // stage: rows past dim and steps past L are zero
-        for (int i = tid; i < 4 * kBCH * T; i += kBW * 32) {
-            const int which = i / (kBCH * T), r = (i / T) % kBCH, t = i % T;
-            const int64_t d = d0 + r;
-            const Tin* src = static_cast<const Tin*>(which == 0 ? p.u : which == 1 ? p.delta
-                                                     : which == 2 ? p.z : p.dy);
-            Tin* dst = which == 0 ? rU : which == 1 ? rDr : which == 2 ? rZ : rDy;
-            Tin v = Tin(0.f);
-            if (d < p.dim && t < valid && src) v = src[(b * p.dim + d) * p.L + t0 + t];
-            dst[r * T + t] = v;
-        }
-        for (int i = tid; i < 2 * 16 * T; i += kBW * 32) {
-            const int which = i / (16 * T), n = (i / T) % 16, t = i % T;
-            const Tin* src = static_cast<const Tin*>(which ? p.C : p.B);
-            float v = 0.f;
-            if (n < p.N && t < valid) v = io<Tin>::to_f(src[(b * p.N + n) * p.L + t0 + t]);
-            (which ? sC : sB)[t * 16 + n] = v;
+        // B and C to fp32 [t][n]: a warp converts two steps of all 16 states per pass
+        for (int i = tid; i < 16 * T; i += kBW * 32) {
+            const int n = i & 15, t = i >> 4;
+            sB[t * 16 + n] = io<Tin>::to_f(rB[n * RR + t]);
+            sC[t * 16 + n] = io<Tin>::to_f(rC[n * RR + t]);
         }
         for (int i = tid; i < T * 32; i += kBW * 32) sAcc[i] = 0.f;
-        __syncthreads();
 
-        // phase A: per (channel, t) of this warp
+        // phase A: Delta for this warp's channels (zero on padded steps: Abar = 1, no input)
         for (int i = lane; i < kBG * T; i += 32) {
             const int c = warp * kBG + i / T, t = i % T;
             const int64_t d = d0 + c;
-            const float bias = (d < p.dim && p.delta_bias) ? p.delta_bias[d] : 0.f;
-            const float x = io<Tin>::to_f(rDr[c * T + t]) + bias;
-            float dt = p.softplus ? softplus(x) : x;
-            dt = t < valid ? dt : 0.f;
-            const float zz = io<Tin>::to_f(rZ[c * T + t]);
-            const float sz = sigmoidf_fast(zz);
-            sDel[c * RS + t] = dt;
-            sQ[c * RS + t] = dt * io<Tin>::to_f(rU[c * T + t]);
-            sSg[c * RS + t] = p.softplus ? sigmoidf_fast(x) : 1.f;
-            sGz[c * RS + t] = has_z ? zz * sz : 1.f;
-            sDs[c * RS + t] = has_z ? sz * (1.f + zz * (1.f - sz)) : 0.f;
+            const float bi = (d < p.dim && p.delta_bias) ? p.delta_bias[d] : 0.f;
+            const float x = io<Tin>::to_f(rDr[c * RR + t]) + bi;
+            const float dt = p.softplus ? softplus(x) : x;
+            sDel[c * RS + t] = t < valid ? dt : 0.f;
         }
-        __syncwarp();
+        __syncthreads();  // B, C converted, sAcc cleared
 
-        // forward: the chunk's states from its checkpoint
-        float hck[4], h[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int n = pp * 4 + j;
-            hck[j] = (chok && n < p.N) ? p.ckpt[((b * p.dim + dch) * p.chunks + k) * p.N + n] : 0.f;
-            h[j] = hck[j];
-        }
-        for (int t = 0; t < T; t += 4) {
-            float yp[4];
-#pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const float dt = sDel[cw * RS + t + s], q = sQ[cw * RS + t + s];
-                const float4 bb = *reinterpret_cast<const float4*>(sB + (t + s) * 16 + pp * 4);
-                const float4 cc = *reinterpret_cast<const float4*>(sC + (t + s) * 16 + pp * 4);
-                const float bv[4] = {bb.x, bb.y, bb.z, bb.w}, cv[4] = {cc.x, cc.y, cc.z, cc.w};
-                float acc = 0.f;
+        // forward: group entry states, dz and dy * silu(z)
+        {
+            f2 hp[2];
+            {
+                float h[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    h[j] = fmaf(ex2(dt * a2[j]), h[j], q * bv[j]);
-                    acc = fmaf(cv[j], h[j], acc);
+                    const int n = pp * 4 + j;
+                    h[j] = (chok && n < p.N)
+                               ? p.ckpt[((b * p.dim + dch) * p.chunks + k) * p.N + n] : 0.f;
                 }
-                *reinterpret_cast<float4*>(sH + ((t + s) * kBCH + cw) * 16 + pp * 4) =
-                    make_float4(h[0], h[1], h[2], h[3]);
-                yp[s] = acc;
+                hp[0] = pack2(h[0], h[1]);
+                hp[1] = pack2(h[2], h[3]);
             }
-            sYt[cw * RS + t + pp] = transpose_reduce4(yp, pp) +
-                                    Dd * io<Tin>::to_f(rU[cw * T + t + pp]);
+            for (int t = 0; t < T; t += 4) {
+                {
+                    float h0, h1, h2, h3;
+                    unpack2(hp[0], h0, h1);
+                    unpack2(hp[1], h2, h3);
+                    *reinterpret_cast<float4*>(sH + ((t / 4) * kBCH + cw) * 16 + pp * 4) =
+                        make_float4(h0, h1, h2, h3);
+                }
+                const float4 d4 = lds4(sDel + cw * RS + t);
+                float uv[4];
+                V4::to_f(*reinterpret_cast<const VT*>(rU + cw * RR + t), uv);
+                const float dts[4] = {d4.x, d4.y, d4.z, d4.w};
+                float yp[4];
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const f2 dd = pack2(dts[s], dts[s]);
+                    const float q = dts[s] * uv[s];
+                    const f2 qq = pack2(q, q);
+                    const float4 bb = lds4(sB + (t + s) * 16 + pp * 4);
+                    const float4 cc = lds4(sC + (t + s) * 16 + pp * 4);
+                    const f2 e0 = ex2x2(mul2(dd, a2p[0])), e1 = ex2x2(mul2(dd, a2p[1]));
+                    hp[0] = fma2(e0, hp[0], mul2(qq, lo2(bb)));
+                    hp[1] = fma2(e1, hp[1], mul2(qq, hi2(bb)));
+                    yp[s] = hsum(fma2(lo2(cc), hp[0], mul2(hi2(cc), hp[1])));
+                }
+                // lane pp finishes step t + pp of its channel
+                const int ts = t + pp;
+                const float yt = transpose_reduce4(yp, pp) + Dd * io<Tin>::to_f(rU[cw * RR + ts]);
+                const float dyv = io<Tin>::to_f(rDy[cw * RR + ts]);
+                float dyt = dyv, dzv = 0.f;
+                if (has_z) {
+                    const float zz = io<Tin>::to_f(rZ[cw * RR + ts]);
+                    const float sz = rcp(1.f + ex2(-zz * kLog2e));
+                    dyt = dyv * zz * sz;
+                    dzv = dyv * yt * sz * (1.f + zz * (1.f - sz));
+                }
+                sDyt[cw * RS + ts] = dyt;
+                rZ[cw * RR + ts] = io<Tin>::from_f(dzv);  // dz replaces z
+            }
         }
         __syncwarp();
 
-        // dz and dy * silu(z) per (channel, t)
-        for (int i = lane; i < kBG * T; i += 32) {
-            const int c = warp * kBG + i / T, t = i % T;
-            const float dyv = io<Tin>::to_f(rDy[c * T + t]);
-            oDz[c * T + t] = io<Tin>::from_f(dyv * sYt[c * RS + t] * sDs[c * RS + t]);
-            sGz[c * RS + t] = dyv * sGz[c * RS + t];
-        }
-        __syncwarp();
-
-        // reverse sweep, four steps per group (last group first)
+        // reverse sweep, one group of four steps at a time (last group first)
         for (int tg = T - 4; tg >= 0; tg -= 4) {
+            const float4 d4 = lds4(sDel + cw * RS + tg), y4 = lds4(sDyt + cw * RS + tg);
+            float uv[4];
+            V4::to_f(*reinterpret_cast<const VT*>(rU + cw * RR + tg), uv);
+            const float dts[4] = {d4.x, d4.y, d4.z, d4.w}, dyts[4] = {y4.x, y4.y, y4.z, y4.w};
+            const float4 h4 = lds4(sH + ((tg / 4) * kBCH + cw) * 16 + pp * 4);
+            const f2 hin[2] = {lo2(h4), hi2(h4)};
+            // the group's Abar and states, recomputed into registers
+            f2 ab[4][2], hs[4][2];
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                const f2 dd = pack2(dts[s], dts[s]);
+                const float q = dts[s] * uv[s];
+                const f2 qq = pack2(q, q);
+                const float4 bb = lds4(sB + (tg + s) * 16 + pp * 4);
+                ab[s][0] = ex2x2(mul2(dd, a2p[0]));
+                ab[s][1] = ex2x2(mul2(dd, a2p[1]));
+                hs[s][0] = fma2(ab[s][0], s ? hs[s - 1][0] : hin[0], mul2(qq, lo2(bb)));
+                hs[s][1] = fma2(ab[s][1], s ? hs[s - 1][1] : hin[1], mul2(qq, hi2(bb)));
+            }
             float dqv[4], ddv[4];
 #pragma unroll
             for (int s = 3; s >= 0; --s) {
                 const int t = tg + s;
-                const float dyt = sGz[cw * RS + t], dt = sDel[cw * RS + t], q = sQ[cw * RS + t];
-                const float4 bb = *reinterpret_cast<const float4*>(sB + t * 16 + pp * 4);
-                const float4 cc = *reinterpret_cast<const float4*>(sC + t * 16 + pp * 4);
-                const float4 hc = *reinterpret_cast<const float4*>(sH + (t * kBCH + cw) * 16 + pp * 4);
-                float hpv[4];
-                if (t > 0) {
-                    const float4 hpr =
-                        *reinterpret_cast<const float4*>(sH + ((t - 1) * kBCH + cw) * 16 + pp * 4);
-                    hpv[0] = hpr.x, hpv[1] = hpr.y, hpv[2] = hpr.z, hpv[3] = hpr.w;
-                } else {
-                    hpv[0] = hck[0], hpv[1] = hck[1], hpv[2] = hck[2], hpv[3] = hck[3];
+                const float4 bb = lds4(sB + t * 16 + pp * 4);
+                const float4 cc = lds4(sC + t * 16 + pp * 4);
+                const f2 yy = pack2(dyts[s], dyts[s]), dd = pack2(dts[s], dts[s]);
+                const float q = dts[s] * uv[s];
+                const f2 qq = pack2(q, q);
+                gp[0] = fma2(yy, lo2(cc), gp[0]);
+                gp[1] = fma2(yy, hi2(cc), gp[1]);
+                const f2 dC0 = mul2(yy, hs[s][0]), dC1 = mul2(yy, hs[s][1]);
+                const f2 dB0 = mul2(gp[0], qq), dB1 = mul2(gp[1], qq);
+                dqv[s] = hsum(fma2(gp[0], lo2(bb), mul2(gp[1], hi2(bb))));
+                const f2 gh0 = mul2(mul2(gp[0], s ? hs[s - 1][0] : hin[0]), ab[s][0]);
+                const f2 gh1 = mul2(mul2(gp[1], s ? hs[s - 1][1] : hin[1]), ab[s][1]);
+                ddv[s] = hsum(fma2(gh0, anp[0], mul2(gh1, anp[1])));
+                dAp[0] = fma2(gh0, dd, dAp[0]);
+                dAp[1] = fma2(gh1, dd, dAp[1]);
+                gp[0] = mul2(gp[0], ab[s][0]);
+                gp[1] = mul2(gp[1], ab[s][1]);
+                // this channel's dB / dC of step t into the warp's exchange rows
+                {
+                    float* row = sRed + (s & 1) * 256 + cl * 32;
+                    float x0, x1, x2, x3;
+                    unpack2(dB0, x0, x1);
+                    unpack2(dB1, x2, x3);
+                    *reinterpret_cast<float4*>(row + red_quad(pp, cl) * 4) = make_float4(x0, x1, x2, x3);
+                    unpack2(dC0, x0, x1);
+                    unpack2(dC1, x2, x3);
+                    *reinterpret_cast<float4*>(row + red_quad(4 + pp, cl) * 4) = make_float4(x0, x1, x2, x3);
                 }
-                const float bv[4] = {bb.x, bb.y, bb.z, bb.w}, cv[4] = {cc.x, cc.y, cc.z, cc.w};
-                const float hv[4] = {hc.x, hc.y, hc.z, hc.w};
-                float part[8], dq = 0.f, dd = 0.f;
+                if ((s & 1) == 0) {
+                    // a step pair is complete: sum it over the warp's 8 channels
+                    __syncwarp();
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    g[j] = fmaf(dyt, cv[j], g[j]);
-                    part[4 + j] = dyt * hv[j];  // dC
-                    part[j] = g[j] * q;         // dB
-                    dq = fmaf(g[j], bv[j], dq);
-                    const float abar = ex2(dt * a2[j]);
-                    const float gh = g[j] * hpv[j] * abar;
-                    dd = fmaf(gh, an[j], dd);
-                    dAacc[j] = fmaf(gh, dt, dAacc[j]);
-                    g[j] *= abar;
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const int ch = rhalf * 4 + kk;
+                        const float4 v = lds4(sRed + rss * 256 + ch * 32 + red_quad(rq, ch) * 4);
+                        acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+                    }
+                    // the two channel halves: lane rhalf keeps slots 2 rhalf, 2 rhalf + 1
+                    const float s0 = rhalf ? acc.x : acc.z, s1 = rhalf ? acc.y : acc.w;
+                    const float k0 = rhalf ? acc.z : acc.x, k1 = rhalf ? acc.w : acc.y;
+                    const float v0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 1);
+                    const float v1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 1);
+                    const int tt = tg + s + rss, slot = rq * 4 + rhalf * 2;
+                    atomicAdd(&sAcc[acc_idx(tt, slot)], v0);
+                    atomicAdd(&sAcc[acc_idx(tt, slot + 1)], v1);
+                    __syncwarp();
                 }
-                dqv[s] = dq;
-                ddv[s] = dd;
-                // dB / dC of step t summed over the warp's 8 channels, then over the CTA
-                const float r = transpose_reduce8(part, lane);
-                const int slot = (cl < 4 ? 0 : 16) + pp * 4 + (cl & 3);
-                atomicAdd(&sAcc[t * 32 + slot], r);
             }
             // lane pp completes step tg + pp of its channel
-            const float dq = transpose_reduce4(dqv, pp), dd = transpose_reduce4(ddv, pp);
+            const float dq = transpose_reduce4(dqv, pp), ddl = transpose_reduce4(ddv, pp);
             const int t = tg + pp;
-            const float uu = io<Tin>::to_f(rU[cw * T + t]);
-            const float dyt = sGz[cw * RS + t], dt = sDel[cw * RS + t];
-            const float ddelta = (dd + dq * uu) * sSg[cw * RS + t];
-            oDu[cw * T + t] = io<Tin>::from_f(fmaf(dyt, Dd, dq * dt));
-            oDd[cw * T + t] = io<Tin>::from_f(ddelta);
+            const float uu = io<Tin>::to_f(rU[cw * RR + t]);
+            const float dt = sDel[cw * RS + t], dyt = sDyt[cw * RS + t];
+            const float xr = io<Tin>::to_f(rDr[cw * RR + t]);
+            float sg = 1.f;
+            if (p.softplus) {
+                float sp;
+                softplus_sigmoid(xr + bias, sp, sg);
+            }
+            const float ddelta = (ddl + dq * uu) * sg;
+            rDy[cw * RR + t] = io<Tin>::from_f(fmaf(dyt, Dd, dq * dt));  // du replaces dy
+            rDr[cw * RR + t] = io<Tin>::from_f(ddelta);                  // ddelta replaces delta
             if (t < valid) {
                 dbacc += ddelta;
                 dDacc = fmaf(dyt, uu, dDacc);
@@ -294,27 +414,41 @@ __global__ void __launch_bounds__(kBW * 32) scan_bwd_kernel(const BParams p) {
         __syncthreads();
 
         // store du, ddelta, dz rows and add the CTA's dB / dC of the chunk
-        for (int i = tid; i < kBCH * T; i += kBW * 32) {
-            const int r = i / T, t = i % T;
-            const int64_t d = d0 + r;
-            if (d >= p.dim || t >= valid) continue;
-            const int64_t off = (b * p.dim + d) * p.L + t0 + t;
-            static_cast<Tin*>(p.du)[off] = oDu[r * T + t];
-            static_cast<Tin*>(p.ddelta)[off] = oDd[r * T + t];
-            if (p.dz) static_cast<Tin*>(p.dz)[off] = oDz[r * T + t];
+        if (p.vec) {
+            constexpr int E = 16 / sizeof(Tin), VPR = T / E;
+            for (int i = tid; i < 3 * kBCH * VPR; i += kBW * 32) {
+                const int which = i / (kBCH * VPR), r = (i / VPR) % kBCH, col = (i % VPR) * E;
+                void* dst = which == 0 ? p.du : which == 1 ? p.ddelta : p.dz;
+                if (!dst || d0 + r >= p.dim || col >= valid) continue;
+                const Tin* src = which == 0 ? rDy : which == 1 ? rDr : rZ;
+                *reinterpret_cast<uint4*>(static_cast<Tin*>(dst) + (b * p.dim + d0 + r) * p.L +
+                                          t0 + col) = *reinterpret_cast<const uint4*>(src + r * RR + col);
+            }
+        } else {
+            for (int i = tid; i < kBCH * T; i += kBW * 32) {
+                const int r = i / T, t = i % T;
+                if (d0 + r >= p.dim || t >= valid) continue;
+                const int64_t off = (b * p.dim + d0 + r) * p.L + t0 + t;
+                static_cast<Tin*>(p.du)[off] = rDy[r * RR + t];
+                static_cast<Tin*>(p.ddelta)[off] = rDr[r * RR + t];
+                if (p.dz) static_cast<Tin*>(p.dz)[off] = rZ[r * RR + t];
+            }
         }
         for (int i = tid; i < T * 32; i += kBW * 32) {
             const int t = i / 32, slot = i % 32, n = slot & 15;
             if (t >= valid || n >= p.N) continue;
             float* dst = slot < 16 ? p.dB : p.dC;
-            atomicAdd(dst + (b * p.N + n) * p.L + t0 + t, sAcc[i]);
+            atomicAdd(dst + (b * p.N + n) * p.L + t0 + t, sAcc[acc_idx(t, slot)]);
         }
     }
 
     if (chok) {
+        float dA[4];
+        unpack2(dAp[0], dA[0], dA[1]);
+        unpack2(dAp[1], dA[2], dA[3]);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-            if (pp * 4 + j < p.N) atomicAdd(p.dA + dch * p.N + pp * 4 + j, dAacc[j]);
+            if (pp * 4 + j < p.N) atomicAdd(p.dA + dch * p.N + pp * 4 + j, dA[j]);
     }
     // dD and dbias: sum the 4 lanes of the channel
     dDacc += __shfl_xor_sync(0xffffffffu, dDacc, 1);
@@ -334,13 +468,17 @@ cudaError_t launch_bwd_typed(const BParams& bp, int64_t batch, int64_t dim, cuda
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Lo::bytes);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((dim + kBCH - 1) / kBCH), (unsigned)batch, 1);
     kern<<<grid, kBW * 32, Lo::bytes, s>>>(bp);
     return cudaGetLastError();
 }
 
 template <typename Tin>
-cudaError_t launch_bwd_io(const BParams& bp, int T, int64_t batch, int64_t dim, cudaStream_t s) {
+cudaError_t launch_bwd_io(BParams bp, int T, int64_t batch, int64_t dim, cudaStream_t s) {
+    // 16-byte staging needs every row start (a multiple of L elements) 16-byte aligned
+    bp.vec = (bp.L * (int64_t)sizeof(Tin)) % 16 == 0 ? 1 : 0;
     if (T == 32) return launch_bwd_typed<32, Tin>(bp, batch, dim, s);
     if (T == 64) return launch_bwd_typed<64, Tin>(bp, batch, dim, s);
     return cudaErrorInvalidConfiguration;
