@@ -12,8 +12,9 @@ ranks (one process per GPU under torchrun) every rank scans its own independent
 batch (weak scaling, no data-path collective) and the max time over ranks is
 used.  The same run measures the decode workload (selective_state_update,
 batch 256, dim 5120, N 16, 1000 fresh tokens, L2 flushed before each token),
-the end-to-end path from pinned host buffers, the SM clocks during the timed
-region, and (rank 0, N = 1) the fp64 CPU oracle on a bounded sample.
+the backward of the same layer's scan (recomputing states from chunk
+checkpoints), the end-to-end path from pinned host buffers, the SM clocks during
+the timed region, and (rank 0, N = 1) the fp64 CPU oracle on bounded samples.
 
 ``--impl reference`` times the CPU oracle itself as the reference arm.
 Rank 0 prints exactly one JSON line.
@@ -196,6 +197,14 @@ def decode_bytes(b, d, n, io_size=2):
     return 2 * b * d * n * 4 + 4 * b * d * io_size + 2 * b * n * io_size + d * n * 4 + 2 * d * 4
 
 
+def backward_bytes(b, d, n, L, in_size=2):
+    """Algorithmic bytes of one scan backward: u, delta, z, dy, B, C read once; du, ddelta,
+    dz (input dtype) and dB, dC (fp32) written once; A, D, bias and their fp32 gradients.
+    Checkpoint traffic is a design choice and is not counted."""
+    return (4 * b * d * L * in_size + 2 * b * n * L * in_size + 3 * b * d * L * in_size +
+            2 * b * n * L * 4 + 2 * d * n * 4 + 4 * d * 4)
+
+
 def flush_l2(buf):
     buf.add_(1)  # reads and writes 2x L2 worth of bytes
 
@@ -294,12 +303,16 @@ def run_ours(args, rank, world, local):
            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     decode = run_decode(dev, stream, world, steps=args.decode_steps)
-    del g, y, last
+    del y, last
+    torch.cuda.empty_cache()
+    backward = run_backward(g, dev, stream, world, w, steps=args.backward_steps)
+    del g
     torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, budget_s=args.cpu_seconds)
+        backward["cpu_baseline"] = cpu_baseline_backward(w, budget_s=args.cpu_seconds / 2)
 
     line = {
         "metric": METRIC, "value": value, "unit": "elems/s", "n_gpus": world,
@@ -313,9 +326,62 @@ def run_ours(args, rank, world, local):
                        (h2d) / 1e6, L2_BYTES >> 20),
                    "parallelism": "replicas x%d (independent batches per GPU)" % world},
         "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
-        "clocks": clocks, "decode": decode, "cpu_baseline": cpu, "impl": "ours",
+        "clocks": clocks, "decode": decode, "backward": backward, "cpu_baseline": cpu,
+        "impl": "ours",
     }
     return line
+
+
+def run_backward(g, dev, stream, world, w, steps=50):
+    """Backward of the m2p8b scan (gradients of every input for a fixed dy), each call
+    timed with events on the launching stream; inputs exceed L2, so no flush."""
+    from selective_state_space_56_b200 import ops
+    b, d, n, L = w.batch, w.dim, w.dstate, w.seqlen
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed + 7)
+    dy = torch.randn((b, d, L), generator=gen, device=dev).to(w.in_dtype)
+    ws = torch.empty(ops.selective_scan_bwd_workspace_size(b, d, n, L), dtype=torch.uint8,
+                     device=dev)
+
+    def call():
+        return ops.selective_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dy, D=g["D"],
+                                      z=g["z"], delta_bias=g["delta_bias"], workspace=ws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b_ in evs:
+        a.record(stream)
+        call()
+        b_.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(statistics.fmean(a.elapsed_time(b_) for a, b_ in evs), world)
+    elems = b * d * L
+    peaks, kind = measured_peaks()
+    fmax_mhz = peaks.get("sm_max_mhz", 1965.0)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    sfu_peak = sms * SFU_OPS_PER_CLK_PER_SM * fmax_mhz * 1e6
+    # SFU results the recomputing backward needs per element: Abar twice (states rebuilt,
+    # then swept), softplus, sigmoid of the step (softplus'), sigmoid of the gate (ex2, rcp)
+    sfu = elems * (2 * n + 4)
+    byts = backward_bytes(b, d, n, L)
+    del dy, ws
+    return {
+        "metric": "selective-scan bwd (b·d·L) elems/s", "unit": "elems/s",
+        "value": world * elems / (ms * 1e-3), "ms_per_call": ms, "steps": steps,
+        "workload": "backward of the m2p8b scan: batch 4, dim 5120, N 16, L 4096, bf16 "
+                    "inputs and du/ddelta/dz, fp32 dA/dB/dC/dD/dbias",
+        "roofline": {"bound": "alu", "unit": "Gop/s (SFU)", "achieved": sfu / (ms * 1e-3) / 1e9,
+                     "peak": sfu_peak / 1e9, "frac": sfu / (ms * 1e-3) / sfu_peak,
+                     "sfu_ops_per_elem": 2 * n + 4,
+                     "algorithmic_bytes": byts, "hbm_GBps": byts / (ms * 1e-3) / 1e9,
+                     "hbm_frac": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "peak_kind": kind,
+                     "traffic": profile_traffic("scan_bwd_m2p8b.txt",
+                                                "selective_state_space_56_b200/csrc/scan_bwd.cu")},
+        "gpu_launches": 2 * steps + 6,
+    }
 
 
 def run_decode(dev, stream, world, steps=1000):
@@ -403,6 +469,35 @@ def cpu_baseline(w, budget_s=10.0):
                       "threads), %.1f s" % (nl, w.batch * w.dim, w.seqlen, cores, t)}
 
 
+def cpu_baseline_backward(w, budget_s=5.0):
+    """The fp64 oracle's backward as it stands, on a bounded channel sample."""
+    import numpy as np
+    import oracle
+    from selective_state_space_56_b200 import inputs
+
+    p = inputs.workload_inputs(w)
+    rng = np.random.default_rng(1)
+    dy_all = None
+
+    def run(nl):
+        nonlocal dy_all
+        bi = rng.integers(0, w.batch, nl)
+        di = rng.integers(0, w.dim, nl)
+        dy = rng.standard_normal((nl, w.seqlen))
+        t = time.perf_counter()
+        oracle.scan_backward_lanes(p["u"][bi, di], p["delta"][bi, di], p["A"][di], p["B"], p["C"],
+                                   bi, dy, D=p["D"][di], z=p["z"][bi, di],
+                                   delta_bias=p["delta_bias"][di])
+        return time.perf_counter() - t
+
+    t = run(8)
+    nl = int(min(w.batch * w.dim, max(8, 8 * budget_s / max(t, 1e-3))))
+    t = run(nl)
+    return {"value": nl * w.seqlen / t, "unit": "elems/s", "cores": 1, "kind": "oracle",
+            "sample": "%d of %d channels x full L=%d (fp64 backward, one thread), %.1f s" % (
+                nl, w.batch * w.dim, w.seqlen, t)}
+
+
 def run_reference(args, rank, world):
     from selective_state_space_56_b200 import inputs
     w = inputs.SCAN_WORKLOADS[WORKLOAD]
@@ -429,7 +524,8 @@ def run_reference(args, rank, world):
 
 
 def profile_target(which):
-    """Three launches of the scan (m2p8b) or eight decode tokens, for ncu captures."""
+    """Three launches of the scan (m2p8b), eight decode tokens, or two backward calls of
+    the m2p8b scan, for ncu captures."""
     from selective_state_space_56_b200 import inputs, ops
     import selective_state_space_56_b200.build as s6build
     s6build.build()
@@ -441,6 +537,15 @@ def profile_target(which):
         for _ in range(3):
             ops.selective_scan_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
                                    delta_bias=p["delta_bias"], y=y)
+    elif which == "backward":
+        w = inputs.SCAN_WORKLOADS[WORKLOAD]
+        p = inputs.scan_inputs(w.batch, w.dim, w.dstate, w.seqlen, w.in_dtype, w.seed, device=dev)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(w.seed + 7)
+        dy = torch.randn((w.batch, w.dim, w.seqlen), generator=gen, device=dev).to(w.in_dtype)
+        for _ in range(2):
+            ops.selective_scan_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"],
+                                   z=p["z"], delta_bias=p["delta_bias"])
     else:
         w = inputs.DECODE_WORKLOAD
         prm = {k: v.to(dev) for k, v in inputs.decode_params(w).items()}
@@ -464,7 +569,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=1000)
-    ap.add_argument("--profile", choices=["scan", "decode"],
+    ap.add_argument("--backward-steps", type=int, default=50)
+    ap.add_argument("--profile", choices=["scan", "decode", "backward"],
                     help="run a few untimed launches of one workload (an ncu capture target) "
                          "and exit")
     args = ap.parse_args(argv)
