@@ -16,10 +16,15 @@ module only marshals numpy arrays.  The definitions it follows:
 * Page "yongjin360.com/news/29389": the serial "MambaMini" scan, initial state
   h_{-1} = 0, Bbar formed as the element-wise product of Delta and B, the
   state shape (batch, d_inner, d_state) and the SiLU gate.
+* With ``zoh=True``: the exact zero-order-hold Bbar = (Delta A)^-1 (exp(Delta A) - I)
+  Delta B of the "Method" section, per state expm1(Delta A_n) / A_n * B_n.
 
 Pins (tests/test_oracle_pins.py): hand-worked examples in tests/golden/, the
 associative-combine prefix of ``oracle.pscan``, the LTI convolution form,
-Abar in (0,1), small/large-Delta limits, the gated-RNN special case.
+Abar in (0,1), small/large-Delta limits, the gated-RNN special case.  The ZOH
+variant (tests/test_oracle_zoh.py): the gated-RNN identity, the continuous-time
+steady state -B u / A, numerical integration of the continuous ODE, the
+small-Delta limit and A = 0.
 """
 from __future__ import annotations
 
@@ -64,11 +69,12 @@ def _load():
             lib.s6o_discretize.argtypes = [ctypes.c_long] * 3 + [_dp, _dp, _dp, ctypes.c_int,
                                                                  _dp, _dp]
             lib.s6o_scan.restype = ctypes.c_int
-            lib.s6o_scan.argtypes = ([ctypes.c_long] * 4 + [_dp] * 8 + [_lp, ctypes.c_int, _dp]
+            lib.s6o_scan.argtypes = ([ctypes.c_long] * 4 + [_dp] * 8 + [_lp, ctypes.c_int,
+                                                                     ctypes.c_int, _dp]
                                      + [_dp] * 3)
             lib.s6o_state_update.restype = ctypes.c_int
             lib.s6o_state_update.argtypes = ([ctypes.c_long] * 3 + [_dp] * 9 + [_lp, ctypes.c_int,
-                                                                             _dp])
+                                                                             ctypes.c_int, _dp])
             lib.s6o_scan_backward.restype = ctypes.c_int
             lib.s6o_scan_backward.argtypes = ([ctypes.c_long] * 4 + [_dp] * 8 + [_lp, ctypes.c_int]
                                               + [_dp] * 9)
@@ -121,11 +127,12 @@ def discretize(delta_raw, A, delta_bias=None, softplus=True):
 
 
 def scan_lanes(u, delta_raw, A, B, C, lane_batch, D=None, z=None, delta_bias=None,
-               softplus=True, h0=None, return_states=False):
+               softplus=True, h0=None, return_states=False, zoh=False):
     """Sequential scan over independent lanes.
 
     u, delta_raw, z: (nlanes, L); A: (nlanes, N); D, delta_bias: (nlanes);
     B, C: (nbatch, N, L); lane_batch: (nlanes) int; h0: (nlanes, N) or None.
+    zoh: Bbar = expm1(Delta A) / A * B (the exact zero-order hold) instead of Delta B.
     Returns y (nlanes, L), h_last (nlanes, N)[, h_all (nlanes, L, N)].
     """
     u, dr, z = _f64(u), _f64(delta_raw), _f64(z)
@@ -144,7 +151,8 @@ def scan_lanes(u, delta_raw, A, B, C, lane_batch, D=None, z=None, delta_bias=Non
     h_all = np.empty((nl, L, N)) if return_states else None
     rc = _load().s6o_scan(nl, N, L, nb, _ptr(u), _ptr(dr), _ptr(z), _ptr(Aa), _ptr(Dd),
                           _ptr(bb), _ptr(Bm), _ptr(Cm), lb.ctypes.data_as(_lp),
-                          int(bool(softplus)), _ptr(h0), _ptr(y), _ptr(h_last), _ptr(h_all))
+                          int(bool(softplus)), int(bool(zoh)), _ptr(h0), _ptr(y), _ptr(h_last),
+                          _ptr(h_all))
     if rc != 0:
         raise ValueError("s6o_scan rejected its arguments")
     if return_states:
@@ -153,7 +161,7 @@ def scan_lanes(u, delta_raw, A, B, C, lane_batch, D=None, z=None, delta_bias=Non
 
 
 def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
-                   h0=None, return_states=False):
+                   h0=None, return_states=False, zoh=False):
     """The selective scan in the library's layouts.
 
     u, delta, z: (batch, dim, L); A: (dim, N); B, C: (batch, N, L);
@@ -171,7 +179,7 @@ def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=
                      D=rep(D), z=None if z is None else _f64(z).reshape(b * d, L),
                      delta_bias=rep(delta_bias), softplus=softplus,
                      h0=None if h0 is None else _f64(h0).reshape(b * d, N),
-                     return_states=return_states)
+                     return_states=return_states, zoh=zoh)
     y = out[0].reshape(b, d, L)
     hl = out[1].reshape(b, d, N)
     if return_states:
@@ -179,7 +187,8 @@ def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=
     return y, hl
 
 
-def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True):
+def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                 zoh=False):
     """One decode token: returns (new_state (batch, dim, N), y (batch, dim)).
 
     state: (batch, dim, N); u, delta, z: (batch, dim); A: (dim, N);
@@ -199,14 +208,14 @@ def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, soft
     y = np.empty(b * d)
     rc = _load().s6o_state_update(
         b * d, N, b, _ptr(st), _ptr(uu), _ptr(dd), _ptr(zz), _ptr(Aa), _ptr(Dd), _ptr(bb),
-        _ptr(Bv), _ptr(Cv), lb.ctypes.data_as(_lp), int(bool(softplus)), _ptr(y))
+        _ptr(Bv), _ptr(Cv), lb.ctypes.data_as(_lp), int(bool(softplus)), int(bool(zoh)), _ptr(y))
     if rc != 0:
         raise ValueError("s6o_state_update rejected its arguments")
     return st, y.reshape(b, d)
 
 
 def state_update_lanes(state, u, delta_raw, A, B, C, lane_batch, D=None, z=None, delta_bias=None,
-                       softplus=True):
+                       softplus=True, zoh=False):
     """One decode token on independent lanes: returns (new_state (nlanes, N), y (nlanes)).
 
     state, A: (nlanes, N); u, delta_raw, z, D, delta_bias: (nlanes);
@@ -222,7 +231,7 @@ def state_update_lanes(state, u, delta_raw, A, B, C, lane_batch, D=None, z=None,
     y = np.empty(nl)
     rc = _load().s6o_state_update(
         nl, N, Bv.shape[0], _ptr(st), _ptr(uu), _ptr(dd), _ptr(zz), _ptr(Aa), _ptr(Dd), _ptr(bb),
-        _ptr(Bv), _ptr(Cv), lb.ctypes.data_as(_lp), int(bool(softplus)), _ptr(y))
+        _ptr(Bv), _ptr(Cv), lb.ctypes.data_as(_lp), int(bool(softplus)), int(bool(zoh)), _ptr(y))
     if rc != 0:
         raise ValueError("s6o_state_update rejected its arguments")
     return st, y

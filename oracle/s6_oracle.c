@@ -15,10 +15,14 @@
  *       x      = delta_raw[t] + delta_bias                 (bias added before tau)
  *       Delta  = softplus(x)  if softplus else x           (tau_Delta = softplus)
  *       for n:  Abar_n = exp(Delta * A[n])                 (ZOH: Abar = exp(Delta A))
- *               h[n]   = Abar_n * h[n] + Delta * B[n,t] * u[t]
- *                                                          (Bbar = Delta * B, the
+ *               h[n]   = Abar_n * h[n] + w_n * B[n,t] * u[t]
+ *               w_n    = Delta                             (Bbar = Delta * B, the
  *                                                           element-wise product the
- *                                                           page-2 Q&A describes)
+ *                                                           page-2 Q&A describes), or
+ *               w_n    = expm1(Delta A[n]) / A[n]          (zoh != 0: the exact ZOH
+ *                                                           Bbar = (Delta A)^-1 (exp(Delta A)
+ *                                                           - I) Delta B of page 4
+ *                                                           "Method"; Delta when A[n] = 0)
  *       y[t]  = (sum_n C[n,t] * h[n] + D * u[t]) * silu(z[t])
  *     last_state = h
  *
@@ -52,6 +56,15 @@ double s6o_softplus(double x) {
 static double step_size(double delta_raw, double bias, int softplus) {
     double x = delta_raw + bias;
     return softplus ? s6o_softplus(x) : x;
+}
+
+/* Weight of the input in one state's update: Bbar = w * B.  The page-2 Q&A forms Bbar as
+ * Delta * B; page 4 "Method" gives the exact zero-order hold Bbar = (Delta A)^-1
+ * (exp(Delta A) - I) Delta B, which for a diagonal A is expm1(Delta A_n) / A_n per state
+ * (its limit Delta as A_n -> 0).  expm1 keeps the small-(Delta A) case exact. */
+static double input_weight(double dt, double a, int zoh) {
+    if (!zoh || a == 0.0) return dt;
+    return expm1(dt * a) / a;
 }
 
 /* SiLU gate: z * sigmoid(z) = z / (1 + e^{-z}) (page 2 Q&A on the gate). */
@@ -94,12 +107,13 @@ int s6o_discretize(long nlanes, long N, long L, const double* delta_raw,
  *   y               : (nlanes, L)          required
  *   h_last          : (nlanes, N) or NULL
  *   h_all           : (nlanes, L, N) or NULL  every state h_t (small inputs only)
+ *   zoh             : 0 for Bbar = Delta B, nonzero for the exact ZOH Bbar
  */
 int s6o_scan(long nlanes, long N, long L, long nbatch,
              const double* u, const double* delta_raw, const double* z,
              const double* A, const double* D, const double* delta_bias,
              const double* Bm, const double* Cm, const long* lane_batch,
-             int softplus, const double* h0,
+             int softplus, int zoh, const double* h0,
              double* y, double* h_last, double* h_all) {
     if (nlanes < 0 || N < 1 || N > S6O_MAX_N || L < 0 || nbatch < 1) return S6O_ERR_ARG;
     if (!u || !delta_raw || !A || !Bm || !Cm || !lane_batch || !y) return S6O_ERR_ARG;
@@ -120,7 +134,8 @@ int s6o_scan(long nlanes, long N, long L, long nbatch,
             double acc = 0.0;
             for (long n = 0; n < N; ++n) {
                 double abar = exp(dt * A[i * N + n]);
-                hv[n] = abar * hv[n] + dt * Bb[n * L + t] * ut;
+                double wt = input_weight(dt, A[i * N + n], zoh);
+                hv[n] = abar * hv[n] + wt * Bb[n * L + t] * ut;
                 acc += Cb[n * L + t] * hv[n];
                 if (h_all) h_all[(i * L + t) * N + n] = hv[n];
             }
@@ -142,13 +157,13 @@ int s6o_scan(long nlanes, long N, long L, long nbatch,
  *   state : (nlanes, N) in/out;   u, delta_raw, z : (nlanes)   z may be NULL
  *   A     : (nlanes, N);          D, delta_bias   : (nlanes) or NULL
  *   Bv, Cv: (nbatch, N); lane i reads row lane_batch[i]
- *   y     : (nlanes)
+ *   y     : (nlanes);                 zoh: as in s6o_scan
  */
 int s6o_state_update(long nlanes, long N, long nbatch, double* state,
                      const double* u, const double* delta_raw, const double* z,
                      const double* A, const double* D, const double* delta_bias,
                      const double* Bv, const double* Cv, const long* lane_batch,
-                     int softplus, double* y) {
+                     int softplus, int zoh, double* y) {
     if (nlanes < 0 || N < 1 || nbatch < 1) return S6O_ERR_ARG;
     if (!state || !u || !delta_raw || !A || !Bv || !Cv || !lane_batch || !y)
         return S6O_ERR_ARG;
@@ -163,7 +178,7 @@ int s6o_state_update(long nlanes, long N, long nbatch, double* state,
         double acc = 0.0;
         for (long n = 0; n < N; ++n) {
             double abar = exp(dt * A[i * N + n]);
-            double hn = abar * state[i * N + n] + dt * Bb[n] * u[i];
+            double hn = abar * state[i * N + n] + input_weight(dt, A[i * N + n], zoh) * Bb[n] * u[i];
             state[i * N + n] = hn;
             acc += Cb[n] * hn;
         }

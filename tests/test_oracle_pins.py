@@ -287,17 +287,17 @@ def test_batches_read_their_own_B_and_C():
 
 MUTATIONS = {
     "drop_D_skip": ("acc += dskip * ut;", "acc += 0.0 * ut;"),
-    "sign_of_exponent": ("exp(dt * A[i * N + n]);\n                hv[n]",
-                         "exp(-dt * A[i * N + n]);\n                hv[n]"),
+    "sign_of_exponent": ("exp(dt * A[i * N + n]);\n                double wt",
+                         "exp(-dt * A[i * N + n]);\n                double wt"),
     "readout_before_update": (
-        "hv[n] = abar * hv[n] + dt * Bb[n * L + t] * ut;\n                acc += Cb[n * L + t] * hv[n];",
-        "acc += Cb[n * L + t] * hv[n];\n                hv[n] = abar * hv[n] + dt * Bb[n * L + t] * ut;"),
-    "B_C_swapped": ("hv[n] = abar * hv[n] + dt * Bb[n * L + t] * ut;\n                acc += Cb[n * L + t]",
-                    "hv[n] = abar * hv[n] + dt * Cb[n * L + t] * ut;\n                acc += Bb[n * L + t]"),
-    "B_time_index_shift": ("dt * Bb[n * L + t] * ut", "dt * Bb[n * L + (t > 0 ? t - 1 : 0)] * ut"),
+        "hv[n] = abar * hv[n] + wt * Bb[n * L + t] * ut;\n                acc += Cb[n * L + t] * hv[n];",
+        "acc += Cb[n * L + t] * hv[n];\n                hv[n] = abar * hv[n] + wt * Bb[n * L + t] * ut;"),
+    "B_C_swapped": ("hv[n] = abar * hv[n] + wt * Bb[n * L + t] * ut;\n                acc += Cb[n * L + t]",
+                    "hv[n] = abar * hv[n] + wt * Cb[n * L + t] * ut;\n                acc += Bb[n * L + t]"),
+    "B_time_index_shift": ("wt * Bb[n * L + t] * ut", "wt * Bb[n * L + (t > 0 ? t - 1 : 0)] * ut"),
     "bias_after_softplus": ("double x = delta_raw + bias;\n    return softplus ? s6o_softplus(x) : x;",
                             "return softplus ? s6o_softplus(delta_raw) + bias : delta_raw + bias;"),
-    "missing_delta_in_B": ("dt * Bb[n * L + t] * ut", "Bb[n * L + t] * ut"),
+    "missing_delta_in_B": ("wt * Bb[n * L + t] * ut", "Bb[n * L + t] * ut"),
     "gate_is_sigmoid": ("if (z) acc *= silu(z[i * L + t]);",
                         "if (z) acc *= 1.0 / (1.0 + exp(-z[i * L + t]));"),
     "softplus_wrong_branch": ("if (x > 0.0) return x + log1p(exp(-x));",
