@@ -13,7 +13,8 @@ batch (weak scaling, no data-path collective) and the max time over ranks is
 used.  The same run measures the decode workload (selective_state_update,
 batch 256, dim 5120, N 16, 1000 fresh tokens, L2 flushed before each token),
 the backward of the same layer's scan (recomputing states from chunk
-checkpoints), the end-to-end path from pinned host buffers, the SM clocks during
+checkpoints), the exact zero-order-hold variant of the scan and of decode, the
+end-to-end path from pinned host buffers, the SM clocks during
 the timed region, and (rank 0, N = 1) the fp64 CPU oracle on bounded samples.
 
 ``--impl reference`` times the CPU oracle itself as the reference arm.
@@ -306,6 +307,7 @@ def run_ours(args, rank, world, local):
     del y, last
     torch.cuda.empty_cache()
     backward = run_backward(g, dev, stream, world, w, steps=args.backward_steps)
+    zoh = run_zoh(g, dev, stream, world, w, steps=args.zoh_steps)
     del g
     torch.cuda.empty_cache()
 
@@ -326,10 +328,88 @@ def run_ours(args, rank, world, local):
                        (h2d) / 1e6, L2_BYTES >> 20),
                    "parallelism": "replicas x%d (independent batches per GPU)" % world},
         "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
-        "clocks": clocks, "decode": decode, "backward": backward, "cpu_baseline": cpu,
+        "clocks": clocks, "decode": decode, "backward": backward, "exact_zoh": zoh,
+        "cpu_baseline": cpu,
         "impl": "ours",
     }
     return line
+
+
+def run_zoh(g, dev, stream, world, w, steps=50):
+    """The exact zero-order-hold variant (MAMBA_FLAG_EXACT_ZOH): the m2p8b scan per launch,
+    and decode tokens after an L2 flush, each timed with events on the launching stream."""
+    from selective_state_space_56_b200 import inputs, ops
+    b, d, n, L = w.batch, w.dim, w.dstate, w.seqlen
+    y = torch.empty((b, d, L), dtype=w.out_dtype, device=dev)
+
+    def scan():
+        ops.selective_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                               delta_bias=g["delta_bias"], y=y, exact_zoh=True)
+
+    for _ in range(3):
+        scan()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b_ in evs:
+        a.record(stream)
+        scan()
+        b_.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(statistics.fmean(a.elapsed_time(b_) for a, b_ in evs), world)
+    elems = b * d * L
+    peaks, kind = measured_peaks()
+    fmax_mhz = peaks.get("sm_max_mhz", 1965.0)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    sfu_peak = sms * SFU_OPS_PER_CLK_PER_SM * fmax_mhz * 1e6
+    exps = elems * (n + 2)
+    del y
+
+    dw = inputs.DECODE_WORKLOAD
+    prm = {k: v.to(dev) for k, v in inputs.decode_params(dw).items()}
+    state = prm["state0"].clone()
+    toks = inputs.decode_tokens_batched(steps, dw, device=dev)
+    yd = torch.empty((dw.batch, dw.dim), dtype=dw.io_dtype, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def tok(s):
+        ops.selective_state_update(state, toks["u"][s], toks["delta"][s], prm["A"], toks["B"][s],
+                                   toks["C"][s], D=prm["D"], z=toks["z"][s],
+                                   delta_bias=prm["delta_bias"], y=yd, exact_zoh=True)
+
+    for s in range(3):
+        tok(s)
+    torch.cuda.synchronize(dev)
+    devs = []
+    for s in range(steps):
+        flush_l2(flush)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        tok(s)
+        b_.record(stream)
+        devs.append((a, b_))
+    torch.cuda.synchronize(dev)
+    ms_tok = max_over_ranks(statistics.fmean(a.elapsed_time(b_) for a, b_ in devs), world)
+    byts = decode_bytes(dw.batch, dw.dim, dw.dstate)
+    del toks, flush, state
+    return {
+        "metric": "selective-scan fwd with exact ZOH Bbar, (b·d·L) elems/s", "unit": "elems/s",
+        "value": world * elems / (ms * 1e-3), "ms_per_call": ms, "steps": steps,
+        "workload": "m2p8b scan (batch 4, dim 5120, N 16, L 4096, bf16 I/O) with "
+                    "Bbar = (exp(Delta A) - 1) / A * B",
+        "roofline": {"bound": "alu", "unit": "Gexp/s", "achieved": exps / (ms * 1e-3) / 1e9,
+                     "peak": sfu_peak / 1e9, "frac": exps / (ms * 1e-3) / sfu_peak,
+                     "note": "same N + 2 SFU exponentials per element as the Delta*B scan; the "
+                             "exact weight adds FMA-pipe work (series + select), not SFU work"},
+        "decode": {"ms_per_token_l2_flushed": ms_tok,
+                   "value": world * dw.batch * dw.dim / (ms_tok * 1e-3),
+                   "unit": "(b,d) lane updates/s",
+                   "roofline": {"bound": "hbm", "unit": "GB/s",
+                                "achieved": byts / (ms_tok * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                                "frac": byts / (ms_tok * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                "peak_kind": kind}},
+        "gpu_launches": 2 * steps + 6,
+    }
 
 
 def run_backward(g, dev, stream, world, w, steps=50):
@@ -570,6 +650,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--backward-steps", type=int, default=50)
+    ap.add_argument("--zoh-steps", type=int, default=50)
     ap.add_argument("--profile", choices=["scan", "decode", "backward"],
                     help="run a few untimed launches of one workload (an ncu capture target) "
                          "and exit")

@@ -54,8 +54,21 @@ typedef enum {
     MAMBA_ERR_DTYPE = -4,     /* an unknown dtype enum                              */
     MAMBA_ERR_WORKSPACE = -5, /* workspace missing or smaller than required          */
     MAMBA_ERR_CUDA = -6,      /* the CUDA runtime reported an error                 */
-    MAMBA_ERR_TIMEOUT = -7    /* a bounded device-side wait gave up                 */
+    MAMBA_ERR_TIMEOUT = -7,   /* a bounded device-side wait gave up                 */
+    MAMBA_ERR_FLAGS = -8      /* unknown bits in a flags argument                   */
 } mamba_status;
+
+/*
+ * Flags of the _ex entry points.
+ *
+ * MAMBA_FLAG_EXACT_ZOH: discretise B with the exact zero-order hold of the "Method"
+ * section, Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B -- for the diagonal A, per
+ * state Bbar_n = (exp(Delta A_n) - 1) / A_n * B_n (Delta B_n when A_n = 0) -- instead of
+ * Bbar = Delta * B.  The kernels form (exp(Delta A_n) - 1) / A_n from the same
+ * exponential as Abar where |Delta A_n| >= 1/2 and from the series of expm1(y) / y
+ * below, so the weight stays accurate as Delta A_n -> 0.
+ */
+#define MAMBA_FLAG_EXACT_ZOH 1u
 
 /* Problem sizes: batch >= 1, dim >= 1, 1 <= dstate <= 16, seqlen >= 0. */
 typedef struct {
@@ -104,6 +117,18 @@ int mamba_selective_scan_fwd(const void* u, const void* delta, const float* A, c
                              void* stream);
 
 /*
+ * mamba_selective_scan_fwd with a flags word (MAMBA_FLAG_EXACT_ZOH, or 0 for exactly
+ * mamba_selective_scan_fwd).  Same arguments, layouts, workspace and errors, plus
+ * MAMBA_ERR_FLAGS for unknown bits.
+ */
+int mamba_selective_scan_fwd_ex(const void* u, const void* delta, const float* A, const void* B,
+                                const void* C, const float* D, const void* z,
+                                const float* delta_bias, int delta_softplus, void* y,
+                                float* last_state, mamba_scan_dims dims, mamba_dtype in_dtype,
+                                mamba_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                unsigned flags, void* stream);
+
+/*
  * One decode token (selective_state_update): the recurrence above for a single
  * t, applied in place to a carried state (the generation mode keeps only a
  * fixed dim x dstate state per layer and costs O(1) per token).
@@ -122,6 +147,16 @@ int mamba_selective_state_update(float* state, const void* u, const void* delta,
                                  const float* delta_bias, int delta_softplus, void* y,
                                  int64_t batch, int64_t dim, int64_t dstate,
                                  mamba_dtype io_dtype, void* stream);
+
+/*
+ * mamba_selective_state_update with a flags word (MAMBA_FLAG_EXACT_ZOH, or 0).  Same
+ * arguments and errors, plus MAMBA_ERR_FLAGS for unknown bits.
+ */
+int mamba_selective_state_update_ex(float* state, const void* u, const void* delta,
+                                    const float* A, const void* B, const void* C, const float* D,
+                                    const void* z, const float* delta_bias, int delta_softplus,
+                                    void* y, int64_t batch, int64_t dim, int64_t dstate,
+                                    mamba_dtype io_dtype, unsigned flags, void* stream);
 
 /*
  * mamba_selective_scan_fwd for callers that cannot allocate device memory.  (This
@@ -183,6 +218,8 @@ size_t mamba_selective_scan_bwd_workspace_size(mamba_scan_dims dims);
  *   workspace   : at least mamba_selective_scan_bwd_workspace_size(dims) bytes; its
  *                 contents on entry do not matter
  *
+ * The backward is that of the Bbar = Delta * B discretisation (the forward without
+ * flags).
  * dA, dB, dC, dD and ddelta_bias are sums over many CTAs, formed with float32
  * atomics: their last bits may differ between runs.  With seqlen == 0 the
  * per-token arrays may be NULL and dA, dD, ddelta_bias are set to zero.

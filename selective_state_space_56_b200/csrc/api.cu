@@ -35,6 +35,18 @@ bool dims_ok(int64_t batch, int64_t dim, int64_t dstate, int64_t L) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA; }
 
+constexpr unsigned kKnownFlags = MAMBA_FLAG_EXACT_ZOH;
+
+int scan_fwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
+             const float* D, const void* z, const float* delta_bias, int delta_softplus, void* y,
+             float* last_state, mamba_scan_dims dims, mamba_dtype in_dtype, mamba_dtype out_dtype,
+             void* workspace, size_t workspace_bytes, unsigned flags, void* stream);
+
+int state_update(float* state, const void* u, const void* delta, const float* A, const void* B,
+                 const void* C, const float* D, const void* z, const float* delta_bias,
+                 int delta_softplus, void* y, int64_t batch, int64_t dim, int64_t dstate,
+                 mamba_dtype io_dtype, unsigned flags, void* stream);
+
 }  // namespace
 
 extern "C" {
@@ -56,6 +68,29 @@ int mamba_selective_scan_fwd(const void* u, const void* delta, const float* A, c
                              float* last_state, mamba_scan_dims dims, mamba_dtype in_dtype,
                              mamba_dtype out_dtype, void* workspace, size_t workspace_bytes,
                              void* stream) {
+    return scan_fwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, last_state, dims,
+                    in_dtype, out_dtype, workspace, workspace_bytes, 0u, stream);
+}
+
+int mamba_selective_scan_fwd_ex(const void* u, const void* delta, const float* A, const void* B,
+                                const void* C, const float* D, const void* z,
+                                const float* delta_bias, int delta_softplus, void* y,
+                                float* last_state, mamba_scan_dims dims, mamba_dtype in_dtype,
+                                mamba_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                unsigned flags, void* stream) {
+    return scan_fwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, last_state, dims,
+                    in_dtype, out_dtype, workspace, workspace_bytes, flags, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+int scan_fwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
+             const float* D, const void* z, const float* delta_bias, int delta_softplus, void* y,
+             float* last_state, mamba_scan_dims dims, mamba_dtype in_dtype, mamba_dtype out_dtype,
+             void* workspace, size_t workspace_bytes, unsigned flags, void* stream) {
+    if (flags & ~kKnownFlags) return MAMBA_ERR_FLAGS;
     // With seqlen == 0 the (batch, dim, 0) and (batch, dstate, 0) arrays are empty and
     // may be NULL; only last_state (zeros) is written.
     const bool empty = dims.seqlen == 0;
@@ -91,6 +126,7 @@ int mamba_selective_scan_fwd(const void* u, const void* delta, const float* A, c
     a.N = dims.dstate;
     a.L = dims.seqlen;
     a.softplus = delta_softplus;
+    a.zoh = (flags & MAMBA_FLAG_EXACT_ZOH) ? 1 : 0;
     a.in_dtype = to_dtype(in_dtype);
     a.out_dtype = to_dtype(out_dtype);
     a.nseg = nseg;
@@ -104,11 +140,11 @@ int mamba_selective_scan_fwd(const void* u, const void* delta, const float* A, c
     return cuda_status(s6::launch_scan(a, static_cast<cudaStream_t>(stream)));
 }
 
-int mamba_selective_state_update(float* state, const void* u, const void* delta, const float* A,
-                                 const void* B, const void* C, const float* D, const void* z,
-                                 const float* delta_bias, int delta_softplus, void* y,
-                                 int64_t batch, int64_t dim, int64_t dstate,
-                                 mamba_dtype io_dtype, void* stream) {
+int state_update(float* state, const void* u, const void* delta, const float* A, const void* B,
+                 const void* C, const float* D, const void* z, const float* delta_bias,
+                 int delta_softplus, void* y, int64_t batch, int64_t dim, int64_t dstate,
+                 mamba_dtype io_dtype, unsigned flags, void* stream) {
+    if (flags & ~kKnownFlags) return MAMBA_ERR_FLAGS;
     if (!state || !u || !delta || !A || !B || !C || !y) return MAMBA_ERR_NULL;
     if (!dtype_ok(io_dtype)) return MAMBA_ERR_DTYPE;
     if (!dims_ok(batch, dim, dstate, 1)) return MAMBA_ERR_DIMS;
@@ -130,8 +166,31 @@ int mamba_selective_state_update(float* state, const void* u, const void* delta,
     a.dim = dim;
     a.N = dstate;
     a.softplus = delta_softplus;
+    a.zoh = (flags & MAMBA_FLAG_EXACT_ZOH) ? 1 : 0;
     a.io_dtype = to_dtype(io_dtype);
     return cuda_status(s6::launch_state_update(a, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+int mamba_selective_state_update(float* state, const void* u, const void* delta, const float* A,
+                                 const void* B, const void* C, const float* D, const void* z,
+                                 const float* delta_bias, int delta_softplus, void* y,
+                                 int64_t batch, int64_t dim, int64_t dstate,
+                                 mamba_dtype io_dtype, void* stream) {
+    return state_update(state, u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, batch, dim,
+                        dstate, io_dtype, 0u, stream);
+}
+
+int mamba_selective_state_update_ex(float* state, const void* u, const void* delta,
+                                    const float* A, const void* B, const void* C, const float* D,
+                                    const void* z, const float* delta_bias, int delta_softplus,
+                                    void* y, int64_t batch, int64_t dim, int64_t dstate,
+                                    mamba_dtype io_dtype, unsigned flags, void* stream) {
+    return state_update(state, u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, batch, dim,
+                        dstate, io_dtype, flags, stream);
 }
 
 size_t mamba_selective_scan_bwd_workspace_size(mamba_scan_dims dims) {
@@ -186,6 +245,7 @@ int mamba_selective_scan_bwd(const void* u, const void* delta, const float* A, c
     a.N = dims.dstate;
     a.L = dims.seqlen;
     a.softplus = delta_softplus;
+    a.zoh = 0;
     a.in_dtype = to_dtype(in_dtype);
     a.out_dtype = a.in_dtype;
     a.nseg = 1;
@@ -223,10 +283,11 @@ const char* mamba_status_string(int status) {
         case MAMBA_ERR_WORKSPACE: return "workspace missing or too small";
         case MAMBA_ERR_CUDA: return "CUDA runtime error";
         case MAMBA_ERR_TIMEOUT: return "a bounded device wait timed out";
+        case MAMBA_ERR_FLAGS: return "unknown flag bits";
         default: return "unknown status";
     }
 }
 
-int mamba_abi_version(void) { return 101; }
+int mamba_abi_version(void) { return 102; }
 
 }  // extern "C"

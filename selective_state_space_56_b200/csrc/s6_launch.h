@@ -22,6 +22,7 @@ struct ScanArgs {
     float* last_state;  // may be null
     int64_t batch, dim, N, L;
     int softplus;
+    int zoh;  // nonzero: exact zero-order-hold Bbar = (exp(Delta A) - 1) / A * B
     DType in_dtype, out_dtype;
     // sequence split (nseg == 1: single pass, no workspace)
     int64_t nseg, seg_len;
@@ -42,6 +43,7 @@ struct StateUpdateArgs {
     void* y;
     int64_t batch, dim, N;
     int softplus;
+    int zoh;  // as in ScanArgs
     DType io_dtype;
 };
 

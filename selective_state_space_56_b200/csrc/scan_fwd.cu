@@ -183,7 +183,8 @@ __device__ __forceinline__ float transpose_reduce(const float* v, int pp) {
     }
 }
 
-template <int NMAX, int P, int WARPS, int T_, typename Tin, typename Tout, int MODE, bool TMA>
+template <int NMAX, int P, int WARPS, int T_, typename Tin, typename Tout, int MODE, bool TMA,
+          bool ZOH = false>
 __global__ void __launch_bounds__(WARPS * 32)
 scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
     using Lo = Layout<NMAX, P, WARPS, T_, Tin, Tout>;
@@ -225,6 +226,7 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
     const int cw = warp * G + lane / P;
     const int64_t dch = d0 + cw;
     f2 a2p[NS / 2], hp[NS / 2];
+    f2 inv_ap[ZOH ? NS / 2 : 1];  // 1 / A per state, for the exact ZOH input weight
 #pragma unroll
     for (int j = 0; j < NS; j += 2) {
         float a[2], h[2];
@@ -239,6 +241,11 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         }
         a2p[j / 2] = pack2(a[0], a[1]);
         hp[j / 2] = pack2(h[0], h[1]);
+        if constexpr (ZOH) {
+            // 1 / A (infinite for A = 0; the weight then takes its series branch)
+            const float ia0 = kLog2e / a[0], ia1 = kLog2e / a[1];
+            inv_ap[j / 2] = pack2(ia0, ia1);
+        }
     }
     float dsum = 0.f;
     __syncthreads();
@@ -397,9 +404,14 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) dt[q] = tb + q < valid ? dt[q] : 0.f;
             }
-            const float q0 = dt[0] * uu[0], q1 = dt[1] * uu[1], q2 = dt[2] * uu[2], q3 = dt[3] * uu[3];
             *reinterpret_cast<float4*>(sDel + c * RS + tb) = make_float4(dt[0], dt[1], dt[2], dt[3]);
-            *reinterpret_cast<float4*>(sDu + c * RS + tb) = make_float4(q0, q1, q2, q3);
+            if constexpr (ZOH) {  // the exact ZOH weight needs u itself
+                *reinterpret_cast<float4*>(sDu + c * RS + tb) = make_float4(uu[0], uu[1], uu[2], uu[3]);
+            } else {
+                const float q0 = dt[0] * uu[0], q1 = dt[1] * uu[1], q2 = dt[2] * uu[2],
+                            q3 = dt[3] * uu[3];
+                *reinterpret_cast<float4*>(sDu + c * RS + tb) = make_float4(q0, q1, q2, q3);
+            }
         }
         __syncwarp();
 
@@ -429,7 +441,9 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 const f2 dd = dd4[kk];
-                const f2 qq = qq4[kk];
+                // ZOH: qq4 holds (u, u); Delta u is formed here
+                const f2 uu = qq4[kk];
+                const f2 qq = ZOH ? mul2(dd, uu) : qq4[kk];
                 f2 acc = pack2(0.f, 0.f);
 #pragma unroll
                 for (int j = 0; j < NS / 4; ++j) {
@@ -453,12 +467,21 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
                             sCt + (t + kk) * NMAX + pp * NS)[j];
                         b01 = f2{bb.x}, b23 = f2{bb.y}, c01 = f2{cc.x}, c23 = f2{cc.y};
                     }
-                    const f2 e0 = ex2x2(mul2(dd, a2p[2 * j]));
-                    const bool on_fma = S6_POLY == 2 || (S6_POLY == 1 && (kk & 1));
-                    const f2 e1 = on_fma ? exp2_fma2(mul2(dd, a2p[2 * j + 1]))
-                                         : ex2x2(mul2(dd, a2p[2 * j + 1]));
-                    hp[2 * j] = fma2(e0, hp[2 * j], mul2(qq, b01));
-                    hp[2 * j + 1] = fma2(e1, hp[2 * j + 1], mul2(qq, b23));
+                    if constexpr (ZOH) {
+                        const f2 x0 = mul2(dd, a2p[2 * j]), x1 = mul2(dd, a2p[2 * j + 1]);
+                        const f2 e0 = ex2x2(x0), e1 = ex2x2(x1);
+                        const f2 m0 = zoh_weight_u2(x0, e0, inv_ap[2 * j], uu, qq);
+                        const f2 m1 = zoh_weight_u2(x1, e1, inv_ap[2 * j + 1], uu, qq);
+                        hp[2 * j] = fma2(e0, hp[2 * j], mul2(m0, b01));
+                        hp[2 * j + 1] = fma2(e1, hp[2 * j + 1], mul2(m1, b23));
+                    } else {
+                        const f2 e0 = ex2x2(mul2(dd, a2p[2 * j]));
+                        const bool on_fma = S6_POLY == 2 || (S6_POLY == 1 && (kk & 1));
+                        const f2 e1 = on_fma ? exp2_fma2(mul2(dd, a2p[2 * j + 1]))
+                                             : ex2x2(mul2(dd, a2p[2 * j + 1]));
+                        hp[2 * j] = fma2(e0, hp[2 * j], mul2(qq, b01));
+                        hp[2 * j + 1] = fma2(e1, hp[2 * j + 1], mul2(qq, b23));
+                    }
                     acc = fma2(c01, hp[2 * j], acc);
                     acc = fma2(c23, hp[2 * j + 1], acc);
                 }
@@ -622,10 +645,11 @@ bool encode_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, u
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NMAX, int P, int WARPS, int T, typename Tin, typename Tout, int MODE, bool TMA>
+template <int NMAX, int P, int WARPS, int T, typename Tin, typename Tout, int MODE, bool TMA,
+          bool ZOH = false>
 cudaError_t launch_one(const KParams& kp, const TMaps& tm, dim3 grid, cudaStream_t s) {
     using Lo = Layout<NMAX, P, WARPS, T, Tin, Tout>;
-    auto kern = scan_kernel<NMAX, P, WARPS, T, Tin, Tout, MODE, TMA>;
+    auto kern = scan_kernel<NMAX, P, WARPS, T, Tin, Tout, MODE, TMA, ZOH>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Lo::bytes);
     if (e != cudaSuccess) return e;
@@ -642,13 +666,13 @@ struct Tile {
     static constexpr int T = NMAX == 16 ? S6_CHUNK : 64;
 };
 
-template <int NMAX, typename Tin, typename Tout, bool TMA>
+template <int NMAX, typename Tin, typename Tout, bool TMA, bool ZOH>
 cudaError_t launch_typed(const ScanArgs& a, const KParams& kp, const TMaps& tm, cudaStream_t s) {
     using TL = Tile<NMAX>;
     using Lo = Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout>;
     const unsigned gx = (unsigned)((a.dim + Lo::CH - 1) / Lo::CH);
     if (a.nseg > 1) {
-        cudaError_t e = launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kAggregate, TMA>(
+        cudaError_t e = launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kAggregate, TMA, ZOH>(
             kp, tm, dim3(gx, (unsigned)a.batch, (unsigned)(a.nseg - 1)), s);
         if (e != cudaSuccess) return e;
         const int64_t lanes = a.batch * a.dim * a.N;
@@ -657,11 +681,11 @@ cudaError_t launch_typed(const ScanArgs& a, const KParams& kp, const TMaps& tm, 
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA>(
+    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA, ZOH>(
         kp, tm, dim3(gx, (unsigned)a.batch, (unsigned)a.nseg), s);
 }
 
-template <int NMAX, typename Tin, typename Tout>
+template <int NMAX, typename Tin, typename Tout, bool ZOH>
 cudaError_t launch_io(const ScanArgs& a, KParams kp, cudaStream_t s) {
     using TL = Tile<NMAX>;
     using Lo = Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout>;
@@ -673,7 +697,7 @@ cudaError_t launch_io(const ScanArgs& a, KParams kp, cudaStream_t s) {
     const bool fits = a.L < (1LL << 31) && a.dim < (1LL << 31) && a.batch < (1LL << 31);
     if (!(rows16 && fits)) {
         kp.y_tma = 0;
-        return launch_typed<NMAX, Tin, Tout, false>(a, kp, tm, s);
+        return launch_typed<NMAX, Tin, Tout, false, ZOH>(a, kp, tm, s);
     }
     bool ok = encode_3d<Tin>(&tm.u, a.u, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
               encode_3d<Tin>(&tm.dr, a.delta, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
@@ -683,7 +707,7 @@ cudaError_t launch_io(const ScanArgs& a, KParams kp, cudaStream_t s) {
     kp.y_tma = out16 ? 1 : 0;
     if (ok && out16) ok = encode_3d<Tout>(&tm.y, a.y, a.L, a.dim, a.batch, Lo::T, Lo::G);
     if (!ok) return cudaErrorInvalidValue;
-    return launch_typed<NMAX, Tin, Tout, true>(a, kp, tm, s);
+    return launch_typed<NMAX, Tin, Tout, true, ZOH>(a, kp, tm, s);
 }
 
 template <int NMAX, typename Tin, bool TMA>
@@ -714,13 +738,18 @@ cudaError_t launch_ckpt_io(const ScanArgs& a, KParams kp, cudaStream_t s) {
     return launch_ckpt_typed<NMAX, Tin, true>(a, kp, tm, s);
 }
 
+template <int NMAX, bool ZOH>
+cudaError_t launch_nmax_z(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
+    const bool ib = a.in_dtype == DType::BF16, ob = a.out_dtype == DType::BF16;
+    if (ib && ob) return launch_io<NMAX, __nv_bfloat16, __nv_bfloat16, ZOH>(a, kp, s);
+    if (ib && !ob) return launch_io<NMAX, __nv_bfloat16, float, ZOH>(a, kp, s);
+    if (!ib && ob) return launch_io<NMAX, float, __nv_bfloat16, ZOH>(a, kp, s);
+    return launch_io<NMAX, float, float, ZOH>(a, kp, s);
+}
+
 template <int NMAX>
 cudaError_t launch_nmax(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
-    const bool ib = a.in_dtype == DType::BF16, ob = a.out_dtype == DType::BF16;
-    if (ib && ob) return launch_io<NMAX, __nv_bfloat16, __nv_bfloat16>(a, kp, s);
-    if (ib && !ob) return launch_io<NMAX, __nv_bfloat16, float>(a, kp, s);
-    if (!ib && ob) return launch_io<NMAX, float, __nv_bfloat16>(a, kp, s);
-    return launch_io<NMAX, float, float>(a, kp, s);
+    return a.zoh ? launch_nmax_z<NMAX, true>(a, kp, s) : launch_nmax_z<NMAX, false>(a, kp, s);
 }
 
 }  // namespace

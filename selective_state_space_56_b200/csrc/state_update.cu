@@ -6,7 +6,8 @@
 // written once in place, so the kernel is laid out for HBM: G = NMAX / 4 adjacent
 // threads share one (batch, channel) lane and each moves 16 contiguous bytes of
 // state, so a warp touches 512 consecutive bytes per access.  The per-lane
-// readout sum_n C_n h_n is finished with log2(G) xor-shuffles.
+// readout sum_n C_n h_n is finished with log2(G) xor-shuffles.  A compile-time
+// variant uses the exact zero-order-hold input weight (e^{Delta A} - 1) / A.
 #include "s6_device.cuh"
 #include "s6_launch.h"
 
@@ -30,7 +31,7 @@ struct UParams {
     int vec;  // N % 4 == 0: 16-byte state / A accesses
 };
 
-template <int NMAX, typename Tio>
+template <int NMAX, typename Tio, bool ZOH>
 __global__ void __launch_bounds__(256) state_update_kernel(const UParams p) {
     constexpr int G = NMAX / 4;
     const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -75,11 +76,30 @@ __global__ void __launch_bounds__(256) state_update_kernel(const UParams p) {
         }
     }
     float acc = 0.f;
+    if constexpr (ZOH) {
+        // exact zero-order hold: Bbar = (e^{Delta A} - 1) / A * B, states in pairs; 1 / A
+        // from rcp.approx (within 1 ulp; infinite for A = 0, where the series branch applies)
+        const f2 uu2 = pack2(uu, uu), qq2 = pack2(du, du);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float abar = ex2(dt * (a[k] * kLog2e));
-        st[k] = fmaf(abar, st[k], du * bv[k]);
-        acc = fmaf(cv[k], st[k], acc);
+        for (int k = 0; k < 4; k += 2) {
+            const f2 x = pack2(dt * (a[k] * kLog2e), dt * (a[k + 1] * kLog2e));
+            const f2 e = ex2x2(x);
+            const f2 m = zoh_weight_u2(x, e, pack2(rcp(a[k]), rcp(a[k + 1])), uu2, qq2);
+            float e0, e1, m0, m1;
+            unpack2(e, e0, e1);
+            unpack2(m, m0, m1);
+            st[k] = fmaf(e0, st[k], m0 * bv[k]);
+            st[k + 1] = fmaf(e1, st[k + 1], m1 * bv[k + 1]);
+            acc = fmaf(cv[k], st[k], acc);
+            acc = fmaf(cv[k + 1], st[k + 1], acc);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float abar = ex2(dt * (a[k] * kLog2e));
+            st[k] = fmaf(abar, st[k], du * bv[k]);
+            acc = fmaf(cv[k], st[k], acc);
+        }
     }
     if (active && jok) {
         if (p.vec) {
@@ -114,7 +134,7 @@ struct Lane16 {
     float u, x, z, dsk;
 };
 
-template <typename Tio>
+template <typename Tio, bool ZOH>
 __global__ void __launch_bounds__(256) state_update16_kernel(const UParams p) {
     using VT = typename vec4<Tio>::type;
     const uint32_t pairs = (uint32_t)(gridDim.x * blockDim.x) / 2;  // lanes per item sweep
@@ -171,8 +191,12 @@ __global__ void __launch_bounds__(256) state_update16_kernel(const UParams p) {
         f2 acc = pack2(0.f, 0.f);
 #pragma unroll
         for (int j = 0; j < 8; j += 2) {
-            const f2 e = ex2x2(mul2(dd, pack2(av[j], av[j + 1])));
-            const f2 hn = fma2(e, pack2(sv[j], sv[j + 1]), mul2(qq, pack2(bv[j], bv[j + 1])));
+            const f2 x = mul2(dd, pack2(av[j], av[j + 1]));
+            const f2 e = ex2x2(x);
+            f2 m = qq;
+            if constexpr (ZOH)  // exact zero-order hold: Bbar = (e^{Delta A} - 1) / A * B
+                m = zoh_weight_u2(x, e, pack2(rcp(av[j]), rcp(av[j + 1])), pack2(w.u, w.u), qq);
+            const f2 hn = fma2(e, pack2(sv[j], sv[j + 1]), mul2(m, pack2(bv[j], bv[j + 1])));
             acc = fma2(pack2(cv[j], cv[j + 1]), hn, acc);
             unpack2(hn, out[j], out[j + 1]);
         }
@@ -193,25 +217,25 @@ __global__ void __launch_bounds__(256) state_update16_kernel(const UParams p) {
     }
 }
 
-template <int NMAX, typename Tio>
+template <int NMAX, typename Tio, bool ZOH>
 cudaError_t launch_u(const UParams& p, cudaStream_t s) {
     constexpr int G = NMAX / 4;
     const int64_t threads = p.lanes * G;
     const unsigned blocks = (unsigned)((threads + 255) / 256);
-    state_update_kernel<NMAX, Tio><<<blocks, 256, 0, s>>>(p);
+    state_update_kernel<NMAX, Tio, ZOH><<<blocks, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 
-template <typename Tio>
+template <typename Tio, bool ZOH>
 cudaError_t launch_u_typed(const UParams& p, cudaStream_t s) {
     if (p.N == 16 && p.lanes < (1LL << 29)) {
         const int64_t threads = 2 * ((p.lanes + kItems - 1) / kItems);
-        state_update16_kernel<Tio><<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(p);
+        state_update16_kernel<Tio, ZOH><<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(p);
         return cudaGetLastError();
     }
-    if (p.N <= 4) return launch_u<4, Tio>(p, s);
-    if (p.N <= 8) return launch_u<8, Tio>(p, s);
-    return launch_u<16, Tio>(p, s);
+    if (p.N <= 4) return launch_u<4, Tio, ZOH>(p, s);
+    if (p.N <= 8) return launch_u<8, Tio, ZOH>(p, s);
+    return launch_u<16, Tio, ZOH>(p, s);
 }
 
 }  // namespace
@@ -234,8 +258,10 @@ cudaError_t launch_state_update(const StateUpdateArgs& a, cudaStream_t stream) {
     p.N = (int)a.N;
     p.softplus = a.softplus ? 1 : 0;
     p.vec = (a.N % 4 == 0) ? 1 : 0;
-    if (a.io_dtype == DType::BF16) return launch_u_typed<__nv_bfloat16>(p, stream);
-    return launch_u_typed<float>(p, stream);
+    const bool bf = a.io_dtype == DType::BF16;
+    if (a.zoh) return bf ? launch_u_typed<__nv_bfloat16, true>(p, stream)
+                         : launch_u_typed<float, true>(p, stream);
+    return bf ? launch_u_typed<__nv_bfloat16, false>(p, stream) : launch_u_typed<float, false>(p, stream);
 }
 
 }  // namespace s6

@@ -19,6 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmamba_s6.so")
 
 MAMBA_F32, MAMBA_BF16 = 0, 1
+MAMBA_FLAG_EXACT_ZOH = 1
 _DTYPES = {torch.float32: MAMBA_F32, torch.bfloat16: MAMBA_BF16}
 
 
@@ -57,6 +58,14 @@ def load_library():
             lib.mamba_selective_scan_bwd.restype = i32
             lib.mamba_selective_scan_bwd.argtypes = [vp] * 8 + [i32] + [vp] * 9 + [
                 ScanDims, i32, vp, ctypes.c_size_t, vp]
+            u32 = ctypes.c_uint
+            lib.mamba_selective_scan_fwd_ex.restype = i32
+            lib.mamba_selective_scan_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp,
+                                                        vp, ScanDims, i32, i32, vp,
+                                                        ctypes.c_size_t, u32, vp]
+            lib.mamba_selective_state_update_ex.restype = i32
+            lib.mamba_selective_state_update_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                                            i32, vp, i64, i64, i64, i32, u32, vp]
             lib.mamba_selective_state_update.restype = i32
             lib.mamba_selective_state_update.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
                                                          vp, i64, i64, i64, i32, vp]
@@ -132,10 +141,11 @@ def selective_scan_workspace_size(batch: int, dim: int, dstate: int, seqlen: int
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
                        out_dtype=None, y=None, last_state=None, return_last_state=False,
-                       workspace=None):
+                       workspace=None, exact_zoh=False):
     """Fused selective scan.  u, delta, z: (batch, dim, L); A: (dim, N) fp32;
     B, C: (batch, N, L); D, delta_bias: (dim) fp32.  Returns y (batch, dim, L)
-    [and last_state (batch, dim, N) fp32]."""
+    [and last_state (batch, dim, N) fp32].  exact_zoh: Bbar = (exp(Delta A) - 1) / A * B
+    instead of Delta * B."""
     if not isinstance(u, torch.Tensor) or u.dim() != 3:
         raise ValueError("u must be a (batch, dim, L) tensor")
     dev = u.device
@@ -169,11 +179,14 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
     if need > 0 and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    with torch.cuda.device(dev):
-        rc = lib.mamba_selective_scan_fwd(
-            _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+    args = (_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
             int(bool(delta_softplus)), _ptr(y), _ptr(last_state), dims, _DTYPES[in_dt],
-            _DTYPES[out_dt], _ptr(workspace), ws_bytes, _stream_handle(dev))
+            _DTYPES[out_dt], _ptr(workspace), ws_bytes)
+    with torch.cuda.device(dev):
+        if exact_zoh:
+            rc = lib.mamba_selective_scan_fwd_ex(*args, MAMBA_FLAG_EXACT_ZOH, _stream_handle(dev))
+        else:
+            rc = lib.mamba_selective_scan_fwd(*args, _stream_handle(dev))
     if rc != 0:
         raise MambaError(rc, "mamba_selective_scan_fwd")
     if return_last_state:
@@ -236,9 +249,10 @@ def selective_scan_bwd_workspace_size(batch: int, dim: int, dstate: int, seqlen:
 
 
 def selective_state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
-                           delta_softplus=True, y=None):
+                           delta_softplus=True, y=None, exact_zoh=False):
     """One decode token, in place on ``state`` (batch, dim, N) fp32.
-    u, delta, z: (batch, dim); B, C: (batch, N); A: (dim, N).  Returns y (batch, dim)."""
+    u, delta, z: (batch, dim); B, C: (batch, N); A: (dim, N).  Returns y (batch, dim).
+    exact_zoh: Bbar = (exp(Delta A) - 1) / A * B instead of Delta * B."""
     if not isinstance(state, torch.Tensor) or state.dim() != 3:
         raise ValueError("state must be a (batch, dim, N) tensor")
     dev = state.device
@@ -260,11 +274,15 @@ def selective_state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=
     if y is None:
         y = torch.empty((b, d), dtype=io_dt, device=dev)
     _check(y, "y", dev, (b, d), (io_dt,))
+    args = (_ptr(state), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+            _ptr(delta_bias), int(bool(delta_softplus)), _ptr(y), b, d, N, _DTYPES[io_dt])
+    lib = load_library()
     with torch.cuda.device(dev):
-        rc = load_library().mamba_selective_state_update(
-            _ptr(state), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
-            _ptr(delta_bias), int(bool(delta_softplus)), _ptr(y), b, d, N, _DTYPES[io_dt],
-            _stream_handle(dev))
+        if exact_zoh:
+            rc = lib.mamba_selective_state_update_ex(*args, MAMBA_FLAG_EXACT_ZOH,
+                                                     _stream_handle(dev))
+        else:
+            rc = lib.mamba_selective_state_update(*args, _stream_handle(dev))
     if rc != 0:
         raise MambaError(rc, "mamba_selective_state_update")
     return y

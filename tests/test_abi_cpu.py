@@ -48,7 +48,7 @@ def test_built_for_sm100a_only():
 
 
 def test_status_strings(lib):
-    for code in range(-7, 1):
+    for code in range(-8, 1):
         assert ops.status_string(code) and ops.status_string(code) != "unknown status"
     assert ops.status_string(-99) == "unknown status"
     assert lib.mamba_abi_version() >= 100
@@ -188,3 +188,21 @@ def test_bwd_workspace_is_one_checkpoint_per_chunk(lib):
     assert ws(1, 3, 5, 65) == (1 * 3 * 2 * 5 * 4 + 255) // 256 * 256
     assert ws(2, 64, 16, 0) == 0
     assert ws(2, 64, 17, 8) == 0
+
+
+ERR_FLAGS = -8
+
+
+def test_ex_entry_points_reject_unknown_flags(lib):
+    vp = lambda v: None if v is None else ctypes.c_void_p(v)  # noqa: E731
+    scan_args = [vp(A16)] * 5 + [None, None, None, 1, vp(A16), None, _dims(), 0, 0, None, 0]
+    for flags in (2, 0x80000000, 3):
+        assert lib.mamba_selective_scan_fwd_ex(*scan_args, flags, None) == ERR_FLAGS
+    # known flags go on to the ordinary checks
+    assert lib.mamba_selective_scan_fwd_ex(*([None] + scan_args[1:]), 1, None) == ERR_NULL
+    assert lib.mamba_selective_scan_fwd_ex(*scan_args[:11], _dims(2, 64, 17, 8), 0, 0, None, 0,
+                                           1, None) == ERR_DIMS
+    upd = [vp(A16)] * 6 + [None, None, None, 1, vp(A16), 4, 64, 16, 1]
+    assert lib.mamba_selective_state_update_ex(*upd, 4, None) == ERR_FLAGS
+    assert lib.mamba_selective_state_update_ex(*([None] + upd[1:]), 1, None) == ERR_NULL
+    assert ops.status_string(ERR_FLAGS) == "unknown flag bits"
