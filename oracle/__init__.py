@@ -24,7 +24,8 @@ associative-combine prefix of ``oracle.pscan``, the LTI convolution form,
 Abar in (0,1), small/large-Delta limits, the gated-RNN special case.  The ZOH
 variant (tests/test_oracle_zoh.py): the gated-RNN identity, the continuous-time
 steady state -B u / A, numerical integration of the continuous ODE, the
-small-Delta limit and A = 0.
+small-Delta limit and A = 0.  The causal conv1d (tests/test_oracle_conv.py): numpy's
+convolution, the impulse response, causality, chunked prefill and decode steps.
 """
 from __future__ import annotations
 
@@ -78,6 +79,12 @@ def _load():
             lib.s6o_scan_backward.restype = ctypes.c_int
             lib.s6o_scan_backward.argtypes = ([ctypes.c_long] * 4 + [_dp] * 8 + [_lp, ctypes.c_int]
                                               + [_dp] * 9)
+            lib.s6o_causal_conv1d.restype = ctypes.c_int
+            lib.s6o_causal_conv1d.argtypes = [ctypes.c_long] * 3 + [_dp] * 4 + [ctypes.c_int,
+                                                                               _dp, _dp]
+            lib.s6o_causal_conv1d_update.restype = ctypes.c_int
+            lib.s6o_causal_conv1d_update.argtypes = [ctypes.c_long] * 2 + [_dp] * 4 + [
+                ctypes.c_int, _dp]
             lib.s6o_num_threads.restype = ctypes.c_int
             lib.s6o_num_threads.argtypes = []
             _lib = lib
@@ -280,3 +287,46 @@ def selective_scan_backward(u, delta, A, B, C, dy, D=None, z=None, delta_bias=No
                 dz=r["dz"].reshape(b, d, L), dA=r["dA"].reshape(b, d, N).sum(0),
                 dD=r["dD"].reshape(b, d).sum(0), dbias=r["dbias"].reshape(b, d).sum(0),
                 dB=r["dB"], dC=r["dC"])
+
+
+def causal_conv1d(x, weight, bias=None, initial_state=None, silu=True):
+    """Causal depthwise conv1d (+ SiLU) in the library's layouts.
+
+    x: (batch, dim, L); weight: (dim, K); bias: (dim) or None; initial_state:
+    (batch, dim, K-1) or None.  Returns out (batch, dim, L) and the final state
+    (batch, dim, K-1): the last K-1 inputs, oldest first."""
+    xx = _f64(x)
+    b, d, L = xx.shape
+    w = _f64(weight)
+    K = w.shape[1]
+    rows = b * d
+    wr = np.ascontiguousarray(np.tile(w, (b, 1)))
+    br = None if bias is None else np.ascontiguousarray(np.tile(_f64(bias), b))
+    init = None if initial_state is None else _f64(initial_state).reshape(rows, K - 1)
+    out = np.empty((rows, L))
+    fin = np.empty((rows, max(K - 1, 0)))
+    rc = _load().s6o_causal_conv1d(rows, L, K, _ptr(np.ascontiguousarray(xx.reshape(rows, L))),
+                                   _ptr(wr), _ptr(br), _ptr(init), int(bool(silu)), _ptr(out),
+                                   _ptr(fin) if K > 1 else None)
+    if rc != 0:
+        raise ValueError("s6o_causal_conv1d rejected its arguments")
+    return out.reshape(b, d, L), fin.reshape(b, d, K - 1)
+
+
+def causal_conv1d_update(state, x, weight, bias=None, silu=True):
+    """One decode token: returns (new_state (batch, dim, K-1), out (batch, dim)).
+    ``state`` is not modified."""
+    w = _f64(weight)
+    d, K = w.shape
+    xx = _f64(x)
+    b = xx.shape[0]
+    st = _f64(state).reshape(b * d, K - 1).copy() if K > 1 else np.empty((b * d, 0))
+    out = np.empty(b * d)
+    rc = _load().s6o_causal_conv1d_update(
+        b * d, K, _ptr(st) if K > 1 else None, _ptr(np.ascontiguousarray(xx.reshape(b * d))),
+        _ptr(np.ascontiguousarray(np.tile(w, (b, 1)))),
+        None if bias is None else _ptr(np.ascontiguousarray(np.tile(_f64(bias), b))),
+        int(bool(silu)), _ptr(out))
+    if rc != 0:
+        raise ValueError("s6o_causal_conv1d_update rejected its arguments")
+    return st.reshape(b, d, K - 1), out.reshape(b, d)

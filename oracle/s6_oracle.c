@@ -289,6 +289,78 @@ int s6o_scan_backward(long nlanes, long N, long L, long nbatch,
     return S6O_OK;
 }
 
+/*
+ * Causal depthwise 1-D convolution with an optional SiLU, per independent row (one
+ * (batch, channel) pair): the step the Mamba block applies to the projected input
+ * before the SSM (page 2 Q&A: a convolution first aggregates local context, an
+ * activation after it adds the non-linearity; page 4 "Mamba Block": input projections,
+ * a 1-D convolution, the selective SSM and multiplicative gating).
+ *
+ *   out[t] = act(bias + sum_{k=0}^{K-1} w[k] * x[t - (K-1) + k])
+ *
+ * Inputs before the sequence (t - (K-1) + k < 0) come from init, the K-1 inputs that
+ * precede it, oldest first (zero when init is NULL).  act is SiLU when silu != 0, the
+ * identity otherwise.  final, when not NULL, receives the last K-1 inputs of the
+ * extended sequence init ++ x, oldest first (the state decode continues from).
+ *
+ *   x, out : (nrows, L);  w : (nrows, K);  bias : (nrows) or NULL
+ *   init, final : (nrows, K-1) or NULL;  1 <= K <= 64
+ */
+int s6o_causal_conv1d(long nrows, long L, long K, const double* x, const double* w,
+                      const double* bias, const double* init, int silu_on, double* out,
+                      double* final_state) {
+    if (nrows < 0 || L < 0 || K < 1 || K > 64 || !w || (L > 0 && (!x || !out)))
+        return S6O_ERR_ARG;
+    for (long i = 0; i < nrows; ++i) {
+        const double* xi = x ? x + i * L : NULL;
+        for (long t = 0; t < L; ++t) {
+            double acc = bias ? bias[i] : 0.0;
+            for (long k = 0; k < K; ++k) {
+                long s = t - (K - 1) + k;  /* position in x; negative: before the sequence */
+                double v;
+                if (s >= 0)
+                    v = xi[s];
+                else
+                    v = init ? init[i * (K - 1) + (K - 1) + s] : 0.0;
+                acc += w[i * K + k] * v;
+            }
+            out[i * L + t] = silu_on ? silu(acc) : acc;
+        }
+        if (final_state) {
+            for (long k = 0; k < K - 1; ++k) {
+                long s = L - (K - 1) + k;
+                double v;
+                if (s >= 0)
+                    v = xi[s];
+                else
+                    v = init ? init[i * (K - 1) + (K - 1) + s] : 0.0;
+                final_state[i * (K - 1) + k] = v;
+            }
+        }
+    }
+    return S6O_OK;
+}
+
+/*
+ * One decode token of the same convolution: state (nrows, K-1) holds the previous K-1
+ * inputs, oldest first.  out = act(bias + sum_{k<K-1} w[k] state[k] + w[K-1] x); then
+ * the state drops its oldest input and appends x.
+ */
+int s6o_causal_conv1d_update(long nrows, long K, double* state, const double* x,
+                             const double* w, const double* bias, int silu_on, double* out) {
+    if (nrows < 0 || K < 1 || K > 64 || !x || !w || !out || (K > 1 && !state))
+        return S6O_ERR_ARG;
+    for (long i = 0; i < nrows; ++i) {
+        double acc = bias ? bias[i] : 0.0;
+        for (long k = 0; k < K - 1; ++k) acc += w[i * K + k] * state[i * (K - 1) + k];
+        acc += w[i * K + K - 1] * x[i];
+        out[i] = silu_on ? silu(acc) : acc;
+        for (long k = 0; k + 1 < K - 1; ++k) state[i * (K - 1) + k] = state[i * (K - 1) + k + 1];
+        if (K > 1) state[i * (K - 1) + K - 2] = x[i];
+    }
+    return S6O_OK;
+}
+
 /* Threads the OpenMP runtime would use for the parallel loops above. */
 #ifdef _OPENMP
 #include <omp.h>

@@ -16,6 +16,12 @@ million    1      2048   16     1048576     bf16 / bf16
 decode     256    5120   16     1 token x 1000 steps, fp32 state
 =========  =====  =====  =====  ==========  ===========================
 
+The causal conv1d producer (conv_inputs) draws, from its own seed, x ~ N(0, 1) with shape
+(batch, dim, L) in the storage dtype, then weight (dim, K) and bias (dim) ~ U(-1/sqrt(K),
+1/sqrt(K)) in fp32, then (when asked) an initial state (batch, dim, K - 1) ~ N(0, 1); the
+bench uses the m2p8b layer's shape (4, 5120, 4096), K = 4, bf16, seed 56010, and decode
+tokens of (256, 5120) from seed 56011.
+
 Recipe: u, delta_raw, z ~ N(0, 1) with shape (batch, dim, L); B, C ~ N(0, 1)
 with shape (batch, N, L), shared by all channels of a batch; A[d, n] = -(n + 1);
 D ~ N(0, 1) per channel; delta_bias = log(expm1(v)) with v ~ U[0.001, 0.1] per
@@ -166,3 +172,23 @@ def decode_tokens_batched(steps: int, w: DecodeWorkload = DECODE_WORKLOAD, devic
 def inverse_softplus_range():
     """The bias range the recipe produces: [log(expm1(0.001)), log(expm1(0.1))]."""
     return math.log(math.expm1(0.001)), math.log(math.expm1(0.1))
+
+
+CONV_WIDTH = 4
+CONV_SEED = 56010
+
+
+def conv_inputs(batch, dim, seqlen, width=CONV_WIDTH, dtype=torch.bfloat16, seed=CONV_SEED,
+                device="cpu", with_bias=True, with_initial_state=False):
+    """x (batch, dim, L), weight (dim, K), bias (dim) [, initial_state (batch, dim, K-1)]."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    x = torch.randn(batch, dim, seqlen, generator=g, dtype=torch.float32, device=device).to(dtype)
+    bound = 1.0 / math.sqrt(width)
+    w = (torch.rand(dim, width, generator=g, dtype=torch.float32, device=device) * 2 - 1) * bound
+    bias = (torch.rand(dim, generator=g, dtype=torch.float32, device=device) * 2 - 1) * bound
+    init = None
+    if with_initial_state:
+        init = torch.randn(batch, dim, width - 1, generator=g, dtype=torch.float32,
+                           device=device).to(dtype)
+    return dict(x=x, weight=w, bias=bias if with_bias else None, initial_state=init)
