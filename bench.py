@@ -14,6 +14,7 @@ used.  The same run measures the decode workload (selective_state_update,
 batch 256, dim 5120, N 16, 1000 fresh tokens, L2 flushed before each token),
 the backward of the same layer's scan (recomputing states from chunk
 checkpoints), the exact zero-order-hold variant of the scan and of decode, the
+causal conv1d + SiLU that produces the scan's input (and its decode update), the
 end-to-end path from pinned host buffers, the SM clocks during
 the timed region, and (rank 0, N = 1) the fp64 CPU oracle on bounded samples.
 
@@ -310,11 +311,14 @@ def run_ours(args, rank, world, local):
     zoh = run_zoh(g, dev, stream, world, w, steps=args.zoh_steps)
     del g
     torch.cuda.empty_cache()
+    conv = run_conv(dev, stream, world, rank, steps=args.conv_steps)
+    torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, budget_s=args.cpu_seconds)
         backward["cpu_baseline"] = cpu_baseline_backward(w, budget_s=args.cpu_seconds / 2)
+        conv["cpu_baseline"] = cpu_baseline_conv(budget_s=args.cpu_seconds / 4)
 
     line = {
         "metric": METRIC, "value": value, "unit": "elems/s", "n_gpus": world,
@@ -329,6 +333,7 @@ def run_ours(args, rank, world, local):
                    "parallelism": "replicas x%d (independent batches per GPU)" % world},
         "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
         "clocks": clocks, "decode": decode, "backward": backward, "exact_zoh": zoh,
+        "conv1d": conv,
         "cpu_baseline": cpu,
         "impl": "ours",
     }
@@ -408,6 +413,81 @@ def run_zoh(g, dev, stream, world, w, steps=50):
                                 "achieved": byts / (ms_tok * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
                                 "frac": byts / (ms_tok * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                 "peak_kind": kind}},
+        "gpu_launches": 2 * steps + 6,
+    }
+
+
+def run_conv(dev, stream, world, rank, steps=50):
+    """The causal conv1d + SiLU producing the m2p8b layer's u (4, 5120, 4096, K = 4, bf16),
+    per launch, and its decode update on (256, 5120) after an L2 flush."""
+    from selective_state_space_56_b200 import inputs, ops
+    b, d, L, K = 4, 5120, 4096, inputs.CONV_WIDTH
+    p = inputs.conv_inputs(b, d, L, K, torch.bfloat16, seed=rank_seed(inputs.CONV_SEED, rank),
+                           device=dev)
+    out = torch.empty_like(p["x"])
+    fin = torch.empty((b, d, K - 1), dtype=torch.bfloat16, device=dev)
+
+    def conv():
+        ops.causal_conv1d_fwd(p["x"], p["weight"], p["bias"], out=out)
+
+    for _ in range(3):
+        conv()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b_ in evs:
+        a.record(stream)
+        conv()
+        b_.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(statistics.fmean(a.elapsed_time(b_) for a, b_ in evs), world)
+    elems = b * d * L
+    byts = 2 * elems * 2 + d * K * 4 + d * 4  # x read, out written (bf16), weights, bias
+    peaks, kind = measured_peaks()
+    del out, fin
+
+    db, dd = 256, 5120
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(inputs.CONV_SEED + 1)
+    state = torch.randn((db, dd, K - 1), generator=gen, device=dev).to(torch.bfloat16)
+    xs = torch.randn((steps, db, dd), generator=gen, device=dev).to(torch.bfloat16)
+    wd, bd = p["weight"][:dd].contiguous(), p["bias"][:dd].contiguous()
+    yd = torch.empty((db, dd), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    for s_ in range(3):
+        ops.causal_conv1d_update(state, xs[s_], wd, bd, out=yd)
+    torch.cuda.synchronize(dev)
+    devs = []
+    for s_ in range(steps):
+        flush_l2(flush)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ops.causal_conv1d_update(state, xs[s_], wd, bd, out=yd)
+        b_.record(stream)
+        devs.append((a, b_))
+    torch.cuda.synchronize(dev)
+    ms_tok = max_over_ranks(statistics.fmean(a.elapsed_time(b_) for a, b_ in devs), world)
+    rows = db * dd
+    dbytes = rows * (2 * (K - 1) * 2 + 2 * 2) + dd * (K + 1) * 4
+    del p, state, xs, flush
+    return {
+        "metric": "causal conv1d + SiLU (b·d·L) elems/s", "unit": "elems/s",
+        "value": world * elems / (ms * 1e-3), "ms_per_call": ms, "steps": steps,
+        "workload": "x (4, 5120, 4096) bf16, weight (5120, 4) and bias fp32, SiLU: the "
+                    "producer of the m2p8b layer's u",
+        "roofline": {"bound": "hbm", "unit": "GB/s", "achieved": byts / (ms * 1e-3) / 1e9,
+                     "peak": peaks["hbm_gbs"], "frac": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "algorithmic_bytes": byts, "peak_kind": kind,
+                     "traffic": profile_traffic("conv1d_m2p8b.txt",
+                                                "selective_state_space_56_b200/csrc/conv1d.cu")},
+        "decode": {"ms_per_token_l2_flushed": ms_tok,
+                   "workload": "conv state (256, 5120, 3) bf16 updated in place, x and out "
+                               "(256, 5120) bf16",
+                   "roofline": {"bound": "hbm", "unit": "GB/s",
+                                "achieved": dbytes / (ms_tok * 1e-3) / 1e9,
+                                "peak": peaks["hbm_gbs"],
+                                "frac": dbytes / (ms_tok * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                "algorithmic_bytes": dbytes}},
         "gpu_launches": 2 * steps + 6,
     }
 
@@ -578,6 +658,25 @@ def cpu_baseline_backward(w, budget_s=5.0):
                 nl, w.batch * w.dim, w.seqlen, t)}
 
 
+def cpu_baseline_conv(budget_s=2.5):
+    """The fp64 oracle's causal conv1d as it stands, on a bounded channel sample of the
+    m2p8b producer workload."""
+    import oracle
+    from selective_state_space_56_b200 import inputs
+    p = inputs.conv_inputs(4, 5120, 4096, inputs.CONV_WIDTH, torch.bfloat16)
+
+    def run(nch):
+        t = time.perf_counter()
+        oracle.causal_conv1d(p["x"][:, :nch], p["weight"][:nch], p["bias"][:nch])
+        return time.perf_counter() - t
+
+    t = run(16)
+    nch = int(min(5120, max(16, 16 * budget_s / max(t, 1e-3))))
+    t = run(nch)
+    return {"value": 4 * nch * 4096 / t, "unit": "elems/s", "cores": 1, "kind": "oracle",
+            "sample": "4 x %d of 5120 channels x L=4096 (fp64, one thread), %.1f s" % (nch, t)}
+
+
 def run_reference(args, rank, world):
     from selective_state_space_56_b200 import inputs
     w = inputs.SCAN_WORKLOADS[WORKLOAD]
@@ -617,6 +716,10 @@ def profile_target(which):
         for _ in range(3):
             ops.selective_scan_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
                                    delta_bias=p["delta_bias"], y=y)
+    elif which == "conv":
+        p = inputs.conv_inputs(4, 5120, 4096, inputs.CONV_WIDTH, torch.bfloat16, device=dev)
+        for _ in range(3):
+            ops.causal_conv1d_fwd(p["x"], p["weight"], p["bias"])
     elif which == "backward":
         w = inputs.SCAN_WORKLOADS[WORKLOAD]
         p = inputs.scan_inputs(w.batch, w.dim, w.dstate, w.seqlen, w.in_dtype, w.seed, device=dev)
@@ -651,7 +754,8 @@ def main(argv=None):
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--backward-steps", type=int, default=50)
     ap.add_argument("--zoh-steps", type=int, default=50)
-    ap.add_argument("--profile", choices=["scan", "decode", "backward"],
+    ap.add_argument("--conv-steps", type=int, default=50)
+    ap.add_argument("--profile", choices=["scan", "decode", "backward", "conv"],
                     help="run a few untimed launches of one workload (an ncu capture target) "
                          "and exit")
     args = ap.parse_args(argv)

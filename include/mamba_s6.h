@@ -1,12 +1,13 @@
 /*
  * mamba_s6.h -- C ABI of the B200 (sm_100a) selective-scan library.
  *
- * Three operations, each a hand-written CUDA kernel sequence launched on the
- * caller's stream:
+ * Operations, each a hand-written CUDA kernel sequence launched on the caller's stream:
  *
  *   mamba_selective_scan_fwd      the fused S6 forward scan over a whole sequence
  *   mamba_selective_state_update  one decode token, updating a carried state in place
  *   mamba_selective_scan_bwd      gradients of the forward scan, states recomputed
+ *   mamba_causal_conv1d_fwd       the block's causal conv1d + SiLU producing the scan's u
+ *   mamba_causal_conv1d_update    its one-token decode step on a rolling conv state
  *
  * Definitions (Mamba: Linear-Time Sequence Modeling with Selective State Spaces,
  * page "xyznot.com/ar/paper/2312.00752", sections "Method", "Selection mechanism
@@ -233,6 +234,43 @@ int mamba_selective_scan_bwd(const void* u, const void* delta, const float* A, c
                              float* dD, float* ddelta_bias, mamba_scan_dims dims,
                              mamba_dtype in_dtype, void* workspace, size_t workspace_bytes,
                              void* stream);
+
+/*
+ * Causal depthwise conv1d with an optional SiLU: the Mamba block's step between the input
+ * projection and the SSM (Mamba, section "Mamba Block": input projections, a 1-D
+ * convolution, the selective SSM and gating; page "yongjin360.com/news/29389", Q&A on
+ * the convolution before the SSM and the activation after it).  Per (batch, channel) row:
+ *
+ *   out[t] = act(bias[d] + sum_{k=0}^{width-1} weight[d, k] * x[t - (width-1) + k])
+ *
+ * where positions before the sequence read initial_state (the width-1 preceding inputs,
+ * oldest first) or zero when it is NULL, and act is SiLU when silu != 0.
+ *
+ *   x, out        : (batch, dim, seqlen) dtype     out must not alias x
+ *   weight        : (dim, width) float32           1 <= width <= 4
+ *   bias          : (dim) float32 or NULL
+ *   initial_state : (batch, dim, width-1) dtype or NULL
+ *   final_state   : (batch, dim, width-1) dtype or NULL; receives the last width-1 inputs
+ *                   of initial_state ++ x, oldest first (the state decode continues from)
+ *   (with seqlen == 0, x and out may be NULL)
+ *
+ * fp32 arithmetic; results rounded to dtype.  Errors: NULL, DIMS, ALIGN, DTYPE, CUDA.
+ */
+int mamba_causal_conv1d_fwd(const void* x, const float* weight, const float* bias,
+                            const void* initial_state, void* out, void* final_state,
+                            int64_t batch, int64_t dim, int64_t seqlen, int width, int silu,
+                            mamba_dtype dtype, void* stream);
+
+/*
+ * One decode token of the convolution above: conv_state (batch, dim, width-1) holds the
+ * previous width-1 inputs, oldest first, and is updated in place (oldest dropped, x
+ * appended); out (batch, dim) = act(bias + weight . [conv_state, x]).  x, out: (batch,
+ * dim) dtype; conv_state may be NULL only when width == 1; batch <= 65535.
+ * Errors: NULL, DIMS, ALIGN, DTYPE, CUDA.
+ */
+int mamba_causal_conv1d_update(void* conv_state, const void* x, const float* weight,
+                               const float* bias, void* out, int64_t batch, int64_t dim,
+                               int width, int silu, mamba_dtype dtype, void* stream);
 
 /*
  * Reads the library's device error word on `stream`, synchronising that stream.

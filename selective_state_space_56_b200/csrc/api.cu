@@ -266,6 +266,60 @@ int mamba_selective_scan_bwd(const void* u, const void* delta, const float* A, c
                                                 static_cast<cudaStream_t>(stream)));
 }
 
+int mamba_causal_conv1d_fwd(const void* x, const float* weight, const float* bias,
+                            const void* initial_state, void* out, void* final_state,
+                            int64_t batch, int64_t dim, int64_t seqlen, int width, int silu,
+                            mamba_dtype dtype, void* stream) {
+    if (!weight || (seqlen > 0 && (!x || !out))) return MAMBA_ERR_NULL;
+    if (!dtype_ok(dtype)) return MAMBA_ERR_DTYPE;
+    if (width < 1 || width > 4 || batch < 1 || dim < 1 || seqlen < 0) return MAMBA_ERR_DIMS;
+    if (!mul_ok(batch, dim) || !mul_ok(batch * dim, seqlen > 0 ? seqlen : 1) ||
+        !mul_ok(batch * dim * (seqlen > 0 ? seqlen : 1), 8))
+        return MAMBA_ERR_DIMS;
+    const void* ptrs[] = {x, weight, bias, initial_state, out, final_state};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MAMBA_ERR_ALIGN;
+    s6::ConvArgs a;
+    a.x = x;
+    a.weight = weight;
+    a.bias = bias;
+    a.initial_state = width > 1 ? initial_state : nullptr;
+    a.out = out;
+    a.final_state = width > 1 ? final_state : nullptr;
+    a.batch = batch;
+    a.dim = dim;
+    a.L = seqlen;
+    a.width = width;
+    a.silu = silu;
+    a.dtype = to_dtype(dtype);
+    return cuda_status(s6::launch_conv1d(a, static_cast<cudaStream_t>(stream)));
+}
+
+int mamba_causal_conv1d_update(void* conv_state, const void* x, const float* weight,
+                               const float* bias, void* out, int64_t batch, int64_t dim,
+                               int width, int silu, mamba_dtype dtype, void* stream) {
+    if (!x || !weight || !out || (width > 1 && !conv_state)) return MAMBA_ERR_NULL;
+    if (!dtype_ok(dtype)) return MAMBA_ERR_DTYPE;
+    if (width < 1 || width > 4 || batch < 1 || dim < 1 || batch > kMaxGridYZ ||
+        !mul_ok(batch, dim) || !mul_ok(batch * dim, 8))
+        return MAMBA_ERR_DIMS;
+    const void* ptrs[] = {conv_state, x, weight, bias, out};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MAMBA_ERR_ALIGN;
+    s6::ConvUpdateArgs a;
+    a.state = conv_state;
+    a.x = x;
+    a.weight = weight;
+    a.bias = bias;
+    a.out = out;
+    a.batch = batch;
+    a.dim = dim;
+    a.width = width;
+    a.silu = silu;
+    a.dtype = to_dtype(dtype);
+    return cuda_status(s6::launch_conv1d_update(a, static_cast<cudaStream_t>(stream)));
+}
+
 int mamba_check_device_error(int clear, void* stream) {
     unsigned word = 0;
     if (s6::read_device_error(&word, clear != 0, static_cast<cudaStream_t>(stream)) != cudaSuccess)
@@ -288,6 +342,6 @@ const char* mamba_status_string(int status) {
     }
 }
 
-int mamba_abi_version(void) { return 102; }
+int mamba_abi_version(void) { return 103; }
 
 }  // extern "C"

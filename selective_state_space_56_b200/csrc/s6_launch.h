@@ -87,6 +87,35 @@ struct BackwardArgs {
 cudaError_t launch_scan_backward(const ScanArgs& a, const BackwardArgs& g, float* ckpt,
                                  cudaStream_t stream);
 
+// Causal depthwise conv1d (+ SiLU) over (batch, dim, L) rows, 1 <= width <= 4.
+struct ConvArgs {
+    const void* x;
+    const float* weight;        // (dim, width)
+    const float* bias;          // (dim) or null
+    const void* initial_state;  // (batch, dim, width - 1) or null
+    void* out;
+    void* final_state;          // (batch, dim, width - 1) or null
+    int64_t batch, dim, L;
+    int width;
+    int silu;
+    DType dtype;
+};
+
+struct ConvUpdateArgs {
+    void* state;  // (batch, dim, width - 1), updated in place
+    const void* x;
+    const float* weight;
+    const float* bias;
+    void* out;
+    int64_t batch, dim;
+    int width;
+    int silu;
+    DType dtype;
+};
+
+cudaError_t launch_conv1d(const ConvArgs& a, cudaStream_t stream);
+cudaError_t launch_conv1d_update(const ConvUpdateArgs& a, cudaStream_t stream);
+
 // Reads (and optionally clears) the device error word on `stream`, synchronising it.
 // Bit 0: a bounded device-side wait gave up.
 cudaError_t read_device_error(unsigned* out, bool clear, cudaStream_t stream);

@@ -66,6 +66,10 @@ def load_library():
             lib.mamba_selective_state_update_ex.restype = i32
             lib.mamba_selective_state_update_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                                             i32, vp, i64, i64, i64, i32, u32, vp]
+            lib.mamba_causal_conv1d_fwd.restype = i32
+            lib.mamba_causal_conv1d_fwd.argtypes = [vp] * 6 + [i64, i64, i64, i32, i32, i32, vp]
+            lib.mamba_causal_conv1d_update.restype = i32
+            lib.mamba_causal_conv1d_update.argtypes = [vp] * 5 + [i64, i64, i32, i32, i32, vp]
             lib.mamba_selective_state_update.restype = i32
             lib.mamba_selective_state_update.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
                                                          vp, i64, i64, i64, i32, vp]
@@ -286,3 +290,68 @@ def selective_state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=
     if rc != 0:
         raise MambaError(rc, "mamba_selective_state_update")
     return y
+
+
+def causal_conv1d_fwd(x, weight, bias=None, initial_state=None, silu=True, out=None,
+                      return_final_state=False):
+    """Causal depthwise conv1d (+ SiLU).  x: (batch, dim, L) bf16/fp32; weight: (dim, K)
+    fp32, 1 <= K <= 4; bias: (dim) fp32; initial_state: (batch, dim, K-1) x.dtype.
+    Returns out (batch, dim, L) [and the final state (batch, dim, K-1)]."""
+    if not isinstance(x, torch.Tensor) or x.dim() != 3:
+        raise ValueError("x must be a (batch, dim, L) tensor")
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("causal_conv1d_fwd runs on CUDA tensors only")
+    b, d, L = x.shape
+    K = weight.shape[1] if weight.dim() == 2 else -1
+    dt = x.dtype
+    if dt not in _DTYPES:
+        raise ValueError("unsupported dtype %s" % dt)
+    _check(x, "x", dev, (b, d, L), (dt,))
+    _check(weight, "weight", dev, (d, K), (torch.float32,))
+    _check(bias, "bias", dev, (d,), (torch.float32,))
+    _check(initial_state, "initial_state", dev, (b, d, K - 1), (dt,))
+    if out is None:
+        out = torch.empty((b, d, L), dtype=dt, device=dev)
+    _check(out, "out", dev, (b, d, L), (dt,))
+    fin = None
+    if return_final_state and K > 1:
+        fin = torch.empty((b, d, K - 1), dtype=dt, device=dev)
+    with torch.cuda.device(dev):
+        rc = load_library().mamba_causal_conv1d_fwd(
+            _ptr(x), _ptr(weight), _ptr(bias), _ptr(initial_state), _ptr(out), _ptr(fin),
+            b, d, L, K, int(bool(silu)), _DTYPES[dt], _stream_handle(dev))
+    if rc != 0:
+        raise MambaError(rc, "mamba_causal_conv1d_fwd")
+    if return_final_state:
+        return out, fin
+    return out
+
+
+def causal_conv1d_update(conv_state, x, weight, bias=None, silu=True, out=None):
+    """One decode token: conv_state (batch, dim, K-1) is updated in place; x (batch, dim).
+    Returns out (batch, dim)."""
+    if not isinstance(x, torch.Tensor) or x.dim() != 2:
+        raise ValueError("x must be a (batch, dim) tensor")
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("causal_conv1d_update runs on CUDA tensors only")
+    b, d = x.shape
+    K = weight.shape[1] if weight.dim() == 2 else -1
+    dt = x.dtype
+    if dt not in _DTYPES:
+        raise ValueError("unsupported dtype %s" % dt)
+    _check(x, "x", dev, (b, d), (dt,))
+    _check(weight, "weight", dev, (d, K), (torch.float32,))
+    _check(bias, "bias", dev, (d,), (torch.float32,))
+    _check(conv_state, "conv_state", dev, (b, d, K - 1), (dt,))
+    if out is None:
+        out = torch.empty((b, d), dtype=dt, device=dev)
+    _check(out, "out", dev, (b, d), (dt,))
+    with torch.cuda.device(dev):
+        rc = load_library().mamba_causal_conv1d_update(
+            _ptr(conv_state), _ptr(x), _ptr(weight), _ptr(bias), _ptr(out), b, d, K,
+            int(bool(silu)), _DTYPES[dt], _stream_handle(dev))
+    if rc != 0:
+        raise MambaError(rc, "mamba_causal_conv1d_update")
+    return out

@@ -206,3 +206,30 @@ def test_ex_entry_points_reject_unknown_flags(lib):
     assert lib.mamba_selective_state_update_ex(*upd, 4, None) == ERR_FLAGS
     assert lib.mamba_selective_state_update_ex(*([None] + upd[1:]), 1, None) == ERR_NULL
     assert ops.status_string(ERR_FLAGS) == "unknown flag bits"
+
+
+def _conv(lib, **kw):
+    args = dict(x=A16, w=A16, bias=None, init=None, out=A16, fin=None, b=2, d=64, L=128, K=4,
+                silu=1, dt=1)
+    args.update(kw)
+    vp = lambda v: None if v is None else ctypes.c_void_p(v)  # noqa: E731
+    return lib.mamba_causal_conv1d_fwd(vp(args["x"]), vp(args["w"]), vp(args["bias"]),
+                                       vp(args["init"]), vp(args["out"]), vp(args["fin"]),
+                                       args["b"], args["d"], args["L"], args["K"], args["silu"],
+                                       args["dt"], None)
+
+
+def test_conv1d_host_checks(lib):
+    for f in ("x", "w", "out"):
+        assert _conv(lib, **{f: None}) == ERR_NULL, f
+    for kw in (dict(K=0), dict(K=5), dict(b=0), dict(d=0), dict(L=-1)):
+        assert _conv(lib, **kw) == ERR_DIMS, kw
+    assert _conv(lib, dt=2) == ERR_DTYPE
+    for f in ("x", "w", "bias", "init", "out", "fin"):
+        assert _conv(lib, **{f: A16 + 2}) == ERR_ALIGN, f
+    vp = ctypes.c_void_p
+    upd = lib.mamba_causal_conv1d_update
+    assert upd(None, vp(A16), vp(A16), None, vp(A16), 2, 64, 4, 1, 1, None) == ERR_NULL
+    assert upd(vp(A16), vp(A16), vp(A16), None, vp(A16), 2, 64, 7, 1, 1, None) == ERR_DIMS
+    assert upd(vp(A16), vp(A16), vp(A16), None, vp(A16), 70000, 4, 4, 1, 1, None) == ERR_DIMS
+    assert upd(vp(A16), vp(A16 + 4), vp(A16), None, vp(A16), 2, 64, 4, 1, 1, None) == ERR_ALIGN
