@@ -14,8 +14,8 @@ used.  The same run measures the decode workload (selective_state_update,
 batch 256, dim 5120, N 16, 1000 fresh tokens, L2 flushed before each token),
 the backward of the same layer's scan (recomputing states from chunk
 checkpoints), the exact zero-order-hold variant of the scan and of decode, the
-causal conv1d + SiLU that produces the scan's input (and its decode update), the
-end-to-end path from pinned host buffers, the SM clocks during
+causal conv1d + SiLU that produces the scan's input (and its decode update), with
+N > 1 the million-length layer split along L over the ranks, the end-to-end path from pinned host buffers, the SM clocks during
 the timed region, and (rank 0, N = 1) the fp64 CPU oracle on bounded samples.
 
 ``--impl reference`` times the CPU oracle itself as the reference arm.
@@ -313,6 +313,13 @@ def run_ours(args, rank, world, local):
     torch.cuda.empty_cache()
     conv = run_conv(dev, stream, world, rank, steps=args.conv_steps)
     torch.cuda.empty_cache()
+    lshard = None
+    if world > 1:
+        try:
+            lshard = run_lshard(dev, stream, world, rank, steps=args.lshard_steps)
+        except Exception as e:  # reported, not fatal: the headline line must still print
+            lshard = {"error": "%s: %s" % (type(e).__name__, str(e)[:200])}
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -333,7 +340,7 @@ def run_ours(args, rank, world, local):
                    "parallelism": "replicas x%d (independent batches per GPU)" % world},
         "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
         "clocks": clocks, "decode": decode, "backward": backward, "exact_zoh": zoh,
-        "conv1d": conv,
+        "conv1d": conv, "lshard": lshard,
         "cpu_baseline": cpu,
         "impl": "ours",
     }
@@ -490,6 +497,42 @@ def run_conv(dev, stream, world, rank, steps=50):
                                 "algorithmic_bytes": dbytes}},
         "gpu_launches": 2 * steps + 6,
     }
+
+
+def run_lshard(dev, stream, world, rank, steps=5):
+    """The million-length layer (1, 2048, 16, 2^20, bf16) split along L over the ranks:
+    each rank scans its consecutive shard after one all-gather of segment summaries
+    (strong scaling: the whole sequence per step)."""
+    from selective_state_space_56_b200 import inputs, sharded
+    import torch.distributed as dist
+    w = inputs.SCAN_WORKLOADS["million"]
+    Ls = w.seqlen // world
+    p = inputs.scan_inputs(w.batch, w.dim, w.dstate, Ls, w.in_dtype,
+                           rank_seed(w.seed + 100, rank), device=dev)
+
+    def step():
+        return sharded.sharded_selective_scan_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"],
+                                                  D=p["D"], z=p["z"], delta_bias=p["delta_bias"])
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b_.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    ms = max_over_ranks(a.elapsed_time(b_) / steps, world)
+    elems = w.batch * w.dim * w.seqlen
+    del p
+    return {"metric": "L-sharded selective-scan fwd (b·d·L) elems/s", "unit": "elems/s",
+            "value": elems / (ms * 1e-3), "ms_per_step": ms, "steps": steps,
+            "scaling": "strong", "n_gpus": world,
+            "workload": "million-length layer (1, 2048, 16, 2^20) bf16, %d steps per rank, one "
+                        "all-gather of b*d*(N+1) fp32 summaries per step" % Ls}
 
 
 def run_backward(g, dev, stream, world, w, steps=50):
@@ -755,6 +798,7 @@ def main(argv=None):
     ap.add_argument("--backward-steps", type=int, default=50)
     ap.add_argument("--zoh-steps", type=int, default=50)
     ap.add_argument("--conv-steps", type=int, default=50)
+    ap.add_argument("--lshard-steps", type=int, default=5)
     ap.add_argument("--profile", choices=["scan", "decode", "backward", "conv"],
                     help="run a few untimed launches of one workload (an ncu capture target) "
                          "and exit")

@@ -130,6 +130,61 @@ int mamba_selective_scan_fwd_ex(const void* u, const void* delta, const float* A
                                 unsigned flags, void* stream);
 
 /*
+ * mamba_selective_scan_fwd_ex starting from a given state instead of h_{-1} = 0.
+ *
+ *   initial_state : (batch, dim, dstate) float32, required; read only
+ *
+ * Everything else as mamba_selective_scan_fwd_ex (last_state receives the state after
+ * the sequence; with seqlen == 0 that is initial_state).  With the two calls below this
+ * lets a sequence be split over devices: the segment of device r starts from the fold of
+ * the summaries of segments 0..r-1.
+ */
+int mamba_selective_scan_fwd_init(const void* u, const void* delta, const float* A,
+                                  const void* B, const void* C, const float* D, const void* z,
+                                  const float* delta_bias, int delta_softplus,
+                                  const float* initial_state, void* y, float* last_state,
+                                  mamba_scan_dims dims, mamba_dtype in_dtype,
+                                  mamba_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                  unsigned flags, void* stream);
+
+/*
+ * Summary of a sequence (segment) for the associative combine of the parallel-scan
+ * derivation (page "yongjin360.com/news/29389", steps 1-4): the segment as one
+ * transformation T = (prod_t Abar_t, h_end) with h_end the state after the segment from
+ * h = 0.  For the diagonal A, prod_t Abar_t,n = exp(A_n * sum_t Delta_t), so the summary is
+ *
+ *   h_end     : (batch, dim, dstate) float32   state after the segment from zero
+ *   delta_sum : (batch, dim) float32           sum over the segment of Delta_t
+ *
+ * Inputs as mamba_selective_scan_fwd (D and z do not enter the state and are not taken).
+ * workspace: at least mamba_selective_scan_workspace_size(dims) bytes (long segments with
+ * few channels are themselves split).  flags: MAMBA_FLAG_EXACT_ZOH or 0.
+ * Errors: NULL, DIMS, ALIGN, DTYPE, WORKSPACE, FLAGS, CUDA.
+ */
+int mamba_selective_scan_summary(const void* u, const void* delta, const float* A, const void* B,
+                                 const void* C, const float* delta_bias, int delta_softplus,
+                                 float* h_end, float* delta_sum, mamba_scan_dims dims,
+                                 mamba_dtype in_dtype, void* workspace, size_t workspace_bytes,
+                                 unsigned flags, void* stream);
+
+/*
+ * Applies `count` consecutive segment summaries, in order, to h0 (NULL = zero): the
+ * combine (prod Abar_j, h_j) (+) state = prod Abar_j * state + h_j, folded left to right
+ * (page "yongjin360.com/news/29389", steps 2-4).
+ *
+ *   h_ends     : (count, batch, dim, dstate) float32     summaries' end states
+ *   delta_sums : (count, batch, dim) float32             summaries' summed steps
+ *   A          : (dim, dstate) float32
+ *   h_out      : (batch, dim, dstate) float32            the state after the segments
+ *   delta_sum_out : (batch, dim) float32 or NULL         the total summed step
+ *
+ * count == 0 gives h_out = h0 (or zero).  Errors: NULL, DIMS, ALIGN, CUDA.
+ */
+int mamba_selective_scan_fold(const float* h_ends, const float* delta_sums, const float* A,
+                              const float* h0, int64_t count, int64_t batch, int64_t dim,
+                              int64_t dstate, float* h_out, float* delta_sum_out, void* stream);
+
+/*
  * One decode token (selective_state_update): the recurrence above for a single
  * t, applied in place to a carried state (the generation mode keeps only a
  * fixed dim x dstate state per layer and costs O(1) per token).

@@ -38,9 +38,10 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_
 constexpr unsigned kKnownFlags = MAMBA_FLAG_EXACT_ZOH;
 
 int scan_fwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
-             const float* D, const void* z, const float* delta_bias, int delta_softplus, void* y,
-             float* last_state, mamba_scan_dims dims, mamba_dtype in_dtype, mamba_dtype out_dtype,
-             void* workspace, size_t workspace_bytes, unsigned flags, void* stream);
+             const float* D, const void* z, const float* delta_bias, int delta_softplus,
+             const float* h0, void* y, float* last_state, mamba_scan_dims dims,
+             mamba_dtype in_dtype, mamba_dtype out_dtype, void* workspace,
+             size_t workspace_bytes, unsigned flags, void* stream);
 
 int state_update(float* state, const void* u, const void* delta, const float* A, const void* B,
                  const void* C, const float* D, const void* z, const float* delta_bias,
@@ -68,8 +69,8 @@ int mamba_selective_scan_fwd(const void* u, const void* delta, const float* A, c
                              float* last_state, mamba_scan_dims dims, mamba_dtype in_dtype,
                              mamba_dtype out_dtype, void* workspace, size_t workspace_bytes,
                              void* stream) {
-    return scan_fwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, last_state, dims,
-                    in_dtype, out_dtype, workspace, workspace_bytes, 0u, stream);
+    return scan_fwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, y, last_state,
+                    dims, in_dtype, out_dtype, workspace, workspace_bytes, 0u, stream);
 }
 
 int mamba_selective_scan_fwd_ex(const void* u, const void* delta, const float* A, const void* B,
@@ -78,8 +79,87 @@ int mamba_selective_scan_fwd_ex(const void* u, const void* delta, const float* A
                                 float* last_state, mamba_scan_dims dims, mamba_dtype in_dtype,
                                 mamba_dtype out_dtype, void* workspace, size_t workspace_bytes,
                                 unsigned flags, void* stream) {
-    return scan_fwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, y, last_state, dims,
-                    in_dtype, out_dtype, workspace, workspace_bytes, flags, stream);
+    return scan_fwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, y, last_state,
+                    dims, in_dtype, out_dtype, workspace, workspace_bytes, flags, stream);
+}
+
+int mamba_selective_scan_fwd_init(const void* u, const void* delta, const float* A,
+                                  const void* B, const void* C, const float* D, const void* z,
+                                  const float* delta_bias, int delta_softplus,
+                                  const float* initial_state, void* y, float* last_state,
+                                  mamba_scan_dims dims, mamba_dtype in_dtype,
+                                  mamba_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                  unsigned flags, void* stream) {
+    if (!initial_state) return MAMBA_ERR_NULL;
+    return scan_fwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, initial_state, y,
+                    last_state, dims, in_dtype, out_dtype, workspace, workspace_bytes, flags,
+                    stream);
+}
+
+int mamba_selective_scan_summary(const void* u, const void* delta, const float* A, const void* B,
+                                 const void* C, const float* delta_bias, int delta_softplus,
+                                 float* h_end, float* delta_sum, mamba_scan_dims dims,
+                                 mamba_dtype in_dtype, void* workspace, size_t workspace_bytes,
+                                 unsigned flags, void* stream) {
+    if (flags & ~kKnownFlags) return MAMBA_ERR_FLAGS;
+    const bool empty = dims.seqlen == 0;
+    if (!A || !h_end || !delta_sum || (!empty && (!u || !delta || !B || !C)))
+        return MAMBA_ERR_NULL;
+    if (!dtype_ok(in_dtype)) return MAMBA_ERR_DTYPE;
+    if (!dims_ok(dims.batch, dims.dim, dims.dstate, dims.seqlen)) return MAMBA_ERR_DIMS;
+    const void* ptrs[] = {u, delta, A, B, C, delta_bias, h_end, delta_sum};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MAMBA_ERR_ALIGN;
+    int64_t nseg = 1, seg_len = 0;
+    s6::plan_segments(dims.batch, dims.dim, dims.seqlen, &nseg, &seg_len);
+    if (nseg > kMaxGridYZ) return MAMBA_ERR_DIMS;
+    const size_t need = mamba_selective_scan_workspace_size(dims);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need) return MAMBA_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return MAMBA_ERR_ALIGN;
+    }
+    s6::ScanArgs a;
+    a.u = u;
+    a.delta = delta;
+    a.z = nullptr;
+    a.A = A;
+    a.B = B;
+    a.C = C;
+    a.D = nullptr;
+    a.delta_bias = delta_bias;
+    a.y = nullptr;
+    a.last_state = nullptr;
+    a.batch = dims.batch;
+    a.dim = dims.dim;
+    a.N = dims.dstate;
+    a.L = dims.seqlen;
+    a.softplus = delta_softplus;
+    a.zoh = (flags & MAMBA_FLAG_EXACT_ZOH) ? 1 : 0;
+    a.in_dtype = to_dtype(in_dtype);
+    a.out_dtype = a.in_dtype;
+    a.nseg = nseg;
+    a.seg_len = seg_len;
+    a.seg_h = nullptr;
+    a.seg_sum = nullptr;
+    a.h0 = nullptr;
+    if (nseg > 1) {
+        a.seg_h = static_cast<float*>(workspace);
+        a.seg_sum = a.seg_h + nseg * dims.batch * dims.dim * dims.dstate;
+    }
+    return cuda_status(s6::launch_scan_summary(a, h_end, delta_sum, static_cast<cudaStream_t>(stream)));
+}
+
+int mamba_selective_scan_fold(const float* h_ends, const float* delta_sums, const float* A,
+                              const float* h0, int64_t count, int64_t batch, int64_t dim,
+                              int64_t dstate, float* h_out, float* delta_sum_out, void* stream) {
+    if (!A || !h_out || (count > 0 && (!h_ends || !delta_sums))) return MAMBA_ERR_NULL;
+    if (count < 0 || !dims_ok(batch, dim, dstate, 0) || !mul_ok(batch * dim * dstate, count + 1))
+        return MAMBA_ERR_DIMS;
+    const void* ptrs[] = {h_ends, delta_sums, A, h0, h_out, delta_sum_out};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MAMBA_ERR_ALIGN;
+    return cuda_status(s6::launch_fold(h_ends, delta_sums, A, h0, count, batch, dim, dstate, h_out,
+                                       delta_sum_out, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"
@@ -87,9 +167,10 @@ int mamba_selective_scan_fwd_ex(const void* u, const void* delta, const float* A
 namespace {
 
 int scan_fwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
-             const float* D, const void* z, const float* delta_bias, int delta_softplus, void* y,
-             float* last_state, mamba_scan_dims dims, mamba_dtype in_dtype, mamba_dtype out_dtype,
-             void* workspace, size_t workspace_bytes, unsigned flags, void* stream) {
+             const float* D, const void* z, const float* delta_bias, int delta_softplus,
+             const float* h0, void* y, float* last_state, mamba_scan_dims dims,
+             mamba_dtype in_dtype, mamba_dtype out_dtype, void* workspace,
+             size_t workspace_bytes, unsigned flags, void* stream) {
     if (flags & ~kKnownFlags) return MAMBA_ERR_FLAGS;
     // With seqlen == 0 the (batch, dim, 0) and (batch, dstate, 0) arrays are empty and
     // may be NULL; only last_state (zeros) is written.
@@ -97,7 +178,7 @@ int scan_fwd(const void* u, const void* delta, const float* A, const void* B, co
     if (!A || (!empty && (!u || !delta || !B || !C || !y))) return MAMBA_ERR_NULL;
     if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return MAMBA_ERR_DTYPE;
     if (!dims_ok(dims.batch, dims.dim, dims.dstate, dims.seqlen)) return MAMBA_ERR_DIMS;
-    const void* ptrs[] = {u, delta, A, B, C, D, z, delta_bias, y, last_state};
+    const void* ptrs[] = {u, delta, A, B, C, D, z, delta_bias, y, last_state, h0};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return MAMBA_ERR_ALIGN;
 
@@ -133,6 +214,7 @@ int scan_fwd(const void* u, const void* delta, const float* A, const void* B, co
     a.seg_len = seg_len;
     a.seg_h = nullptr;
     a.seg_sum = nullptr;
+    a.h0 = h0;
     if (nseg > 1) {
         a.seg_h = static_cast<float*>(workspace);
         a.seg_sum = a.seg_h + nseg * dims.batch * dims.dim * dims.dstate;
@@ -252,6 +334,7 @@ int mamba_selective_scan_bwd(const void* u, const void* delta, const float* A, c
     a.seg_len = dims.seqlen;
     a.seg_h = nullptr;
     a.seg_sum = nullptr;
+    a.h0 = nullptr;
     s6::BackwardArgs g;
     g.dy = dy;
     g.du = du;
@@ -342,6 +425,6 @@ const char* mamba_status_string(int status) {
     }
 }
 
-int mamba_abi_version(void) { return 103; }
+int mamba_abi_version(void) { return 104; }
 
 }  // extern "C"

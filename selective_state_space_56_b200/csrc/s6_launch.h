@@ -28,6 +28,7 @@ struct ScanArgs {
     int64_t nseg, seg_len;
     float* seg_h;    // (nseg, batch, dim, N)
     float* seg_sum;  // (nseg, batch, dim)
+    const float* h0;  // (batch, dim, N) initial state or null (zero)
 };
 
 struct StateUpdateArgs {
@@ -57,6 +58,17 @@ void plan_segments(int64_t batch, int64_t dim, int64_t L, int64_t* nseg, int64_t
 // Each returns a cudaError_t from the launches (cudaSuccess when all were enqueued).
 cudaError_t launch_scan(const ScanArgs& a, cudaStream_t stream);
 cudaError_t launch_state_update(const StateUpdateArgs& a, cudaStream_t stream);
+
+// Summary of the whole sequence in `a` (its plan's segments folded): the end state from
+// h = 0 into h_end (batch, dim, N) and the summed step into dsum (batch, dim).  With
+// a.nseg > 1 the segment aggregates go through a.seg_h / a.seg_sum.
+cudaError_t launch_scan_summary(const ScanArgs& a, float* h_end, float* dsum, cudaStream_t stream);
+
+// Inclusive fold of `count` summaries (hend (count, batch, dim, N), dsum (count, batch, dim))
+// applied to h0 (or zero): the state after them and (when dsum_out) their total step.
+cudaError_t launch_fold(const float* hend, const float* dsum, const float* A, const float* h0,
+                        int64_t count, int64_t batch, int64_t dim, int64_t N, float* h_out,
+                        float* dsum_out, cudaStream_t stream);
 
 // Steps per chunk of the forward kernel for state width N (the backward recomputes
 // states chunk by chunk from checkpoints taken at these boundaries).

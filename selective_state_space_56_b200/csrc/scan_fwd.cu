@@ -235,7 +235,8 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
             const int nn = pp * NS + j + q;
             const bool ok = dch < p.dim && nn < p.N;
             a[q] = ok ? p.A[dch * p.N + nn] * kLog2e : 0.f;  // padded states: Abar = 1, b = 0
-            h[q] = (MODE == kFull && p.nseg > 1 && ok)
+            // initial state: the segment's start (split sequences) or the caller's h0
+            h[q] = (MODE == kFull && p.seg_h != nullptr && ok)
                        ? p.seg_h[(((int64_t)seg * p.batch + b) * p.dim + dch) * p.N + nn]
                        : 0.f;
         }
@@ -590,9 +591,10 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
 
 // Fold the segments left to right.  Thread per (batch, channel, state):
 // on entry seg_h[s] holds segment s's end state from h = 0 (s < nseg - 1) and
-// seg_sum[s] its summed step; on exit seg_h[s] holds segment s's true start state.
+// seg_sum[s] its summed step; on exit seg_h[s] holds segment s's true start state
+// (segment 0 starts from h0, or from zero when h0 is null).
 __global__ void carry_kernel(float* seg_h, const float* seg_sum, const float* A, int64_t batch,
-                             int64_t dim, int N, int nseg) {
+                             int64_t dim, int N, int nseg, const float* h0) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t lanes = batch * dim * N;
     if (i >= lanes) return;
@@ -600,7 +602,7 @@ __global__ void carry_kernel(float* seg_h, const float* seg_sum, const float* A,
     const int64_t bd = i / N;
     const int64_t d = bd % dim;
     const float a2 = A[d * N + n] * kLog2e;
-    float H = 0.f;
+    float H = h0 ? h0[bd * N + n] : 0.f;
     for (int s = 0; s < nseg - 1; ++s) {
         const int64_t row = (int64_t)s * batch * dim + bd;
         const float hend = seg_h[row * N + n];
@@ -608,6 +610,30 @@ __global__ void carry_kernel(float* seg_h, const float* seg_sum, const float* A,
         H = fmaf(ex2(a2 * seg_sum[row]), H, hend);  // (prod Abar, h_end) (+) (., H)
     }
     seg_h[((int64_t)(nseg - 1) * batch * dim + bd) * N + n] = H;
+}
+
+// Inclusive fold of `count` segment summaries (h_end from zero, summed step) applied to h0:
+// h_out = the state after all of them, dsum_out = their total step.  Thread per
+// (batch, channel, state); the pair (exp(A * dsum), h_end) is the associative combine's
+// element, so folding consecutive summaries is applying them in order.
+__global__ void fold_kernel(const float* hend, const float* dsum, const float* A, const float* h0,
+                            int64_t count, int64_t batch, int64_t dim, int N, float* h_out,
+                            float* dsum_out) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t lanes = batch * dim * N;
+    if (i >= lanes) return;
+    const int n = (int)(i % N);
+    const int64_t bd = i / N;
+    const int64_t d = bd % dim;
+    const float a2 = A[d * N + n] * kLog2e;
+    float H = h0 ? h0[bd * N + n] : 0.f, S = 0.f;
+    for (int64_t s = 0; s < count; ++s) {
+        const int64_t row = s * batch * dim + bd;
+        H = fmaf(ex2(a2 * dsum[row]), H, hend[row * N + n]);
+        S += dsum[row];
+    }
+    h_out[bd * N + n] = H;
+    if (dsum_out && n == 0) dsum_out[bd] = S;
 }
 
 // ---- host side ---------------------------------------------------------------------------
@@ -677,7 +703,7 @@ cudaError_t launch_typed(const ScanArgs& a, const KParams& kp, const TMaps& tm, 
         if (e != cudaSuccess) return e;
         const int64_t lanes = a.batch * a.dim * a.N;
         carry_kernel<<<(unsigned)((lanes + 255) / 256), 256, 0, s>>>(
-            a.seg_h, a.seg_sum, a.A, a.batch, a.dim, (int)a.N, (int)a.nseg);
+            a.seg_h, a.seg_sum, a.A, a.batch, a.dim, (int)a.N, (int)a.nseg, a.h0);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -738,6 +764,41 @@ cudaError_t launch_ckpt_io(const ScanArgs& a, KParams kp, cudaStream_t s) {
     return launch_ckpt_typed<NMAX, Tin, true>(a, kp, tm, s);
 }
 
+// Segment summaries: kAggregate over `nseg` segments (all of them) into seg_h / seg_sum.
+template <int NMAX, typename Tin, bool ZOH>
+cudaError_t launch_summary_io(const ScanArgs& a, KParams kp, cudaStream_t s) {
+    using TL = Tile<NMAX>;
+    using Lo = Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin>;
+    TMaps tm;
+    memset(&tm, 0, sizeof(tm));
+    kp.y_tma = 0;
+    const unsigned gx = (unsigned)((a.dim + Lo::CH - 1) / Lo::CH);
+    const dim3 grid(gx, (unsigned)a.batch, (unsigned)a.nseg);
+    const bool rows16 = (a.L * (int64_t)sizeof(Tin)) % 16 == 0 && a.L > 0;
+    const bool fits = a.L < (1LL << 31) && a.dim < (1LL << 31) && a.batch < (1LL << 31);
+    if (!(rows16 && fits))
+        return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kAggregate, false, ZOH>(kp, tm, grid, s);
+    const bool ok = encode_3d<Tin>(&tm.u, a.u, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
+                    encode_3d<Tin>(&tm.dr, a.delta, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
+                    encode_3d<Tin>(&tm.B, a.B, a.L, a.N, a.batch, Lo::T, NMAX) &&
+                    encode_3d<Tin>(&tm.C, a.C, a.L, a.N, a.batch, Lo::T, NMAX);
+    if (!ok) return cudaErrorInvalidValue;
+    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kAggregate, true, ZOH>(kp, tm, grid, s);
+}
+
+template <int NMAX, bool ZOH>
+cudaError_t launch_summary_n(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
+    return a.in_dtype == DType::BF16 ? launch_summary_io<NMAX, __nv_bfloat16, ZOH>(a, kp, s)
+                                     : launch_summary_io<NMAX, float, ZOH>(a, kp, s);
+}
+
+template <bool ZOH>
+cudaError_t launch_summary_z(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
+    if (a.N <= 4) return launch_summary_n<4, ZOH>(a, kp, s);
+    if (a.N <= 8) return launch_summary_n<8, ZOH>(a, kp, s);
+    return launch_summary_n<16, ZOH>(a, kp, s);
+}
+
 template <int NMAX, bool ZOH>
 cudaError_t launch_nmax_z(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
     const bool ib = a.in_dtype == DType::BF16, ob = a.out_dtype == DType::BF16;
@@ -781,6 +842,40 @@ cudaError_t launch_scan_checkpoints(const ScanArgs& a, float* ckpt, cudaStream_t
     if (a.N <= 4) return ib ? launch_ckpt_io<4, __nv_bfloat16>(a, kp, stream) : launch_ckpt_io<4, float>(a, kp, stream);
     if (a.N <= 8) return ib ? launch_ckpt_io<8, __nv_bfloat16>(a, kp, stream) : launch_ckpt_io<8, float>(a, kp, stream);
     return ib ? launch_ckpt_io<16, __nv_bfloat16>(a, kp, stream) : launch_ckpt_io<16, float>(a, kp, stream);
+}
+
+cudaError_t launch_fold(const float* hend, const float* dsum, const float* A, const float* h0,
+                        int64_t count, int64_t batch, int64_t dim, int64_t N, float* h_out,
+                        float* dsum_out, cudaStream_t stream) {
+    const int64_t lanes = batch * dim * N;
+    fold_kernel<<<(unsigned)((lanes + 255) / 256), 256, 0, stream>>>(
+        hend, dsum, A, h0, count, batch, dim, (int)N, h_out, dsum_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scan_summary(const ScanArgs& a, float* h_end, float* dsum, cudaStream_t stream) {
+    KParams kp;
+    memset(&kp, 0, sizeof(kp));
+    kp.u = a.u;
+    kp.delta = a.delta;
+    kp.A = a.A;
+    kp.B = a.B;
+    kp.C = a.C;
+    kp.delta_bias = a.delta_bias;
+    kp.batch = a.batch;
+    kp.dim = a.dim;
+    kp.L = a.L;
+    kp.seg_len = a.nseg > 1 ? a.seg_len : (a.L > 0 ? a.L : 1);
+    kp.N = (int)a.N;
+    kp.nseg = (int)a.nseg;
+    kp.softplus = a.softplus ? 1 : 0;
+    // one segment: the aggregate pass writes the outputs directly
+    kp.seg_h = a.nseg > 1 ? a.seg_h : h_end;
+    kp.seg_sum = a.nseg > 1 ? a.seg_sum : dsum;
+    cudaError_t e = a.zoh ? launch_summary_z<true>(a, kp, stream) : launch_summary_z<false>(a, kp, stream);
+    if (e != cudaSuccess || a.nseg <= 1) return e;
+    return launch_fold(a.seg_h, a.seg_sum, a.A, nullptr, a.nseg, a.batch, a.dim, a.N, h_end, dsum,
+                       stream);
 }
 
 cudaError_t read_device_error(unsigned* out, bool clear, cudaStream_t stream) {
@@ -829,7 +924,8 @@ cudaError_t launch_scan(const ScanArgs& a, cudaStream_t stream) {
     kp.delta_bias = a.delta_bias;
     kp.y = a.y;
     kp.last_state = a.last_state;
-    kp.seg_h = a.seg_h;
+    // with one segment the kernel reads its initial state through seg_h (read only)
+    kp.seg_h = a.nseg > 1 ? a.seg_h : const_cast<float*>(a.h0);
     kp.seg_sum = a.seg_sum;
     kp.batch = a.batch;
     kp.dim = a.dim;

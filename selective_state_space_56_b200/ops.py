@@ -63,6 +63,14 @@ def load_library():
             lib.mamba_selective_scan_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp,
                                                         vp, ScanDims, i32, i32, vp,
                                                         ctypes.c_size_t, u32, vp]
+            lib.mamba_selective_scan_fwd_init.restype = i32
+            lib.mamba_selective_scan_fwd_init.argtypes = [vp] * 8 + [i32] + [vp] * 3 + [
+                ScanDims, i32, i32, vp, ctypes.c_size_t, u32, vp]
+            lib.mamba_selective_scan_summary.restype = i32
+            lib.mamba_selective_scan_summary.argtypes = [vp] * 6 + [i32, vp, vp, ScanDims, i32, vp,
+                                                                 ctypes.c_size_t, u32, vp]
+            lib.mamba_selective_scan_fold.restype = i32
+            lib.mamba_selective_scan_fold.argtypes = [vp] * 4 + [i64] * 4 + [vp, vp, vp]
             lib.mamba_selective_state_update_ex.restype = i32
             lib.mamba_selective_state_update_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                                             i32, vp, i64, i64, i64, i32, u32, vp]
@@ -145,11 +153,12 @@ def selective_scan_workspace_size(batch: int, dim: int, dstate: int, seqlen: int
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
                        out_dtype=None, y=None, last_state=None, return_last_state=False,
-                       workspace=None, exact_zoh=False):
+                       workspace=None, exact_zoh=False, initial_state=None):
     """Fused selective scan.  u, delta, z: (batch, dim, L); A: (dim, N) fp32;
     B, C: (batch, N, L); D, delta_bias: (dim) fp32.  Returns y (batch, dim, L)
     [and last_state (batch, dim, N) fp32].  exact_zoh: Bbar = (exp(Delta A) - 1) / A * B
-    instead of Delta * B."""
+    instead of Delta * B.  initial_state: (batch, dim, N) fp32 state before the sequence
+    (zero when None)."""
     if not isinstance(u, torch.Tensor) or u.dim() != 3:
         raise ValueError("u must be a (batch, dim, L) tensor")
     dev = u.device
@@ -177,6 +186,7 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
     if last_state is None and return_last_state:
         last_state = torch.empty((b, d, N), dtype=torch.float32, device=dev)
     _check(last_state, "last_state", dev, (b, d, N), (torch.float32,))
+    _check(initial_state, "initial_state", dev, (b, d, N), (torch.float32,))
     lib = load_library()
     dims = ScanDims(b, d, N, L)
     need = int(lib.mamba_selective_scan_workspace_size(dims))
@@ -186,9 +196,13 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
     args = (_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
             int(bool(delta_softplus)), _ptr(y), _ptr(last_state), dims, _DTYPES[in_dt],
             _DTYPES[out_dt], _ptr(workspace), ws_bytes)
+    flags = MAMBA_FLAG_EXACT_ZOH if exact_zoh else 0
     with torch.cuda.device(dev):
-        if exact_zoh:
-            rc = lib.mamba_selective_scan_fwd_ex(*args, MAMBA_FLAG_EXACT_ZOH, _stream_handle(dev))
+        if initial_state is not None:
+            rc = lib.mamba_selective_scan_fwd_init(*args[:9], _ptr(initial_state), *args[9:], flags,
+                                                   _stream_handle(dev))
+        elif exact_zoh:
+            rc = lib.mamba_selective_scan_fwd_ex(*args, flags, _stream_handle(dev))
         else:
             rc = lib.mamba_selective_scan_fwd(*args, _stream_handle(dev))
     if rc != 0:
@@ -355,3 +369,63 @@ def causal_conv1d_update(conv_state, x, weight, bias=None, silu=True, out=None):
     if rc != 0:
         raise MambaError(rc, "mamba_causal_conv1d_update")
     return out
+
+
+def selective_scan_summary(u, delta, A, B, C, delta_bias=None, delta_softplus=True,
+                           exact_zoh=False, workspace=None):
+    """Summary of a sequence segment for the associative combine: (h_end (batch, dim, N),
+    delta_sum (batch, dim)), the state after the segment from zero and its summed step."""
+    if not isinstance(u, torch.Tensor) or u.dim() != 3:
+        raise ValueError("u must be a (batch, dim, L) tensor")
+    dev = u.device
+    if dev.type != "cuda":
+        raise ValueError("selective_scan_summary runs on CUDA tensors only")
+    b, d, L = u.shape
+    N = A.shape[1] if A.dim() == 2 else -1
+    dt = u.dtype
+    if dt not in _DTYPES:
+        raise ValueError("unsupported input dtype %s" % dt)
+    for t, name, shape, dts in ((u, "u", (b, d, L), (dt,)), (delta, "delta", (b, d, L), (dt,)),
+                                (A, "A", (d, N), (torch.float32,)), (B, "B", (b, N, L), (dt,)),
+                                (C, "C", (b, N, L), (dt,)),
+                                (delta_bias, "delta_bias", (d,), (torch.float32,))):
+        _check(t, name, dev, shape, dts)
+    h_end = torch.empty((b, d, N), dtype=torch.float32, device=dev)
+    dsum = torch.empty((b, d), dtype=torch.float32, device=dev)
+    lib = load_library()
+    dims = ScanDims(b, d, N, L)
+    need = int(lib.mamba_selective_scan_workspace_size(dims))
+    if need > 0 and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        rc = lib.mamba_selective_scan_summary(
+            _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(delta_bias),
+            int(bool(delta_softplus)), _ptr(h_end), _ptr(dsum), dims, _DTYPES[dt],
+            _ptr(workspace), ws_bytes, MAMBA_FLAG_EXACT_ZOH if exact_zoh else 0,
+            _stream_handle(dev))
+    if rc != 0:
+        raise MambaError(rc, "mamba_selective_scan_summary")
+    return h_end, dsum
+
+
+def selective_scan_fold(h_ends, delta_sums, A, h0=None, return_delta_sum=False):
+    """Apply summaries h_ends (count, batch, dim, N), delta_sums (count, batch, dim) in order
+    to h0 (batch, dim, N) or zero; returns the resulting state [and the total step]."""
+    dev = A.device
+    if dev.type != "cuda":
+        raise ValueError("selective_scan_fold runs on CUDA tensors only")
+    cnt, b, d, N = h_ends.shape
+    _check(h_ends, "h_ends", dev, (cnt, b, d, N), (torch.float32,))
+    _check(delta_sums, "delta_sums", dev, (cnt, b, d), (torch.float32,))
+    _check(A, "A", dev, (d, N), (torch.float32,))
+    _check(h0, "h0", dev, (b, d, N), (torch.float32,))
+    h_out = torch.empty((b, d, N), dtype=torch.float32, device=dev)
+    s_out = torch.empty((b, d), dtype=torch.float32, device=dev) if return_delta_sum else None
+    with torch.cuda.device(dev):
+        rc = load_library().mamba_selective_scan_fold(
+            _ptr(h_ends) if cnt else None, _ptr(delta_sums) if cnt else None, _ptr(A), _ptr(h0),
+            cnt, b, d, N, _ptr(h_out), _ptr(s_out), _stream_handle(dev))
+    if rc != 0:
+        raise MambaError(rc, "mamba_selective_scan_fold")
+    return (h_out, s_out) if return_delta_sum else h_out
