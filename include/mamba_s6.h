@@ -246,7 +246,7 @@ int mamba_selective_scan_fwd_noalloc(const void* u, const void* delta, const flo
 
 /*
  * Bytes of device workspace mamba_selective_scan_bwd needs for `dims`:
- * batch x dim x ceil(seqlen / T) x dstate x 4, T = 32 steps for dstate > 8 and 64
+ * batch x dim x ceil(seqlen / T) x dstate x 4, T = 16 steps for dstate > 8 and 64
  * otherwise, rounded up to 256 bytes (0 when seqlen == 0).  Returns 0 for invalid dims.
  */
 size_t mamba_selective_scan_bwd_workspace_size(mamba_scan_dims dims);
@@ -255,7 +255,7 @@ size_t mamba_selective_scan_bwd_workspace_size(mamba_scan_dims dims);
  * Backward of mamba_selective_scan_fwd: given dy = dLoss/dy, writes the gradients of
  * every input.  The intermediate states are not read from memory (the forward never
  * stored them); as the method's hardware-aware algorithm prescribes, they are
- * recomputed: a forward pass records the state entering every T-step chunk in the
+ * recomputed: a forward pass records the state entering every T-step block in the
  * workspace, and a reverse sweep rebuilds each chunk's states from its record
  * before propagating the adjoint state backwards through it (Mamba, section
  * "Hardware-aware state expansion").

@@ -277,7 +277,7 @@ int mamba_selective_state_update_ex(float* state, const void* u, const void* del
 
 size_t mamba_selective_scan_bwd_workspace_size(mamba_scan_dims dims) {
     if (!dims_ok(dims.batch, dims.dim, dims.dstate, dims.seqlen)) return 0;
-    const int64_t T = s6::scan_chunk_steps(dims.dstate);
+    const int64_t T = s6::checkpoint_steps(dims.dstate);
     const int64_t chunks = (dims.seqlen + T - 1) / T;
     if (!mul_ok(dims.batch * dims.dim, chunks) || !mul_ok(dims.batch * dims.dim * chunks, dims.dstate * 4))
         return 0;

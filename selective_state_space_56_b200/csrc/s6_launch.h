@@ -70,12 +70,15 @@ cudaError_t launch_fold(const float* hend, const float* dsum, const float* A, co
                         int64_t count, int64_t batch, int64_t dim, int64_t N, float* h_out,
                         float* dsum_out, cudaStream_t stream);
 
-// Steps per chunk of the forward kernel for state width N (the backward recomputes
-// states chunk by chunk from checkpoints taken at these boundaries).
+// Steps per chunk of the forward kernel for state width N.
 int scan_chunk_steps(int64_t N);
 
-// Forward pass that writes the state entering every chunk to
-// ckpt[((b * dim + d) * chunks + k) * N + n], chunks = ceil(L / scan_chunk_steps(N)),
+// Steps between the backward's checkpoints (a divisor of scan_chunk_steps(N)); the
+// backward recomputes states block by block from them.
+int checkpoint_steps(int64_t N);
+
+// Forward pass that writes the state entering every checkpoint block to
+// ckpt[((b * dim + d) * blocks + k) * N + n], blocks = ceil(L / checkpoint_steps(N)),
 // and no output.  Uses a.u, delta, A, B, C, delta_bias, softplus, dims and in_dtype.
 cudaError_t launch_scan_checkpoints(const ScanArgs& a, float* ckpt, cudaStream_t stream);
 
@@ -94,7 +97,7 @@ struct BackwardArgs {
 
 // Backward of the scan described by `a` (its y, last_state and segment fields are
 // unused): zeroes the accumulated outputs, runs the checkpointing forward into
-// `ckpt` (batch * dim * ceil(L / scan_chunk_steps(N)) * N floats) and then the
+// `ckpt` (batch * dim * ceil(L / checkpoint_steps(N)) * N floats) and then the
 // reverse sweep.
 cudaError_t launch_scan_backward(const ScanArgs& a, const BackwardArgs& g, float* ckpt,
                                  cudaStream_t stream);

@@ -2,8 +2,9 @@
 //
 // Mamba ("Hardware-aware state expansion"): the intermediate states are not stored for
 // the backward pass; they are recomputed on chip.  The forward kernel first records
-// only the state entering every chunk (checkpoints, one N-vector per chunk of T steps
-// per channel).  This kernel then walks the chunks of a channel tile in reverse:
+// only the state entering every block of T steps (checkpoints, one N-vector per block per
+// channel; T = 16 for N > 8, so that a CTA's shared memory stays small enough for every
+// CTA of the 2.8B-shaped layer to be resident at once).  This kernel then walks the chunks of a channel tile in reverse:
 //
 //   stage     u, delta, z, dy rows and the batch's B, C for the chunk -> shared memory
 //             (16-byte cp.async copies into rows padded against bank conflicts);
@@ -60,7 +61,9 @@ struct BParams {
     int64_t batch, dim, L;
     int N;
     int softplus;
-    int chunks;
+    int chunks;     // blocks of T steps this kernel walks
+    int ck_blocks;  // checkpoints per channel (blocks of checkpoint_steps(N))
+    int ck_stride;  // checkpoints per block of T steps
     int vec;  // rows start on 16-byte boundaries: stage them with 16-byte copies
 };
 
@@ -271,7 +274,9 @@ __global__ void __launch_bounds__(kBW * 32) scan_bwd_kernel(const BParams p) {
                 for (int j = 0; j < 4; ++j) {
                     const int n = pp * 4 + j;
                     h[j] = (chok && n < p.N)
-                               ? p.ckpt[((b * p.dim + dch) * p.chunks + k) * p.N + n] : 0.f;
+                               ? p.ckpt[((b * p.dim + dch) * p.ck_blocks +
+                                         (int64_t)k * p.ck_stride) * p.N + n]
+                               : 0.f;
                 }
                 hp[0] = pack2(h[0], h[1]);
                 hp[1] = pack2(h[2], h[3]);
@@ -479,17 +484,48 @@ template <typename Tin>
 cudaError_t launch_bwd_io(BParams bp, int T, int64_t batch, int64_t dim, cudaStream_t s) {
     // 16-byte staging needs every row start (a multiple of L elements) 16-byte aligned
     bp.vec = (bp.L * (int64_t)sizeof(Tin)) % 16 == 0 ? 1 : 0;
+    if (T == 16) return launch_bwd_typed<16, Tin>(bp, batch, dim, s);
     if (T == 32) return launch_bwd_typed<32, Tin>(bp, batch, dim, s);
     if (T == 64) return launch_bwd_typed<64, Tin>(bp, batch, dim, s);
     return cudaErrorInvalidConfiguration;
+}
+
+// Resident CTAs of the T-step backward kernel per SM on the current device.
+template <int T, typename Tin>
+int resident_ctas() {
+    int n = 0;
+    if (cudaFuncSetAttribute(scan_bwd_kernel<T, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)BLayout<T, Tin>::bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(scan_bwd_kernel<T, Tin>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, scan_bwd_kernel<T, Tin>, kBW * 32,
+                                                      BLayout<T, Tin>::bytes) != cudaSuccess)
+        return 0;
+    return n;
+}
+
+// Block length for N > 8: 32 steps (half the per-block overhead) when every CTA of the
+// grid is resident at once with it, else 16 (less shared memory per CTA, so more fit).
+template <typename Tin>
+int pick_block_steps(int64_t ctas) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 16;
+    return ctas <= (int64_t)sms * resident_ctas<32, Tin>() ? 32 : 16;
 }
 
 }  // namespace
 
 cudaError_t launch_scan_backward(const ScanArgs& a, const BackwardArgs& g, float* ckpt,
                                  cudaStream_t stream) {
-    // the backward walks the chunks the forward checkpointed
-    const int T = scan_chunk_steps(a.N);
+    // checkpoints every CK steps; the kernel walks blocks of T = CK (or 2 CK) steps
+    const int CK = checkpoint_steps(a.N);
+    const int64_t ctas = (a.dim + kBCH - 1) / kBCH * a.batch;
+    int T = CK;
+    if (a.N > 8 && CK == 16)
+        T = a.in_dtype == DType::BF16 ? pick_block_steps<__nv_bfloat16>(ctas)
+                                      : pick_block_steps<float>(ctas);
     const int64_t chunks = (a.L + T - 1) / T;
     cudaError_t e;
     // outputs accumulated with atomics start at zero
@@ -531,6 +567,8 @@ cudaError_t launch_scan_backward(const ScanArgs& a, const BackwardArgs& g, float
     bp.N = (int)a.N;
     bp.softplus = a.softplus ? 1 : 0;
     bp.chunks = (int)chunks;
+    bp.ck_blocks = (int)((a.L + CK - 1) / CK);
+    bp.ck_stride = T / CK;
     if (a.in_dtype == DType::BF16) return launch_bwd_io<__nv_bfloat16>(bp, T, a.batch, a.dim, stream);
     return launch_bwd_io<float>(bp, T, a.batch, a.dim, stream);
 }

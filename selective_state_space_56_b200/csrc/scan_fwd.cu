@@ -416,10 +416,14 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         }
         __syncwarp();
 
-        if (MODE == kCheckpoint && dch < p.dim) {
-            // state entering chunk k: ckpt[((b * dim + d) * chunks + k) * N + n]
-            const int64_t chunks = (p.L + T - 1) / T;
-            float* ck = p.seg_h + ((b * p.dim + dch) * chunks + k) * p.N;
+        // checkpoint mode: the state entering every CKPT-step block of the sequence,
+        // ckpt[((b * dim + d) * blocks + kb) * N + n], blocks = ceil(L / CKPT)
+        constexpr int CKPT = NMAX == 16 ? 16 : T;
+        auto write_ckpt = [&](int t) {
+            const int64_t blocks = (p.L + CKPT - 1) / CKPT;
+            const int64_t kb = (t0 + t) / CKPT;
+            if (dch >= p.dim || t0 + t >= p.L) return;
+            float* ck = p.seg_h + ((b * p.dim + dch) * blocks + kb) * p.N;
 #pragma unroll
             for (int j = 0; j < NS / 2; ++j) {
                 float h0, h1;
@@ -427,11 +431,13 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
                 if (pp * NS + 2 * j < p.N) ck[pp * NS + 2 * j] = h0;
                 if (pp * NS + 2 * j + 1 < p.N) ck[pp * NS + 2 * j + 1] = h1;
             }
-        }
+        };
+        if (MODE == kCheckpoint) write_ckpt(0);
 
         // Phase B: the recurrence, four steps per iteration, states in packed pairs.
 #pragma unroll
         for (int t = 0; t < T; t += 4) {
+            if (MODE == kCheckpoint && t > 0 && t % CKPT == 0) write_ckpt(t);
             const float4 d4 = *reinterpret_cast<const float4*>(sDel + cw * RS + t);
             const float4 q4 = *reinterpret_cast<const float4*>(sDu + cw * RS + t);
             const f2 dd4[4] = {pack2(d4.x, d4.x), pack2(d4.y, d4.y), pack2(d4.z, d4.z),
@@ -820,6 +826,8 @@ int scan_chunk_steps(int64_t N) {
     if (N <= 8) return Tile<8>::T;
     return Tile<16>::T;
 }
+
+int checkpoint_steps(int64_t N) { return N <= 8 ? scan_chunk_steps(N) : 16; }
 
 cudaError_t launch_scan_checkpoints(const ScanArgs& a, float* ckpt, cudaStream_t stream) {
     KParams kp;

@@ -181,9 +181,9 @@ def test_bwd_dims_dtype_align_workspace(lib):
 
 def test_bwd_workspace_is_one_checkpoint_per_chunk(lib):
     ws = lambda *d: lib.mamba_selective_scan_bwd_workspace_size(_dims(*d))  # noqa: E731
-    # 32-step chunks for dstate > 8, 64-step chunks otherwise; fp32 states
-    assert ws(4, 5120, 16, 4096) == 4 * 5120 * 128 * 16 * 4
-    assert ws(2, 64, 16, 33) == 2 * 64 * 2 * 16 * 4
+    # 16-step blocks for dstate > 8, 64-step blocks otherwise; fp32 states
+    assert ws(4, 5120, 16, 4096) == 4 * 5120 * 256 * 16 * 4
+    assert ws(2, 64, 16, 33) == 2 * 64 * 3 * 16 * 4
     assert ws(2, 64, 8, 64) == 2 * 64 * 1 * 8 * 4
     assert ws(1, 3, 5, 65) == (1 * 3 * 2 * 5 * 4 + 255) // 256 * 256
     assert ws(2, 64, 16, 0) == 0
