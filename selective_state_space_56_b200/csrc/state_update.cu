@@ -125,7 +125,10 @@ __global__ void __launch_bounds__(256) state_update_kernel(const UParams p) {
 // (1 KiB of state) per instruction pair.  Each thread serves kItems lanes, one grid
 // stride apart, and issues every load of all of them before any arithmetic, keeping
 // 64 bytes of state per thread in flight.  Math runs on packed fp32 pairs.
-constexpr int kItems = 2;
+#ifndef S6_DEC_ITEMS
+#define S6_DEC_ITEMS 2
+#endif
+constexpr int kItems = S6_DEC_ITEMS;
 
 template <typename Tio>
 struct Lane16 {
