@@ -178,7 +178,8 @@ def profile_traffic(name: str, source: str):
             k, v = line.split(":", 1)
             vals[k.strip()] = v.strip()
     digest = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()[:16]
-    if vals.get("source_sha256_16") != digest:
+    recorded = vals.get("source_sha256_16", "").split()
+    if not recorded or recorded[0] != digest:  # the kernel changed since the capture
         return None
     try:
         return float(vals["dram_bytes_per_launch"])

@@ -60,3 +60,20 @@ def test_weak_scaling_value_counts_every_rank(n):
     elems = 4 * 5120 * 4096
     ms_total, steps = 637.0, 1000
     assert n * elems * steps / (ms_total * 1e-3) == pytest.approx(n * 1.3168e11, rel=1e-3)
+
+
+def test_committed_profile_traffic_is_found_for_unchanged_kernels(tmp_path, monkeypatch):
+    """bench.py reads a kernel's DRAM bytes from its committed ncu summary only while the
+    kernel source still has the digest recorded there."""
+    import hashlib
+    import bench
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1")
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    digest = hashlib.sha256(b"kernel v1").hexdigest()[:16]
+    (prof / "k.txt").write_text("source_sha256_16: %s   (k.cu)\ndram_bytes_per_launch: 1234\n" % digest)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profile_traffic("k.txt", "k.cu") == 1234.0
+    src.write_text("kernel v2")
+    assert bench.profile_traffic("k.txt", "k.cu") is None
