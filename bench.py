@@ -167,8 +167,19 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}, "fallback"
 
 
+def source_digest(path: str) -> str:
+    """First 16 hex digits of the SHA-256 of a CUDA source with its comments and blank-space
+    differences removed: it changes when the code changes, not when a comment does."""
+    import re
+    text = open(path, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    code = "\n".join(" ".join(line.split()) for line in text.splitlines() if line.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
+
+
 def profile_traffic(name: str, source: str):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    """DRAM bytes per launch from a committed ncu summary, if the kernel code is unchanged."""
     path = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(path):
         return None
@@ -177,7 +188,7 @@ def profile_traffic(name: str, source: str):
         if ":" in line:
             k, v = line.split(":", 1)
             vals[k.strip()] = v.strip()
-    digest = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()[:16]
+    digest = source_digest(os.path.join(ROOT, source))
     recorded = vals.get("source_sha256_16", "").split()
     if not recorded or recorded[0] != digest:  # the kernel changed since the capture
         return None

@@ -2,9 +2,10 @@
 //
 // Mamba ("Hardware-aware state expansion"): the intermediate states are not stored for
 // the backward pass; they are recomputed on chip.  The forward kernel first records
-// only the state entering every block of T steps (checkpoints, one N-vector per block per
-// channel; T = 16 for N > 8, so that a CTA's shared memory stays small enough for every
-// CTA of the 2.8B-shaped layer to be resident at once).  This kernel then walks the chunks of a channel tile in reverse:
+// only the state entering every 16 steps (checkpoints, one N-vector per channel; every 64
+// steps for N <= 8).  This kernel then walks blocks of T steps of a channel tile in
+// reverse -- T = 16, or 32 (every other checkpoint) when the whole grid is resident at
+// once with the larger shared-memory footprint of 32-step blocks:
 //
 //   stage     u, delta, z, dy rows and the batch's B, C for the chunk -> shared memory
 //             (16-byte cp.async copies into rows padded against bank conflicts);

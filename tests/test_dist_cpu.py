@@ -65,15 +65,16 @@ def test_weak_scaling_value_counts_every_rank(n):
 def test_committed_profile_traffic_is_found_for_unchanged_kernels(tmp_path, monkeypatch):
     """bench.py reads a kernel's DRAM bytes from its committed ncu summary only while the
     kernel source still has the digest recorded there."""
-    import hashlib
     import bench
     src = tmp_path / "k.cu"
     src.write_text("kernel v1")
     prof = tmp_path / "profiles"
     prof.mkdir()
-    digest = hashlib.sha256(b"kernel v1").hexdigest()[:16]
+    digest = bench.source_digest(str(src))
     (prof / "k.txt").write_text("source_sha256_16: %s   (k.cu)\ndram_bytes_per_launch: 1234\n" % digest)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profile_traffic("k.txt", "k.cu") == 1234.0
+    src.write_text("kernel v1 // a comment\n/* another */")
     assert bench.profile_traffic("k.txt", "k.cu") == 1234.0
     src.write_text("kernel v2")
     assert bench.profile_traffic("k.txt", "k.cu") is None
