@@ -120,6 +120,9 @@ enum Mode : int { kFull = 0, kAggregate = 1, kCheckpoint = 2 };
 #ifndef S6_PREEXP
 #define S6_PREEXP 1  // Abar of a whole 4-step group before its updates (measured +1.7%)
 #endif
+#ifndef S6_WS
+#define S6_WS 0  // TMA path: a producer warp stages and converts, compute warps never meet
+#endif
 #ifndef S6_POLY
 #define S6_POLY 0
 #endif
@@ -157,8 +160,10 @@ struct Layout {
     static constexpr size_t off_out = align128(off_y + (size_t)CH * RS * 4);  // Tout [CH][T]
     static constexpr size_t out_bytes = align128((size_t)CH * T * sizeof(Tout));
     static constexpr size_t off_par = off_out + out_bytes;               // bias[CH], D[CH]
-    static constexpr size_t off_bar = align128(off_par + (size_t)2 * CH * 4);  // 2 mbarriers
-    static constexpr size_t bytes = off_bar + 16;
+    // mbarriers: full[2] (TMA bytes landed), then, for the producer-warp variant,
+    // ready[2] (coefficients converted) and empty[2] (compute warps done with a stage)
+    static constexpr size_t off_bar = align128(off_par + (size_t)2 * CH * 4);
+    static constexpr size_t bytes = off_bar + 6 * 8;
     static_assert(NS % 4 == 0, "states per lane must be a multiple of 4");
     static_assert(T % 4 == 0 && kChunk % T == 0, "chunks of whole 4-step groups");
     static_assert(T * sizeof(Tin) % 16 == 0 && T * sizeof(Tout) % 16 == 0, "TMA rows");
@@ -187,9 +192,10 @@ __device__ __forceinline__ float transpose_reduce(const float* v, int pp) {
 }
 
 template <int NMAX, int P, int WARPS, int T_, typename Tin, typename Tout, int MODE, bool TMA,
-          bool ZOH = false>
-__global__ void __launch_bounds__(WARPS * 32)
+          bool ZOH = false, bool WS = false>
+__global__ void __launch_bounds__(WARPS * 32 + (WS ? 32 : 0))
 scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
+    static_assert(!WS || (TMA && MODE == kFull), "producer warp: TMA full scans only");
     using Lo = Layout<NMAX, P, WARPS, T_, Tin, Tout>;
     using V4 = vec4<Tin>;
     using VT = typename V4::type;
@@ -221,6 +227,12 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
     if (TMA && tid == 0) {
         mbar_init(&bar[0], 1);
         mbar_init(&bar[1], 1);
+        if (WS) {
+            mbar_init(&bar[2], 1);
+            mbar_init(&bar[3], 1);
+            mbar_init(&bar[4], WARPS);
+            mbar_init(&bar[5], WARPS);
+        }
         fence_barrier_init();
     }
 
@@ -298,31 +310,13 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         }
     };
 
-    if constexpr (TMA) {
-        if (tid == 0 && nchunks > 0) issue_chunk(0);
-    }
-    bool aborted = false;
-    for (int64_t k = 0; k < nchunks; ++k) {
-        bool ok = true;
-        if constexpr (TMA) {
-            ok = mbar_wait_bounded(&bar[k & 1], (uint32_t)((k >> 1) & 1), kWaitLimitCycles);
-        } else {
-            load_chunk_elementwise(k);
-            __syncthreads();
-        }
-
-        const Tin* st = stage_ptr(k);
-        const unsigned char* stb = reinterpret_cast<const unsigned char*>(st);
-        const Tin* rU = st;
-        const Tin* rDr = reinterpret_cast<const Tin*>(stb + Lo::off_dr);
-        const Tin* rZ = reinterpret_cast<const Tin*>(stb + Lo::off_z);
+    // B, C of chunk k into its coefficient buffer (work items first, first + stride, ...).
+    auto convert_chunk = [&](int64_t k, int first, int stride) {
+        const unsigned char* stb = reinterpret_cast<const unsigned char*>(stage_ptr(k));
         const Tin* rB = reinterpret_cast<const Tin*>(stb + Lo::off_B);
         const Tin* rC = reinterpret_cast<const Tin*>(stb + Lo::off_C);
-        const int64_t t0 = t_begin + k * T;
-        const int valid = (int)min((int64_t)T, t_end - t0);
         float* sBt = reinterpret_cast<float*>(smem + Lo::off_coef + (k & 1) * Lo::coef_bytes_all);
-        float* sCt = sBt + T * NMAX;  // formats 0 and 2: what follows the fp32 B tile
-
+        float* sCt = sBt + T * NMAX;
         // B, C of the chunk, time-major: every lane then reads the coefficients of its four
         // states for step t with one 16-byte load (bf16: B[4] and C[4] as pairs; fp32: a
         // 16-byte vector from each of two tiles, transposed through 4x4 register blocks).
@@ -331,7 +325,7 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
             // format 2: the C half only, [C0|C1][C2|C3] per (step, group), after the B tile.
             // Work item: (4-state group, step pair, B or C) -> two 8-byte half-groups.
             constexpr int kWhich = Lo::kBC == 1 ? 2 : 1;
-            for (int i = tid; i < (NMAX / 4) * (T / 2) * kWhich; i += Lo::THREADS) {
+            for (int i = first; i < (NMAX / 4) * (T / 2) * kWhich; i += stride) {
                 const int which = kWhich == 2 ? (i & 1) : 1;
                 const int i2 = kWhich == 2 ? (i >> 1) : i;
                 const int n4 = i2 % (NMAX / 4), t2 = i2 / (NMAX / 4);
@@ -357,7 +351,7 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         if constexpr (Lo::kBC == 0 || Lo::kBC == 2) {
             // fp32 tiles [T][NMAX], transposed through 4x4 register blocks
             constexpr int kTiles = Lo::kBC == 0 ? 2 : 1;
-            for (int i = tid; i < (NMAX / 4) * (T / 4) * kTiles; i += Lo::THREADS) {
+            for (int i = first; i < (NMAX / 4) * (T / 4) * kTiles; i += stride) {
                 const int which = kTiles == 2 ? (i & 1) : 0;
                 const int i2 = kTiles == 2 ? (i >> 1) : i;
                 const int n4 = i2 % (NMAX / 4), t4 = i2 / (NMAX / 4);
@@ -373,17 +367,90 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
                         make_float4(v[0][q], v[1][q], v[2][q], v[3][q]);
             }
         }
-        // The one CTA-wide barrier of a chunk: coefficients visible to every warp, and
-        // every warp done with chunk k-1, so its stage can take chunk k+1.
-        if (__syncthreads_or(!ok)) {  // every thread agrees to stop if any wait gave up
-            if (tid == 0) atomicOr(&g_device_error, 1u);
-            aborted = true;
-            break;
+    };
+
+    // Producer warp (variant WS): stages every chunk with TMA and converts its
+    // coefficients; the compute warps wait only for a chunk to be ready and release its
+    // stage when done, so they never wait for one another.
+    if constexpr (WS) {
+        if (warp == WARPS) {
+            bool pok = true;
+            int64_t issued = -1, landed = -1;
+            for (int64_t k = 0; k < nchunks; ++k) {
+                const int s = (int)(k & 1);
+                if (k >= 2) {  // the compute warps are done with chunk k - 2 in this stage
+                    pok = __all_sync(0xffffffffu, mbar_wait_bounded(
+                        &bar[4 + s], (uint32_t)(((k >> 1) & 1) ^ 1), kWaitLimitCycles));
+                    if (!pok) break;
+                }
+                if (lane == 0) {
+                    fence_proxy_async();  // the stage was last read through the generic proxy
+                    issue_chunk(k);
+                }
+                issued = k;
+                pok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar[s], (uint32_t)((k >> 1) & 1),
+                                                                kWaitLimitCycles));
+                if (!pok) break;
+                landed = k;
+                convert_chunk(k, lane, 32);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[2 + s]);
+            }
+            if (!pok) {
+                if (lane == 0) atomicOr(&g_device_error, 1u);
+                if (lane == 0 && issued > landed)  // let the copy in flight land first
+                    mbar_wait_bounded(&bar[issued & 1], (uint32_t)((issued >> 1) & 1),
+                                      kWaitLimitCycles);
+            }
+            return;
         }
-        if constexpr (TMA) {
-            if (tid == 0 && k + 1 < nchunks) {
-                fence_proxy_async();  // stage (k+1)&1 was last read through the generic proxy
-                issue_chunk(k + 1);
+    }
+
+    if constexpr (TMA && !WS) {
+        if (tid == 0 && nchunks > 0) issue_chunk(0);
+    }
+    bool aborted = false;
+    for (int64_t k = 0; k < nchunks; ++k) {
+        bool ok = true;
+        if constexpr (WS) {
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar[2 + (k & 1)], (uint32_t)((k >> 1) & 1),
+                                                           kWaitLimitCycles));
+            if (!ok) {
+                if (lane == 0) atomicOr(&g_device_error, 1u);
+                aborted = true;
+                break;
+            }
+        } else if constexpr (TMA) {
+            ok = mbar_wait_bounded(&bar[k & 1], (uint32_t)((k >> 1) & 1), kWaitLimitCycles);
+        } else {
+            load_chunk_elementwise(k);
+            __syncthreads();
+        }
+
+        const Tin* st = stage_ptr(k);
+        const unsigned char* stb = reinterpret_cast<const unsigned char*>(st);
+        const Tin* rU = st;
+        const Tin* rDr = reinterpret_cast<const Tin*>(stb + Lo::off_dr);
+        const Tin* rZ = reinterpret_cast<const Tin*>(stb + Lo::off_z);
+        const int64_t t0 = t_begin + k * T;
+        const int valid = (int)min((int64_t)T, t_end - t0);
+        float* sBt = reinterpret_cast<float*>(smem + Lo::off_coef + (k & 1) * Lo::coef_bytes_all);
+        float* sCt = sBt + T * NMAX;  // formats 0 and 2: what follows the fp32 B tile
+
+        if constexpr (!WS) {
+            convert_chunk(k, tid, Lo::THREADS);
+            // The one CTA-wide barrier of a chunk: coefficients visible to every warp, and
+            // every warp done with chunk k-1, so its stage can take chunk k+1.
+            if (__syncthreads_or(!ok)) {  // every thread agrees to stop if any wait gave up
+                if (tid == 0) atomicOr(&g_device_error, 1u);
+                aborted = true;
+                break;
+            }
+            if constexpr (TMA) {
+                if (tid == 0 && k + 1 < nchunks) {
+                    fence_proxy_async();  // stage (k+1)&1 was last read through the generic proxy
+                    issue_chunk(k + 1);
+                }
             }
         }
 
@@ -592,9 +659,13 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
                 }
             }
         }
+        if constexpr (WS) {  // this warp is done with the chunk's stage and coefficients
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[4 + (k & 1)]);
+        }
     }
 
-    if constexpr (TMA) {
+    if constexpr (TMA && !WS) {
         if (tid == 0) {
             if (aborted) {  // let copies still in flight land before the CTA exits
                 mbar_wait_bounded(&bar[0], 0, kWaitLimitCycles);
@@ -712,14 +783,14 @@ bool encode_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, u
 }
 
 template <int NMAX, int P, int WARPS, int T, typename Tin, typename Tout, int MODE, bool TMA,
-          bool ZOH = false>
+          bool ZOH = false, bool WS = false>
 cudaError_t launch_one(const KParams& kp, const TMaps& tm, dim3 grid, cudaStream_t s) {
     using Lo = Layout<NMAX, P, WARPS, T, Tin, Tout>;
-    auto kern = scan_kernel<NMAX, P, WARPS, T, Tin, Tout, MODE, TMA, ZOH>;
+    auto kern = scan_kernel<NMAX, P, WARPS, T, Tin, Tout, MODE, TMA, ZOH, WS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Lo::bytes);
     if (e != cudaSuccess) return e;
-    kern<<<grid, Lo::THREADS, Lo::bytes, s>>>(kp, tm);
+    kern<<<grid, Lo::THREADS + (WS ? 32 : 0), Lo::bytes, s>>>(kp, tm);
     return cudaGetLastError();
 }
 
@@ -747,7 +818,7 @@ cudaError_t launch_typed(const ScanArgs& a, const KParams& kp, const TMaps& tm, 
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA, ZOH>(
+    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA, ZOH, TMA && S6_WS>(
         kp, tm, dim3(gx, (unsigned)a.batch, (unsigned)a.nseg), s);
 }
 
