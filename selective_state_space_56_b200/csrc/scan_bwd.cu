@@ -9,19 +9,19 @@
 //
 //   stage     u, delta, z, dy rows and the batch's B, C for the chunk -> shared memory
 //             (16-byte cp.async copies into rows padded against bank conflicts);
-//   phase A   per (channel, t): Delta = softplus(delta + bias);
+//   phase A   per (channel, t): Delta = softplus(delta + bias) and the gated output
+//             gradient dyt_t = dy_t silu(z_t);
 //   forward   from the checkpoint, the chunk's states are recomputed; the state
-//             entering every group of 4 steps is kept in shared memory, and the
-//             pre-gate output yt_t = C_t . h_t + D u_t (4-lane transpose-reduce) gives
-//             dz_t = dy_t yt_t silu'(z_t) and the gated gradient dyt_t = dy_t silu(z_t);
+//             entering every group of 4 steps is kept in shared memory;
 //   reverse   per group of 4 steps, last group first: the group's states and Abar are
 //             recomputed into registers from the group's entry state; then the adjoint
 //             state g (registers) is swept from the group's last step to its first:
 //               g += dyt C;  dC += dyt h;  dB += g Delta u;  dq = g . B;
 //               dDelta = dq u + sum_n g h_{t-1} Abar A;  dA += g h_{t-1} Abar Delta;
 //               g *= Abar.
-//             dq and the state part of dDelta are summed over a channel's 4 lanes once
-//             per group.  dB and dC, shared by all channels of a batch, go through a
+//             dq, the state part of dDelta and C_t . h_t are summed over a channel's 4
+//             lanes once per group; C_t . h_t + D u_t gives dz_t = dy_t yt_t silu'(z_t).
+//             dB and dC, shared by all channels of a batch, go through a
 //             per-warp exchange buffer: every channel stores its 32 values of a step,
 //             and after each pair of steps the warp's lanes sum them over the warp's 8
 //             channels (16-byte loads), add the sums into the CTA's chunk accumulator
@@ -195,7 +195,7 @@ __device__ __forceinline__ void stage_chunk(const BParams& p, unsigned char* st,
 }
 
 template <int T, typename Tin>
-__global__ void __launch_bounds__(kBW * 32) scan_bwd_kernel(const BParams p) {
+__global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) {
     using Lo = BLayout<T, Tin>;
     constexpr int RS = Lo::RS, RR = Lo::RR;
     using V4 = vec4<Tin>;
@@ -255,7 +255,8 @@ __global__ void __launch_bounds__(kBW * 32) scan_bwd_kernel(const BParams p) {
         }
         for (int i = tid; i < T * 32; i += kBW * 32) sAcc[i] = 0.f;
 
-        // phase A: Delta for this warp's channels (zero on padded steps: Abar = 1, no input)
+        // phase A, per (channel, t) of this warp: Delta (zero on padded steps: Abar = 1, no
+        // input) and the gated output gradient dyt = dy silu(z)
         for (int i = lane; i < kBG * T; i += 32) {
             const int c = warp * kBG + i / T, t = i % T;
             const int64_t d = d0 + c;
@@ -263,10 +264,12 @@ __global__ void __launch_bounds__(kBW * 32) scan_bwd_kernel(const BParams p) {
             const float x = io<Tin>::to_f(rDr[c * RR + t]) + bi;
             const float dt = p.softplus ? softplus(x) : x;
             sDel[c * RS + t] = t < valid ? dt : 0.f;
+            const float dyv = io<Tin>::to_f(rDy[c * RR + t]);
+            sDyt[c * RS + t] = has_z ? dyv * silu(io<Tin>::to_f(rZ[c * RR + t])) : dyv;
         }
         __syncthreads();  // B, C converted, sAcc cleared
 
-        // forward: group entry states, dz and dy * silu(z)
+        // forward: the state entering every group of four steps
         {
             f2 hp[2];
             {
@@ -294,32 +297,16 @@ __global__ void __launch_bounds__(kBW * 32) scan_bwd_kernel(const BParams p) {
                 float uv[4];
                 V4::to_f(*reinterpret_cast<const VT*>(rU + cw * RR + t), uv);
                 const float dts[4] = {d4.x, d4.y, d4.z, d4.w};
-                float yp[4];
 #pragma unroll
                 for (int s = 0; s < 4; ++s) {
                     const f2 dd = pack2(dts[s], dts[s]);
                     const float q = dts[s] * uv[s];
                     const f2 qq = pack2(q, q);
                     const float4 bb = lds4(sB + (t + s) * 16 + pp * 4);
-                    const float4 cc = lds4(sC + (t + s) * 16 + pp * 4);
                     const f2 e0 = ex2x2(mul2(dd, a2p[0])), e1 = ex2x2(mul2(dd, a2p[1]));
                     hp[0] = fma2(e0, hp[0], mul2(qq, lo2(bb)));
                     hp[1] = fma2(e1, hp[1], mul2(qq, hi2(bb)));
-                    yp[s] = hsum(fma2(lo2(cc), hp[0], mul2(hi2(cc), hp[1])));
                 }
-                // lane pp finishes step t + pp of its channel
-                const int ts = t + pp;
-                const float yt = transpose_reduce4(yp, pp) + Dd * io<Tin>::to_f(rU[cw * RR + ts]);
-                const float dyv = io<Tin>::to_f(rDy[cw * RR + ts]);
-                float dyt = dyv, dzv = 0.f;
-                if (has_z) {
-                    const float zz = io<Tin>::to_f(rZ[cw * RR + ts]);
-                    const float sz = rcp(1.f + ex2(-zz * kLog2e));
-                    dyt = dyv * zz * sz;
-                    dzv = dyv * yt * sz * (1.f + zz * (1.f - sz));
-                }
-                sDyt[cw * RS + ts] = dyt;
-                rZ[cw * RR + ts] = io<Tin>::from_f(dzv);  // dz replaces z
             }
         }
         __syncwarp();
@@ -345,7 +332,7 @@ __global__ void __launch_bounds__(kBW * 32) scan_bwd_kernel(const BParams p) {
                 hs[s][0] = fma2(ab[s][0], s ? hs[s - 1][0] : hin[0], mul2(qq, lo2(bb)));
                 hs[s][1] = fma2(ab[s][1], s ? hs[s - 1][1] : hin[1], mul2(qq, hi2(bb)));
             }
-            float dqv[4], ddv[4];
+            float dqv[4], ddv[4], ypv[4];
 #pragma unroll
             for (int s = 3; s >= 0; --s) {
                 const int t = tg + s;
@@ -356,6 +343,7 @@ __global__ void __launch_bounds__(kBW * 32) scan_bwd_kernel(const BParams p) {
                 const f2 qq = pack2(q, q);
                 gp[0] = fma2(yy, lo2(cc), gp[0]);
                 gp[1] = fma2(yy, hi2(cc), gp[1]);
+                ypv[s] = hsum(fma2(lo2(cc), hs[s][0], mul2(hi2(cc), hs[s][1])));  // C_t . h_t
                 const f2 dC0 = mul2(yy, hs[s][0]), dC1 = mul2(yy, hs[s][1]);
                 const f2 dB0 = mul2(gp[0], qq), dB1 = mul2(gp[1], qq);
                 dqv[s] = hsum(fma2(gp[0], lo2(bb), mul2(gp[1], hi2(bb))));
@@ -400,8 +388,16 @@ __global__ void __launch_bounds__(kBW * 32) scan_bwd_kernel(const BParams p) {
             }
             // lane pp completes step tg + pp of its channel
             const float dq = transpose_reduce4(dqv, pp), ddl = transpose_reduce4(ddv, pp);
+            const float cy = transpose_reduce4(ypv, pp);
             const int t = tg + pp;
             const float uu = io<Tin>::to_f(rU[cw * RR + t]);
+            if (has_z) {  // dz = dy * (C . h + D u) * silu'(z), replacing z in its row
+                const float zz = io<Tin>::to_f(rZ[cw * RR + t]);
+                const float sz = rcp(1.f + ex2(-zz * kLog2e));
+                const float yt = fmaf(Dd, uu, cy);
+                rZ[cw * RR + t] = io<Tin>::from_f(io<Tin>::to_f(rDy[cw * RR + t]) * yt * sz *
+                                                  (1.f + zz * (1.f - sz)));
+            }
             const float dt = sDel[cw * RS + t], dyt = sDyt[cw * RS + t];
             const float xr = io<Tin>::to_f(rDr[cw * RR + t]);
             float sg = 1.f;
