@@ -708,9 +708,30 @@ def cpu_baseline(w, budget_s=10.0):
     t = run(probe)
     nl = int(min(w.batch * w.dim, max(probe, probe * budget_s / max(t, 1e-3))))
     t = run(nl)
+    # the same loop on one thread, on a quarter of the time budget
+    prev = oracle.set_num_threads(1)
+    try:
+        t1 = run(8)
+        n1 = int(min(w.batch * w.dim, max(8, 8 * budget_s / 4 / max(t1, 1e-3))))
+        t1 = run(n1)
+    finally:
+        oracle.set_num_threads(prev)
     return {"value": nl * w.seqlen / t, "unit": "elems/s", "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(), "single_thread_value": n1 * w.seqlen / t1,
             "sample": "%d of %d channels x full L=%d (fp64, sequential per channel, %d OpenMP "
-                      "threads), %.1f s" % (nl, w.batch * w.dim, w.seqlen, cores, t)}
+                      "threads), %.1f s; single thread: %d channels, %.1f s" % (
+                          nl, w.batch * w.dim, w.seqlen, cores, t, n1, t1)}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def cpu_baseline_backward(w, budget_s=5.0):

@@ -87,6 +87,8 @@ def _load():
                 ctypes.c_int, _dp]
             lib.s6o_num_threads.restype = ctypes.c_int
             lib.s6o_num_threads.argtypes = []
+            lib.s6o_set_num_threads.restype = ctypes.c_int
+            lib.s6o_set_num_threads.argtypes = [ctypes.c_int]
             _lib = lib
     return _lib
 
@@ -108,6 +110,11 @@ def _ptr(a):
 def num_threads() -> int:
     """OpenMP threads the oracle's lane loops use."""
     return int(_load().s6o_num_threads())
+
+
+def set_num_threads(n: int) -> int:
+    """Use n OpenMP threads from now on; returns the previous count."""
+    return int(_load().s6o_set_num_threads(int(n)))
 
 
 def softplus(x: float) -> float:

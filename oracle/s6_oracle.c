@@ -365,6 +365,13 @@ int s6o_causal_conv1d_update(long nrows, long K, double* state, const double* x,
 #ifdef _OPENMP
 #include <omp.h>
 int s6o_num_threads(void) { return omp_get_max_threads(); }
+/* Threads for the following parallel loops (n >= 1); returns the previous setting. */
+int s6o_set_num_threads(int n) {
+    int old = omp_get_max_threads();
+    if (n >= 1) omp_set_num_threads(n);
+    return old;
+}
 #else
 int s6o_num_threads(void) { return 1; }
+int s6o_set_num_threads(int n) { (void)n; return 1; }
 #endif

@@ -78,3 +78,14 @@ def test_committed_profile_traffic_is_found_for_unchanged_kernels(tmp_path, monk
     assert bench.profile_traffic("k.txt", "k.cu") == 1234.0
     src.write_text("kernel v2")
     assert bench.profile_traffic("k.txt", "k.cu") is None
+
+
+def test_cpu_baseline_reports_all_cores_and_one_thread():
+    import bench
+    import oracle
+    from selective_state_space_56_b200 import inputs
+    before = oracle.num_threads()
+    r = bench.cpu_baseline(inputs.SCAN_WORKLOADS["tiny_fp32"], budget_s=0.05)
+    assert r["kind"] == "oracle" and r["value"] > 0 and r["single_thread_value"] > 0
+    assert r["cores"] == before and oracle.num_threads() == before  # setting restored
+    assert r["cpu_model"]
