@@ -338,6 +338,16 @@ int mamba_causal_conv1d_update(void* conv_state, const void* x, const float* wei
 int mamba_check_device_error(int clear, void* stream);
 
 /*
+ * Diagnostic for the failure-detection path: launches one bounded device-side wait on a
+ * barrier that nothing completes.  It gives up after limit_cycles SM clocks (1 to 4e9;
+ * about 2e6 per millisecond) and sets the device error word exactly as a lost transfer
+ * in the scan would, so mamba_check_device_error then returns MAMBA_ERR_TIMEOUT.  No
+ * fault, trap or unbounded wait is involved and the context stays usable.
+ * Errors: DIMS (limit out of range), CUDA.
+ */
+int mamba_diag_wait_timeout(int64_t limit_cycles, void* stream);
+
+/*
  * Diagnostic: evaluates 2^x for n floats three ways on the device -- the FMA-pipe
  * polynomial the scan uses for part of its Abar factors (out_fma), the SFU
  * ex2.approx instruction (out_sfu) and CUDA's exp2f (out_lib) -- so tests can bound

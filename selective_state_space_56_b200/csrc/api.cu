@@ -403,6 +403,12 @@ int mamba_causal_conv1d_update(void* conv_state, const void* x, const float* wei
     return cuda_status(s6::launch_conv1d_update(a, static_cast<cudaStream_t>(stream)));
 }
 
+int mamba_diag_wait_timeout(int64_t limit_cycles, void* stream) {
+    if (limit_cycles < 1 || limit_cycles > 4000000000LL) return MAMBA_ERR_DIMS;
+    return cuda_status(s6::launch_wait_timeout_probe((long long)limit_cycles,
+                                                     static_cast<cudaStream_t>(stream)));
+}
+
 int mamba_check_device_error(int clear, void* stream) {
     unsigned word = 0;
     if (s6::read_device_error(&word, clear != 0, static_cast<cudaStream_t>(stream)) != cudaSuccess)

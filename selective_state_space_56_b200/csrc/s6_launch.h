@@ -131,6 +131,10 @@ struct ConvUpdateArgs {
 cudaError_t launch_conv1d(const ConvArgs& a, cudaStream_t stream);
 cudaError_t launch_conv1d_update(const ConvUpdateArgs& a, cudaStream_t stream);
 
+// One bounded device wait that nothing completes: sets bit 0 of the device error word
+// after limit_cycles SM clocks.
+cudaError_t launch_wait_timeout_probe(long long limit_cycles, cudaStream_t stream);
+
 // Reads (and optionally clears) the device error word on `stream`, synchronising it.
 // Bit 0: a bounded device-side wait gave up.
 cudaError_t read_device_error(unsigned* out, bool clear, cudaStream_t stream);

@@ -700,6 +700,19 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
     }
 }
 
+// Failure-detection probe: one bounded wait on an mbarrier that nothing ever completes.
+// It gives up after limit_cycles SM clocks and records that in the device error word, as
+// any bounded wait of the scan does -- so the host's detection path can be exercised
+// without a fault.
+__global__ void wait_timeout_probe_kernel(long long limit_cycles) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+        if (!mbar_wait_bounded(&bar, 0, limit_cycles)) atomicOr(&g_device_error, 1u);
+    }
+}
+
 // Fold the segments left to right.  Thread per (batch, channel, state):
 // on entry seg_h[s] holds segment s's end state from h = 0 (s < nseg - 1) and
 // seg_sum[s] its summed step; on exit seg_h[s] holds segment s's true start state
@@ -989,6 +1002,11 @@ cudaError_t launch_scan_summary(const ScanArgs& a, float* h_end, float* dsum, cu
     if (e != cudaSuccess || a.nseg <= 1) return e;
     return launch_fold(a.seg_h, a.seg_sum, a.A, nullptr, a.nseg, a.batch, a.dim, a.N, h_end, dsum,
                        stream);
+}
+
+cudaError_t launch_wait_timeout_probe(long long limit_cycles, cudaStream_t stream) {
+    wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(limit_cycles);
+    return cudaGetLastError();
 }
 
 cudaError_t read_device_error(unsigned* out, bool clear, cudaStream_t stream) {

@@ -85,6 +85,8 @@ def load_library():
             lib.mamba_status_string.argtypes = [i32]
             lib.mamba_check_device_error.restype = i32
             lib.mamba_check_device_error.argtypes = [i32, vp]
+            lib.mamba_diag_wait_timeout.restype = i32
+            lib.mamba_diag_wait_timeout.argtypes = [i64, vp]
             lib.mamba_diag_exp2.restype = i32
             lib.mamba_diag_exp2.argtypes = [vp, vp, vp, vp, i64, vp]
             lib.mamba_abi_version.restype = i32
@@ -130,6 +132,16 @@ def check_device_error(clear: bool = True, device=None) -> None:
         rc = load_library().mamba_check_device_error(int(bool(clear)), _stream_handle(dev))
     if rc != 0:
         raise MambaError(rc, "mamba_check_device_error")
+
+
+def diag_wait_timeout(limit_cycles: int = 2_000_000, device=None) -> None:
+    """Launch one bounded device wait that nothing completes (it gives up after
+    limit_cycles SM clocks and sets the device error word); for testing detection."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        rc = load_library().mamba_diag_wait_timeout(int(limit_cycles), _stream_handle(dev))
+    if rc != 0:
+        raise MambaError(rc, "mamba_diag_wait_timeout")
 
 
 def diag_exp2(x):

@@ -233,3 +233,9 @@ def test_conv1d_host_checks(lib):
     assert upd(vp(A16), vp(A16), vp(A16), None, vp(A16), 2, 64, 7, 1, 1, None) == ERR_DIMS
     assert upd(vp(A16), vp(A16), vp(A16), None, vp(A16), 70000, 4, 4, 1, 1, None) == ERR_DIMS
     assert upd(vp(A16), vp(A16 + 4), vp(A16), None, vp(A16), 2, 64, 4, 1, 1, None) == ERR_ALIGN
+
+
+def test_diag_wait_timeout_rejects_bad_limits(lib):
+    assert lib.mamba_diag_wait_timeout(0, None) == ERR_DIMS
+    assert lib.mamba_diag_wait_timeout(-5, None) == ERR_DIMS
+    assert lib.mamba_diag_wait_timeout(5_000_000_000, None) == ERR_DIMS
