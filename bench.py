@@ -611,7 +611,37 @@ def run_backward(g, dev, stream, world, w, steps=50):
     # then swept), softplus, sigmoid of the step (softplus'), sigmoid of the gate (ex2, rcp)
     sfu = elems * (2 * n + 4)
     byts = backward_bytes(b, d, n, L)
-    del dy, ws
+
+    # a training step: the forward recording the checkpoints, then the backward from them
+    y = torch.empty((b, d, L), dtype=w.out_dtype, device=dev)
+
+    def train_step():
+        ops.selective_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                               delta_bias=g["delta_bias"], y=y, checkpoints=ws)
+        return ops.selective_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dy, D=g["D"],
+                                      z=g["z"], delta_bias=g["delta_bias"], checkpoints=ws)
+
+    for _ in range(3):
+        train_step()
+    torch.cuda.synchronize(dev)
+    tevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(steps)]
+    for a, b_ in tevs:
+        a.record(stream)
+        train_step()
+        b_.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_train = max_over_ranks(statistics.fmean(a.elapsed_time(b_) for a, b_ in tevs), world)
+    sfu_train = elems * (3 * n + 6)  # forward N + 2, backward 2N + 4
+    train = {"ms_per_step": ms_train, "value": world * elems / (ms_train * 1e-3),
+             "unit": "elems/s",
+             "what": "forward recording the backward's checkpoints, then the backward from "
+                     "them (no checkpointing pass of its own)",
+             "roofline": {"bound": "alu", "unit": "Gop/s (SFU)",
+                          "achieved": sfu_train / (ms_train * 1e-3) / 1e9,
+                          "peak": sfu_peak / 1e9, "frac": sfu_train / (ms_train * 1e-3) / sfu_peak,
+                          "sfu_ops_per_elem": 3 * n + 6}}
+    del dy, ws, y
     return {
         "metric": "selective-scan bwd (b·d·L) elems/s", "unit": "elems/s",
         "value": world * elems / (ms * 1e-3), "ms_per_call": ms, "steps": steps,
@@ -624,7 +654,8 @@ def run_backward(g, dev, stream, world, w, steps=50):
                      "hbm_frac": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "peak_kind": kind,
                      "traffic": profile_traffic("scan_bwd_m2p8b.txt",
                                                 "selective_state_space_56_b200/csrc/scan_bwd.cu")},
-        "gpu_launches": 2 * steps + 6,
+        "train_step": train,
+        "gpu_launches": 2 * steps + 6 + 2 * (steps + 3),
     }
 
 

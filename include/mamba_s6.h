@@ -291,6 +291,39 @@ int mamba_selective_scan_bwd(const void* u, const void* delta, const float* A, c
                              void* stream);
 
 /*
+ * Training forward: mamba_selective_scan_fwd that also records the backward's checkpoints
+ * (the state entering every 16 steps for dstate > 8, every 64 otherwise -- the layout the
+ * backward's own recomputing pass writes), so that a following
+ * mamba_selective_scan_bwd_from_checkpoints needs no forward pass of its own.
+ *
+ *   checkpoints      : device buffer of at least mamba_selective_scan_bwd_workspace_size(dims)
+ *                      bytes, written (may be NULL when seqlen == 0)
+ *   everything else  : as mamba_selective_scan_fwd (no flags: the Delta * B form)
+ *
+ * Errors: as mamba_selective_scan_fwd, plus WORKSPACE when checkpoint_bytes is too small.
+ */
+int mamba_selective_scan_fwd_train(const void* u, const void* delta, const float* A,
+                                   const void* B, const void* C, const float* D, const void* z,
+                                   const float* delta_bias, int delta_softplus, void* y,
+                                   float* last_state, mamba_scan_dims dims, mamba_dtype in_dtype,
+                                   mamba_dtype out_dtype, void* workspace,
+                                   size_t workspace_bytes, float* checkpoints,
+                                   size_t checkpoint_bytes, void* stream);
+
+/*
+ * mamba_selective_scan_bwd from the checkpoints a mamba_selective_scan_fwd_train call
+ * recorded for the same inputs (read only): the same gradients, without the backward's
+ * own checkpointing forward pass.  Arguments as mamba_selective_scan_bwd with the
+ * checkpoints in place of the workspace.
+ */
+int mamba_selective_scan_bwd_from_checkpoints(
+    const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int delta_softplus, const void* dy,
+    void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC, float* dD,
+    float* ddelta_bias, mamba_scan_dims dims, mamba_dtype in_dtype, const float* checkpoints,
+    size_t checkpoint_bytes, void* stream);
+
+/*
  * Causal depthwise conv1d with an optional SiLU: the Mamba block's step between the input
  * projection and the SSM (Mamba, section "Mamba Block": input projections, a 1-D
  * convolution, the selective SSM and gating; page "yongjin360.com/news/29389", Q&A on

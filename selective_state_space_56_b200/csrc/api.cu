@@ -41,7 +41,14 @@ int scan_fwd(const void* u, const void* delta, const float* A, const void* B, co
              const float* D, const void* z, const float* delta_bias, int delta_softplus,
              const float* h0, void* y, float* last_state, mamba_scan_dims dims,
              mamba_dtype in_dtype, mamba_dtype out_dtype, void* workspace,
-             size_t workspace_bytes, unsigned flags, void* stream);
+             size_t workspace_bytes, unsigned flags, void* stream, float* ckpt = nullptr,
+             size_t ckpt_bytes = 0);
+
+int scan_bwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
+             const float* D, const void* z, const float* delta_bias, int delta_softplus,
+             const void* dy, void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC,
+             float* dD, float* ddelta_bias, mamba_scan_dims dims, mamba_dtype in_dtype,
+             void* ckpt, size_t ckpt_bytes, bool ckpt_ready, void* stream);
 
 int state_update(float* state, const void* u, const void* delta, const float* A, const void* B,
                  const void* C, const float* D, const void* z, const float* delta_bias,
@@ -142,6 +149,7 @@ int mamba_selective_scan_summary(const void* u, const void* delta, const float* 
     a.seg_h = nullptr;
     a.seg_sum = nullptr;
     a.h0 = nullptr;
+    a.ckpt = nullptr;
     if (nseg > 1) {
         a.seg_h = static_cast<float*>(workspace);
         a.seg_sum = a.seg_h + nseg * dims.batch * dims.dim * dims.dstate;
@@ -170,7 +178,8 @@ int scan_fwd(const void* u, const void* delta, const float* A, const void* B, co
              const float* D, const void* z, const float* delta_bias, int delta_softplus,
              const float* h0, void* y, float* last_state, mamba_scan_dims dims,
              mamba_dtype in_dtype, mamba_dtype out_dtype, void* workspace,
-             size_t workspace_bytes, unsigned flags, void* stream) {
+             size_t workspace_bytes, unsigned flags, void* stream, float* ckpt,
+             size_t ckpt_bytes) {
     if (flags & ~kKnownFlags) return MAMBA_ERR_FLAGS;
     // With seqlen == 0 the (batch, dim, 0) and (batch, dstate, 0) arrays are empty and
     // may be NULL; only last_state (zeros) is written.
@@ -178,9 +187,11 @@ int scan_fwd(const void* u, const void* delta, const float* A, const void* B, co
     if (!A || (!empty && (!u || !delta || !B || !C || !y))) return MAMBA_ERR_NULL;
     if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return MAMBA_ERR_DTYPE;
     if (!dims_ok(dims.batch, dims.dim, dims.dstate, dims.seqlen)) return MAMBA_ERR_DIMS;
-    const void* ptrs[] = {u, delta, A, B, C, D, z, delta_bias, y, last_state, h0};
+    const void* ptrs[] = {u, delta, A, B, C, D, z, delta_bias, y, last_state, h0, ckpt};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return MAMBA_ERR_ALIGN;
+    if (ckpt && ckpt_bytes < mamba_selective_scan_bwd_workspace_size(dims))
+        return MAMBA_ERR_WORKSPACE;
 
     int64_t nseg = 1, seg_len = 0;
     s6::plan_segments(dims.batch, dims.dim, dims.seqlen, &nseg, &seg_len);
@@ -215,6 +226,7 @@ int scan_fwd(const void* u, const void* delta, const float* A, const void* B, co
     a.seg_h = nullptr;
     a.seg_sum = nullptr;
     a.h0 = h0;
+    a.ckpt = ckpt;
     if (nseg > 1) {
         a.seg_h = static_cast<float*>(workspace);
         a.seg_sum = a.seg_h + nseg * dims.batch * dims.dim * dims.dstate;
@@ -292,6 +304,44 @@ int mamba_selective_scan_bwd(const void* u, const void* delta, const float* A, c
                              float* dD, float* ddelta_bias, mamba_scan_dims dims,
                              mamba_dtype in_dtype, void* workspace, size_t workspace_bytes,
                              void* stream) {
+    return scan_bwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, dy, du, ddelta, dz, dA,
+                    dB, dC, dD, ddelta_bias, dims, in_dtype, workspace, workspace_bytes, false,
+                    stream);
+}
+
+int mamba_selective_scan_fwd_train(const void* u, const void* delta, const float* A,
+                                   const void* B, const void* C, const float* D, const void* z,
+                                   const float* delta_bias, int delta_softplus, void* y,
+                                   float* last_state, mamba_scan_dims dims, mamba_dtype in_dtype,
+                                   mamba_dtype out_dtype, void* workspace,
+                                   size_t workspace_bytes, float* checkpoints,
+                                   size_t checkpoint_bytes, void* stream) {
+    if (!checkpoints && dims.seqlen > 0) return MAMBA_ERR_NULL;
+    return scan_fwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, y, last_state,
+                    dims, in_dtype, out_dtype, workspace, workspace_bytes, 0u, stream,
+                    dims.seqlen > 0 ? checkpoints : nullptr, checkpoint_bytes);
+}
+
+int mamba_selective_scan_bwd_from_checkpoints(
+    const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int delta_softplus, const void* dy,
+    void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC, float* dD,
+    float* ddelta_bias, mamba_scan_dims dims, mamba_dtype in_dtype, const float* checkpoints,
+    size_t checkpoint_bytes, void* stream) {
+    return scan_bwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, dy, du, ddelta, dz, dA,
+                    dB, dC, dD, ddelta_bias, dims, in_dtype, const_cast<float*>(checkpoints),
+                    checkpoint_bytes, true, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+int scan_bwd(const void* u, const void* delta, const float* A, const void* B, const void* C,
+             const float* D, const void* z, const float* delta_bias, int delta_softplus,
+             const void* dy, void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC,
+             float* dD, float* ddelta_bias, mamba_scan_dims dims, mamba_dtype in_dtype,
+             void* workspace, size_t workspace_bytes, bool ckpt_ready, void* stream) {
     const bool empty = dims.seqlen == 0;
     if (!A || !dA) return MAMBA_ERR_NULL;
     if (!empty && (!u || !delta || !B || !C || !dy || !du || !ddelta || !dB || !dC))
@@ -335,6 +385,7 @@ int mamba_selective_scan_bwd(const void* u, const void* delta, const float* A, c
     a.seg_h = nullptr;
     a.seg_sum = nullptr;
     a.h0 = nullptr;
+    a.ckpt = nullptr;
     s6::BackwardArgs g;
     g.dy = dy;
     g.du = du;
@@ -346,8 +397,12 @@ int mamba_selective_scan_bwd(const void* u, const void* delta, const float* A, c
     g.dD = dD;
     g.ddelta_bias = ddelta_bias;
     return cuda_status(s6::launch_scan_backward(a, g, static_cast<float*>(workspace),
-                                                static_cast<cudaStream_t>(stream)));
+                                                static_cast<cudaStream_t>(stream), ckpt_ready));
 }
+
+}  // namespace
+
+extern "C" {
 
 int mamba_causal_conv1d_fwd(const void* x, const float* weight, const float* bias,
                             const void* initial_state, void* out, void* final_state,

@@ -29,6 +29,7 @@ struct ScanArgs {
     float* seg_h;    // (nseg, batch, dim, N)
     float* seg_sum;  // (nseg, batch, dim)
     const float* h0;  // (batch, dim, N) initial state or null (zero)
+    float* ckpt;      // backward checkpoints to record, or null (layout of launch_scan_checkpoints)
 };
 
 struct StateUpdateArgs {
@@ -97,10 +98,10 @@ struct BackwardArgs {
 
 // Backward of the scan described by `a` (its y, last_state and segment fields are
 // unused): zeroes the accumulated outputs, runs the checkpointing forward into
-// `ckpt` (batch * dim * ceil(L / checkpoint_steps(N)) * N floats) and then the
-// reverse sweep.
+// `ckpt` (batch * dim * ceil(L / checkpoint_steps(N)) * N floats) -- unless ckpt_ready,
+// when a training forward has recorded them already -- and then the reverse sweep.
 cudaError_t launch_scan_backward(const ScanArgs& a, const BackwardArgs& g, float* ckpt,
-                                 cudaStream_t stream);
+                                 cudaStream_t stream, bool ckpt_ready = false);
 
 // Causal depthwise conv1d (+ SiLU) over (batch, dim, L) rows, 1 <= width <= 4.
 struct ConvArgs {

@@ -515,7 +515,7 @@ int pick_block_steps(int64_t ctas) {
 }  // namespace
 
 cudaError_t launch_scan_backward(const ScanArgs& a, const BackwardArgs& g, float* ckpt,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, bool ckpt_ready) {
     // checkpoints every CK steps; the kernel walks blocks of T = CK (or 2 CK) steps
     const int CK = checkpoint_steps(a.N);
     const int64_t ctas = (a.dim + kBCH - 1) / kBCH * a.batch;
@@ -537,7 +537,7 @@ cudaError_t launch_scan_backward(const ScanArgs& a, const BackwardArgs& g, float
         (e = cudaMemsetAsync(g.ddelta_bias, 0, (size_t)a.dim * sizeof(float), stream)) != cudaSuccess)
         return e;
     if (a.L == 0) return cudaSuccess;
-    if ((e = launch_scan_checkpoints(a, ckpt, stream)) != cudaSuccess) return e;
+    if (!ckpt_ready && (e = launch_scan_checkpoints(a, ckpt, stream)) != cudaSuccess) return e;
     BParams bp;
     memset(&bp, 0, sizeof(bp));
     bp.u = a.u;

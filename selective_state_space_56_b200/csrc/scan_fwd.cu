@@ -67,6 +67,7 @@ struct KParams {
     float* last_state;
     float* seg_h;
     float* seg_sum;
+    float* ckpt;  // checkpoint modes: (batch, dim, blocks, N)
     int64_t batch, dim, L, seg_len;
     int N;
     int nseg;
@@ -95,8 +96,9 @@ __device__ __forceinline__ void store4(__nv_bfloat16* dst, const float (&o)[4]) 
 
 // kFull: the scan itself; kAggregate: split-sequence pass 1 (end state and summed step
 // per segment, no output); kCheckpoint: the backward's forward pass (the state at the
-// start of every chunk, no output).
-enum Mode : int { kFull = 0, kAggregate = 1, kCheckpoint = 2 };
+// start of every checkpoint block, no output); kFullCkpt: the scan that also records
+// those checkpoints (a training forward, so the backward needs no pass of its own).
+enum Mode : int { kFull = 0, kAggregate = 1, kCheckpoint = 2, kFullCkpt = 3 };
 
 // Tuning of the N = 16 instantiation: lanes per channel, warps per CTA, chunk length.
 #ifndef S6_P16
@@ -196,6 +198,8 @@ template <int NMAX, int P, int WARPS, int T_, typename Tin, typename Tout, int M
 __global__ void __launch_bounds__(WARPS * 32 + (WS ? 32 : 0))
 scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
     static_assert(!WS || (TMA && MODE == kFull), "producer warp: TMA full scans only");
+    constexpr bool kOut = MODE == kFull || MODE == kFullCkpt;         // writes y
+    constexpr bool kCk = MODE == kCheckpoint || MODE == kFullCkpt;    // writes checkpoints
     using Lo = Layout<NMAX, P, WARPS, T_, Tin, Tout>;
     using V4 = vec4<Tin>;
     using VT = typename V4::type;
@@ -215,8 +219,8 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
     const int64_t t_begin = (int64_t)seg * p.seg_len;
     const int64_t t_end = min(p.L, t_begin + p.seg_len);
     const int64_t nchunks = t_end > t_begin ? (t_end - t_begin + T - 1) / T : 0;
-    const bool has_z = (MODE == kFull) && p.z != nullptr;
-    const bool out_tma = TMA && (MODE == kFull) && p.y_tma;
+    const bool has_z = kOut && p.z != nullptr;
+    const bool out_tma = TMA && kOut && p.y_tma;
 
     for (int c = tid; c < CH; c += Lo::THREADS) {
         const int64_t d = d0 + c;
@@ -251,7 +255,7 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
             const bool ok = dch < p.dim && nn < p.N;
             a[q] = ok ? p.A[dch * p.N + nn] * kLog2e : 0.f;  // padded states: Abar = 1, b = 0
             // initial state: the segment's start (split sequences) or the caller's h0
-            h[q] = (MODE == kFull && p.seg_h != nullptr && ok)
+            h[q] = (kOut && p.seg_h != nullptr && ok)
                        ? p.seg_h[(((int64_t)seg * p.batch + b) * p.dim + dch) * p.N + nn]
                        : 0.f;
         }
@@ -493,7 +497,7 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
             const int64_t blocks = (p.L + CKPT - 1) / CKPT;
             const int64_t kb = (t0 + t) / CKPT;
             if (dch >= p.dim || t0 + t >= p.L) return;
-            float* ck = p.seg_h + ((b * p.dim + dch) * blocks + kb) * p.N;
+            float* ck = p.ckpt + ((b * p.dim + dch) * blocks + kb) * p.N;
 #pragma unroll
             for (int j = 0; j < NS / 2; ++j) {
                 float h0, h1;
@@ -502,12 +506,12 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
                 if (pp * NS + 2 * j + 1 < p.N) ck[pp * NS + 2 * j + 1] = h1;
             }
         };
-        if (MODE == kCheckpoint) write_ckpt(0);
+        if (kCk) write_ckpt(0);
 
         // Phase B: the recurrence, four steps per iteration, states in packed pairs.
 #pragma unroll
         for (int t = 0; t < T; t += 4) {
-            if (MODE == kCheckpoint && t > 0 && t % CKPT == 0) write_ckpt(t);
+            if (kCk && t > 0 && t % CKPT == 0) write_ckpt(t);
             const float4 d4 = *reinterpret_cast<const float4*>(sDel + cw * RS + t);
             const float4 q4 = *reinterpret_cast<const float4*>(sDu + cw * RS + t);
             const f2 dd4[4] = {pack2(d4.x, d4.x), pack2(d4.y, d4.y), pack2(d4.z, d4.z),
@@ -612,7 +616,7 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
             }
         }
 
-        if (MODE == kFull) {
+        if (kOut) {
             // Phase C: skip term, gate; four steps per lane into this warp's rows of the
             // output tile, which its lane 0 then stores with TMA (or straight to global
             // memory when rows cannot be described to TMA).  The warp's previous store
@@ -680,7 +684,7 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         float h[NS];
 #pragma unroll
         for (int j = 0; j < NS / 2; ++j) unpack2(hp[j], h[2 * j], h[2 * j + 1]);
-        if (MODE == kFull) {
+        if (kOut) {
             if (p.last_state && seg == (int)gridDim.z - 1) {
 #pragma unroll
                 for (int n = 0; n < NS; ++n) {
@@ -831,6 +835,11 @@ cudaError_t launch_typed(const ScanArgs& a, const KParams& kp, const TMaps& tm, 
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
+    if constexpr (!ZOH) {
+        if (a.ckpt)
+            return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFullCkpt, TMA, false>(
+                kp, tm, dim3(gx, (unsigned)a.batch, (unsigned)a.nseg), s);
+    }
     return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA, ZOH, TMA && S6_WS>(
         kp, tm, dim3(gx, (unsigned)a.batch, (unsigned)a.nseg), s);
 }
@@ -956,7 +965,7 @@ cudaError_t launch_scan_checkpoints(const ScanArgs& a, float* ckpt, cudaStream_t
     kp.B = a.B;
     kp.C = a.C;
     kp.delta_bias = a.delta_bias;
-    kp.seg_h = ckpt;
+    kp.ckpt = ckpt;
     kp.batch = a.batch;
     kp.dim = a.dim;
     kp.L = a.L;
@@ -1057,6 +1066,7 @@ cudaError_t launch_scan(const ScanArgs& a, cudaStream_t stream) {
     kp.last_state = a.last_state;
     // with one segment the kernel reads its initial state through seg_h (read only)
     kp.seg_h = a.nseg > 1 ? a.seg_h : const_cast<float*>(a.h0);
+    kp.ckpt = a.ckpt;
     kp.seg_sum = a.seg_sum;
     kp.batch = a.batch;
     kp.dim = a.dim;

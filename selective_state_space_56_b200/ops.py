@@ -63,6 +63,13 @@ def load_library():
             lib.mamba_selective_scan_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp,
                                                         vp, ScanDims, i32, i32, vp,
                                                         ctypes.c_size_t, u32, vp]
+            lib.mamba_selective_scan_fwd_train.restype = i32
+            lib.mamba_selective_scan_fwd_train.argtypes = [vp] * 8 + [i32, vp, vp, ScanDims, i32,
+                                                               i32, vp, ctypes.c_size_t, vp,
+                                                               ctypes.c_size_t, vp]
+            lib.mamba_selective_scan_bwd_from_checkpoints.restype = i32
+            lib.mamba_selective_scan_bwd_from_checkpoints.argtypes = [vp] * 8 + [i32] + [vp] * 9 + [
+                ScanDims, i32, vp, ctypes.c_size_t, vp]
             lib.mamba_selective_scan_fwd_init.restype = i32
             lib.mamba_selective_scan_fwd_init.argtypes = [vp] * 8 + [i32] + [vp] * 3 + [
                 ScanDims, i32, i32, vp, ctypes.c_size_t, u32, vp]
@@ -165,12 +172,14 @@ def selective_scan_workspace_size(batch: int, dim: int, dstate: int, seqlen: int
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
                        out_dtype=None, y=None, last_state=None, return_last_state=False,
-                       workspace=None, exact_zoh=False, initial_state=None):
+                       workspace=None, exact_zoh=False, initial_state=None, checkpoints=None):
     """Fused selective scan.  u, delta, z: (batch, dim, L); A: (dim, N) fp32;
     B, C: (batch, N, L); D, delta_bias: (dim) fp32.  Returns y (batch, dim, L)
     [and last_state (batch, dim, N) fp32].  exact_zoh: Bbar = (exp(Delta A) - 1) / A * B
     instead of Delta * B.  initial_state: (batch, dim, N) fp32 state before the sequence
-    (zero when None)."""
+    (zero when None).  checkpoints: a uint8 CUDA tensor of at least
+    selective_scan_bwd_workspace_size(...) bytes to record the backward's checkpoints in
+    (a training forward; not with exact_zoh or initial_state)."""
     if not isinstance(u, torch.Tensor) or u.dim() != 3:
         raise ValueError("u must be a (batch, dim, L) tensor")
     dev = u.device
@@ -209,8 +218,15 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
             int(bool(delta_softplus)), _ptr(y), _ptr(last_state), dims, _DTYPES[in_dt],
             _DTYPES[out_dt], _ptr(workspace), ws_bytes)
     flags = MAMBA_FLAG_EXACT_ZOH if exact_zoh else 0
+    if checkpoints is not None and (exact_zoh or initial_state is not None):
+        raise ValueError("checkpoints are recorded by the plain forward only")
     with torch.cuda.device(dev):
-        if initial_state is not None:
+        if checkpoints is not None:
+            _check(checkpoints, "checkpoints", dev)
+            rc = lib.mamba_selective_scan_fwd_train(
+                *args, _ptr(checkpoints), checkpoints.numel() * checkpoints.element_size(),
+                _stream_handle(dev))
+        elif initial_state is not None:
             rc = lib.mamba_selective_scan_fwd_init(*args[:9], _ptr(initial_state), *args[9:], flags,
                                                    _stream_handle(dev))
         elif exact_zoh:
@@ -225,11 +241,13 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
 
 
 def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
-                       delta_softplus=True, workspace=None):
+                       delta_softplus=True, workspace=None, checkpoints=None):
     """Gradients of ``selective_scan_fwd`` for the upstream gradient dy (batch, dim, L),
     in the inputs' dtype.  Returns a dict with du, ddelta, dz (input dtype, dz None
     without a gate), dA (dim, N), dB, dC (batch, N, L), dD, ddelta_bias (dim) in fp32
-    (None where the input is None)."""
+    (None where the input is None).  checkpoints: the buffer a training forward
+    (selective_scan_fwd(..., checkpoints=...)) filled for the same inputs; the backward
+    then skips its own checkpointing pass."""
     if not isinstance(u, torch.Tensor) or u.dim() != 3:
         raise ValueError("u must be a (batch, dim, L) tensor")
     dev = u.device
@@ -257,6 +275,18 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
              ddelta_bias=None if delta_bias is None else torch.empty(d, dtype=f32, device=dev))
     lib = load_library()
     dims = ScanDims(b, d, N, L)
+    if checkpoints is not None:
+        _check(checkpoints, "checkpoints", dev)
+        with torch.cuda.device(dev):
+            rc = lib.mamba_selective_scan_bwd_from_checkpoints(
+                _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                _ptr(delta_bias), int(bool(delta_softplus)), _ptr(dy), _ptr(g["du"]),
+                _ptr(g["ddelta"]), _ptr(g["dz"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]),
+                _ptr(g["dD"]), _ptr(g["ddelta_bias"]), dims, _DTYPES[dt], _ptr(checkpoints),
+                checkpoints.numel() * checkpoints.element_size(), _stream_handle(dev))
+        if rc != 0:
+            raise MambaError(rc, "mamba_selective_scan_bwd_from_checkpoints")
+        return g
     need = int(lib.mamba_selective_scan_bwd_workspace_size(dims))
     if need > 0 and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)

@@ -239,3 +239,17 @@ def test_diag_wait_timeout_rejects_bad_limits(lib):
     assert lib.mamba_diag_wait_timeout(0, None) == ERR_DIMS
     assert lib.mamba_diag_wait_timeout(-5, None) == ERR_DIMS
     assert lib.mamba_diag_wait_timeout(5_000_000_000, None) == ERR_DIMS
+
+
+def test_training_entry_points_check_the_checkpoint_buffer(lib):
+    vp = ctypes.c_void_p
+    need = lib.mamba_selective_scan_bwd_workspace_size(_dims())
+    base = [vp(A16)] * 5 + [None, None, None, 1, vp(A16), None, _dims(), 0, 0, None, 0]
+    assert lib.mamba_selective_scan_fwd_train(*base, None, 0, None) == ERR_NULL
+    assert lib.mamba_selective_scan_fwd_train(*base, vp(A16), need - 1, None) == ERR_WORKSPACE
+    assert lib.mamba_selective_scan_fwd_train(*base, vp(A16 + 8), need, None) == ERR_ALIGN
+    bw = [vp(A16)] * 5 + [None, None, None, 1] + [vp(A16)] * 3 + [None] + [vp(A16)] * 3 + \
+        [None, None, _dims(), 1]
+    assert lib.mamba_selective_scan_bwd_from_checkpoints(*bw, vp(A16), need - 1, None) == \
+        ERR_WORKSPACE
+    assert lib.mamba_selective_scan_bwd_from_checkpoints(*bw, None, need, None) == ERR_WORKSPACE

@@ -1,0 +1,68 @@
+"""The training path (needs a B200): a forward that records the backward's checkpoints
+(mamba_selective_scan_fwd_train) and the backward that reads them
+(mamba_selective_scan_bwd_from_checkpoints).  The forward's outputs must equal the plain
+forward's bit for bit, and the gradients must equal those of the recomputing backward:
+bit for bit where no atomics are involved, when the sequence is scanned in one pass; dA,
+dB, dC, dD and ddelta_bias are sums formed with atomics, whose order varies, so they are
+compared to 1e-5 relative.  A sequence long enough to be split has its segment starts
+folded from segment summaries in the training forward but recomputed straight through by
+the backward's own pass, so the states -- and the gradients that depend on them -- agree
+to rounding there (du, which depends on no state, still bit for bit)."""
+import pytest
+import torch
+
+from selective_state_space_56_b200 import inputs, ops
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.mark.parametrize("shape,dtype", [((2, 40, 16, 200), torch.bfloat16),
+                                         ((1, 64, 16, 40000), torch.bfloat16),  # split plan
+                                         ((2, 33, 5, 130), torch.float32),      # 64-step blocks
+                                         ((3, 24, 16, 77), torch.float32),      # ragged, no TMA
+                                         ((1, 16, 16, 1), torch.float32)],
+                         ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
+def test_training_forward_and_backward_match(cuda_ok, shape, dtype):
+    b, d, N, L = shape
+    p = inputs.scan_inputs(b, d, N, L, dtype, seed=L + d, device=DEV)
+    gen = torch.Generator(device=DEV).manual_seed(3)
+    dy = torch.randn(b, d, L, generator=gen, device=DEV).to(dtype)
+    ck = torch.empty(ops.selective_scan_bwd_workspace_size(b, d, N, L), dtype=torch.uint8,
+                     device=DEV)
+    y_t, st_t = ops.selective_scan_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"],
+                                       z=p["z"], delta_bias=p["delta_bias"],
+                                       return_last_state=True, checkpoints=ck)
+    y_p, st_p = ops.selective_scan_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"],
+                                       z=p["z"], delta_bias=p["delta_bias"],
+                                       return_last_state=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y_t, y_p) and torch.equal(st_t, st_p)
+    g_c = ops.selective_scan_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"],
+                                 z=p["z"], delta_bias=p["delta_bias"], checkpoints=ck)
+    g_r = ops.selective_scan_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"],
+                                 z=p["z"], delta_bias=p["delta_bias"])
+    torch.cuda.synchronize()
+    split = ops.selective_scan_workspace_size(b, d, N, L) > 0
+    assert torch.equal(g_c["du"], g_r["du"])
+    for k in ("ddelta", "dz"):
+        if not split:
+            assert torch.equal(g_c[k], g_r[k]), k
+        else:  # within one unit of the output dtype's rounding of the larger value
+            diff = (g_c[k].float() - g_r[k].float()).abs()
+            tol = (g_r[k].float().abs() * (2.0 ** -7 if dtype == torch.bfloat16 else 1e-5) +
+                   1e-6 * g_r[k].float().abs().max())
+            assert bool((diff <= tol).all()), k
+    for k in ("dA", "dB", "dC", "dD", "ddelta_bias"):
+        torch.testing.assert_close(g_c[k], g_r[k], rtol=1e-4 if split else 1e-5,
+                                   atol=1e-6 * g_r[k].abs().max().item())
+    ops.check_device_error()
+
+
+def test_training_forward_rejects_zoh_and_initial_state(cuda_ok):
+    p = inputs.scan_inputs(1, 8, 16, 16, torch.float32, seed=1, device=DEV)
+    ck = torch.empty(ops.selective_scan_bwd_workspace_size(1, 8, 16, 16), dtype=torch.uint8,
+                     device=DEV)
+    with pytest.raises(ValueError):
+        ops.selective_scan_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], checkpoints=ck,
+                               exact_zoh=True)
