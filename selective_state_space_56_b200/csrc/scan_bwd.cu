@@ -8,7 +8,9 @@
 // once with the larger shared-memory footprint of 32-step blocks:
 //
 //   stage     u, delta, z, dy rows and the batch's B, C for the chunk -> shared memory
-//             (16-byte cp.async copies into rows padded against bank conflicts);
+//             (16-byte cp.async copies into rows padded against bank conflicts); B, C
+//             then re-laid out per (4-step group, 4-state quad): fp32, or bf16 for bf16
+//             inputs (fewer shared-memory wavefronts for loads all 8 channels repeat);
 //   phase A   per (channel, t): Delta = softplus(delta + bias) and the gated output
 //             gradient dyt_t = dy_t silu(z_t);
 //   forward   from the checkpoint, the chunk's states are recomputed; the state
@@ -21,11 +23,11 @@
 //               g *= Abar.
 //             dq, the state part of dDelta and C_t . h_t are summed over a channel's 4
 //             lanes once per group; C_t . h_t + D u_t gives dz_t = dy_t yt_t silu'(z_t).
-//             dB and dC, shared by all channels of a batch, go through a
-//             per-warp exchange buffer: every channel stores its 32 values of a step,
-//             and after each pair of steps the warp's lanes sum them over the warp's 8
-//             channels (16-byte loads), add the sums into the CTA's chunk accumulator
-//             (shared atomics), which is added to global memory once per (t, n) and CTA;
+//             dB and dC, shared by all channels of a batch, are summed over the warp's
+//             8 channels every step (shuffles; for blocks of 16 steps) or every group
+//             (a per-warp exchange buffer, one lane per (step, quad), for longer
+//             blocks), added into the CTA's chunk accumulator (shared atomics), which is
+//             added to global memory once per (t, n) and CTA;
 //   store     du, dDelta_raw (= dDelta softplus'(x)), dz rows; dA, dD, dbias by atomics.
 //
 // State arithmetic runs on packed fp32 pairs (two states per instruction).  Gradients
@@ -71,6 +73,12 @@ struct BParams {
 #ifndef S6_BWD_WARPS
 #define S6_BWD_WARPS 4
 #endif
+// Steps per dB / dC exchange buffer.  16-step blocks sum each step's dB / dC over the
+// warp's 8 channels with shuffles (no buffer: the shared memory then holds five CTAs per
+// SM for either input type); longer blocks store them to a per-warp buffer and sum a
+// group of 4 steps at once (fewer instructions; measured faster there).
+template <int T> constexpr int exchange_steps() { return T == 16 ? 0 : 4; }
+
 constexpr int kBW = S6_BWD_WARPS;  // warps per CTA
 constexpr int kBP = 4;             // lanes per channel, 4 states each
 constexpr int kBG = 32 / kBP;      // channels per warp
@@ -95,8 +103,9 @@ struct BLayout {
     static constexpr size_t off_dyt = off_del + f;               // dy * silu(z)
     static constexpr size_t off_h = off_dyt + f;                 // fp32 [T/4][CH][16]
     static constexpr size_t off_acc = off_h + (size_t)(T / 4) * kBCH * 16 * 4;  // fp32 [T][32]
-    static constexpr size_t off_red = off_acc + (size_t)T * 32 * 4;  // per warp fp32 [2][8][32]
-    static constexpr size_t bytes = off_red + (size_t)kBW * 2 * 8 * 32 * 4;
+    static constexpr int XS = exchange_steps<T>();
+    static constexpr size_t off_red = off_acc + (size_t)T * 32 * 4;  // per warp fp32 [XS][8][32]
+    static constexpr size_t bytes = off_red + (size_t)kBW * XS * 8 * 32 * 4;
     static_assert(T % 8 == 0, "chunk length");
     static_assert((RR * sizeof(Tin)) % 16 == 0, "raw rows must stay 16-byte aligned");
 };
@@ -127,6 +136,33 @@ __device__ __forceinline__ float hsum(f2 v) {
     unpack2(v, a, b);
     return a + b;
 }
+
+// B or C of one lane's 4 states at the steps of a group.  fp32 inputs: tile fp32
+// [t][16], one 16-byte load per step.  bf16 inputs: tile of bf16 blocks
+// [t / 4][quad][step][4 states], one 8-byte load per step, widened in registers: half
+// the shared-memory wavefronts of the fp32 rows, which all 8 channels of a warp re-read.
+struct f2x2 {
+    f2 lo, hi;
+};
+template <typename Tin> struct Coef;
+template <> struct Coef<float> {
+    const float* p;
+    __device__ __forceinline__ void load(const float* tile, int tg, int pp) { p = tile + tg * 16 + pp * 4; }
+    __device__ __forceinline__ f2x2 at(int s) const {
+        const float4 v = lds4(p + s * 16);
+        return {lo2(v), hi2(v)};
+    }
+};
+template <> struct Coef<__nv_bfloat16> {
+    const uint2* p;
+    __device__ __forceinline__ void load(const float* tile, int tg, int pp) {
+        p = reinterpret_cast<const uint2*>(tile) + ((tg / 4) * 4 + pp) * 4;
+    }
+    __device__ __forceinline__ f2x2 at(int s) const {
+        const uint2 w = p[s];
+        return {bf16pair(w.x), bf16pair(w.y)};
+    }
+};
 
 // dB / dC exchange rows: channel ch of a warp stores its 32 values (8 quads: dB states
 // 0-15, then dC states 0-15) with the quad index XOR-ed by 4 for half of the channels,
@@ -218,7 +254,8 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int pp = lane & 3, cl = lane >> 2;
     const int cw = warp * kBG + cl;
-    float* sRed = reinterpret_cast<float*>(smem + Lo::off_red) + warp * (2 * 8 * 32);
+    constexpr int XS = Lo::XS;
+    float* sRed = reinterpret_cast<float*>(smem + Lo::off_red) + warp * (XS * 8 * 32);
     const int64_t b = blockIdx.y, d0 = (int64_t)blockIdx.x * kBCH, dch = d0 + cw;
     const bool chok = dch < p.dim;
     const bool has_z = p.z != nullptr;
@@ -237,8 +274,6 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
     const float Dd = (chok && p.D) ? p.D[dch] : 0.f;
     const float bias = (chok && p.delta_bias) ? p.delta_bias[dch] : 0.f;
     float dDacc = 0.f, dbacc = 0.f;
-    // reduction lane roles: step ss of a step pair, quad q of the 32 slots, channel half
-    const int rss = lane >> 4, rq = (lane >> 1) & 7, rhalf = lane & 1;
 
     for (int k = p.chunks - 1; k >= 0; --k) {
         const int64_t t0 = (int64_t)k * T;
@@ -247,11 +282,24 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
         stage_chunk<T, Tin>(p, st, b, d0, k, tid);
         __syncthreads();  // chunk k staged
 
-        // B and C to fp32 [t][n]: a warp converts two steps of all 16 states per pass
-        for (int i = tid; i < 16 * T; i += kBW * 32) {
-            const int n = i & 15, t = i >> 4;
-            sB[t * 16 + n] = io<Tin>::to_f(rB[n * RR + t]);
-            sC[t * 16 + n] = io<Tin>::to_f(rC[n * RR + t]);
+        if constexpr (sizeof(Tin) == 2) {
+            // B and C to bf16 blocks [t / 4][quad][t % 4][4 states], one (step, quad) per item
+            for (int i = tid; i < 2 * 4 * T; i += kBW * 32) {
+                const int which = i / (4 * T), t = (i / 4) % T, pq = i % 4;
+                const unsigned short* src =
+                    reinterpret_cast<const unsigned short*>(which ? rC : rB) + pq * 4 * RR + t;
+                uint2 w;
+                w.x = (uint32_t)src[0] | ((uint32_t)src[RR] << 16);
+                w.y = (uint32_t)src[2 * RR] | ((uint32_t)src[3 * RR] << 16);
+                reinterpret_cast<uint2*>(which ? sC : sB)[((t / 4) * 4 + pq) * 4 + t % 4] = w;
+            }
+        } else {
+            // B and C to fp32 [t][n]: a warp converts two steps of all 16 states per pass
+            for (int i = tid; i < 16 * T; i += kBW * 32) {
+                const int n = i & 15, t = i >> 4;
+                sB[t * 16 + n] = io<Tin>::to_f(rB[n * RR + t]);
+                sC[t * 16 + n] = io<Tin>::to_f(rC[n * RR + t]);
+            }
         }
         for (int i = tid; i < T * 32; i += kBW * 32) sAcc[i] = 0.f;
 
@@ -285,7 +333,7 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
                 hp[0] = pack2(h[0], h[1]);
                 hp[1] = pack2(h[2], h[3]);
             }
-            for (int t = 0; t < T; t += 4) {
+                        for (int t = 0; t < T; t += 4) {
                 {
                     float h0, h1, h2, h3;
                     unpack2(hp[0], h0, h1);
@@ -297,22 +345,24 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
                 float uv[4];
                 V4::to_f(*reinterpret_cast<const VT*>(rU + cw * RR + t), uv);
                 const float dts[4] = {d4.x, d4.y, d4.z, d4.w};
+                Coef<Tin> bq;
+                bq.load(sB, t, pp);
 #pragma unroll
                 for (int s = 0; s < 4; ++s) {
                     const f2 dd = pack2(dts[s], dts[s]);
                     const float q = dts[s] * uv[s];
                     const f2 qq = pack2(q, q);
-                    const float4 bb = lds4(sB + (t + s) * 16 + pp * 4);
+                    const f2x2 bb = bq.at(s);
                     const f2 e0 = ex2x2(mul2(dd, a2p[0])), e1 = ex2x2(mul2(dd, a2p[1]));
-                    hp[0] = fma2(e0, hp[0], mul2(qq, lo2(bb)));
-                    hp[1] = fma2(e1, hp[1], mul2(qq, hi2(bb)));
+                    hp[0] = fma2(e0, hp[0], mul2(qq, bb.lo));
+                    hp[1] = fma2(e1, hp[1], mul2(qq, bb.hi));
                 }
             }
         }
         __syncwarp();
 
         // reverse sweep, one group of four steps at a time (last group first)
-        for (int tg = T - 4; tg >= 0; tg -= 4) {
+                for (int tg = T - 4; tg >= 0; tg -= 4) {
             const float4 d4 = lds4(sDel + cw * RS + tg), y4 = lds4(sDyt + cw * RS + tg);
             float uv[4];
             V4::to_f(*reinterpret_cast<const VT*>(rU + cw * RR + tg), uv);
@@ -321,42 +371,70 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
             const f2 hin[2] = {lo2(h4), hi2(h4)};
             // the group's Abar and states, recomputed into registers
             f2 ab[4][2], hs[4][2];
+            Coef<Tin> bq, cq;
+            bq.load(sB, tg, pp);
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
                 const f2 dd = pack2(dts[s], dts[s]);
                 const float q = dts[s] * uv[s];
                 const f2 qq = pack2(q, q);
-                const float4 bb = lds4(sB + (tg + s) * 16 + pp * 4);
+                const f2x2 bb = bq.at(s);
                 ab[s][0] = ex2x2(mul2(dd, a2p[0]));
                 ab[s][1] = ex2x2(mul2(dd, a2p[1]));
-                hs[s][0] = fma2(ab[s][0], s ? hs[s - 1][0] : hin[0], mul2(qq, lo2(bb)));
-                hs[s][1] = fma2(ab[s][1], s ? hs[s - 1][1] : hin[1], mul2(qq, hi2(bb)));
+                hs[s][0] = fma2(ab[s][0], s ? hs[s - 1][0] : hin[0], mul2(qq, bb.lo));
+                hs[s][1] = fma2(ab[s][1], s ? hs[s - 1][1] : hin[1], mul2(qq, bb.hi));
             }
+            cq.load(sC, tg, pp);
+
             float dqv[4], ddv[4], ypv[4];
 #pragma unroll
             for (int s = 3; s >= 0; --s) {
-                const int t = tg + s;
-                const float4 bb = lds4(sB + t * 16 + pp * 4);
-                const float4 cc = lds4(sC + t * 16 + pp * 4);
+                const f2x2 bb = bq.at(s), cc = cq.at(s);
                 const f2 yy = pack2(dyts[s], dyts[s]), dd = pack2(dts[s], dts[s]);
                 const float q = dts[s] * uv[s];
                 const f2 qq = pack2(q, q);
-                gp[0] = fma2(yy, lo2(cc), gp[0]);
-                gp[1] = fma2(yy, hi2(cc), gp[1]);
-                ypv[s] = hsum(fma2(lo2(cc), hs[s][0], mul2(hi2(cc), hs[s][1])));  // C_t . h_t
+                gp[0] = fma2(yy, cc.lo, gp[0]);
+                gp[1] = fma2(yy, cc.hi, gp[1]);
+                ypv[s] = hsum(fma2(cc.lo, hs[s][0], mul2(cc.hi, hs[s][1])));  // C_t . h_t
                 const f2 dC0 = mul2(yy, hs[s][0]), dC1 = mul2(yy, hs[s][1]);
                 const f2 dB0 = mul2(gp[0], qq), dB1 = mul2(gp[1], qq);
-                dqv[s] = hsum(fma2(gp[0], lo2(bb), mul2(gp[1], hi2(bb))));
-                const f2 gh0 = mul2(mul2(gp[0], s ? hs[s - 1][0] : hin[0]), ab[s][0]);
-                const f2 gh1 = mul2(mul2(gp[1], s ? hs[s - 1][1] : hin[1]), ab[s][1]);
+                dqv[s] = hsum(fma2(gp[0], bb.lo, mul2(gp[1], bb.hi)));
+                // g Abar is the adjoint carried to step t - 1; times h_{t-1} it gives the
+                // terms of dA and of the state part of dDelta
+                gp[0] = mul2(gp[0], ab[s][0]);
+                gp[1] = mul2(gp[1], ab[s][1]);
+                const f2 gh0 = mul2(gp[0], s ? hs[s - 1][0] : hin[0]);
+                const f2 gh1 = mul2(gp[1], s ? hs[s - 1][1] : hin[1]);
                 ddv[s] = hsum(fma2(gh0, anp[0], mul2(gh1, anp[1])));
                 dAp[0] = fma2(gh0, dd, dAp[0]);
                 dAp[1] = fma2(gh1, dd, dAp[1]);
-                gp[0] = mul2(gp[0], ab[s][0]);
-                gp[1] = mul2(gp[1], ab[s][1]);
-                // this channel's dB / dC of step t into the warp's exchange rows
-                {
-                    float* row = sRed + (s & 1) * 256 + cl * 32;
+                if constexpr (XS == 0) {
+                    // sum this step's 32 values over the warp's 8 channels: each of three
+                    // rounds (lane bits 4, 3, 2) keeps half the values and adds the
+                    // partner's copy of that half; lane (cl, pp) ends with value
+                    // 4 b4 + 2 b3 + b2 of quad pp: dB states 0-3, then dC states 0-3
+                    float v[8];
+                    unpack2(dB0, v[0], v[1]);
+                    unpack2(dB1, v[2], v[3]);
+                    unpack2(dC0, v[4], v[5]);
+                    unpack2(dC1, v[6], v[7]);
+                    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+                    float r1[4], r2[2];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        r1[i] = (b4 ? v[4 + i] : v[i]) +
+                                __shfl_xor_sync(0xffffffffu, b4 ? v[i] : v[4 + i], 16);
+#pragma unroll
+                    for (int i = 0; i < 2; ++i)
+                        r2[i] = (b3 ? r1[2 + i] : r1[i]) +
+                                __shfl_xor_sync(0xffffffffu, b3 ? r1[i] : r1[2 + i], 8);
+                    const float r3 = (b2 ? r2[1] : r2[0]) +
+                                     __shfl_xor_sync(0xffffffffu, b2 ? r2[0] : r2[1], 4);
+                    const int idx = (lane >> 2) & 7;  // = 4 b4 + 2 b3 + b2
+                    const int slot = (idx & 4) * 4 + pp * 4 + (idx & 3);
+                    atomicAdd(&sAcc[acc_idx(tg + s, slot)], r3);
+                } else {  // this channel's dB / dC of step t into the warp's exchange rows
+                    float* row = sRed + s * 256 + cl * 32;
                     float x0, x1, x2, x3;
                     unpack2(dB0, x0, x1);
                     unpack2(dB1, x2, x3);
@@ -365,24 +443,27 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
                     unpack2(dC1, x2, x3);
                     *reinterpret_cast<float4*>(row + red_quad(4 + pp, cl) * 4) = make_float4(x0, x1, x2, x3);
                 }
-                if ((s & 1) == 0) {
-                    // a step pair is complete: sum it over the warp's 8 channels
+                if (XS == 4 && s == 0) {
+                    // the group is complete: lane (xs, xq) sums quad xq of step tg + xs over
+                    // the warp's 8 channels
                     __syncwarp();
-                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    const int xs = lane >> 3, xq = lane & 7;
+                    float4 v = lds4(sRed + xs * 256 + red_quad(xq, 0) * 4);
+                    f2 a01 = lo2(v), a23 = hi2(v);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const int ch = rhalf * 4 + kk;
-                        const float4 v = lds4(sRed + rss * 256 + ch * 32 + red_quad(rq, ch) * 4);
-                        acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+                    for (int ch = 1; ch < 8; ++ch) {
+                        v = lds4(sRed + xs * 256 + ch * 32 + red_quad(xq, ch) * 4);
+                        a01 = add2(a01, lo2(v));
+                        a23 = add2(a23, hi2(v));
                     }
-                    // the two channel halves: lane rhalf keeps slots 2 rhalf, 2 rhalf + 1
-                    const float s0 = rhalf ? acc.x : acc.z, s1 = rhalf ? acc.y : acc.w;
-                    const float k0 = rhalf ? acc.z : acc.x, k1 = rhalf ? acc.w : acc.y;
-                    const float v0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 1);
-                    const float v1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 1);
-                    const int tt = tg + s + rss, slot = rq * 4 + rhalf * 2;
+                    float v0, v1, v2, v3;
+                    unpack2(a01, v0, v1);
+                    unpack2(a23, v2, v3);
+                    const int tt = tg + xs, slot = xq * 4;
                     atomicAdd(&sAcc[acc_idx(tt, slot)], v0);
                     atomicAdd(&sAcc[acc_idx(tt, slot + 1)], v1);
+                    atomicAdd(&sAcc[acc_idx(tt, slot + 2)], v2);
+                    atomicAdd(&sAcc[acc_idx(tt, slot + 3)], v3);
                     __syncwarp();
                 }
             }
