@@ -154,16 +154,15 @@ __device__ __forceinline__ f2 exp2_fma2(f2 x) {
 // (Delta A)^-1 (exp(Delta A) - I) Delta B, per diagonal state w = (e^{Delta A} - 1) / A).
 // Inputs: x = Delta A log2(e) (so Abar = e = 2^x), e, 1/A, uu = (u, u), qq = (Delta u,
 // Delta u).  Returns m = w u, the factor of B in the state update.
-//   |Delta A| >= 1/2:  m = u (e - 1) / A;
-//   |Delta A| <  1/2:  m = Delta u phi(Delta A), phi(y) = expm1(y) / y = sum_k y^k / (k+1)!
-//                      truncated after y^6 (truncation below 2e-7 relative), evaluated in x
-//                      with coefficients ln2^k / (k+1)!; this avoids the cancellation of
-//                      e - 1 as Delta A -> 0 (and covers A = 0, where 1/A is infinite).
+//   |Delta A| >= 1/16: m = u (e - 1) / A  (|e - 1| >= 0.0606 there, so an error of a few
+//                      1e-7 in e costs at most about 4e-6 relative);
+//   |Delta A| <  1/16: m = Delta u phi(Delta A), phi(y) = expm1(y) / y = sum_k y^k / (k+1)!
+//                      truncated after y^3 (the first dropped term, y^4 / 120, is below
+//                      1.3e-7 relative), evaluated in x with coefficients ln2^k / (k+1)!;
+//                      this avoids the cancellation of e - 1 as Delta A -> 0 (and covers
+//                      A = 0, where 1/A is infinite).
 __device__ __forceinline__ f2 zoh_weight_u2(f2 x, f2 e, f2 inv_a, f2 uu, f2 qq) {
-    f2 p = fma2(pack2(2.2005043e-05f, 2.2005043e-05f), x, pack2(2.2222597e-04f, 2.2222597e-04f));
-    p = fma2(p, x, pack2(1.9236258e-03f, 1.9236258e-03f));
-    p = fma2(p, x, pack2(1.3876027e-02f, 1.3876027e-02f));
-    p = fma2(p, x, pack2(8.0075502e-02f, 8.0075502e-02f));
+    f2 p = fma2(pack2(1.3876027e-02f, 1.3876027e-02f), x, pack2(8.0075502e-02f, 8.0075502e-02f));
     p = fma2(p, x, pack2(3.4657359e-01f, 3.4657359e-01f));
     p = fma2(p, x, pack2(1.0f, 1.0f));
     const f2 small = mul2(qq, p);
@@ -172,7 +171,7 @@ __device__ __forceinline__ f2 zoh_weight_u2(f2 x, f2 e, f2 inv_a, f2 uu, f2 qq) 
     unpack2(x, x0, x1);
     unpack2(small, s0, s1);
     unpack2(large, l0, l1);
-    constexpr float kTau = 0.72134752f;  // |Delta A| = 1/2 in log2 units
+    constexpr float kTau = 0.09016844f;  // |Delta A| = 1/16 in log2 units
     return pack2(fabsf(x0) < kTau ? s0 : l0, fabsf(x1) < kTau ? s1 : l1);
 }
 
