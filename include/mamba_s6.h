@@ -66,7 +66,7 @@ typedef enum {
  * section, Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B -- for the diagonal A, per
  * state Bbar_n = (exp(Delta A_n) - 1) / A_n * B_n (Delta B_n when A_n = 0) -- instead of
  * Bbar = Delta * B.  The kernels form (exp(Delta A_n) - 1) / A_n from the same
- * exponential as Abar where |Delta A_n| >= 1/2 and from the series of expm1(y) / y
+ * exponential as Abar where |Delta A_n| >= 1/16 and from the series of expm1(y) / y
  * below, so the weight stays accurate as Delta A_n -> 0.
  */
 #define MAMBA_FLAG_EXACT_ZOH 1u

@@ -1,7 +1,7 @@
 """Parity of the exact zero-order-hold variant (MAMBA_FLAG_EXACT_ZOH) with the fp64 oracle's
 ZOH scan (pinned in test_oracle_zoh.py), through the C ABI.  Bbar = (exp(Delta A) - 1) / A * B
 replaces Delta * B (Mamba, "Method" section); the kernels evaluate the weight from the same
-exponential as Abar where |Delta A| >= 1/2 and from the series of expm1(y) / y below, so the
+exponential as Abar where |Delta A| >= 1/16 and from the series of expm1(y) / y below, so the
 cases cover both branches (small, mixed and large steps), A = 0 and A > 0, a split sequence
 (segment aggregates with the ZOH weight), and the decode step.  Tolerances are those of the
 plain scan (s6_compare).
@@ -47,8 +47,8 @@ def test_tiny_fp32_workload_zoh(cuda_ok):
 def test_zoh_fp32_regimes(cuda_ok, shape, regime):
     b, d, N, L = shape
     p = inputs.scan_inputs(b, d, N, L, torch.float32, seed=sum(shape) + len(regime))
-    # step bias: Delta ~ 1e-4 (every |Delta A| < 1/2), the recipe's [0.001, 0.1] (both
-    # branches), or Delta ~ 3 (most |Delta A| >= 1/2)
+    # step bias: Delta ~ 1e-4 (every |Delta A| < 1/16), the recipe's [0.001, 0.1] (both
+    # branches), or Delta ~ 3 (most |Delta A| >= 1/16)
     shift = {"small_steps": -9.0, "mixed": 0.0, "large_steps": 3.0}[regime]
     p["delta"] = p["delta"] * 0.3
     p["delta_bias"] = p["delta_bias"] + shift
