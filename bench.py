@@ -362,6 +362,8 @@ def run_ours(args, rank, world, local):
             lshard = {"error": "%s: %s" % (type(e).__name__, str(e)[:200])}
         torch.cuda.empty_cache()
 
+    probes = run_probes(dev, stream, sms, fmax_mhz)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, budget_s=args.cpu_seconds)
@@ -381,11 +383,43 @@ def run_ours(args, rank, world, local):
                    "parallelism": "replicas x%d (independent batches per GPU)" % world},
         "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
         "clocks": clocks, "decode": decode, "backward": backward, "exact_zoh": zoh,
-        "conv1d": conv, "lshard": lshard,
+        "conv1d": conv, "lshard": lshard, "pipe_probes": probes,
         "cpu_baseline": cpu,
         "impl": "ours",
     }
     return line
+
+
+def run_probes(dev, stream, sms, fmax_mhz, reps=3):
+    """Measured throughput of the pipes the rooflines are stated against (the library's
+    probe: 8 independent chains per thread, 8 CTAs of 256 threads per SM): SFU ex2,
+    fp32 FMA, packed fp32x2 FMA, each the best of `reps` launches of a few ms, beside the
+    rate derived from unit counts and the maximum SM clock."""
+    from selective_state_space_56_b200 import ops
+    blocks = sms * 8
+    sink = torch.empty(blocks * 256, dtype=torch.float32, device=dev)
+    derived = {"sfu_ex2": sms * SFU_OPS_PER_CLK_PER_SM * fmax_mhz * 1e6,
+               "ffma": sms * 128 * fmax_mhz * 1e6, "ffma2": sms * 128 * fmax_mhz * 1e6}
+    iters = {"sfu_ex2": 8192, "ffma": 65536, "ffma2": 32768}
+    out = {}
+    with torch.cuda.stream(stream):
+        for kind in ("sfu_ex2", "ffma", "ffma2"):
+            ops.diag_throughput(kind, blocks, 64, sink)  # warm-up
+            best = float("inf")
+            for _ in range(reps):
+                a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                n = ops.diag_throughput(kind, blocks, iters[kind], sink)
+                e.record(stream)
+                e.synchronize()
+                best = min(best, a.elapsed_time(e))
+            rate = n / (best * 1e-3)
+            out[kind] = {"results_per_s": rate, "derived_per_s": derived[kind],
+                         "frac_of_derived": rate / derived[kind], "ms": best}
+    ops.check_device_error()
+    out["note"] = ("derived: %d SMs x (SFU 16, FMA 128 fp32 results)/clk x %.0f MHz; ffma2 counts "
+                   "two fp32 results per instruction" % (sms, fmax_mhz))
+    return out
 
 
 def run_zoh(g, dev, stream, world, w, steps=50):

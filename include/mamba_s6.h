@@ -390,6 +390,18 @@ int mamba_diag_wait_timeout(int64_t limit_cycles, void* stream);
 int mamba_diag_exp2(const float* x, float* out_fma, float* out_sfu, float* out_lib, int64_t n,
                     void* stream);
 
+/*
+ * Diagnostic: throughput probe of the pipes the scan's roofline is stated against.
+ * Launches `blocks` CTAs of 256 threads (1 to 2^20); every thread runs `iters` rounds
+ * (1 to 2^24) of 8 independent chains of one instruction: kind 0 = SFU ex2.approx.f32,
+ * 1 = fp32 FMA, 2 = packed fp32x2 FMA (two fp32 results each).  The caller times the
+ * launch on `stream`; results per launch = blocks * 256 * iters * 8 (kind 2: * 16).
+ * sink: device array of blocks * 256 floats (caller-owned) that receives one value per
+ * thread, so no chain is optimised away.  Reads nothing.
+ * Errors: NULL, DIMS (kind, blocks or iters out of range), CUDA.
+ */
+int mamba_diag_throughput(int kind, int64_t blocks, int64_t iters, float* sink, void* stream);
+
 /* A static, human-readable name for a status code. */
 const char* mamba_status_string(int status);
 

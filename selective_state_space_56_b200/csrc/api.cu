@@ -486,6 +486,6 @@ const char* mamba_status_string(int status) {
     }
 }
 
-int mamba_abi_version(void) { return 104; }
+int mamba_abi_version(void) { return 105; }
 
 }  // extern "C"

@@ -96,6 +96,8 @@ def load_library():
             lib.mamba_diag_wait_timeout.argtypes = [i64, vp]
             lib.mamba_diag_exp2.restype = i32
             lib.mamba_diag_exp2.argtypes = [vp, vp, vp, vp, i64, vp]
+            lib.mamba_diag_throughput.restype = i32
+            lib.mamba_diag_throughput.argtypes = [i32, i64, i64, vp, vp]
             lib.mamba_abi_version.restype = i32
             lib.mamba_abi_version.argtypes = []
             _lib = lib
@@ -162,6 +164,24 @@ def diag_exp2(x):
     if rc != 0:
         raise MambaError(rc, "mamba_diag_exp2")
     return tuple(outs)
+
+
+THROUGHPUT_KINDS = {"sfu_ex2": 0, "ffma": 1, "ffma2": 2}
+
+
+def diag_throughput(kind: str, blocks: int, iters: int, sink):
+    """Launch the pipe-throughput probe (kind "sfu_ex2", "ffma" or "ffma2") on the current
+    stream; sink is a float32 CUDA tensor of at least blocks * 256 elements.  Returns the
+    number of fp32 results the launch computes (the caller times it)."""
+    k = THROUGHPUT_KINDS[kind]
+    if sink.dtype != torch.float32 or sink.device.type != "cuda" or sink.numel() < blocks * 256:
+        raise ValueError("sink must be a float32 CUDA tensor of at least blocks * 256 elements")
+    with torch.cuda.device(sink.device):
+        rc = load_library().mamba_diag_throughput(k, int(blocks), int(iters), _ptr(sink),
+                                                  _stream_handle(sink.device))
+    if rc != 0:
+        raise MambaError(rc, "mamba_diag_throughput")
+    return blocks * 256 * iters * (16 if k == 2 else 8)
 
 
 def selective_scan_workspace_size(batch: int, dim: int, dstate: int, seqlen: int) -> int:

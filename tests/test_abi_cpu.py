@@ -241,6 +241,16 @@ def test_diag_wait_timeout_rejects_bad_limits(lib):
     assert lib.mamba_diag_wait_timeout(5_000_000_000, None) == ERR_DIMS
 
 
+def test_diag_throughput_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    probe = lib.mamba_diag_throughput
+    probe.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int64, vp, vp]
+    assert probe(0, 8, 16, None, None) == ERR_NULL
+    for kind, blocks, iters in ((3, 8, 16), (-1, 8, 16), (0, 0, 16), (0, 1 << 21, 16),
+                                (0, 8, 0), (0, 8, 1 << 25)):
+        assert probe(kind, blocks, iters, vp(A16), None) == ERR_DIMS, (kind, blocks, iters)
+
+
 def test_training_entry_points_check_the_checkpoint_buffer(lib):
     vp = ctypes.c_void_p
     need = lib.mamba_selective_scan_bwd_workspace_size(_dims())
