@@ -105,7 +105,7 @@ enum Mode : int { kFull = 0, kAggregate = 1, kCheckpoint = 2, kFullCkpt = 3 };
 #define S6_P16 4
 #endif
 #ifndef S6_WARPS16
-#define S6_WARPS16 3
+#define S6_WARPS16 6
 #endif
 #ifndef S6_CHUNK
 #define S6_CHUNK 32
