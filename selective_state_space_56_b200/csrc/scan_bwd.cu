@@ -73,10 +73,6 @@ struct BParams {
 #ifndef S6_BWD_WARPS
 #define S6_BWD_WARPS 4
 #endif
-// CTAs per SM the register budget is sized for (96 registers a thread at 4 warps and 5)
-#ifndef S6_BWD_MINB
-#define S6_BWD_MINB 5
-#endif
 // Steps per dB / dC exchange buffer.  16-step blocks sum each step's dB / dC over the
 // warp's 8 channels with shuffles (no buffer: the shared memory then holds five CTAs per
 // SM for either input type); longer blocks store them to a per-warp buffer and sum a
@@ -235,7 +231,7 @@ __device__ __forceinline__ void stage_chunk(const BParams& p, unsigned char* st,
 }
 
 template <int T, typename Tin>
-__global__ void __launch_bounds__(kBW * 32, S6_BWD_MINB) scan_bwd_kernel(const BParams p) {
+__global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) {
     using Lo = BLayout<T, Tin>;
     constexpr int RS = Lo::RS, RR = Lo::RR;
     using V4 = vec4<Tin>;
