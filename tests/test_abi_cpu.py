@@ -251,6 +251,15 @@ def test_diag_throughput_rejects_bad_arguments(lib):
         assert probe(kind, blocks, iters, vp(A16), None) == ERR_DIMS, (kind, blocks, iters)
 
 
+def test_diag_throughput_binding_checks_its_sink():
+    import torch
+    with pytest.raises(ValueError):
+        ops.diag_throughput("sfu_ex2", 1, 1, torch.empty(256))  # host tensor
+    with pytest.raises(KeyError):
+        ops.diag_throughput("dfma", 1, 1, torch.empty(256))
+    assert set(ops.THROUGHPUT_KINDS) == {"sfu_ex2", "ffma", "ffma2"}
+
+
 def test_training_entry_points_check_the_checkpoint_buffer(lib):
     vp = ctypes.c_void_p
     need = lib.mamba_selective_scan_bwd_workspace_size(_dims())
