@@ -169,13 +169,16 @@ def measured_peaks():
 
 def source_digest(path: str) -> str:
     """First 16 hex digits of the SHA-256 of a CUDA source with its comments and blank-space
-    differences removed: it changes when the code changes, not when a comment does."""
+    differences removed: it changes when the code changes, not when a comment does.
+    Several sources joined by '+' are digested together, in that order."""
     import re
-    text = open(path, encoding="utf-8").read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    text = re.sub(r"//[^\n]*", "", text)
-    code = "\n".join(" ".join(line.split()) for line in text.splitlines() if line.strip())
-    return hashlib.sha256(code.encode()).hexdigest()[:16]
+    codes = []
+    for part in path.split("+"):
+        text = open(part, encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        codes.append("\n".join(" ".join(line.split()) for line in text.splitlines() if line.strip()))
+    return hashlib.sha256("\n".join(codes).encode()).hexdigest()[:16]
 
 
 def profile_traffic(name: str, source: str):
@@ -188,7 +191,7 @@ def profile_traffic(name: str, source: str):
         if ":" in line:
             k, v = line.split(":", 1)
             vals[k.strip()] = v.strip()
-    digest = source_digest(os.path.join(ROOT, source))
+    digest = source_digest("+".join(os.path.join(ROOT, s) for s in source.split("+")))
     recorded = vals.get("source_sha256_16", "").split()
     if not recorded or recorded[0] != digest:  # the kernel changed since the capture
         return None
@@ -486,6 +489,9 @@ def run_zoh(g, dev, stream, world, w, steps=50):
                     "Bbar = (exp(Delta A) - 1) / A * B",
         "roofline": {"bound": "alu", "unit": "Gexp/s", "achieved": exps / (ms * 1e-3) / 1e9,
                      "peak": sfu_peak / 1e9, "frac": exps / (ms * 1e-3) / sfu_peak,
+                     "traffic": profile_traffic(
+                         "scan_zoh_m2p8b.txt", "selective_state_space_56_b200/csrc/scan_fwd.cu+"
+                         "selective_state_space_56_b200/csrc/s6_device.cuh"),
                      "note": "same N + 2 SFU exponentials per element as the Delta*B scan; the "
                              "exact weight adds FMA-pipe work (series + select), not SFU work"},
         "decode": {"ms_per_token_l2_flushed": ms_tok,
@@ -896,19 +902,19 @@ def run_reference(args, rank, world):
 
 
 def profile_target(which):
-    """Three launches of the scan (m2p8b), eight decode tokens, or two backward calls of
-    the m2p8b scan, for ncu captures."""
+    """Three launches of the scan (m2p8b) or of its exact-ZOH variant, eight decode tokens,
+    two backward calls of the m2p8b scan, or three conv1d launches, for ncu captures."""
     from selective_state_space_56_b200 import inputs, ops
     import selective_state_space_56_b200.build as s6build
     s6build.build()
     dev = torch.device("cuda", 0)
-    if which == "scan":
+    if which in ("scan", "zoh"):
         w = inputs.SCAN_WORKLOADS[WORKLOAD]
         p = inputs.scan_inputs(w.batch, w.dim, w.dstate, w.seqlen, w.in_dtype, w.seed, device=dev)
         y = torch.empty((w.batch, w.dim, w.seqlen), dtype=w.out_dtype, device=dev)
         for _ in range(3):
             ops.selective_scan_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
-                                   delta_bias=p["delta_bias"], y=y)
+                                   delta_bias=p["delta_bias"], y=y, exact_zoh=which == "zoh")
     elif which == "conv":
         p = inputs.conv_inputs(4, 5120, 4096, inputs.CONV_WIDTH, torch.bfloat16, device=dev)
         for _ in range(3):
@@ -949,7 +955,7 @@ def main(argv=None):
     ap.add_argument("--zoh-steps", type=int, default=50)
     ap.add_argument("--conv-steps", type=int, default=50)
     ap.add_argument("--lshard-steps", type=int, default=5)
-    ap.add_argument("--profile", choices=["scan", "decode", "backward", "conv"],
+    ap.add_argument("--profile", choices=["scan", "zoh", "decode", "backward", "conv"],
                     help="run a few untimed launches of one workload (an ncu capture target) "
                          "and exit")
     args = ap.parse_args(argv)

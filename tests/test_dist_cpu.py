@@ -78,6 +78,15 @@ def test_committed_profile_traffic_is_found_for_unchanged_kernels(tmp_path, monk
     assert bench.profile_traffic("k.txt", "k.cu") == 1234.0
     src.write_text("kernel v2")
     assert bench.profile_traffic("k.txt", "k.cu") is None
+    # a summary can depend on several sources ('+'-joined): a change in any of them counts
+    hdr = tmp_path / "k.cuh"
+    hdr.write_text("helper v1")
+    both = bench.source_digest(str(src) + "+" + str(hdr))
+    assert both != bench.source_digest(str(src))
+    (prof / "kk.txt").write_text("source_sha256_16: %s   (k.cu+k.cuh)\ndram_bytes_per_launch: 99\n" % both)
+    assert bench.profile_traffic("kk.txt", "k.cu+k.cuh") == 99.0
+    hdr.write_text("helper v2")
+    assert bench.profile_traffic("kk.txt", "k.cu+k.cuh") is None
 
 
 def test_cpu_baseline_reports_all_cores_and_one_thread():
