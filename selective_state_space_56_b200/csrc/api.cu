@@ -61,8 +61,8 @@ extern "C" {
 
 size_t mamba_selective_scan_workspace_size(mamba_scan_dims dims) {
     if (!dims_ok(dims.batch, dims.dim, dims.dstate, dims.seqlen)) return 0;
-    int64_t nseg = 1, seg_len = 0;
-    s6::plan_segments(dims.batch, dims.dim, dims.seqlen, &nseg, &seg_len);
+    // sized for the most segments the plan can take, so the size depends on the sizes alone
+    const int64_t nseg = s6::split_segments_bound(dims.batch, dims.dim, dims.seqlen);
     if (nseg <= 1) return 0;
     const int64_t rows = nseg * dims.batch * dims.dim;
     // seg_h (rows x N) then seg_sum (rows), fp32; the tail rounded to 256 bytes
@@ -118,7 +118,7 @@ int mamba_selective_scan_summary(const void* u, const void* delta, const float* 
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return MAMBA_ERR_ALIGN;
     int64_t nseg = 1, seg_len = 0;
-    s6::plan_segments(dims.batch, dims.dim, dims.seqlen, &nseg, &seg_len);
+    s6::plan_segments(dims.batch, dims.dim, dims.dstate, dims.seqlen, &nseg, &seg_len);
     if (nseg > kMaxGridYZ) return MAMBA_ERR_DIMS;
     const size_t need = mamba_selective_scan_workspace_size(dims);
     if (need > 0) {
@@ -194,7 +194,7 @@ int scan_fwd(const void* u, const void* delta, const float* A, const void* B, co
         return MAMBA_ERR_WORKSPACE;
 
     int64_t nseg = 1, seg_len = 0;
-    s6::plan_segments(dims.batch, dims.dim, dims.seqlen, &nseg, &seg_len);
+    s6::plan_segments(dims.batch, dims.dim, dims.dstate, dims.seqlen, &nseg, &seg_len);
     if (nseg > kMaxGridYZ) return MAMBA_ERR_DIMS;
     const size_t need = mamba_selective_scan_workspace_size(dims);
     if (need > 0) {

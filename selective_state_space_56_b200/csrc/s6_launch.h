@@ -54,7 +54,10 @@ struct StateUpdateArgs {
 constexpr int kChunk = 128;
 
 // Split plan for a problem: number of segments and their length (a multiple of kChunk).
-void plan_segments(int64_t batch, int64_t dim, int64_t L, int64_t* nseg, int64_t* seg_len);
+void plan_segments(int64_t batch, int64_t dim, int64_t dstate, int64_t L, int64_t* nseg,
+                   int64_t* seg_len);
+// Most segments plan_segments can return for these sizes (what the workspace is sized for).
+int64_t split_segments_bound(int64_t batch, int64_t dim, int64_t L);
 
 // Each returns a cudaError_t from the launches (cudaSuccess when all were enqueued).
 cudaError_t launch_scan(const ScanArgs& a, cudaStream_t stream);

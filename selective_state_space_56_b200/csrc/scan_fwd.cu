@@ -1033,10 +1033,46 @@ cudaError_t read_device_error(unsigned* out, bool clear, cudaStream_t stream) {
     return e;
 }
 
-void plan_segments(int64_t batch, int64_t dim, int64_t L, int64_t* nseg, int64_t* seg_len) {
-    // Split only when the channels alone cannot fill the GPU (fewer than 4096 lanes
-    // of 32 channels... i.e. under ~1 warp per SM sub-partition) and L is long:
-    // a split costs a second pass over all but the last segment.
+namespace {
+
+// CTAs of the N-state tile resident at once on a B200 (148 SMs; residency from the tile's
+// shared memory and threads with bf16 inputs): one wave.
+template <int NMAX>
+constexpr int64_t wave_ctas() {
+    using TL = Tile<NMAX>;
+    using Lo = Layout<NMAX, TL::P, TL::WARPS, TL::T, __nv_bfloat16, __nv_bfloat16>;
+    constexpr int64_t by_smem = 233472 / ((int64_t)Lo::bytes + 1024);
+    constexpr int64_t by_threads = 2048 / Lo::THREADS;
+    constexpr int64_t r = by_smem < by_threads ? by_smem : by_threads;
+    return 148 * (r < 32 ? r : 32);
+}
+
+template <int NMAX>
+constexpr int64_t tile_channels() {
+    using TL = Tile<NMAX>;
+    return Layout<NMAX, TL::P, TL::WARPS, TL::T, __nv_bfloat16, __nv_bfloat16>::CH;
+}
+
+}  // namespace
+
+namespace {
+
+// Segment length for n segments of L steps: a multiple of kChunk; returns the count that
+// length gives.
+int64_t segment_len(int64_t L, int64_t n, int64_t* len_out) {
+    int64_t len = (L + n - 1) / n;
+    len = (len + kChunk - 1) / kChunk * kChunk;
+    if (len == 0) len = kChunk;
+    *len_out = len;
+    return std::max<int64_t>(1, (L + len - 1) / len);
+}
+
+}  // namespace
+
+int64_t split_segments_bound(int64_t batch, int64_t dim, int64_t L) {
+    // Split only when the channels alone cannot fill the GPU (fewer than 4096, so under
+    // about a warp per SM sub-partition) and L is long; at most enough segments for
+    // 32768 channel-segments and none shorter than 4096 steps.
     const int64_t channels = batch * dim;
     const int64_t kMinSeg = 4096;
     int64_t n = 1;
@@ -1044,12 +1080,26 @@ void plan_segments(int64_t batch, int64_t dim, int64_t L, int64_t* nseg, int64_t
         const int64_t want = (32768 + channels - 1) / channels;
         n = std::max<int64_t>(1, std::min<int64_t>(want, L / kMinSeg));
     }
-    int64_t len = (L + n - 1) / n;
-    len = (len + kChunk - 1) / kChunk * kChunk;
-    if (len == 0) len = kChunk;
-    n = std::max<int64_t>(1, (L + len - 1) / len);
-    *nseg = n;
-    *seg_len = len;
+    int64_t len;
+    return segment_len(L, n, &len);
+}
+
+void plan_segments(int64_t batch, int64_t dim, int64_t dstate, int64_t L, int64_t* nseg,
+                   int64_t* seg_len) {
+    // Each CTA of a split sweeps a whole segment, so a second, partial wave of CTAs costs a
+    // whole segment's time again, while the split's extra pass costs about the same for
+    // any number of segments: take no more segments than one wave of CTAs holds (and
+    // never more than the bound the workspace is sized for).
+    int64_t n = split_segments_bound(batch, dim, L);
+    if (n > 1) {
+        const int64_t ch = dstate <= 4 ? tile_channels<4>() : dstate <= 8 ? tile_channels<8>()
+                                                                           : tile_channels<16>();
+        const int64_t wave = dstate <= 4 ? wave_ctas<4>() : dstate <= 8 ? wave_ctas<8>()
+                                                                         : wave_ctas<16>();
+        const int64_t per_seg = (dim + ch - 1) / ch * batch;
+        n = std::max<int64_t>(1, std::min<int64_t>(n, wave / per_seg));
+    }
+    *nseg = segment_len(L, n, seg_len);
 }
 
 cudaError_t launch_scan(const ScanArgs& a, cudaStream_t stream) {
