@@ -155,7 +155,7 @@ __device__ __forceinline__ f2 exp2_fma2(f2 x) {
 // Inputs: x = Delta A log2(e) (so Abar = e = 2^x), e, 1/A, uu = (u, u), qq = (Delta u,
 // Delta u).  Returns m = w u, the factor of B in the state update.
 //   |Delta A| >= 1/16: m = u (e - 1) / A  (|e - 1| >= 0.0606 there, so an error of a few
-//                      1e-7 in e costs at most about 4e-6 relative);
+//                      1e-7 in e costs under 5e-6 relative);
 //   |Delta A| <  1/16: m = Delta u phi(Delta A), phi(y) = expm1(y) / y = sum_k y^k / (k+1)!
 //                      truncated after y^3 (the first dropped term, y^4 / 120, is below
 //                      1.3e-7 relative), evaluated in x with coefficients ln2^k / (k+1)!;
