@@ -87,7 +87,9 @@ typedef struct {
  * aggregates (the segment's state from h = 0 and its summed step), the exclusive
  * prefix of the associative combine (Abar_j Abar_i, Abar_j b_i + b_j) across
  * segments (parallel-scan derivation, steps 2-4), and a final pass from each
- * segment's true initial state -- and the workspace holds the aggregates.
+ * segment's true initial state -- and the workspace holds the aggregates.  The size
+ * covers the most segments a plan for `dims` may take (segments x batch x dim x
+ * (dstate + 1) x 4 bytes); a launch may use fewer, e.g. to keep its CTAs in one wave.
  * Depends on `dims` only.  Returns 0 for invalid dims.
  */
 size_t mamba_selective_scan_workspace_size(mamba_scan_dims dims);
