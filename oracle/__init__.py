@@ -229,13 +229,21 @@ def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, soft
 
 
 def state_update_lanes(state, u, delta_raw, A, B, C, lane_batch, D=None, z=None, delta_bias=None,
-                       softplus=True, zoh=False):
+                       softplus=True, zoh=False, inplace=False):
     """One decode token on independent lanes: returns (new_state (nlanes, N), y (nlanes)).
 
     state, A: (nlanes, N); u, delta_raw, z, D, delta_bias: (nlanes);
-    B, C: (nbatch, N); lane i reads row lane_batch[i].  ``state`` is not modified.
+    B, C: (nbatch, N); lane i reads row lane_batch[i].  ``state`` is not modified, unless
+    ``inplace``: then it must be a C-contiguous float64 numpy array, which is updated and
+    returned (long decode runs carry millions of lanes without a copy per token).
     """
-    st = _f64(state).copy()
+    if inplace:
+        if not (isinstance(state, np.ndarray) and state.dtype == np.float64
+                and state.flags["C_CONTIGUOUS"]):
+            raise TypeError("inplace needs a C-contiguous float64 numpy state")
+        st = state
+    else:
+        st = _f64(state).copy()
     nl, N = st.shape
     uu, dd, zz = _f64(u).reshape(nl), _f64(delta_raw).reshape(nl), _f64(z)
     Aa, Dd, bb = _f64(A), _f64(D), _f64(delta_bias)
