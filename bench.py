@@ -19,7 +19,10 @@ N > 1 the million-length layer split along L over the ranks, the end-to-end path
 the timed region, and (rank 0, N = 1) the fp64 CPU oracle on bounded samples.
 
 ``--impl reference`` times the CPU oracle itself as the reference arm.
-Rank 0 prints exactly one JSON line.
+Rank 0 prints exactly one JSON line on stdout: the contract keys plus short objects
+for decode (last), the backward, the exact-ZOH variant, the conv1d producer and the
+other scan workloads.  The full record (samples, notes, probe results) goes to stderr
+on a line starting with ``DETAIL``.
 """
 from __future__ import annotations
 
@@ -226,6 +229,11 @@ def flush_l2(buf):
     buf.add_(1)  # reads and writes 2x L2 worth of bytes
 
 
+def med_ms(evs):
+    """Median duration (ms) of (start, end) CUDA event pairs recorded on one stream."""
+    return statistics.median(a.elapsed_time(b) for a, b in evs)
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def run_ours(args, rank, world, local):
@@ -272,7 +280,7 @@ def run_ours(args, rank, world, local):
         torch.cuda.synchronize(dev)
         barrier(world)
     ms_total = t0.elapsed_time(t1)
-    ms_kernel = statistics.fmean(a.elapsed_time(bb) for a, bb in ev)
+    ms_kernel = med_ms(ev)
     ms_total = max_over_ranks(ms_total, world)
     ms_step = ms_total / args.steps
     elems = b * d * L
@@ -365,6 +373,7 @@ def run_ours(args, rank, world, local):
             lshard = {"error": "%s: %s" % (type(e).__name__, str(e)[:200])}
         torch.cuda.empty_cache()
 
+    workloads = run_workloads(dev, stream, world)
     probes = run_probes(dev, stream, sms, fmax_mhz)
 
     cpu = None
@@ -386,11 +395,70 @@ def run_ours(args, rank, world, local):
                    "parallelism": "replicas x%d (independent batches per GPU)" % world},
         "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
         "clocks": clocks, "decode": decode, "backward": backward, "exact_zoh": zoh,
-        "conv1d": conv, "lshard": lshard, "pipe_probes": probes,
+        "conv1d": conv, "lshard": lshard, "workloads": workloads, "pipe_probes": probes,
         "cpu_baseline": cpu,
         "impl": "ours",
     }
     return line
+
+
+def _r(x, sig=5):
+    """x rounded to `sig` significant digits (ints and non-numbers unchanged)."""
+    if isinstance(x, float):
+        return float("%.*g" % (sig, x))
+    return x
+
+
+def compact_line(line):
+    """The one stdout line: every contract key, the other halves of the metric and the
+    side measurements as short objects, floats to five significant digits, and the decode
+    workload last (the consumer keeps the end of long output).  The full record, with
+    samples, notes and probe details, goes to stderr."""
+    rf, cb, e2e, ck = line["roofline"], line["cpu_baseline"], line["e2e"], line["clocks"]
+    out = {k: _r(line[k]) for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup",
+                                     "ms_per_step", "higher_is_better", "scaling",
+                                     "vs_baseline", "dtype", "io_dtype", "data", "impl")}
+    cfg = line["config"]
+    out["config"] = {"workload": "m2p8b layer scan (4, 5120, 16, 4096), bf16 I/O, fp32 state",
+                     "batch": cfg["batch"], "dim": cfg["dim"], "dstate": cfg["dstate"],
+                     "seqlen": cfg["seqlen"], "l2": "no flush: 504 MB inputs per step > 126 MB L2",
+                     "parallelism": cfg["parallelism"]}
+    out["roofline"] = {k: _r(rf[k]) for k in ("bound", "achieved", "peak", "unit", "frac",
+                                               "traffic", "kernel_ms", "hbm_frac")}
+    out["cpu_baseline"] = None if cb is None else {
+        "value": _r(cb["value"]), "unit": cb["unit"], "cores": cb["cores"], "kind": cb["kind"],
+        "sample": cb["sample"].split(";")[0]}
+    out["e2e"] = {k: _r(e2e[k]) for k in ("value", "unit", "h2d_bytes_per_step",
+                                           "d2h_bytes_per_step", "ms_per_step")}
+    out["gpu_launches"] = line["gpu_launches"]
+    out["clocks"] = {k: _r(ck.get(k)) for k in ("sm_mhz", "sm_max_mhz", "reasons")}
+    wl = line.get("workloads") or {}
+    out["workloads"] = {k: {"ms": _r(v["ms"], 4), "frac": _r(v["frac"], 4)}
+                        for k, v in wl.items() if isinstance(v, dict)}
+    bw, z, cv = line["backward"], line["exact_zoh"], line["conv1d"]
+    out["backward"] = {"ms": _r(bw["ms_per_call"], 4), "value": _r(bw["value"], 4),
+                       "frac": _r(bw["roofline"]["frac"], 4),
+                       "train_ms": _r(bw["train_step"]["ms_per_step"], 4),
+                       "train_frac": _r(bw["train_step"]["roofline"]["frac"], 4)}
+    out["exact_zoh"] = {"ms": _r(z["ms_per_call"], 4), "frac": _r(z["roofline"]["frac"], 4),
+                        "decode_us": _r(z["decode"]["ms_per_token_l2_flushed"] * 1e3, 4),
+                        "decode_hbm_frac": _r(z["decode"]["roofline"]["frac"], 4)}
+    out["conv1d"] = {"ms": _r(cv["ms_per_call"], 4), "hbm_frac": _r(cv["roofline"]["frac"], 4),
+                     "decode_us": _r(cv["decode"]["ms_per_token_l2_flushed"] * 1e3, 4),
+                     "decode_hbm_frac": _r(cv["decode"]["roofline"]["frac"], 4)}
+    if line.get("lshard") is not None:
+        ls = line["lshard"]
+        out["lshard"] = {k: _r(ls[k]) for k in ("value", "ms_per_step", "n_gpus")} \
+            if "value" in ls else ls
+    d = line["decode"]
+    dr = d["roofline"]
+    out["decode"] = {"metric": d["metric"], "value": _r(d["value"]), "unit": d["unit"],
+                     "steps_per_s": _r(d["steps_per_s"]),
+                     "us_per_token_l2_flushed": _r(d["ms_per_token_l2_flushed"] * 1e3, 4),
+                     "us_per_token_back_to_back": _r(d["ms_per_token_back_to_back"] * 1e3, 4),
+                     "roofline": {k: _r(dr[k]) for k in ("bound", "achieved", "peak", "unit",
+                                                          "frac", "traffic")}}
+    return out
 
 
 def run_probes(dev, stream, sms, fmax_mhz, reps=3):
@@ -446,7 +514,7 @@ def run_zoh(g, dev, stream, world, w, steps=50):
         scan()
         b_.record(stream)
     torch.cuda.synchronize(dev)
-    ms = max_over_ranks(statistics.fmean(a.elapsed_time(b_) for a, b_ in evs), world)
+    ms = max_over_ranks(med_ms(evs), world)
     elems = b * d * L
     peaks, kind = measured_peaks()
     fmax_mhz = peaks.get("sm_max_mhz", 1965.0)
@@ -479,7 +547,7 @@ def run_zoh(g, dev, stream, world, w, steps=50):
         b_.record(stream)
         devs.append((a, b_))
     torch.cuda.synchronize(dev)
-    ms_tok = max_over_ranks(statistics.fmean(a.elapsed_time(b_) for a, b_ in devs), world)
+    ms_tok = max_over_ranks(med_ms(devs), world)
     byts = decode_bytes(dw.batch, dw.dim, dw.dstate)
     del toks, flush, state
     return {
@@ -528,7 +596,7 @@ def run_conv(dev, stream, world, rank, steps=50):
         conv()
         b_.record(stream)
     torch.cuda.synchronize(dev)
-    ms = max_over_ranks(statistics.fmean(a.elapsed_time(b_) for a, b_ in evs), world)
+    ms = max_over_ranks(med_ms(evs), world)
     elems = b * d * L
     byts = 2 * elems * 2 + d * K * 4 + d * 4  # x read, out written (bf16), weights, bias
     peaks, kind = measured_peaks()
@@ -554,7 +622,7 @@ def run_conv(dev, stream, world, rank, steps=50):
         b_.record(stream)
         devs.append((a, b_))
     torch.cuda.synchronize(dev)
-    ms_tok = max_over_ranks(statistics.fmean(a.elapsed_time(b_) for a, b_ in devs), world)
+    ms_tok = max_over_ranks(med_ms(devs), world)
     rows = db * dd
     dbytes = rows * (2 * (K - 1) * 2 + 2 * 2) + dd * (K + 1) * 4
     del p, state, xs, flush
@@ -641,7 +709,7 @@ def run_backward(g, dev, stream, world, w, steps=50):
         call()
         b_.record(stream)
     torch.cuda.synchronize(dev)
-    ms = max_over_ranks(statistics.fmean(a.elapsed_time(b_) for a, b_ in evs), world)
+    ms = max_over_ranks(med_ms(evs), world)
     elems = b * d * L
     peaks, kind = measured_peaks()
     fmax_mhz = peaks.get("sm_max_mhz", 1965.0)
@@ -671,7 +739,7 @@ def run_backward(g, dev, stream, world, w, steps=50):
         train_step()
         b_.record(stream)
     torch.cuda.synchronize(dev)
-    ms_train = max_over_ranks(statistics.fmean(a.elapsed_time(b_) for a, b_ in tevs), world)
+    ms_train = max_over_ranks(med_ms(tevs), world)
     sfu_train = elems * (3 * n + 6)  # forward N + 2, backward 2N + 4
     train = {"ms_per_step": ms_train, "value": world * elems / (ms_train * 1e-3),
              "unit": "elems/s",
@@ -697,6 +765,50 @@ def run_backward(g, dev, stream, world, w, steps=50):
         "train_step": train,
         "gpu_launches": 2 * steps + 6 + 2 * (steps + 3),
     }
+
+
+def run_workloads(dev, stream, world, steps=20):
+    """The forward scan on the other scan workloads of the metric: the Mamba-130M-shaped
+    layer (8, 1536, 16, 2048) and the million-length layer (1, 2048, 16, 2^20, split along
+    L inside the call), each call timed with events (median), against the same SFU
+    roofline of N + 2 exponentials per element."""
+    from selective_state_space_56_b200 import inputs, ops
+    peaks, _ = measured_peaks()
+    fmax_mhz = peaks.get("sm_max_mhz", 1965.0)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    sfu_peak = sms * SFU_OPS_PER_CLK_PER_SM * fmax_mhz * 1e6
+    out = {}
+    launches = 0
+    for name, reps in (("m130m", steps), ("million", max(3, steps // 4))):
+        w = inputs.SCAN_WORKLOADS[name]
+        p = inputs.scan_inputs(w.batch, w.dim, w.dstate, w.seqlen, w.in_dtype, w.seed, device=dev)
+        y = torch.empty((w.batch, w.dim, w.seqlen), dtype=w.out_dtype, device=dev)
+        nws = ops.selective_scan_workspace_size(w.batch, w.dim, w.dstate, w.seqlen)
+        ws = torch.empty(nws, dtype=torch.uint8, device=dev) if nws else None
+
+        def call():
+            ops.selective_scan_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"],
+                                   z=p["z"], delta_bias=p["delta_bias"], y=y, workspace=ws)
+
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize(dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        for a, b_ in evs:
+            a.record(stream)
+            call()
+            b_.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = max_over_ranks(med_ms(evs), world)
+        elems = w.batch * w.dim * w.seqlen
+        out[name] = {"ms": ms, "value": world * elems / (ms * 1e-3),
+                     "frac": elems * (w.dstate + 2) / (ms * 1e-3) / sfu_peak}
+        launches += (reps + 3) * (3 if nws else 1)
+        del p, y, ws
+        torch.cuda.empty_cache()
+    out["gpu_launches"] = launches
+    return out
 
 
 def run_decode(dev, stream, world, steps=1000):
@@ -727,7 +839,7 @@ def run_decode(dev, stream, world, steps=1000):
         b_.record(stream)
         evs.append((a, b_))
     torch.cuda.synchronize(dev)
-    ms_cold = statistics.fmean(a.elapsed_time(b_) for a, b_ in evs)
+    ms_cold = med_ms(evs)
     # back to back (state L2-resident between tokens), for context
     a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
@@ -977,7 +1089,8 @@ def main(argv=None):
     try:
         line = run_ours(args, rank, world, local)
         if rank == 0:
-            print(json.dumps(line), flush=True)
+            print("DETAIL " + json.dumps(line), file=sys.stderr, flush=True)
+            print(json.dumps(compact_line(line)), flush=True)
     finally:
         dist_teardown(world)
 
