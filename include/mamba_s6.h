@@ -235,6 +235,10 @@ int mamba_selective_state_update_ex(float* state, const void* u, const void* del
  *   - The array exists on every GPU that loads the library and stays allocated until
  *     the process exits.  The first call on a device (with that device current) looks
  *     up the array's device address; make that first call before any stream capture.
+ *     The address is kept per device and driver context: a call under a different
+ *     current context looks it up again.  After cudaDeviceReset the module may be
+ *     loaded at a new address under an identical context handle, so do not use this
+ *     entry point on a device after resetting it.
  *   - Every call shares the one array and it keeps the last call's contents; the scan
  *     writes each entry before reading it, so nothing needs clearing.  Calls whose
  *     kernels overlap on the GPU (e.g. on two streams at once) race on the array:
@@ -395,7 +399,8 @@ int mamba_diag_exp2(const float* x, float* out_fma, float* out_sfu, float* out_l
 /*
  * Diagnostic: throughput probe of the pipes the scan's roofline is stated against.
  * Launches `blocks` CTAs of 256 threads (1 to 2^20); every thread runs `iters` rounds
- * (1 to 2^24) of 8 independent chains of one instruction: kind 0 = SFU ex2.approx.f32,
+ * (1 to 2^24, with blocks * iters at most 2^28 so that one launch stays well under a
+ * second) of 8 independent chains of one instruction: kind 0 = SFU ex2.approx.f32,
  * 1 = fp32 FMA, 2 = packed fp32x2 FMA (two fp32 results each).  The caller times the
  * launch on `stream`; results per launch = blocks * 256 * iters * 8 (kind 2: * 16).
  * sink: device array of blocks * 256 floats (caller-owned) that receives one value per

@@ -67,8 +67,9 @@ __global__ void __launch_bounds__(256) throughput_kernel(int kind, int64_t iters
 extern "C" int mamba_diag_throughput(int kind, int64_t blocks, int64_t iters, float* sink,
                                      void* stream) {
     if (!sink) return MAMBA_ERR_NULL;
+    // blocks x iters <= 2^28 keeps one launch well under a second on a B200
     if (kind < 0 || kind > 2 || blocks < 1 || blocks > (1LL << 20) || iters < 1 ||
-        iters > (1LL << 24))
+        iters > (1LL << 24) || blocks * iters > (1LL << 28))
         return MAMBA_ERR_DIMS;
     throughput_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(kind, iters,
                                                                                       sink);

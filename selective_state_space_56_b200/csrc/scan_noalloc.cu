@@ -10,8 +10,14 @@
 //
 // The array lives in device global memory on every GPU that loads the library and
 // stays allocated until the process exits.  Its device address is looked up once per
-// device (cudaGetSymbolAddress on the first call made with that device current); host
-// code never passes the array's name itself, which on the host side is only a stand-in.
+// device and context (cudaGetSymbolAddress on the first call made with that device and
+// context current; a call under another context, such as one the caller made current
+// with the driver API, looks it up again); host code never passes the array's name
+// itself, which on the host side is only a stand-in.  After cudaDeviceReset the
+// runtime may load the module again at a new address under a context whose handle
+// equals the old one, so callers that reset a device must not use this entry point
+// on that device afterwards.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -29,19 +35,47 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 constexpr int kMaxDevices = 64;
 std::mutex g_lock;
-void* g_scratch_addr[kMaxDevices] = {};
+struct CachedAddr {
+    CUcontext ctx;  // the context the address was looked up under
+    void* addr;
+};
+CachedAddr g_scratch[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (set up on first use).
+using CtxGetCurrent = CUresult (*)(CUcontext*);
+
+// cuCtxGetCurrent through the runtime's driver entry-point query (no link to libcuda).
+CtxGetCurrent ctx_get_current() {
+    static CtxGetCurrent fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrent>(ptr);
+    });
+    return fn;
+}
+
+// Device address of the scratch array on the current device and context (looked up on
+// the first use there).
 int scratch_on_current_device(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MAMBA_ERR_CUDA;
+    const CtxGetCurrent get_ctx = ctx_get_current();
+    if (!get_ctx) return MAMBA_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return MAMBA_ERR_CUDA;
     std::lock_guard<std::mutex> guard(g_lock);
-    if (!g_scratch_addr[dev]) {
+    if (!ctx || g_scratch[dev].ctx != ctx || !g_scratch[dev].addr) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MAMBA_ERR_CUDA;
-        g_scratch_addr[dev] = p;
+        // the lookup makes the runtime's context current on this thread if none was
+        if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return MAMBA_ERR_CUDA;
+        g_scratch[dev].ctx = ctx;
+        g_scratch[dev].addr = p;
     }
-    *out = g_scratch_addr[dev];
+    *out = g_scratch[dev].addr;
     return MAMBA_OK;
 }
 

@@ -108,6 +108,9 @@ def test_workspace_plan(lib):
     assert ws(8, 1536, 16, 2048) == 0
     assert ws(1, 2048, 16, 1 << 20) > 0        # million-length: split
     assert ws(1, 2048, 16, 1 << 20) < 64 << 20
+    # the no-allocation entry point's fixed 2.25 MiB scratch covers the million-length layer
+    assert ws(1, 2048, 16, 1 << 20) <= 9 << 18
+    assert ws(1, 3300, 16, 40960) <= 9 << 18 < ws(1, 3300, 16, 40960) * 1.06  # just under it
     assert ws(0, 2048, 16, 1 << 20) == 0       # invalid dims report 0
 
 
@@ -247,7 +250,8 @@ def test_diag_throughput_rejects_bad_arguments(lib):
     probe.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int64, vp, vp]
     assert probe(0, 8, 16, None, None) == ERR_NULL
     for kind, blocks, iters in ((3, 8, 16), (-1, 8, 16), (0, 0, 16), (0, 1 << 21, 16),
-                                (0, 8, 0), (0, 8, 1 << 25)):
+                                (0, 8, 0), (0, 8, 1 << 25), (0, 1 << 20, 1 << 9),
+                                (1, 1 << 5, 1 << 24)):  # the last two: blocks x iters > 2^28
         assert probe(kind, blocks, iters, vp(A16), None) == ERR_DIMS, (kind, blocks, iters)
 
 

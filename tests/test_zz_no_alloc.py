@@ -73,6 +73,25 @@ def test_noalloc_matches_regular_entry_point_twice(cuda_ok, shape, in_dt, out_dt
     ops.check_device_error(clear=True)
 
 
+def test_noalloc_just_under_its_limit_is_bit_identical(cuda_ok):
+    # 1 x 3300 channels, L = 40960: ten segments, 2.24 MB of scratch (95% of the array).
+    b, d, n, L = 1, 3300, 16, 40960
+    assert (9 << 18) * 0.9 < ops.selective_scan_workspace_size(b, d, n, L) <= (9 << 18)
+    p = inputs.scan_inputs(b, d, n, L, in_dtype=torch.bfloat16, seed=905, device=DEV)
+    y_ref, st_ref = ops.selective_scan_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"],
+                                           z=p["z"], delta_bias=p["delta_bias"],
+                                           return_last_state=True)
+    for call in range(2):
+        y = torch.full_like(y_ref, float("nan"))
+        st = torch.full_like(st_ref, float("nan"))
+        assert _noalloc(p, y, st, torch.bfloat16) == 0, "call %d" % call
+        torch.cuda.synchronize()
+        # the same plan and kernels on the same inputs: identical bits
+        assert torch.equal(y, y_ref), "y, call %d" % call
+        assert torch.equal(st, st_ref), "last_state, call %d" % call
+    ops.check_device_error(clear=True)
+
+
 def test_noalloc_rejects_scratch_beyond_its_limit(cuda_ok):
     # 1 x 4095 channels, L = 65536: the split plan needs ~2.4 MiB > 2.25 MiB.
     assert ops.selective_scan_workspace_size(1, 4095, 16, 65536) > (9 << 18)
