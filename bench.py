@@ -225,8 +225,13 @@ def backward_bytes(b, d, n, L, in_size=2):
             2 * b * n * L * 4 + 2 * d * n * 4 + 4 * d * 4)
 
 
-def flush_l2(buf):
+def flush_l2(buf, rbuf=None):
+    """Evict L2: write a buffer of twice its size, then (when rbuf is given) read another
+    such buffer, so the write-back of the lines the first pass left dirty happens here
+    and not inside the timed launch that follows."""
     buf.add_(1)  # reads and writes 2x L2 worth of bytes
+    if rbuf is not None:
+        rbuf.amax()  # reads 2x L2 worth of bytes, writes one scalar
 
 
 def med_ms(evs):
@@ -456,6 +461,7 @@ def compact_line(line):
                      "steps_per_s": _r(d["steps_per_s"]),
                      "us_per_token_l2_flushed": _r(d["ms_per_token_l2_flushed"] * 1e3, 4),
                      "us_per_token_back_to_back": _r(d["ms_per_token_back_to_back"] * 1e3, 4),
+                     "l2": "252 MB written then read before each token",
                      "roofline": {k: _r(dr[k]) for k in ("bound", "achieved", "peak", "unit",
                                                           "frac", "traffic")}}
     return out
@@ -529,6 +535,7 @@ def run_zoh(g, dev, stream, world, w, steps=50):
     toks = inputs.decode_tokens_batched(steps, dw, device=dev)
     yd = torch.empty((dw.batch, dw.dim), dtype=dw.io_dtype, device=dev)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    rflush = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
     def tok(s):
         ops.selective_state_update(state, toks["u"][s], toks["delta"][s], prm["A"], toks["B"][s],
@@ -540,7 +547,7 @@ def run_zoh(g, dev, stream, world, w, steps=50):
     torch.cuda.synchronize(dev)
     devs = []
     for s in range(steps):
-        flush_l2(flush)
+        flush_l2(flush, rflush)
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         tok(s)
@@ -549,7 +556,7 @@ def run_zoh(g, dev, stream, world, w, steps=50):
     torch.cuda.synchronize(dev)
     ms_tok = max_over_ranks(med_ms(devs), world)
     byts = decode_bytes(dw.batch, dw.dim, dw.dstate)
-    del toks, flush, state
+    del toks, flush, rflush, state
     return {
         "metric": "selective-scan fwd with exact ZOH Bbar, (b·d·L) elems/s", "unit": "elems/s",
         "value": world * elems / (ms * 1e-3), "ms_per_call": ms, "steps": steps,
@@ -610,12 +617,13 @@ def run_conv(dev, stream, world, rank, steps=50):
     wd, bd = p["weight"][:dd].contiguous(), p["bias"][:dd].contiguous()
     yd = torch.empty((db, dd), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    rflush = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     for s_ in range(3):
         ops.causal_conv1d_update(state, xs[s_], wd, bd, out=yd)
     torch.cuda.synchronize(dev)
     devs = []
     for s_ in range(steps):
-        flush_l2(flush)
+        flush_l2(flush, rflush)
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         ops.causal_conv1d_update(state, xs[s_], wd, bd, out=yd)
@@ -625,7 +633,7 @@ def run_conv(dev, stream, world, rank, steps=50):
     ms_tok = max_over_ranks(med_ms(devs), world)
     rows = db * dd
     dbytes = rows * (2 * (K - 1) * 2 + 2 * 2) + dd * (K + 1) * 4
-    del p, state, xs, flush
+    del p, state, xs, flush, rflush
     return {
         "metric": "causal conv1d + SiLU (b·d·L) elems/s", "unit": "elems/s",
         "value": world * elems / (ms * 1e-3), "ms_per_call": ms, "steps": steps,
@@ -822,6 +830,7 @@ def run_decode(dev, stream, world, steps=1000):
     toks = [{k: v[s] for k, v in allt.items()} for s in range(steps)]
     y = torch.empty((w.batch, w.dim), dtype=w.io_dtype, device=dev)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    rflush = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
     def tok(x):
         ops.selective_state_update(state, x["u"], x["delta"], prm["A"], x["B"], x["C"],
@@ -832,7 +841,7 @@ def run_decode(dev, stream, world, steps=1000):
     torch.cuda.synchronize(dev)
     evs = []
     for x in toks:
-        flush_l2(flush)
+        flush_l2(flush, rflush)
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         tok(x)
@@ -840,6 +849,18 @@ def run_decode(dev, stream, world, steps=1000):
         evs.append((a, b_))
     torch.cuda.synchronize(dev)
     ms_cold = med_ms(evs)
+    # with the write-only flush, the flush's own dirty lines are written back during the
+    # token: for context
+    wevs = []
+    for x in toks[: max(5, len(toks) // 5)]:
+        flush_l2(flush)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        tok(x)
+        b_.record(stream)
+        wevs.append((a, b_))
+    torch.cuda.synchronize(dev)
+    ms_wflush = med_ms(wevs)
     # back to back (state L2-resident between tokens), for context
     a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
@@ -852,18 +873,20 @@ def run_decode(dev, stream, world, steps=1000):
     peaks, kind = measured_peaks()
     byts = decode_bytes(w.batch, w.dim, w.dstate)
     lanes = w.batch * w.dim
-    del toks, allt, flush
+    del toks, allt, flush, rflush
     return {
         "metric": "decode state-updates/s", "unit": "(b,d) lane updates/s",
         "value": world * lanes / (ms_cold * 1e-3), "steps_per_s": 1e3 / ms_cold,
         "ms_per_token_l2_flushed": ms_cold, "ms_per_token_back_to_back": ms_warm,
+        "ms_per_token_write_flush_only": ms_wflush,
+        "l2": "flushed before every token: 252 MB written, then 252 MB read",
         "workload": "decode: batch 256, dim 5120, N 16, bf16 I/O, fp32 state, %d fresh tokens" % steps,
         "roofline": {"bound": "hbm", "unit": "GB/s", "achieved": byts / (ms_cold * 1e-3) / 1e9,
                      "peak": peaks["hbm_gbs"], "frac": byts / (ms_cold * 1e-3) / 1e9 / peaks["hbm_gbs"],
                      "algorithmic_bytes": byts, "peak_kind": kind,
                      "traffic": profile_traffic("state_update_decode.txt",
                                                 "selective_state_space_56_b200/csrc/state_update.cu")},
-        "gpu_launches": 2 * steps + 5,
+        "gpu_launches": 2 * steps + 5 + len(wevs),
     }
 
 
@@ -1014,7 +1037,8 @@ def run_reference(args, rank, world):
 
 
 def profile_target(which):
-    """Three launches of the scan (m2p8b) or of its exact-ZOH variant, eight decode tokens,
+    """Three launches of the scan (m2p8b) or of its exact-ZOH variant, eight decode tokens
+    (each after an L2 flush),
     two backward calls of the m2p8b scan, or three conv1d launches, for ncu captures."""
     from selective_state_space_56_b200 import inputs, ops
     import selective_state_space_56_b200.build as s6build
@@ -1046,7 +1070,10 @@ def profile_target(which):
         state = prm["state0"].clone()
         toks = inputs.decode_tokens_batched(8, w, device=dev)
         y = torch.empty((w.batch, w.dim), dtype=w.io_dtype, device=dev)
-        for s in range(8):
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        rflush = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        for s in range(8):  # every token after an L2 flush, as the bench times them
+            flush_l2(flush, rflush)
             ops.selective_state_update(state, toks["u"][s], toks["delta"][s], prm["A"], toks["B"][s],
                                        toks["C"][s], D=prm["D"], z=toks["z"][s],
                                        delta_bias=prm["delta_bias"], y=y)

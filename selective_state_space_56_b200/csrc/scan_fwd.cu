@@ -74,6 +74,7 @@ struct KParams {
     int softplus;
     int y_vec;  // L % 4 == 0: four outputs per vector store
     int y_tma;  // output rows are 16-byte multiples: tiles go back by TMA store
+    int seg_first;  // kCorr: the segment of blockIdx.z = 0
 };
 
 // TMA descriptors of the operands (unused when rows are not 16-byte multiples).
@@ -96,9 +97,13 @@ __device__ __forceinline__ void store4(__nv_bfloat16* dst, const float (&o)[4]) 
 
 // kFull: the scan itself; kAggregate: split-sequence pass 1 (end state and summed step
 // per segment, no output); kCheckpoint: the backward's forward pass (the state at the
-// start of every checkpoint block, no output); kFullCkpt: the scan that also records
+// start of every checkpoint block, no output); kFullAgg: the one-pass split -- every
+// segment scanned from h = 0, writing y and its end state and summed step; kCorr: its
+// correction -- from the segment's true start state with no input (h = Abar h), adding
+// (C.h) * silu(z) to y until the state has decayed below fp32 resolution; kFullCkpt: the
+// scan that also records
 // those checkpoints (a training forward, so the backward needs no pass of its own).
-enum Mode : int { kFull = 0, kAggregate = 1, kCheckpoint = 2, kFullCkpt = 3 };
+enum Mode : int { kFull = 0, kAggregate = 1, kCheckpoint = 2, kFullCkpt = 3, kFullAgg = 4, kCorr = 5 };
 
 // Tuning of the N = 16 instantiation: lanes per channel, warps per CTA, chunk length.
 #ifndef S6_P16
@@ -128,17 +133,45 @@ enum Mode : int { kFull = 0, kAggregate = 1, kCheckpoint = 2, kFullCkpt = 3 };
 #ifndef S6_POLY
 #define S6_POLY 0
 #endif
+// Channels per lane of the plain N = 16 forward: 2 lets one load and widening of a step's
+// B and C serve two channels, halving the coefficient traffic through shared memory.
+#ifndef S6_CPL16
+#define S6_CPL16 1
+#endif
+#ifndef S6_WARPS16F
+#define S6_WARPS16F S6_WARPS16
+#endif
+// Delta * A log2(e) formed for two consecutive steps of one state at once (the pair
+// (Delta_t, Delta_t+1) is already adjacent in registers) instead of for two states of one
+// step, which needs Delta copied into both halves of a pair first.  Measured 1.5% slower
+// on the 2.8B-shaped layer (no fewer instructions, six more registers): off, except for
+// the correction pass, which has no input term and always uses this form.
+#ifndef S6_TPX
+#define S6_TPX 0
+#endif
+// Abar of the next 4-step group computed while the current group's states update (one
+// step's worth of exponentials before each step), instead of all of a group's before its
+// own updates.
+#ifndef S6_PIPE
+#define S6_PIPE 0
+#endif
+// SiLU of four outputs with one shared reciprocal (silu4) instead of one each.
+#ifndef S6_SILU4
+#define S6_SILU4 1
+#endif
 
 constexpr size_t align128(size_t x) { return (x + 127) / 128 * 128; }
 
 // Shared-memory carve-up for one instantiation.
-template <int NMAX, int P, int WARPS_, int T_, typename Tin, typename Tout>
+template <int NMAX, int P, int WARPS_, int T_, typename Tin, typename Tout, int CPL_ = 1>
 struct Layout {
     static constexpr int T = T_;
-    static constexpr int NS = NMAX / P;        // states per lane
-    static constexpr int G = 32 / P;           // channels per warp
+    static constexpr int CPL = CPL_;           // channels per lane
+    static constexpr int NS = NMAX / P;        // states per lane and channel
+    static constexpr int G = 32 / P;           // lane groups per warp
+    static constexpr int CW = G * CPL;         // channels per warp
     static constexpr int WARPS = WARPS_;
-    static constexpr int CH = WARPS * G;       // channels per CTA
+    static constexpr int CH = WARPS * CW;      // channels per CTA
     static constexpr int THREADS = WARPS * 32;
     static constexpr int RS = T + 4;           // fp32 row stride: rows land 16 B apart in banks
     static constexpr size_t rows_bytes = (size_t)CH * T * sizeof(Tin);    // one of u, delta, z
@@ -194,16 +227,24 @@ __device__ __forceinline__ float transpose_reduce(const float* v, int pp) {
 }
 
 template <int NMAX, int P, int WARPS, int T_, typename Tin, typename Tout, int MODE, bool TMA,
-          bool ZOH = false, bool WS = false>
+          bool ZOH = false, bool WS = false, int CPL = 1>
 __global__ void __launch_bounds__(WARPS * 32 + (WS ? 32 : 0))
 scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
     static_assert(!WS || (TMA && MODE == kFull), "producer warp: TMA full scans only");
-    constexpr bool kOut = MODE == kFull || MODE == kFullCkpt;         // writes y
+    static_assert(CPL == 1 || (MODE == kFull && !ZOH && !WS), "two channels per lane: plain scan");
+    constexpr bool kOut = MODE == kFull || MODE == kFullCkpt || MODE == kFullAgg ||
+                          MODE == kCorr;                              // writes y
     constexpr bool kCk = MODE == kCheckpoint || MODE == kFullCkpt;    // writes checkpoints
-    using Lo = Layout<NMAX, P, WARPS, T_, Tin, Tout>;
+    constexpr bool kCorrM = MODE == kCorr;                            // input-free correction
+    constexpr bool kSum = MODE == kAggregate || MODE == kFullAgg;     // segment summaries
+    // time-paired exponent arguments (the FMA-pipe exponential and the exact ZOH weight
+    // keep the state-paired form)
+    constexpr bool kTPX = (MODE == kCorr) || (S6_TPX && !ZOH && S6_POLY == 0);
+    static_assert(CPL == 1 || kTPX, "two channels per lane use the time-paired form");
+    using Lo = Layout<NMAX, P, WARPS, T_, Tin, Tout, CPL>;
     using V4 = vec4<Tin>;
     using VT = typename V4::type;
-    constexpr int T = Lo::T, NS = Lo::NS, G = Lo::G, CH = Lo::CH, RS = Lo::RS;
+    constexpr int T = Lo::T, NS = Lo::NS, G = Lo::G, CW = Lo::CW, CH = Lo::CH, RS = Lo::RS;
     extern __shared__ __align__(128) unsigned char smem[];
     float* sDel = reinterpret_cast<float*>(smem + Lo::off_del);
     float* sDu = reinterpret_cast<float*>(smem + Lo::off_du);
@@ -215,12 +256,12 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t b = blockIdx.y;
     const int64_t d0 = (int64_t)blockIdx.x * CH;
-    const int seg = blockIdx.z;
+    const int seg = (int)blockIdx.z + (kCorrM ? p.seg_first : 0);
     const int64_t t_begin = (int64_t)seg * p.seg_len;
     const int64_t t_end = min(p.L, t_begin + p.seg_len);
     const int64_t nchunks = t_end > t_begin ? (t_end - t_begin + T - 1) / T : 0;
     const bool has_z = kOut && p.z != nullptr;
-    const bool out_tma = TMA && kOut && p.y_tma;
+    const bool out_tma = TMA && kOut && !kCorrM && p.y_tma;
 
     for (int c = tid; c < CH; c += Lo::THREADS) {
         const int64_t d = d0 + c;
@@ -240,34 +281,67 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         fence_barrier_init();
     }
 
-    // This lane's channel and states.
+    // This lane's channels (CPL of them, G apart) and states (NS of each).
     const int pp = lane % P;
-    const int cw = warp * G + lane / P;
-    const int64_t dch = d0 + cw;
-    f2 a2p[NS / 2], hp[NS / 2];
+    int cwk[CPL];
+    int64_t dchk[CPL];
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) {
+        cwk[k] = warp * CW + k * G + lane / P;
+        dchk[k] = d0 + cwk[k];
+    }
+    const int cw = cwk[0];
+    const int64_t dch = dchk[0];
+    f2 a2p[CPL][NS / 2], hp[CPL][NS / 2];
+    f2 a2d[kTPX ? CPL : 1][kTPX ? NS : 1];  // (a_n, a_n): one state's factor for two steps
     f2 inv_ap[ZOH ? NS / 2 : 1];  // 1 / A per state, for the exact ZOH input weight
 #pragma unroll
-    for (int j = 0; j < NS; j += 2) {
-        float a[2], h[2];
+    for (int k = 0; k < CPL; ++k) {
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const int nn = pp * NS + j + q;
-            const bool ok = dch < p.dim && nn < p.N;
-            a[q] = ok ? p.A[dch * p.N + nn] * kLog2e : 0.f;  // padded states: Abar = 1, b = 0
-            // initial state: the segment's start (split sequences) or the caller's h0
-            h[q] = (kOut && p.seg_h != nullptr && ok)
-                       ? p.seg_h[(((int64_t)seg * p.batch + b) * p.dim + dch) * p.N + nn]
-                       : 0.f;
-        }
-        a2p[j / 2] = pack2(a[0], a[1]);
-        hp[j / 2] = pack2(h[0], h[1]);
-        if constexpr (ZOH) {
-            // 1 / A (infinite for A = 0; the weight then takes its series branch)
-            const float ia0 = kLog2e / a[0], ia1 = kLog2e / a[1];
-            inv_ap[j / 2] = pack2(ia0, ia1);
+        for (int j = 0; j < NS; j += 2) {
+            float a[2], h[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int nn = pp * NS + j + q;
+                const bool ok = dchk[k] < p.dim && nn < p.N;
+                a[q] = ok ? p.A[dchk[k] * p.N + nn] * kLog2e : 0.f;  // padded states: Abar = 1, b = 0
+                // initial state: the segment's start (split sequences) or the caller's h0
+                h[q] = ((kOut && MODE != kFullAgg) && p.seg_h != nullptr && ok)
+                           ? p.seg_h[(((int64_t)seg * p.batch + b) * p.dim + dchk[k]) * p.N + nn]
+                           : 0.f;
+            }
+            a2p[k][j / 2] = pack2(a[0], a[1]);
+            hp[k][j / 2] = pack2(h[0], h[1]);
+            if constexpr (kTPX) {
+                a2d[k][j] = pack2(a[0], a[0]);
+                a2d[k][j + 1] = pack2(a[1], a[1]);
+            }
+            if constexpr (ZOH) {
+                // 1 / A (infinite for A = 0; the weight then takes its series branch)
+                const float ia0 = kLog2e / a[0], ia1 = kLog2e / a[1];
+                inv_ap[j / 2] = pack2(ia0, ia1);
+            }
         }
     }
     float dsum = 0.f;
+    // Correction pass: the state it carries decays monotonically when every A of the lane
+    // is <= 0 and Delta >= 0 (softplus); then it may stop once every state is below
+    // 2^-24 of the largest it started from.
+    bool decay_ok = kCorrM && p.softplus != 0;
+    float decay_thr = 0.f;
+    if constexpr (kCorrM) {
+#pragma unroll
+        for (int k = 0; k < CPL; ++k)
+#pragma unroll
+            for (int j = 0; j < NS / 2; ++j) {
+                float a0, a1, h0v, h1v;
+                unpack2(a2p[k][j], a0, a1);
+                unpack2(hp[k][j], h0v, h1v);
+                decay_ok = decay_ok && a0 <= 0.f && a1 <= 0.f;
+                decay_thr = fmaxf(decay_thr, fmaxf(fabsf(h0v), fabsf(h1v)));
+            }
+        decay_thr *= 5.9604645e-8f;  // 2^-24
+    }
     __syncthreads();
 
     // Stage chunk k of this CTA's segment into stage buffer k & 1.
@@ -277,13 +351,15 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
     auto issue_chunk = [&](int64_t k) {  // TMA: called by one thread
         unsigned char* st = smem + (k & 1) * Lo::stage_bytes;
         const int tt = (int)(t_begin + k * T);
-        const uint32_t bytes = (uint32_t)((has_z ? 3 : 2) * Lo::rows_bytes + 2 * Lo::coef_bytes);
+        // the correction has no input: neither u nor B is needed
+        const uint32_t bytes = kCorrM ? (uint32_t)((has_z ? 2 : 1) * Lo::rows_bytes + Lo::coef_bytes)
+                                      : (uint32_t)((has_z ? 3 : 2) * Lo::rows_bytes + 2 * Lo::coef_bytes);
         uint64_t* bk = &bar[k & 1];
         mbar_arrive_expect_tx(bk, bytes);
-        tma_load_3d(st, &tm.u, tt, (int)d0, (int)b, bk);
+        if (!kCorrM) tma_load_3d(st, &tm.u, tt, (int)d0, (int)b, bk);
         tma_load_3d(st + Lo::off_dr, &tm.dr, tt, (int)d0, (int)b, bk);
         if (has_z) tma_load_3d(st + Lo::off_z, &tm.z, tt, (int)d0, (int)b, bk);
-        tma_load_3d(st + Lo::off_B, &tm.B, tt, 0, (int)b, bk);
+        if (!kCorrM) tma_load_3d(st + Lo::off_B, &tm.B, tt, 0, (int)b, bk);
         tma_load_3d(st + Lo::off_C, &tm.C, tt, 0, (int)b, bk);
     };
     auto load_chunk_elementwise = [&](int64_t k) {  // rows not 16-byte multiples
@@ -414,6 +490,8 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         if (tid == 0 && nchunks > 0) issue_chunk(0);
     }
     bool aborted = false;
+    bool drained = false;      // the correction stopped early (its remainder is negligible)
+    int64_t abort_chunk = -1;  // the chunk whose copy may still be in flight when stopping
     for (int64_t k = 0; k < nchunks; ++k) {
         bool ok = true;
         if constexpr (WS) {
@@ -448,6 +526,7 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
             if (__syncthreads_or(!ok)) {  // every thread agrees to stop if any wait gave up
                 if (tid == 0) atomicOr(&g_device_error, 1u);
                 aborted = true;
+                abort_chunk = k;  // chunk k was issued; chunk k + 1 was not
                 break;
             }
             if constexpr (TMA) {
@@ -460,11 +539,11 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
 
         // Phase A: step sizes of this warp's channels, four steps per lane.  Steps past
         // the end of the segment get Delta = 0 (Abar = 1, no input): the state passes.
-        for (int i = lane; i < G * (T / 4); i += 32) {
-            const int c = warp * G + i / (T / 4), tb = 4 * (i % (T / 4));
-            float x[4], uu[4];
+        for (int i = lane; i < CW * (T / 4); i += 32) {
+            const int c = warp * CW + i / (T / 4), tb = 4 * (i % (T / 4));
+            float x[4], uu[4] = {0.f, 0.f, 0.f, 0.f};
             V4::to_f(*reinterpret_cast<const VT*>(rDr + c * T + tb), x);
-            V4::to_f(*reinterpret_cast<const VT*>(rU + c * T + tb), uu);
+            if (!kCorrM) V4::to_f(*reinterpret_cast<const VT*>(rU + c * T + tb), uu);
             const float bias = sBias[c];
             float dt[4], xb[4];
 #pragma unroll
@@ -480,7 +559,9 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
                 for (int q = 0; q < 4; ++q) dt[q] = tb + q < valid ? dt[q] : 0.f;
             }
             *reinterpret_cast<float4*>(sDel + c * RS + tb) = make_float4(dt[0], dt[1], dt[2], dt[3]);
-            if constexpr (ZOH) {  // the exact ZOH weight needs u itself
+            if constexpr (kCorrM) {
+                // no input term
+            } else if constexpr (ZOH) {  // the exact ZOH weight needs u itself
                 *reinterpret_cast<float4*>(sDu + c * RS + tb) = make_float4(uu[0], uu[1], uu[2], uu[3]);
             } else {
                 const float q0 = dt[0] * uu[0], q1 = dt[1] * uu[1], q2 = dt[2] * uu[2],
@@ -501,7 +582,7 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
 #pragma unroll
             for (int j = 0; j < NS / 2; ++j) {
                 float h0, h1;
-                unpack2(hp[j], h0, h1);
+                unpack2(hp[0][j], h0, h1);
                 if (pp * NS + 2 * j < p.N) ck[pp * NS + 2 * j] = h0;
                 if (pp * NS + 2 * j + 1 < p.N) ck[pp * NS + 2 * j + 1] = h1;
             }
@@ -509,110 +590,171 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         if (kCk) write_ckpt(0);
 
         // Phase B: the recurrence, four steps per iteration, states in packed pairs.
+        f2 ee_next[4][NS / 2];  // the lookahead's Abar of the next group (S6_PIPE)
 #pragma unroll
         for (int t = 0; t < T; t += 4) {
             if (kCk && t > 0 && t % CKPT == 0) write_ckpt(t);
-            const float4 d4 = *reinterpret_cast<const float4*>(sDel + cw * RS + t);
-            const float4 q4 = *reinterpret_cast<const float4*>(sDu + cw * RS + t);
-            const f2 dd4[4] = {pack2(d4.x, d4.x), pack2(d4.y, d4.y), pack2(d4.z, d4.z),
-                               pack2(d4.w, d4.w)};
-            const f2 qq4[4] = {pack2(q4.x, q4.x), pack2(q4.y, q4.y), pack2(q4.z, q4.z),
-                               pack2(q4.w, q4.w)};
-            float yp[4];
-            // all Abar factors of the four steps first, so their SFU latency overlaps
-            f2 ee[4][NS / 2];
-            if constexpr (S6_PREEXP && !ZOH && S6_POLY == 0) {
+            float4 d4[CPL], q4[CPL];
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-                    for (int j = 0; j < NS / 2; ++j) ee[kk][j] = ex2x2(mul2(dd4[kk], a2p[j]));
+            for (int k = 0; k < CPL; ++k) {
+                d4[k] = *reinterpret_cast<const float4*>(sDel + cwk[k] * RS + t);
+                if (!kCorrM) q4[k] = *reinterpret_cast<const float4*>(sDu + cwk[k] * RS + t);
             }
-#if S6_PREEXP >= 2
-            // the group's coefficients too (format 2: fp32 B pairs, bf16 C pairs)
-            ulonglong2 bpre[4][NS / 4];
-            uint2 cpre[4][NS / 4];
-            if constexpr (Lo::kBC == 2) {
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-                    for (int j = 0; j < NS / 4; ++j) {
-                        bpre[kk][j] = reinterpret_cast<const ulonglong2*>(sBt + (t + kk) * NMAX + pp * NS)[j];
-                        cpre[kk][j] = reinterpret_cast<const uint2*>(sCt)[(t + kk) * (NMAX / 4) +
-                                                                          pp * (NS / 4) + j];
-                    }
-            }
-#endif
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const f2 dd = dd4[kk];
-                // ZOH: qq4 holds (u, u); Delta u is formed here
-                const f2 uu = qq4[kk];
-                const f2 qq = ZOH ? mul2(dd, uu) : qq4[kk];
-                f2 acc = pack2(0.f, 0.f);
+            float yp[CPL][4];
+            // this lane's B and C of step t + kk, as fp32 pairs (states 2j, 2j + 1)
+            auto coefs = [&](int kk, f2 (&bq)[NS / 2], f2 (&cq)[NS / 2]) {
 #pragma unroll
                 for (int j = 0; j < NS / 4; ++j) {
-                    f2 b01, b23, c01, c23;
                     if constexpr (Lo::kBC == 1) {
                         const uint4 g = reinterpret_cast<const uint4*>(sBt)[(t + kk) * (NMAX / 4) +
                                                                             pp * (NS / 4) + j];
-                        b01 = bf16pair(g.x), b23 = bf16pair(g.y);
-                        c01 = bf16pair(g.z), c23 = bf16pair(g.w);
+                        bq[2 * j] = bf16pair(g.x), bq[2 * j + 1] = bf16pair(g.y);
+                        cq[2 * j] = bf16pair(g.z), cq[2 * j + 1] = bf16pair(g.w);
                     } else if constexpr (Lo::kBC == 2) {
-#if S6_PREEXP >= 2
-                        const ulonglong2 bb = bpre[kk][j];
-                        const uint2 g = cpre[kk][j];
-#else
                         const ulonglong2 bb = reinterpret_cast<const ulonglong2*>(
                             sBt + (t + kk) * NMAX + pp * NS)[j];
                         const uint2 g = reinterpret_cast<const uint2*>(sCt)[(t + kk) * (NMAX / 4) +
                                                                           pp * (NS / 4) + j];
-#endif
-                        b01 = f2{bb.x}, b23 = f2{bb.y};
-                        c01 = bf16pair(g.x), c23 = bf16pair(g.y);
+                        bq[2 * j] = f2{bb.x}, bq[2 * j + 1] = f2{bb.y};
+                        cq[2 * j] = bf16pair(g.x), cq[2 * j + 1] = bf16pair(g.y);
                     } else {
                         const ulonglong2 bb = reinterpret_cast<const ulonglong2*>(
                             sBt + (t + kk) * NMAX + pp * NS)[j];
                         const ulonglong2 cc = reinterpret_cast<const ulonglong2*>(
                             sCt + (t + kk) * NMAX + pp * NS)[j];
-                        b01 = f2{bb.x}, b23 = f2{bb.y}, c01 = f2{cc.x}, c23 = f2{cc.y};
+                        bq[2 * j] = f2{bb.x}, bq[2 * j + 1] = f2{bb.y};
+                        cq[2 * j] = f2{cc.x}, cq[2 * j + 1] = f2{cc.y};
                     }
-                    if constexpr (ZOH) {
-                        const f2 x0 = mul2(dd, a2p[2 * j]), x1 = mul2(dd, a2p[2 * j + 1]);
-                        const f2 e0 = ex2x2(x0), e1 = ex2x2(x1);
-                        const f2 m0 = zoh_weight_u2(x0, e0, inv_ap[2 * j], uu, qq);
-                        const f2 m1 = zoh_weight_u2(x1, e1, inv_ap[2 * j + 1], uu, qq);
-                        hp[2 * j] = fma2(e0, hp[2 * j], mul2(m0, b01));
-                        hp[2 * j + 1] = fma2(e1, hp[2 * j + 1], mul2(m1, b23));
-                    } else if constexpr (S6_PREEXP && S6_POLY == 0) {
-                        hp[2 * j] = fma2(ee[kk][2 * j], hp[2 * j], mul2(qq, b01));
-                        hp[2 * j + 1] = fma2(ee[kk][2 * j + 1], hp[2 * j + 1], mul2(qq, b23));
-                    } else {
-                        const f2 e0 = ex2x2(mul2(dd, a2p[2 * j]));
-                        const bool on_fma = S6_POLY == 2 || (S6_POLY == 1 && (kk & 1));
-                        const f2 e1 = on_fma ? exp2_fma2(mul2(dd, a2p[2 * j + 1]))
-                                             : ex2x2(mul2(dd, a2p[2 * j + 1]));
-                        hp[2 * j] = fma2(e0, hp[2 * j], mul2(qq, b01));
-                        hp[2 * j + 1] = fma2(e1, hp[2 * j + 1], mul2(qq, b23));
-                    }
-                    acc = fma2(c01, hp[2 * j], acc);
-                    acc = fma2(c23, hp[2 * j + 1], acc);
                 }
-                float lo, hi;
-                unpack2(acc, lo, hi);
-                yp[kk] = lo + hi;
-            }
-            if (MODE == kCheckpoint) {
-                // states only
-            } else if (MODE == kAggregate) {
-                float dv[4], dup;
+            };
+            if constexpr (kTPX) {
+                // Abar of the four steps first (their SFU latency overlaps): per state, the
+                // arguments of steps (t, t+1) and (t+2, t+3) as two packed products.
+                float ee[CPL][4][NS];
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) unpack2(dd4[kk], dv[kk], dup);
-                dsum += (dv[0] + dv[1]) + (dv[2] + dv[3]);
-            } else if constexpr (P == 1) {
-                *reinterpret_cast<float4*>(sY + cw * RS + t) = make_float4(yp[0], yp[1], yp[2], yp[3]);
+                for (int k = 0; k < CPL; ++k)
+#pragma unroll
+                    for (int j = 0; j < NS; ++j) {
+                        float x0, x1, x2, x3;
+                        unpack2(mul2(pack2(d4[k].x, d4[k].y), a2d[k][j]), x0, x1);
+                        unpack2(mul2(pack2(d4[k].z, d4[k].w), a2d[k][j]), x2, x3);
+                        ee[k][0][j] = ex2(x0);
+                        ee[k][1][j] = ex2(x1);
+                        ee[k][2][j] = ex2(x2);
+                        ee[k][3][j] = ex2(x3);
+                    }
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    f2 bq[NS / 2], cq[NS / 2];
+                    coefs(kk, bq, cq);
+#pragma unroll
+                    for (int k = 0; k < CPL; ++k) {
+                        f2 acc = pack2(0.f, 0.f);
+#pragma unroll
+                        for (int j = 0; j < NS / 2; ++j) {
+                            const f2 e = pack2(ee[k][kk][2 * j], ee[k][kk][2 * j + 1]);
+                            if constexpr (kCorrM) {
+                                hp[k][j] = mul2(e, hp[k][j]);  // no input: h = Abar h
+                            } else {
+                                const float qa[4] = {q4[k].x, q4[k].y, q4[k].z, q4[k].w};
+                                const f2 qq = pack2(qa[kk], qa[kk]);
+                                hp[k][j] = fma2(e, hp[k][j], mul2(qq, bq[j]));
+                            }
+                            acc = fma2(cq[j], hp[k][j], acc);
+                        }
+                        float lo, hi;
+                        unpack2(acc, lo, hi);
+                        yp[k][kk] = lo + hi;
+                    }
+                }
             } else {
+                const float4 dv = d4[0], qv = q4[0];
+                const f2 dd4[4] = {pack2(dv.x, dv.x), pack2(dv.y, dv.y), pack2(dv.z, dv.z),
+                                   pack2(dv.w, dv.w)};
+                const f2 qq4[4] = {pack2(qv.x, qv.x), pack2(qv.y, qv.y), pack2(qv.z, qv.z),
+                                   pack2(qv.w, qv.w)};
+                constexpr bool kPipe = S6_PIPE && S6_PREEXP && !ZOH && S6_POLY == 0;
+                // all Abar factors of the four steps first, so their SFU latency overlaps
+                // (with the lookahead, they were formed during the previous group)
+                f2 ee[4][NS / 2];
+                if constexpr (kPipe) {
+                    if (t == 0) {
 #pragma unroll
-                for (int g = 0; g < 4; g += P) sY[cw * RS + t + g + pp] = transpose_reduce<P>(yp + g, pp);
+                        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                            for (int j = 0; j < NS / 2; ++j)
+                                ee_next[kk][j] = ex2x2(mul2(dd4[kk], a2p[0][j]));
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                        for (int j = 0; j < NS / 2; ++j) ee[kk][j] = ee_next[kk][j];
+                } else if constexpr (S6_PREEXP && !ZOH && S6_POLY == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                        for (int j = 0; j < NS / 2; ++j) ee[kk][j] = ex2x2(mul2(dd4[kk], a2p[0][j]));
+                }
+                // the next group's step sizes, for the lookahead
+                f2 ddn[4];
+                if constexpr (kPipe) {
+                    if (t + 4 < T) {
+                        const float4 dn = *reinterpret_cast<const float4*>(sDel + cwk[0] * RS + t + 4);
+                        ddn[0] = pack2(dn.x, dn.x), ddn[1] = pack2(dn.y, dn.y);
+                        ddn[2] = pack2(dn.z, dn.z), ddn[3] = pack2(dn.w, dn.w);
+                    }
+                }
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    if constexpr (kPipe) {
+                        if (t + 4 < T) {
+#pragma unroll
+                            for (int j = 0; j < NS / 2; ++j)
+                                ee_next[kk][j] = ex2x2(mul2(ddn[kk], a2p[0][j]));
+                        }
+                    }
+                    const f2 dd = dd4[kk];
+                    // ZOH: qq4 holds (u, u); Delta u is formed here
+                    const f2 uu = qq4[kk];
+                    const f2 qq = ZOH ? mul2(dd, uu) : qq4[kk];
+                    f2 bq[NS / 2], cq[NS / 2];
+                    coefs(kk, bq, cq);
+                    f2 acc = pack2(0.f, 0.f);
+#pragma unroll
+                    for (int j = 0; j < NS / 2; ++j) {
+                        if constexpr (ZOH) {
+                            const f2 x0 = mul2(dd, a2p[0][j]);
+                            const f2 e0 = ex2x2(x0);
+                            const f2 m0 = zoh_weight_u2(x0, e0, inv_ap[j], uu, qq);
+                            hp[0][j] = fma2(e0, hp[0][j], mul2(m0, bq[j]));
+                        } else if constexpr (S6_PREEXP && S6_POLY == 0) {
+                            hp[0][j] = fma2(ee[kk][j], hp[0][j], mul2(qq, bq[j]));
+                        } else {
+                            const bool on_fma = (j & 1) && (S6_POLY == 2 || (S6_POLY == 1 && (kk & 1)));
+                            const f2 e0 = on_fma ? exp2_fma2(mul2(dd, a2p[0][j]))
+                                                 : ex2x2(mul2(dd, a2p[0][j]));
+                            hp[0][j] = fma2(e0, hp[0][j], mul2(qq, bq[j]));
+                        }
+                        acc = fma2(cq[j], hp[0][j], acc);
+                    }
+                    float lo, hi;
+                    unpack2(acc, lo, hi);
+                    yp[0][kk] = lo + hi;
+                }
+            }
+            if constexpr (kSum) dsum += (d4[0].x + d4[0].y) + (d4[0].z + d4[0].w);
+            if constexpr (kOut) {
+#pragma unroll
+                for (int k = 0; k < CPL; ++k) {
+                    if constexpr (P == 1) {
+                        *reinterpret_cast<float4*>(sY + cwk[k] * RS + t) =
+                            make_float4(yp[k][0], yp[k][1], yp[k][2], yp[k][3]);
+                    } else {
+#pragma unroll
+                        for (int g = 0; g < 4; g += P)
+                            sY[cwk[k] * RS + t + g + pp] = transpose_reduce<P>(yp[k] + g, pp);
+                    }
+                }
             }
         }
 
@@ -625,19 +767,27 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
             __syncwarp();
             Tout* sOut = reinterpret_cast<Tout*>(smem + Lo::off_out);
             Tout* gy = static_cast<Tout*>(p.y);
-            for (int i = lane; i < G * (T / 4); i += 32) {
-                const int c = warp * G + i / (T / 4), tb = 4 * (i % (T / 4));
+            for (int i = lane; i < CW * (T / 4); i += 32) {
+                const int c = warp * CW + i / (T / 4), tb = 4 * (i % (T / 4));
                 const float4 y4 = *reinterpret_cast<const float4*>(sY + c * RS + tb);
-                float uu[4], zz[4];
-                V4::to_f(*reinterpret_cast<const VT*>(rU + c * T + tb), uu);
+                float uu[4] = {0.f, 0.f, 0.f, 0.f}, zz[4];
+                if (!kCorrM) V4::to_f(*reinterpret_cast<const VT*>(rU + c * T + tb), uu);
                 if (has_z) V4::to_f(*reinterpret_cast<const VT*>(rZ + c * T + tb), zz);
                 const float yv[4] = {y4.x, y4.y, y4.z, y4.w};
                 const float dsk = sDsk[c];
-                float o[4];
+                float o[4], sz[4];
+                if (has_z) {
+                    if constexpr (S6_SILU4) {
+                        silu4(zz, sz);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) sz[q] = silu(zz[q]);
+                    }
+                }
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    o[q] = fmaf(dsk, uu[q], yv[q]);
-                    if (has_z) o[q] *= silu(zz[q]);
+                    o[q] = kCorrM ? yv[q] : fmaf(dsk, uu[q], yv[q]);  // D u is in y already
+                    if (has_z) o[q] *= sz[q];
                 }
                 if (out_tma) {
                     store4(sOut + c * T + tb, o);
@@ -645,6 +795,18 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
                     const int64_t d = d0 + c;
                     if (d >= p.dim || tb >= valid) continue;
                     Tout* dst = gy + (b * p.dim + d) * p.L + t0 + tb;
+                    if constexpr (kCorrM) {  // the correction adds to the first pass's output
+                        if (p.y_vec && tb + 4 <= valid) {
+                            float yo[4];
+                            vec4<Tout>::to_f(*reinterpret_cast<const typename vec4<Tout>::type*>(dst), yo);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) o[q] += yo[q];
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                if (tb + q < valid) o[q] += io<Tout>::to_f(dst[q]);
+                        }
+                    }
                     if (p.y_vec && tb + 4 <= valid) {
                         store4(dst, o);
                     } else {
@@ -657,8 +819,8 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
             if (out_tma) {
                 fence_proxy_async();  // this lane's tile writes, before the async-proxy read
                 __syncwarp();
-                if (lane == 0 && d0 + warp * G < p.dim) {  // rows past dim are clipped
-                    tma_store_3d(&tm.y, sOut + warp * G * T, (int)t0, (int)(d0 + warp * G), (int)b);
+                if (lane == 0 && d0 + warp * CW < p.dim) {  // rows past dim are clipped
+                    tma_store_3d(&tm.y, sOut + warp * CW * T, (int)t0, (int)(d0 + warp * CW), (int)b);
                     tma_store_commit();
                 }
             }
@@ -667,32 +829,54 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[4 + (k & 1)]);
         }
+        if constexpr (kCorrM) {
+            // The carried start state only decays (Abar in (0, 1] when A <= 0 and Delta >= 0):
+            // once every state of every channel of the CTA is below 2^-24 of where it
+            // started, the rest of the correction is below fp32 resolution and the CTA stops.
+            bool small = decay_ok;
+#pragma unroll
+            for (int kc = 0; kc < CPL; ++kc)
+#pragma unroll
+                for (int j = 0; j < NS / 2; ++j) {
+                    float h0v, h1v;
+                    unpack2(hp[kc][j], h0v, h1v);
+                    small = small && fabsf(h0v) <= decay_thr && fabsf(h1v) <= decay_thr;
+                }
+            if (__syncthreads_and(small)) {
+                if (TMA && k + 1 < nchunks) abort_chunk = k + 1;  // issued, still in flight
+                drained = true;
+                break;
+            }
+        }
     }
 
     if constexpr (TMA && !WS) {
         if (tid == 0) {
-            if (aborted) {  // let copies still in flight land before the CTA exits
-                mbar_wait_bounded(&bar[0], 0, kWaitLimitCycles);
-                mbar_wait_bounded(&bar[1], 0, kWaitLimitCycles);
-            }
+            // let the copy still in flight (the chunk the loop stopped at) land before the
+            // CTA exits; earlier chunks completed their phases already
+            if ((aborted || drained) && abort_chunk >= 0)
+                mbar_wait_bounded(&bar[abort_chunk & 1], (uint32_t)((abort_chunk >> 1) & 1),
+                                  kWaitLimitCycles);
         }
     }
     if (out_tma && lane == 0) tma_store_wait_all();
     if (aborted) return;
 
-    if (dch < p.dim) {
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) {
+        if (dchk[k] >= p.dim) continue;
         float h[NS];
 #pragma unroll
-        for (int j = 0; j < NS / 2; ++j) unpack2(hp[j], h[2 * j], h[2 * j + 1]);
-        if (kOut) {
+        for (int j = 0; j < NS / 2; ++j) unpack2(hp[k][j], h[2 * j], h[2 * j + 1]);
+        if constexpr (MODE == kFull || MODE == kFullCkpt) {
             if (p.last_state && seg == (int)gridDim.z - 1) {
 #pragma unroll
                 for (int n = 0; n < NS; ++n) {
                     const int nn = pp * NS + n;
-                    if (nn < p.N) p.last_state[(b * p.dim + dch) * p.N + nn] = h[n];
+                    if (nn < p.N) p.last_state[(b * p.dim + dchk[k]) * p.N + nn] = h[n];
                 }
             }
-        } else if (MODE == kAggregate) {
+        } else if constexpr (kSum) {
             const int64_t row = ((int64_t)seg * p.batch + b) * p.dim + dch;
 #pragma unroll
             for (int n = 0; n < NS; ++n) {
@@ -738,6 +922,29 @@ __global__ void carry_kernel(float* seg_h, const float* seg_sum, const float* A,
         H = fmaf(ex2(a2 * seg_sum[row]), H, hend);  // (prod Abar, h_end) (+) (., H)
     }
     seg_h[((int64_t)(nseg - 1) * batch * dim + bd) * N + n] = H;
+}
+
+// The one-pass split's fold.  Thread per (batch, channel, state): on entry seg_h[s]
+// holds the end state of segment s scanned from h = 0 and seg_sum[s] its summed step,
+// for every segment; on exit seg_h[s] holds segment s's true start state (segment 0
+// from h0, or zero), and last_state (when not null) the state after the whole sequence.
+__global__ void carry_all_kernel(float* seg_h, const float* seg_sum, const float* A, int64_t batch,
+                                 int64_t dim, int N, int nseg, const float* h0, float* last_state) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t lanes = batch * dim * N;
+    if (i >= lanes) return;
+    const int n = (int)(i % N);
+    const int64_t bd = i / N;
+    const int64_t d = bd % dim;
+    const float a2 = A[d * N + n] * kLog2e;
+    float H = h0 ? h0[bd * N + n] : 0.f;
+    for (int s = 0; s < nseg; ++s) {
+        const int64_t row = (int64_t)s * batch * dim + bd;
+        const float hend = seg_h[row * N + n];
+        seg_h[row * N + n] = H;
+        H = fmaf(ex2(a2 * seg_sum[row]), H, hend);  // (prod Abar, h_end) (+) (., H)
+    }
+    if (last_state) last_state[bd * N + n] = H;
 }
 
 // Inclusive fold of `count` segment summaries (h_end from zero, summed step) applied to h0:
@@ -799,20 +1006,54 @@ bool encode_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, u
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor maps of one launch: boxes of T steps x the tile's channels for u, delta (and z
+// when gated), of T steps x NMAX states for B and C, and of T steps x one warp's channels
+// for y when the output rows can be stored by TMA.
+template <typename Lo, int NMAX, typename Tin, typename Tout>
+bool make_maps(const ScanArgs& a, bool want_z, bool want_y, TMaps* tm) {
+    memset(tm, 0, sizeof(*tm));
+    bool ok = encode_3d<Tin>(&tm->u, a.u, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
+              encode_3d<Tin>(&tm->dr, a.delta, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
+              encode_3d<Tin>(&tm->B, a.B, a.L, a.N, a.batch, Lo::T, NMAX) &&
+              encode_3d<Tin>(&tm->C, a.C, a.L, a.N, a.batch, Lo::T, NMAX);
+    if (ok && want_z && a.z) ok = encode_3d<Tin>(&tm->z, a.z, a.L, a.dim, a.batch, Lo::T, Lo::CH);
+    if (ok && want_y) ok = encode_3d<Tout>(&tm->y, a.y, a.L, a.dim, a.batch, Lo::T, Lo::CW);
+    return ok;
+}
+
+// Rows that TMA can describe: a 16-byte multiple of elements, coordinates in int32.
+template <typename T>
+bool tma_rows(const ScanArgs& a) {
+    const bool fits = a.L < (1LL << 31) && a.dim < (1LL << 31) && a.batch < (1LL << 31);
+    return fits && a.L > 0 && (a.L * (int64_t)sizeof(T)) % 16 == 0;
+}
+
+// One launch of the scan kernel over (channel tiles, batch, segments); `nz` segments
+// (the grid's z extent).  TMA launches build their tensor maps from the kernel's layout.
 template <int NMAX, int P, int WARPS, int T, typename Tin, typename Tout, int MODE, bool TMA,
-          bool ZOH = false, bool WS = false>
-cudaError_t launch_one(const KParams& kp, const TMaps& tm, dim3 grid, cudaStream_t s) {
-    using Lo = Layout<NMAX, P, WARPS, T, Tin, Tout>;
-    auto kern = scan_kernel<NMAX, P, WARPS, T, Tin, Tout, MODE, TMA, ZOH, WS>;
+          bool ZOH = false, bool WS = false, int CPL = 1>
+cudaError_t launch_one(const ScanArgs& a, KParams kp, int64_t nz, cudaStream_t s) {
+    using Lo = Layout<NMAX, P, WARPS, T, Tin, Tout, CPL>;
+    constexpr bool kOut = MODE == kFull || MODE == kFullCkpt || MODE == kFullAgg || MODE == kCorr;
+    TMaps tm;
+    memset(&tm, 0, sizeof(tm));
+    kp.y_tma = 0;
+    if constexpr (TMA) {
+        const bool out16 = kOut && tma_rows<Tout>(a);
+        if (!make_maps<Lo, NMAX, Tin, Tout>(a, kOut, out16, &tm)) return cudaErrorInvalidValue;
+        kp.y_tma = out16 ? 1 : 0;
+    }
+    auto kern = scan_kernel<NMAX, P, WARPS, T, Tin, Tout, MODE, TMA, ZOH, WS, CPL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Lo::bytes);
     if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)((a.dim + Lo::CH - 1) / Lo::CH), (unsigned)a.batch, (unsigned)nz);
     kern<<<grid, Lo::THREADS + (WS ? 32 : 0), Lo::bytes, s>>>(kp, tm);
     return cudaGetLastError();
 }
 
-// Instantiation per state width: N = 16 uses the tuned tile; narrower states keep four
-// states per lane.
+// Instantiation per state width for the split passes, checkpoints and the exact ZOH scan:
+// N = 16 uses the tuned tile; narrower states keep four states per lane.
 template <int NMAX>
 struct Tile {
     static constexpr int P = NMAX == 16 ? S6_P16 : NMAX / 4;
@@ -820,14 +1061,39 @@ struct Tile {
     static constexpr int T = NMAX == 16 ? S6_CHUNK : 64;
 };
 
+// The plain forward (one pass, no checkpoints, Delta * B weight).
+template <int NMAX>
+struct TileFwd {
+    static constexpr int P = Tile<NMAX>::P;
+    static constexpr int CPL = NMAX == 16 ? S6_CPL16 : 1;
+    static constexpr int WARPS = NMAX == 16 ? S6_WARPS16F : Tile<NMAX>::WARPS;
+    static constexpr int T = Tile<NMAX>::T;
+};
+
 template <int NMAX, typename Tin, typename Tout, bool TMA, bool ZOH>
-cudaError_t launch_typed(const ScanArgs& a, const KParams& kp, const TMaps& tm, cudaStream_t s) {
+cudaError_t launch_typed(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
     using TL = Tile<NMAX>;
-    using Lo = Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout>;
-    const unsigned gx = (unsigned)((a.dim + Lo::CH - 1) / Lo::CH);
-    if (a.nseg > 1) {
+    using TF = TileFwd<NMAX>;
+    if (a.nseg > 1 && !a.ckpt) {
+        // One pass over every segment from h = 0 (y, end states, summed steps), the fold,
+        // then the input-free correction of every segment that starts from a nonzero state
+        // (segment 0 only when the caller gave h0), for as long as that state matters.
+        cudaError_t e = launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFullAgg, TMA, ZOH>(
+            a, kp, a.nseg, s);
+        if (e != cudaSuccess) return e;
+        const int64_t lanes = a.batch * a.dim * a.N;
+        carry_all_kernel<<<(unsigned)((lanes + 255) / 256), 256, 0, s>>>(
+            a.seg_h, a.seg_sum, a.A, a.batch, a.dim, (int)a.N, (int)a.nseg, a.h0, a.last_state);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        KParams kc = kp;
+        kc.seg_first = a.h0 ? 0 : 1;
+        return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kCorr, TMA, ZOH>(
+            a, kc, a.nseg - kc.seg_first, s);
+    }
+    if (a.nseg > 1) {  // a training forward: exact starts first, so the checkpoints are true
         cudaError_t e = launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kAggregate, TMA, ZOH>(
-            kp, tm, dim3(gx, (unsigned)a.batch, (unsigned)(a.nseg - 1)), s);
+            a, kp, a.nseg - 1, s);
         if (e != cudaSuccess) return e;
         const int64_t lanes = a.batch * a.dim * a.N;
         carry_kernel<<<(unsigned)((lanes + 255) / 256), 256, 0, s>>>(
@@ -838,85 +1104,37 @@ cudaError_t launch_typed(const ScanArgs& a, const KParams& kp, const TMaps& tm, 
     if constexpr (!ZOH) {
         if (a.ckpt)
             return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFullCkpt, TMA, false>(
-                kp, tm, dim3(gx, (unsigned)a.batch, (unsigned)a.nseg), s);
+                a, kp, a.nseg, s);
+        // the split's rescan keeps the tile its segment plan was made for
+        if (a.nseg == 1)
+            return launch_one<NMAX, TF::P, TF::WARPS, TF::T, Tin, Tout, kFull, TMA, false,
+                              TMA && S6_WS, TF::CPL>(a, kp, 1, s);
     }
-    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA, ZOH, TMA && S6_WS>(
-        kp, tm, dim3(gx, (unsigned)a.batch, (unsigned)a.nseg), s);
+    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA, ZOH, TMA && S6_WS && !ZOH>(
+        a, kp, a.nseg, s);
 }
 
 template <int NMAX, typename Tin, typename Tout, bool ZOH>
-cudaError_t launch_io(const ScanArgs& a, KParams kp, cudaStream_t s) {
-    using TL = Tile<NMAX>;
-    using Lo = Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout>;
-    TMaps tm;
-    memset(&tm, 0, sizeof(tm));
-    const bool rows16 = (a.L * (int64_t)sizeof(Tin)) % 16 == 0 && a.L > 0;
-    const bool out16 = (a.L * (int64_t)sizeof(Tout)) % 16 == 0 && a.L > 0;
-    // TMA coordinates are 32-bit signed integers.
-    const bool fits = a.L < (1LL << 31) && a.dim < (1LL << 31) && a.batch < (1LL << 31);
-    if (!(rows16 && fits)) {
-        kp.y_tma = 0;
-        return launch_typed<NMAX, Tin, Tout, false, ZOH>(a, kp, tm, s);
-    }
-    bool ok = encode_3d<Tin>(&tm.u, a.u, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
-              encode_3d<Tin>(&tm.dr, a.delta, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
-              encode_3d<Tin>(&tm.B, a.B, a.L, a.N, a.batch, Lo::T, NMAX) &&
-              encode_3d<Tin>(&tm.C, a.C, a.L, a.N, a.batch, Lo::T, NMAX);
-    if (ok && a.z) ok = encode_3d<Tin>(&tm.z, a.z, a.L, a.dim, a.batch, Lo::T, Lo::CH);
-    kp.y_tma = out16 ? 1 : 0;
-    if (ok && out16) ok = encode_3d<Tout>(&tm.y, a.y, a.L, a.dim, a.batch, Lo::T, Lo::G);
-    if (!ok) return cudaErrorInvalidValue;
-    return launch_typed<NMAX, Tin, Tout, true, ZOH>(a, kp, tm, s);
-}
-
-template <int NMAX, typename Tin, bool TMA>
-cudaError_t launch_ckpt_typed(const ScanArgs& a, const KParams& kp, const TMaps& tm,
-                              cudaStream_t s) {
-    using TL = Tile<NMAX>;
-    using Lo = Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin>;
-    const unsigned gx = (unsigned)((a.dim + Lo::CH - 1) / Lo::CH);
-    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kCheckpoint, TMA>(
-        kp, tm, dim3(gx, (unsigned)a.batch, 1), s);
+cudaError_t launch_io(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
+    return tma_rows<Tin>(a) ? launch_typed<NMAX, Tin, Tout, true, ZOH>(a, kp, s)
+                            : launch_typed<NMAX, Tin, Tout, false, ZOH>(a, kp, s);
 }
 
 template <int NMAX, typename Tin>
-cudaError_t launch_ckpt_io(const ScanArgs& a, KParams kp, cudaStream_t s) {
+cudaError_t launch_ckpt_io(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
     using TL = Tile<NMAX>;
-    using Lo = Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin>;
-    TMaps tm;
-    memset(&tm, 0, sizeof(tm));
-    kp.y_tma = 0;
-    const bool rows16 = (a.L * (int64_t)sizeof(Tin)) % 16 == 0 && a.L > 0;
-    const bool fits = a.L < (1LL << 31) && a.dim < (1LL << 31) && a.batch < (1LL << 31);
-    if (!(rows16 && fits)) return launch_ckpt_typed<NMAX, Tin, false>(a, kp, tm, s);
-    const bool ok = encode_3d<Tin>(&tm.u, a.u, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
-                    encode_3d<Tin>(&tm.dr, a.delta, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
-                    encode_3d<Tin>(&tm.B, a.B, a.L, a.N, a.batch, Lo::T, NMAX) &&
-                    encode_3d<Tin>(&tm.C, a.C, a.L, a.N, a.batch, Lo::T, NMAX);
-    if (!ok) return cudaErrorInvalidValue;
-    return launch_ckpt_typed<NMAX, Tin, true>(a, kp, tm, s);
+    return tma_rows<Tin>(a)
+               ? launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kCheckpoint, true>(a, kp, 1, s)
+               : launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kCheckpoint, false>(a, kp, 1, s);
 }
 
 // Segment summaries: kAggregate over `nseg` segments (all of them) into seg_h / seg_sum.
 template <int NMAX, typename Tin, bool ZOH>
-cudaError_t launch_summary_io(const ScanArgs& a, KParams kp, cudaStream_t s) {
+cudaError_t launch_summary_io(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
     using TL = Tile<NMAX>;
-    using Lo = Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin>;
-    TMaps tm;
-    memset(&tm, 0, sizeof(tm));
-    kp.y_tma = 0;
-    const unsigned gx = (unsigned)((a.dim + Lo::CH - 1) / Lo::CH);
-    const dim3 grid(gx, (unsigned)a.batch, (unsigned)a.nseg);
-    const bool rows16 = (a.L * (int64_t)sizeof(Tin)) % 16 == 0 && a.L > 0;
-    const bool fits = a.L < (1LL << 31) && a.dim < (1LL << 31) && a.batch < (1LL << 31);
-    if (!(rows16 && fits))
-        return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kAggregate, false, ZOH>(kp, tm, grid, s);
-    const bool ok = encode_3d<Tin>(&tm.u, a.u, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
-                    encode_3d<Tin>(&tm.dr, a.delta, a.L, a.dim, a.batch, Lo::T, Lo::CH) &&
-                    encode_3d<Tin>(&tm.B, a.B, a.L, a.N, a.batch, Lo::T, NMAX) &&
-                    encode_3d<Tin>(&tm.C, a.C, a.L, a.N, a.batch, Lo::T, NMAX);
-    if (!ok) return cudaErrorInvalidValue;
-    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kAggregate, true, ZOH>(kp, tm, grid, s);
+    return tma_rows<Tin>(a)
+               ? launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kAggregate, true, ZOH>(a, kp, a.nseg, s)
+               : launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kAggregate, false, ZOH>(a, kp, a.nseg, s);
 }
 
 template <int NMAX, bool ZOH>
@@ -1127,6 +1345,7 @@ cudaError_t launch_scan(const ScanArgs& a, cudaStream_t stream) {
     kp.softplus = a.softplus ? 1 : 0;
     kp.y_vec = a.L % 4 == 0 ? 1 : 0;
     kp.y_tma = 0;
+    kp.seg_first = 0;
     if (a.N <= 4) return launch_nmax<4>(a, kp, stream);
     if (a.N <= 8) return launch_nmax<8>(a, kp, stream);
     return launch_nmax<16>(a, kp, stream);

@@ -8,6 +8,8 @@
 // state, so a warp touches 512 consecutive bytes per access.  The per-lane
 // readout sum_n C_n h_n is finished with log2(G) xor-shuffles.  A compile-time
 // variant uses the exact zero-order-hold input weight (e^{Delta A} - 1) / A.
+#include <algorithm>
+
 #include "s6_device.cuh"
 #include "s6_launch.h"
 
@@ -128,6 +130,10 @@ __global__ void __launch_bounds__(256) state_update_kernel(const UParams p) {
 #ifndef S6_DEC_ITEMS
 #define S6_DEC_ITEMS 2
 #endif
+// Nonzero: the persistent variant with that many CTAs per SM.
+#ifndef S6_DEC_PERSIST
+#define S6_DEC_PERSIST 0
+#endif
 constexpr int kItems = S6_DEC_ITEMS;
 
 template <typename Tio>
@@ -137,14 +143,66 @@ struct Lane16 {
     float u, x, z, dsk;
 };
 
+// Every load of lane li's half h (state, A, B, C, u, delta, z, D) into w.
+template <typename Tio>
+__device__ __forceinline__ void load_lane16(const UParams& p, uint32_t li, bool act, int h,
+                                            Lane16<Tio>& w) {
+    using VT = typename vec4<Tio>::type;
+    const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    const uint32_t dim = (uint32_t)p.dim;
+    const uint32_t bb = li / dim, d = li - bb * dim;
+    const float* sp = p.state + (size_t)li * 16;
+    const float* ap = p.A + (size_t)d * 16;
+    const Tio* bp = static_cast<const Tio*>(p.B) + (size_t)bb * 16;
+    const Tio* cp = static_cast<const Tio*>(p.C) + (size_t)bb * 16;
+    w.s0 = act ? *reinterpret_cast<const float4*>(sp + 4 * h) : z4;
+    w.s1 = act ? *reinterpret_cast<const float4*>(sp + 8 + 4 * h) : z4;
+    w.a0 = __ldg(reinterpret_cast<const float4*>(ap + 4 * h));
+    w.a1 = __ldg(reinterpret_cast<const float4*>(ap + 8 + 4 * h));
+    w.b0 = *reinterpret_cast<const VT*>(bp + 4 * h);
+    w.b1 = *reinterpret_cast<const VT*>(bp + 8 + 4 * h);
+    w.c0 = *reinterpret_cast<const VT*>(cp + 4 * h);
+    w.c1 = *reinterpret_cast<const VT*>(cp + 8 + 4 * h);
+    w.u = io<Tio>::load(static_cast<const Tio*>(p.u) + li);
+    w.x = io<Tio>::load(static_cast<const Tio*>(p.delta) + li) + (p.delta_bias ? p.delta_bias[d] : 0.f);
+    w.z = p.z ? io<Tio>::load(static_cast<const Tio*>(p.z) + li) : 0.f;
+    w.dsk = p.D ? p.D[d] : 0.f;
+}
+
+template <typename Tio, bool ZOH>
+__device__ __forceinline__ void step_lane16(const UParams& p, uint32_t li, bool act, int h,
+                                            const Lane16<Tio>& w);
+
+// Persistent variant: a grid of a few CTAs per SM; each thread walks its half of lanes
+// one grid stride apart, loading the next lane's data before computing the current one.
+// Every thread of a warp runs the same number of rounds (the readout's shuffle needs the
+// whole warp); threads past the last lane compute on placeholder data and store nothing.
+template <typename Tio, bool ZOH>
+__global__ void __launch_bounds__(256) state_update16p_kernel(const UParams p) {
+    const uint32_t pairs = (uint32_t)(gridDim.x * blockDim.x) / 2;
+    const uint32_t gid = blockIdx.x * blockDim.x + threadIdx.x;
+    const int h = gid & 1;
+    const uint32_t lanes = (uint32_t)p.lanes;
+    uint32_t li = gid >> 1;
+    bool act = li < lanes;
+    Lane16<Tio> cur, nxt;
+    load_lane16<Tio>(p, act ? li : 0, act, h, cur);
+    while (__any_sync(0xffffffffu, act)) {
+        const uint32_t nl = li + pairs;
+        const bool nact = nl < lanes;
+        load_lane16<Tio>(p, nact ? nl : 0, nact, h, nxt);
+        step_lane16<Tio, ZOH>(p, act ? li : 0, act, h, cur);
+        cur = nxt;
+        li = nl;
+        act = nact;
+    }
+}
+
 template <typename Tio, bool ZOH>
 __global__ void __launch_bounds__(256) state_update16_kernel(const UParams p) {
-    using VT = typename vec4<Tio>::type;
     const uint32_t pairs = (uint32_t)(gridDim.x * blockDim.x) / 2;  // lanes per item sweep
     const uint32_t gid = blockIdx.x * blockDim.x + threadIdx.x;
     const int h = gid & 1;
-    const uint32_t dim = (uint32_t)p.dim;
-    const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
     Lane16<Tio> v[kItems];
     uint32_t lid[kItems];
     bool act[kItems];
@@ -152,30 +210,18 @@ __global__ void __launch_bounds__(256) state_update16_kernel(const UParams p) {
     for (int it = 0; it < kItems; ++it) {
         const uint32_t lane_id = (gid >> 1) + it * pairs;
         act[it] = lane_id < (uint32_t)p.lanes;
-        const uint32_t li = act[it] ? lane_id : 0;
-        lid[it] = li;
-        const uint32_t bb = li / dim, d = li - bb * dim;
-        const float* sp = p.state + (size_t)li * 16;
-        const float* ap = p.A + (size_t)d * 16;
-        const Tio* bp = static_cast<const Tio*>(p.B) + (size_t)bb * 16;
-        const Tio* cp = static_cast<const Tio*>(p.C) + (size_t)bb * 16;
-        v[it].s0 = act[it] ? *reinterpret_cast<const float4*>(sp + 4 * h) : z4;
-        v[it].s1 = act[it] ? *reinterpret_cast<const float4*>(sp + 8 + 4 * h) : z4;
-        v[it].a0 = __ldg(reinterpret_cast<const float4*>(ap + 4 * h));
-        v[it].a1 = __ldg(reinterpret_cast<const float4*>(ap + 8 + 4 * h));
-        v[it].b0 = *reinterpret_cast<const VT*>(bp + 4 * h);
-        v[it].b1 = *reinterpret_cast<const VT*>(bp + 8 + 4 * h);
-        v[it].c0 = *reinterpret_cast<const VT*>(cp + 4 * h);
-        v[it].c1 = *reinterpret_cast<const VT*>(cp + 8 + 4 * h);
-        v[it].u = io<Tio>::load(static_cast<const Tio*>(p.u) + li);
-        v[it].x = io<Tio>::load(static_cast<const Tio*>(p.delta) + li) +
-                  (p.delta_bias ? p.delta_bias[d] : 0.f);
-        v[it].z = p.z ? io<Tio>::load(static_cast<const Tio*>(p.z) + li) : 0.f;
-        v[it].dsk = p.D ? p.D[d] : 0.f;
+        lid[it] = act[it] ? lane_id : 0;
+        load_lane16<Tio>(p, lid[it], act[it], h, v[it]);
     }
 #pragma unroll
-    for (int it = 0; it < kItems; ++it) {
-        const Lane16<Tio>& w = v[it];
+    for (int it = 0; it < kItems; ++it) step_lane16<Tio, ZOH>(p, lid[it], act[it], h, v[it]);
+}
+
+// The token for one lane half: Delta, Abar, the state update, the readout, y.
+template <typename Tio, bool ZOH>
+__device__ __forceinline__ void step_lane16(const UParams& p, uint32_t li, bool act, int h,
+                                            const Lane16<Tio>& w) {
+    {
         float bv[8], cv[8], t[4];
         vec4<Tio>::to_f(w.b0, t);
         bv[0] = t[0], bv[1] = t[1], bv[2] = t[2], bv[3] = t[3];
@@ -203,8 +249,8 @@ __global__ void __launch_bounds__(256) state_update16_kernel(const UParams p) {
             acc = fma2(pack2(cv[j], cv[j + 1]), hn, acc);
             unpack2(hn, out[j], out[j + 1]);
         }
-        if (act[it]) {
-            float* wp = p.state + (size_t)lid[it] * 16;
+        if (act) {
+            float* wp = p.state + (size_t)li * 16;
             *reinterpret_cast<float4*>(wp + 4 * h) = make_float4(out[0], out[1], out[2], out[3]);
             *reinterpret_cast<float4*>(wp + 8 + 4 * h) = make_float4(out[4], out[5], out[6], out[7]);
         }
@@ -212,10 +258,10 @@ __global__ void __launch_bounds__(256) state_update16_kernel(const UParams p) {
         unpack2(acc, lo, hi);
         float yv = lo + hi;
         yv += __shfl_xor_sync(0xffffffffu, yv, 1);
-        if (act[it] && h == 0) {
+        if (act && h == 0) {
             yv = fmaf(w.dsk, w.u, yv);
             if (p.z) yv *= silu(w.z);
-            static_cast<Tio*>(p.y)[lid[it]] = io<Tio>::from_f(yv);
+            static_cast<Tio*>(p.y)[li] = io<Tio>::from_f(yv);
         }
     }
 }
@@ -232,8 +278,18 @@ cudaError_t launch_u(const UParams& p, cudaStream_t s) {
 template <typename Tio, bool ZOH>
 cudaError_t launch_u_typed(const UParams& p, cudaStream_t s) {
     if (p.N == 16 && p.lanes < (1LL << 29)) {
+#if S6_DEC_PERSIST
+        // a whole number of waves: S6_DEC_PERSIST CTAs of 256 threads per SM
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int64_t need = (2 * p.lanes + 255) / 256;
+        const int64_t blocks = std::min<int64_t>(need, (int64_t)sms * S6_DEC_PERSIST);
+        state_update16p_kernel<Tio, ZOH><<<(unsigned)blocks, 256, 0, s>>>(p);
+#else
         const int64_t threads = 2 * ((p.lanes + kItems - 1) / kItems);
         state_update16_kernel<Tio, ZOH><<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(p);
+#endif
         return cudaGetLastError();
     }
     if (p.N <= 4) return launch_u<4, Tio, ZOH>(p, s);

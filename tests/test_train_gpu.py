@@ -1,7 +1,11 @@
 """The training path (needs a B200): a forward that records the backward's checkpoints
 (mamba_selective_scan_fwd_train) and the backward that reads them
 (mamba_selective_scan_bwd_from_checkpoints).  The forward's outputs must equal the plain
-forward's bit for bit, and the gradients must equal those of the recomputing backward:
+forward's bit for bit when the sequence is scanned in one pass; a sequence long enough to
+be split is scanned by the plain forward in one pass over all segments from zero plus a
+correction from each segment's true start, while the training forward rescans every
+segment from its start (so its checkpoints are true states), and the two agree to
+rounding.  The gradients must equal those of the recomputing backward:
 bit for bit where no atomics are involved, when the sequence is scanned in one pass; dA,
 dB, dC, dD and ddelta_bias are sums formed with atomics, whose order varies, so they are
 compared to 1e-5 relative.  A sequence long enough to be split has its segment starts
@@ -37,13 +41,20 @@ def test_training_forward_and_backward_match(cuda_ok, shape, dtype):
                                        z=p["z"], delta_bias=p["delta_bias"],
                                        return_last_state=True)
     torch.cuda.synchronize()
-    assert torch.equal(y_t, y_p) and torch.equal(st_t, st_p)
+    split = ops.selective_scan_workspace_size(b, d, N, L) > 0
+    if not split:
+        assert torch.equal(y_t, y_p) and torch.equal(st_t, st_p)
+    else:  # y within one unit of the output dtype's rounding (plus a sliver of the range)
+        diff = (y_t.float() - y_p.float()).abs()
+        tol = (y_p.float().abs() * (2.0 ** -7 if dtype == torch.bfloat16 else 1e-5) +
+               1e-6 * y_p.float().abs().max())
+        assert bool((diff <= tol).all())
+        torch.testing.assert_close(st_t, st_p, rtol=1e-4, atol=1e-6 * st_p.abs().max().item())
     g_c = ops.selective_scan_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"],
                                  z=p["z"], delta_bias=p["delta_bias"], checkpoints=ck)
     g_r = ops.selective_scan_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"],
                                  z=p["z"], delta_bias=p["delta_bias"])
     torch.cuda.synchronize()
-    split = ops.selective_scan_workspace_size(b, d, N, L) > 0
     assert torch.equal(g_c["du"], g_r["du"])
     for k in ("ddelta", "dz"):
         if not split:
