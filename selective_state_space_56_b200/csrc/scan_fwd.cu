@@ -127,8 +127,15 @@ enum Mode : int { kFull = 0, kAggregate = 1, kCheckpoint = 2, kFullCkpt = 3, kFu
 #ifndef S6_PREEXP
 #define S6_PREEXP 1  // Abar of a whole 4-step group before its updates (measured +1.7%)
 #endif
+// TMA path, producer warps: 0 = none (one CTA barrier per chunk); 1 = one producer warp
+// stages every chunk and converts its coefficients; 2 = S6_WSP producer warps also form
+// Delta and Delta u for every channel into a double-buffered ring.  With 1 or 2 the
+// compute warps wait only on mbarriers and never for one another.
 #ifndef S6_WS
-#define S6_WS 0  // TMA path: a producer warp stages and converts, compute warps never meet
+#define S6_WS 0
+#endif
+#ifndef S6_WSP
+#define S6_WSP 1
 #endif
 #ifndef S6_POLY
 #define S6_POLY 0
@@ -163,7 +170,8 @@ enum Mode : int { kFull = 0, kAggregate = 1, kCheckpoint = 2, kFullCkpt = 3, kFu
 constexpr size_t align128(size_t x) { return (x + 127) / 128 * 128; }
 
 // Shared-memory carve-up for one instantiation.
-template <int NMAX, int P, int WARPS_, int T_, typename Tin, typename Tout, int CPL_ = 1>
+template <int NMAX, int P, int WARPS_, int T_, typename Tin, typename Tout, int CPL_ = 1,
+          int DQ = 1>
 struct Layout {
     static constexpr int T = T_;
     static constexpr int CPL = CPL_;           // channels per lane
@@ -190,8 +198,9 @@ struct Layout {
         kBC == 0 ? 2 * coef_fp32_bytes : (kBC == 1 ? coef_fp32_bytes : coef_fp32_bytes * 3 / 2);
     static constexpr size_t off_coef = 2 * stage_bytes;
     static constexpr size_t off_del = off_coef + 2 * coef_bytes_all;   // float [CH][RS]
-    static constexpr size_t off_du = off_del + (size_t)CH * RS * 4;
-    static constexpr size_t off_y = off_du + (size_t)CH * RS * 4;
+    static constexpr size_t dq_stride = (size_t)CH * RS;                // floats per Delta buffer
+    static constexpr size_t off_du = off_del + DQ * (size_t)CH * RS * 4;
+    static constexpr size_t off_y = off_du + DQ * (size_t)CH * RS * 4;
     static constexpr size_t off_out = align128(off_y + (size_t)CH * RS * 4);  // Tout [CH][T]
     static constexpr size_t out_bytes = align128((size_t)CH * T * sizeof(Tout));
     static constexpr size_t off_par = off_out + out_bytes;               // bias[CH], D[CH]
@@ -199,7 +208,7 @@ struct Layout {
     // ready[2] (coefficients converted) and empty[2] (compute warps done with a stage)
     static constexpr size_t off_bar = align128(off_par + (size_t)2 * CH * 4);
     static constexpr size_t bytes = off_bar + 6 * 8;
-    static_assert(NS % 4 == 0, "states per lane must be a multiple of 4");
+    static_assert(NS % 4 == 0 || NS == 2, "states per lane: a multiple of 4, or 2");
     static_assert(T % 4 == 0 && kChunk % T == 0, "chunks of whole 4-step groups");
     static_assert(T * sizeof(Tin) % 16 == 0 && T * sizeof(Tout) % 16 == 0, "TMA rows");
     static_assert(T <= 256 && CH <= 256, "TMA box extents");
@@ -216,21 +225,33 @@ __device__ __forceinline__ float transpose_reduce(const float* v, int pp) {
         float keep = hi ? v[1] : v[0];
         float send = hi ? v[0] : v[1];
         return keep + __shfl_xor_sync(0xffffffffu, send, 1);
-    } else {
-        static_assert(P == 4, "P must be 1, 2 or 4");
+    } else if constexpr (P == 4) {
         const bool hi2 = pp & 2;
         float w0 = (hi2 ? v[2] : v[0]) + __shfl_xor_sync(0xffffffffu, hi2 ? v[0] : v[2], 2);
         float w1 = (hi2 ? v[3] : v[1]) + __shfl_xor_sync(0xffffffffu, hi2 ? v[1] : v[3], 2);
         const bool hi1 = pp & 1;
         return (hi1 ? w1 : w0) + __shfl_xor_sync(0xffffffffu, hi1 ? w0 : w1, 1);
+    } else {
+        static_assert(P == 8, "P must be 1, 2, 4 or 8");
+        const bool hi4 = pp & 4;
+        float w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            w[i] = (hi4 ? v[i + 4] : v[i]) + __shfl_xor_sync(0xffffffffu, hi4 ? v[i] : v[i + 4], 4);
+        const bool hi2 = pp & 2;
+        const float x0 = (hi2 ? w[2] : w[0]) + __shfl_xor_sync(0xffffffffu, hi2 ? w[0] : w[2], 2);
+        const float x1 = (hi2 ? w[3] : w[1]) + __shfl_xor_sync(0xffffffffu, hi2 ? w[1] : w[3], 2);
+        const bool hi1 = pp & 1;
+        return (hi1 ? x1 : x0) + __shfl_xor_sync(0xffffffffu, hi1 ? x0 : x1, 1);
     }
 }
 
 template <int NMAX, int P, int WARPS, int T_, typename Tin, typename Tout, int MODE, bool TMA,
-          bool ZOH = false, bool WS = false, int CPL = 1>
-__global__ void __launch_bounds__(WARPS * 32 + (WS ? 32 : 0))
+          bool ZOH = false, int WS = 0, int CPL = 1>
+__global__ void __launch_bounds__(WARPS * 32 + 32 * (WS == 0 ? 0 : (WS == 1 ? 1 : S6_WSP)))
 scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
     static_assert(!WS || (TMA && MODE == kFull), "producer warp: TMA full scans only");
+    constexpr int NPROD = WS == 0 ? 0 : (WS == 1 ? 1 : S6_WSP);  // producer warps
     static_assert(CPL == 1 || (MODE == kFull && !ZOH && !WS), "two channels per lane: plain scan");
     constexpr bool kOut = MODE == kFull || MODE == kFullCkpt || MODE == kFullAgg ||
                           MODE == kCorr;                              // writes y
@@ -241,7 +262,7 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
     // keep the state-paired form)
     constexpr bool kTPX = (MODE == kCorr) || (S6_TPX && !ZOH && S6_POLY == 0);
     static_assert(CPL == 1 || kTPX, "two channels per lane use the time-paired form");
-    using Lo = Layout<NMAX, P, WARPS, T_, Tin, Tout, CPL>;
+    using Lo = Layout<NMAX, P, WARPS, T_, Tin, Tout, CPL, WS == 2 ? 2 : 1>;
     using V4 = vec4<Tin>;
     using VT = typename V4::type;
     constexpr int T = Lo::T, NS = Lo::NS, G = Lo::G, CW = Lo::CW, CH = Lo::CH, RS = Lo::RS;
@@ -273,8 +294,8 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         mbar_init(&bar[0], 1);
         mbar_init(&bar[1], 1);
         if (WS) {
-            mbar_init(&bar[2], 1);
-            mbar_init(&bar[3], 1);
+            mbar_init(&bar[2], NPROD);
+            mbar_init(&bar[3], NPROD);
             mbar_init(&bar[4], WARPS);
             mbar_init(&bar[5], WARPS);
         }
@@ -449,11 +470,54 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         }
     };
 
+    // Phase A on chunk k: work items i0, i0 + istride, ... below nitems, item i being channel
+    // cfirst + i / (T/4) at steps 4 (i % (T/4)) .. +3: Delta = softplus(delta + bias) and
+    // Delta u (u itself for the exact ZOH weight) into dl, du.  Steps past the end of the
+    // segment get Delta = 0 (Abar = 1, no input): the state passes.
+    auto phase_a = [&](int64_t k, int cfirst, int nitems, int i0, int istride, float* dl, float* du) {
+        const unsigned char* stb = smem + (k & 1) * Lo::stage_bytes;
+        const Tin* rU = reinterpret_cast<const Tin*>(stb);
+        const Tin* rDr = reinterpret_cast<const Tin*>(stb + Lo::off_dr);
+        const int valid = (int)min((int64_t)T, t_end - (t_begin + k * T));
+        for (int i = i0; i < nitems; i += istride) {
+            const int c = cfirst + i / (T / 4), tb = 4 * (i % (T / 4));
+            float x[4], uu[4] = {0.f, 0.f, 0.f, 0.f};
+            V4::to_f(*reinterpret_cast<const VT*>(rDr + c * T + tb), x);
+            if (!kCorrM) V4::to_f(*reinterpret_cast<const VT*>(rU + c * T + tb), uu);
+            const float bias = sBias[c];
+            float dt[4], xb[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) xb[q] = x[q] + bias;
+            if (p.softplus) {
+                softplus4(xb, dt);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) dt[q] = xb[q];
+            }
+            if (valid < T) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) dt[q] = tb + q < valid ? dt[q] : 0.f;
+            }
+            *reinterpret_cast<float4*>(dl + c * RS + tb) = make_float4(dt[0], dt[1], dt[2], dt[3]);
+            if constexpr (kCorrM) {
+                // no input term
+            } else if constexpr (ZOH) {  // the exact ZOH weight needs u itself
+                *reinterpret_cast<float4*>(du + c * RS + tb) = make_float4(uu[0], uu[1], uu[2], uu[3]);
+            } else {
+                const float q0 = dt[0] * uu[0], q1 = dt[1] * uu[1], q2 = dt[2] * uu[2],
+                            q3 = dt[3] * uu[3];
+                *reinterpret_cast<float4*>(du + c * RS + tb) = make_float4(q0, q1, q2, q3);
+            }
+        }
+        __syncwarp();
+    };
+
     // Producer warp (variant WS): stages every chunk with TMA and converts its
     // coefficients; the compute warps wait only for a chunk to be ready and release its
     // stage when done, so they never wait for one another.
     if constexpr (WS) {
-        if (warp == WARPS) {
+        if (warp >= WARPS) {
+            const int pw = warp - WARPS;  // producer warp index
             bool pok = true;
             int64_t issued = -1, landed = -1;
             for (int64_t k = 0; k < nchunks; ++k) {
@@ -463,7 +527,7 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
                         &bar[4 + s], (uint32_t)(((k >> 1) & 1) ^ 1), kWaitLimitCycles));
                     if (!pok) break;
                 }
-                if (lane == 0) {
+                if (pw == 0 && lane == 0) {
                     fence_proxy_async();  // the stage was last read through the generic proxy
                     issue_chunk(k);
                 }
@@ -472,13 +536,16 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
                                                                 kWaitLimitCycles));
                 if (!pok) break;
                 landed = k;
-                convert_chunk(k, lane, 32);
+                convert_chunk(k, pw * 32 + lane, 32 * NPROD);
+                if constexpr (WS == 2)
+                    phase_a(k, 0, CH * (T / 4), pw * 32 + lane, 32 * NPROD, sDel + s * Lo::dq_stride,
+                            sDu + s * Lo::dq_stride);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar[2 + s]);
             }
             if (!pok) {
                 if (lane == 0) atomicOr(&g_device_error, 1u);
-                if (lane == 0 && issued > landed)  // let the copy in flight land first
+                if (pw == 0 && lane == 0 && issued > landed)  // let the copy in flight land first
                     mbar_wait_bounded(&bar[issued & 1], (uint32_t)((issued >> 1) & 1),
                                       kWaitLimitCycles);
             }
@@ -537,39 +604,10 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
             }
         }
 
-        // Phase A: step sizes of this warp's channels, four steps per lane.  Steps past
-        // the end of the segment get Delta = 0 (Abar = 1, no input): the state passes.
-        for (int i = lane; i < CW * (T / 4); i += 32) {
-            const int c = warp * CW + i / (T / 4), tb = 4 * (i % (T / 4));
-            float x[4], uu[4] = {0.f, 0.f, 0.f, 0.f};
-            V4::to_f(*reinterpret_cast<const VT*>(rDr + c * T + tb), x);
-            if (!kCorrM) V4::to_f(*reinterpret_cast<const VT*>(rU + c * T + tb), uu);
-            const float bias = sBias[c];
-            float dt[4], xb[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) xb[q] = x[q] + bias;
-            if (p.softplus) {
-                softplus4(xb, dt);
-            } else {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) dt[q] = xb[q];
-            }
-            if (valid < T) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) dt[q] = tb + q < valid ? dt[q] : 0.f;
-            }
-            *reinterpret_cast<float4*>(sDel + c * RS + tb) = make_float4(dt[0], dt[1], dt[2], dt[3]);
-            if constexpr (kCorrM) {
-                // no input term
-            } else if constexpr (ZOH) {  // the exact ZOH weight needs u itself
-                *reinterpret_cast<float4*>(sDu + c * RS + tb) = make_float4(uu[0], uu[1], uu[2], uu[3]);
-            } else {
-                const float q0 = dt[0] * uu[0], q1 = dt[1] * uu[1], q2 = dt[2] * uu[2],
-                            q3 = dt[3] * uu[3];
-                *reinterpret_cast<float4*>(sDu + c * RS + tb) = make_float4(q0, q1, q2, q3);
-            }
-        }
-        __syncwarp();
+        // Phase A for this warp's channels (with S6_WS=2 the producer warps do it).
+        float* sDelK = sDel + (WS == 2 ? (k & 1) * Lo::dq_stride : 0);
+        float* sDuK = sDu + (WS == 2 ? (k & 1) * Lo::dq_stride : 0);
+        if constexpr (WS != 2) phase_a(k, warp * CW, CW * (T / 4), lane, 32, sDelK, sDuK);
 
         // checkpoint mode: the state entering every CKPT-step block of the sequence,
         // ckpt[((b * dim + d) * blocks + kb) * N + n], blocks = ceil(L / CKPT)
@@ -591,18 +629,35 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
 
         // Phase B: the recurrence, four steps per iteration, states in packed pairs.
         f2 ee_next[4][NS / 2];  // the lookahead's Abar of the next group (S6_PIPE)
+        float yp8[CPL][8];      // P = 8: partial outputs of two groups for one transpose-reduce
 #pragma unroll
         for (int t = 0; t < T; t += 4) {
             if (kCk && t > 0 && t % CKPT == 0) write_ckpt(t);
             float4 d4[CPL], q4[CPL];
 #pragma unroll
             for (int k = 0; k < CPL; ++k) {
-                d4[k] = *reinterpret_cast<const float4*>(sDel + cwk[k] * RS + t);
-                if (!kCorrM) q4[k] = *reinterpret_cast<const float4*>(sDu + cwk[k] * RS + t);
+                d4[k] = *reinterpret_cast<const float4*>(sDelK + cwk[k] * RS + t);
+                if (!kCorrM) q4[k] = *reinterpret_cast<const float4*>(sDuK + cwk[k] * RS + t);
             }
             float yp[CPL][4];
             // this lane's B and C of step t + kk, as fp32 pairs (states 2j, 2j + 1)
             auto coefs = [&](int kk, f2 (&bq)[NS / 2], f2 (&cq)[NS / 2]) {
+                if constexpr (NS == 2) {  // one state pair per lane: half of a 4-state group
+                    const int q = pp >> 1, hw = pp & 1;
+                    if constexpr (Lo::kBC == 1) {
+                        const uint32_t* g = reinterpret_cast<const uint32_t*>(sBt) +
+                                            ((t + kk) * (NMAX / 4) + q) * 4;
+                        bq[0] = bf16pair(g[hw]);
+                        cq[0] = bf16pair(g[2 + hw]);
+                    } else {
+                        bq[0] = f2{*reinterpret_cast<const unsigned long long*>(sBt + (t + kk) * NMAX + 2 * pp)};
+                        if constexpr (Lo::kBC == 2)
+                            cq[0] = bf16pair(reinterpret_cast<const uint32_t*>(sCt)[((t + kk) * (NMAX / 4) + q) * 2 + hw]);
+                        else
+                            cq[0] = f2{*reinterpret_cast<const unsigned long long*>(sCt + (t + kk) * NMAX + 2 * pp)};
+                    }
+                    return;
+                }
 #pragma unroll
                 for (int j = 0; j < NS / 4; ++j) {
                     if constexpr (Lo::kBC == 1) {
@@ -699,7 +754,7 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
                 f2 ddn[4];
                 if constexpr (kPipe) {
                     if (t + 4 < T) {
-                        const float4 dn = *reinterpret_cast<const float4*>(sDel + cwk[0] * RS + t + 4);
+                        const float4 dn = *reinterpret_cast<const float4*>(sDelK + cwk[0] * RS + t + 4);
                         ddn[0] = pack2(dn.x, dn.x), ddn[1] = pack2(dn.y, dn.y);
                         ddn[2] = pack2(dn.z, dn.z), ddn[3] = pack2(dn.w, dn.w);
                     }
@@ -749,6 +804,11 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
                     if constexpr (P == 1) {
                         *reinterpret_cast<float4*>(sY + cwk[k] * RS + t) =
                             make_float4(yp[k][0], yp[k][1], yp[k][2], yp[k][3]);
+                    } else if constexpr (P == 8) {
+                        // eight steps per transpose-reduce: this group's and the previous one's
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) yp8[k][(t & 4) + q] = yp[k][q];
+                        if (t & 4) sY[cwk[k] * RS + (t - 4) + pp] = transpose_reduce<P>(yp8[k], pp);
                     } else {
 #pragma unroll
                         for (int g = 0; g < 4; g += P)
@@ -1031,9 +1091,10 @@ bool tma_rows(const ScanArgs& a) {
 // One launch of the scan kernel over (channel tiles, batch, segments); `nz` segments
 // (the grid's z extent).  TMA launches build their tensor maps from the kernel's layout.
 template <int NMAX, int P, int WARPS, int T, typename Tin, typename Tout, int MODE, bool TMA,
-          bool ZOH = false, bool WS = false, int CPL = 1>
+          bool ZOH = false, int WS = 0, int CPL = 1>
 cudaError_t launch_one(const ScanArgs& a, KParams kp, int64_t nz, cudaStream_t s) {
-    using Lo = Layout<NMAX, P, WARPS, T, Tin, Tout, CPL>;
+    using Lo = Layout<NMAX, P, WARPS, T, Tin, Tout, CPL, WS == 2 ? 2 : 1>;
+    constexpr int kProd = WS == 0 ? 0 : (WS == 1 ? 1 : S6_WSP);
     constexpr bool kOut = MODE == kFull || MODE == kFullCkpt || MODE == kFullAgg || MODE == kCorr;
     TMaps tm;
     memset(&tm, 0, sizeof(tm));
@@ -1048,7 +1109,7 @@ cudaError_t launch_one(const ScanArgs& a, KParams kp, int64_t nz, cudaStream_t s
                                          (int)Lo::bytes);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((a.dim + Lo::CH - 1) / Lo::CH), (unsigned)a.batch, (unsigned)nz);
-    kern<<<grid, Lo::THREADS + (WS ? 32 : 0), Lo::bytes, s>>>(kp, tm);
+    kern<<<grid, Lo::THREADS + 32 * kProd, Lo::bytes, s>>>(kp, tm);
     return cudaGetLastError();
 }
 
@@ -1108,9 +1169,9 @@ cudaError_t launch_typed(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
         // the split's rescan keeps the tile its segment plan was made for
         if (a.nseg == 1)
             return launch_one<NMAX, TF::P, TF::WARPS, TF::T, Tin, Tout, kFull, TMA, false,
-                              TMA && S6_WS, TF::CPL>(a, kp, 1, s);
+                              TMA ? S6_WS : 0, TF::CPL>(a, kp, 1, s);
     }
-    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA, ZOH, TMA && S6_WS && !ZOH>(
+    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA, ZOH, (TMA && !ZOH) ? S6_WS : 0>(
         a, kp, a.nseg, s);
 }
 

@@ -124,16 +124,34 @@ __global__ void __launch_bounds__(256) state_update_kernel(const UParams p) {
 // N = 16 fast path.  Two threads per (batch, channel) lane, each owning eight states:
 // thread h holds states 4h..4h+3 and 8+4h..8+4h+3, so for every 16-byte access the two
 // threads of a lane cover one whole 32-byte sector and a warp moves 16 contiguous lanes
-// (1 KiB of state) per instruction pair.  Each thread serves kItems lanes, one grid
-// stride apart, and issues every load of all of them before any arithmetic, keeping
-// 64 bytes of state per thread in flight.  Math runs on packed fp32 pairs.
+// (1 KiB of state) per instruction pair.  The default (persistent) kernel keeps one wave of
+// CTAs resident; each thread walks its lanes a grid stride apart with the next lane's loads
+// issued before the current lane's arithmetic, and one thread per CTA bulk-prefetches into
+// L2 the state block the CTA reaches two strides later.  The other form serves kItems lanes
+// per thread and issues every load of all of them before any arithmetic.  Math runs on
+// packed fp32 pairs.
 #ifndef S6_DEC_ITEMS
 #define S6_DEC_ITEMS 2
 #endif
-// Nonzero: the persistent variant with that many CTAs per SM.
+// Nonzero: the persistent variant with up to that many CTAs per SM (fewer when the
+// instantiation's registers allow fewer); 0: one lane pair per S6_DEC_ITEMS, one wave after
+// another.  Measured on the decode workload (256 x 5120 x 16, bf16, L2 flushed before the
+// token): 35.6 us with two items per thread, 35.0 us persistent without prefetch, 33.5 us
+// persistent with the prefetch two rounds ahead.
 #ifndef S6_DEC_PERSIST
-#define S6_DEC_PERSIST 0
+#define S6_DEC_PERSIST 3
 #endif
+// Persistent variant: one thread per CTA prefetches into L2 the state (and u, delta, z)
+// of the lanes this CTA takes S6_DEC_PREFETCH grid strides ahead (0 = no prefetch), so
+// the HBM reads of later rounds are in flight while this round computes.
+#ifndef S6_DEC_PREFETCH
+#define S6_DEC_PREFETCH 2
+#endif
+
+// Bulk prefetch of `bytes` (a multiple of 16, from a 16-byte aligned address) into L2.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 constexpr int kItems = S6_DEC_ITEMS;
 
 template <typename Tio>
@@ -187,7 +205,34 @@ __global__ void __launch_bounds__(256) state_update16p_kernel(const UParams p) {
     bool act = li < lanes;
     Lane16<Tio> cur, nxt;
     load_lane16<Tio>(p, act ? li : 0, act, h, cur);
+#if S6_DEC_PREFETCH
+    // this CTA's lanes in a round: blockDim.x / 2 consecutive ones
+    const uint32_t cta_lanes = blockDim.x / 2;
+    const uint32_t cta_first = blockIdx.x * cta_lanes;
+    auto prefetch_round = [&](uint32_t round) {
+        const uint64_t first = (uint64_t)cta_first + (uint64_t)round * pairs;
+        if (threadIdx.x != 0 || first >= lanes) return;
+        const uint32_t n = (uint32_t)min((uint64_t)cta_lanes, (uint64_t)lanes - first);
+        prefetch_l2(p.state + first * 16, n * 64u);
+        const size_t esz = sizeof(Tio);
+        // u, delta, z of these lanes: the whole 16-byte chunks inside [first, first + n)
+        // rounded outwards, but never past the last whole chunk of the buffers
+        const uint64_t end = (uint64_t)lanes * esz / 16 * 16;
+        const uint64_t b0 = first * esz / 16 * 16;
+        const uint64_t b1 = min(((first + n) * esz + 15) / 16 * 16, end);
+        if (b1 <= b0) return;
+        prefetch_l2(static_cast<const char*>(p.u) + b0, (uint32_t)(b1 - b0));
+        prefetch_l2(static_cast<const char*>(p.delta) + b0, (uint32_t)(b1 - b0));
+        if (p.z) prefetch_l2(static_cast<const char*>(p.z) + b0, (uint32_t)(b1 - b0));
+    };
+#pragma unroll
+    for (uint32_t r = 1; r <= S6_DEC_PREFETCH; ++r) prefetch_round(r);
+    uint32_t round = 0;
+#endif
     while (__any_sync(0xffffffffu, act)) {
+#if S6_DEC_PREFETCH
+        prefetch_round(++round + S6_DEC_PREFETCH);
+#endif
         const uint32_t nl = li + pairs;
         const bool nact = nl < lanes;
         load_lane16<Tio>(p, nact ? nl : 0, nact, h, nxt);
@@ -279,12 +324,17 @@ template <typename Tio, bool ZOH>
 cudaError_t launch_u_typed(const UParams& p, cudaStream_t s) {
     if (p.N == 16 && p.lanes < (1LL << 29)) {
 #if S6_DEC_PERSIST
-        // a whole number of waves: S6_DEC_PERSIST CTAs of 256 threads per SM
-        int dev = 0, sms = 148;
-        if (cudaGetDevice(&dev) == cudaSuccess)
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        // one wave: up to S6_DEC_PERSIST resident CTAs of 256 threads on every SM
+        int dev = 0, sms = 0, occ = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, state_update16p_kernel<Tio, ZOH>,
+                                                              256, 0);
+        if (e != cudaSuccess) return e;
+        const int64_t per_sm = std::max(1, std::min(occ, S6_DEC_PERSIST));
         const int64_t need = (2 * p.lanes + 255) / 256;
-        const int64_t blocks = std::min<int64_t>(need, (int64_t)sms * S6_DEC_PERSIST);
+        const int64_t blocks = std::min<int64_t>(need, (int64_t)sms * per_sm);
         state_update16p_kernel<Tio, ZOH><<<(unsigned)blocks, 256, 0, s>>>(p);
 #else
         const int64_t threads = 2 * ((p.lanes + kItems - 1) / kItems);
