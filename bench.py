@@ -302,7 +302,8 @@ def run_ours(args, rank, world, local):
     roofline = {
         "bound": "alu", "unit": "Gexp/s",
         "achieved": achieved / 1e9, "peak": sfu_peak / 1e9, "frac": achieved / sfu_peak,
-        "traffic": profile_traffic("scan_fwd_m2p8b.txt", "selective_state_space_56_b200/csrc/scan_fwd.cu"),
+        "traffic": profile_traffic("scan_fwd_m2p8b.txt", "selective_state_space_56_b200/csrc/scan_fwd.cu+"
+                                  "selective_state_space_56_b200/csrc/s6_device.cuh"),
         "algorithmic_bytes": byts,
         "hbm_GBps": byts / (ms_kernel * 1e-3) / 1e9,
         "hbm_frac": byts / (ms_kernel * 1e-3) / 1e9 / peaks["hbm_gbs"],

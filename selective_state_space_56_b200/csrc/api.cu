@@ -118,7 +118,8 @@ int mamba_selective_scan_summary(const void* u, const void* delta, const float* 
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return MAMBA_ERR_ALIGN;
     int64_t nseg = 1, seg_len = 0;
-    s6::plan_segments(dims.batch, dims.dim, dims.dstate, dims.seqlen, &nseg, &seg_len);
+    s6::plan_segments(dims.batch, dims.dim, dims.dstate, dims.seqlen, &nseg, &seg_len,
+                      in_dtype == MAMBA_F32);
     if (nseg > kMaxGridYZ) return MAMBA_ERR_DIMS;
     const size_t need = mamba_selective_scan_workspace_size(dims);
     if (need > 0) {
@@ -194,7 +195,8 @@ int scan_fwd(const void* u, const void* delta, const float* A, const void* B, co
         return MAMBA_ERR_WORKSPACE;
 
     int64_t nseg = 1, seg_len = 0;
-    s6::plan_segments(dims.batch, dims.dim, dims.dstate, dims.seqlen, &nseg, &seg_len);
+    s6::plan_segments(dims.batch, dims.dim, dims.dstate, dims.seqlen, &nseg, &seg_len,
+                      in_dtype == MAMBA_F32);
     if (nseg > kMaxGridYZ) return MAMBA_ERR_DIMS;
     const size_t need = mamba_selective_scan_workspace_size(dims);
     if (need > 0) {

@@ -53,9 +53,10 @@ struct StateUpdateArgs {
 // chunk length a scan kernel stages at once).
 constexpr int kChunk = 128;
 
-// Split plan for a problem: number of segments and their length (a multiple of kChunk).
+// Split plan for a problem: number of segments and their length (a multiple of kChunk),
+// no more segments than one wave of the current device's CTAs holds for the input type.
 void plan_segments(int64_t batch, int64_t dim, int64_t dstate, int64_t L, int64_t* nseg,
-                   int64_t* seg_len);
+                   int64_t* seg_len, bool fp32_in);
 // Most segments plan_segments can return for these sizes (what the workspace is sized for).
 int64_t split_segments_bound(int64_t batch, int64_t dim, int64_t L);
 

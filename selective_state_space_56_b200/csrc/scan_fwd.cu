@@ -130,12 +130,16 @@ enum Mode : int { kFull = 0, kAggregate = 1, kCheckpoint = 2, kFullCkpt = 3, kFu
 // TMA path, producer warps: 0 = none (one CTA barrier per chunk); 1 = one producer warp
 // stages every chunk and converts its coefficients; 2 = S6_WSP producer warps also form
 // Delta and Delta u for every channel into a double-buffered ring.  With 1 or 2 the
-// compute warps wait only on mbarriers and never for one another.
-#ifndef S6_WS
-#define S6_WS 0
-#endif
+// compute warps wait only on mbarriers and never for one another.  S6_WS forces a form
+// for every plain forward; by default the plan picks form 2 for a grid of one wave at
+// 2.5 to 3 CTAs per SM and form 0 otherwise (measured on one B200: the 2.8B-shaped layer,
+// 428 CTAs, 609.8 -> 584.2 us with form 2; at batch 12, 1284 CTAs, 1602 -> 1640 us).
 #ifndef S6_WSP
-#define S6_WSP 1
+#define S6_WSP 2
+#endif
+// The exact-ZOH forward with the same plan-based producer form.
+#ifndef S6_ZOH_WS
+#define S6_ZOH_WS 0
 #endif
 #ifndef S6_POLY
 #define S6_POLY 0
@@ -251,6 +255,7 @@ template <int NMAX, int P, int WARPS, int T_, typename Tin, typename Tout, int M
 __global__ void __launch_bounds__(WARPS * 32 + 32 * (WS == 0 ? 0 : (WS == 1 ? 1 : S6_WSP)))
 scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
     static_assert(!WS || (TMA && MODE == kFull), "producer warp: TMA full scans only");
+    static_assert(!(WS && ZOH) || WS == 2, "exact ZOH with producers: form 2 only");
     constexpr int NPROD = WS == 0 ? 0 : (WS == 1 ? 1 : S6_WSP);  // producer warps
     static_assert(CPL == 1 || (MODE == kFull && !ZOH && !WS), "two channels per lane: plain scan");
     constexpr bool kOut = MODE == kFull || MODE == kFullCkpt || MODE == kFullAgg ||
@@ -1081,6 +1086,15 @@ bool make_maps(const ScanArgs& a, bool want_z, bool want_y, TMaps* tm) {
     return ok;
 }
 
+// Multiprocessors of the current device (148 on a B200 if the query fails).
+int64_t sm_count() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        return 148;
+    return sms;
+}
+
 // Rows that TMA can describe: a 16-byte multiple of elements, coordinates in int32.
 template <typename T>
 bool tma_rows(const ScanArgs& a) {
@@ -1167,11 +1181,42 @@ cudaError_t launch_typed(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
             return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFullCkpt, TMA, false>(
                 a, kp, a.nseg, s);
         // the split's rescan keeps the tile its segment plan was made for
-        if (a.nseg == 1)
+        if (a.nseg == 1) {
+#ifdef S6_WS
             return launch_one<NMAX, TF::P, TF::WARPS, TF::T, Tin, Tout, kFull, TMA, false,
                               TMA ? S6_WS : 0, TF::CPL>(a, kp, 1, s);
+#else
+            if constexpr (TMA && TF::CPL == 1) {
+                using LoF = Layout<NMAX, TF::P, TF::WARPS, TF::T, Tin, Tout, 1>;
+                const int64_t ctas = (a.dim + LoF::CH - 1) / LoF::CH * a.batch;
+                const int64_t sms = sm_count();
+                if (2 * ctas >= 5 * sms && ctas <= 3 * sms)
+                    return launch_one<NMAX, TF::P, TF::WARPS, TF::T, Tin, Tout, kFull, TMA, false,
+                                      2>(a, kp, 1, s);
+            }
+            return launch_one<NMAX, TF::P, TF::WARPS, TF::T, Tin, Tout, kFull, TMA, false, 0,
+                              TF::CPL>(a, kp, 1, s);
+#endif
+        }
     }
-    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA, ZOH, (TMA && !ZOH) ? S6_WS : 0>(
+#ifdef S6_WS
+    constexpr int kWsSplit = (TMA && !ZOH) ? S6_WS : 0;
+#else
+    constexpr int kWsSplit = 0;
+#endif
+#if S6_ZOH_WS
+    // the exact-ZOH forward in one pass: the same plan as the Delta*B forward
+    if constexpr (ZOH && TMA) {
+        if (a.nseg == 1) {
+            using LoZ = Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, 1>;
+            const int64_t ctas = (a.dim + LoZ::CH - 1) / LoZ::CH * a.batch;
+            const int64_t sms = sm_count();
+            if (2 * ctas >= 5 * sms && ctas <= 3 * sms)
+                return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA, ZOH, 2>(a, kp, 1, s);
+        }
+    }
+#endif
+    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA, ZOH, kWsSplit>(
         a, kp, a.nseg, s);
 }
 
@@ -1314,16 +1359,17 @@ cudaError_t read_device_error(unsigned* out, bool clear, cudaStream_t stream) {
 
 namespace {
 
-// CTAs of the N-state tile resident at once on a B200 (148 SMs; residency from the tile's
-// shared memory and threads with bf16 inputs): one wave.
-template <int NMAX>
-constexpr int64_t wave_ctas() {
+// CTAs of the N-state tile (input and output of type Tio) resident at once on the current
+// device: its SM count times the CTAs an SM holds by the tile's shared memory (228 KB per
+// SM, 1 KB reserved per CTA) and threads.  One wave.
+template <int NMAX, typename Tio>
+int64_t wave_ctas() {
     using TL = Tile<NMAX>;
-    using Lo = Layout<NMAX, TL::P, TL::WARPS, TL::T, __nv_bfloat16, __nv_bfloat16>;
+    using Lo = Layout<NMAX, TL::P, TL::WARPS, TL::T, Tio, Tio>;
     constexpr int64_t by_smem = 233472 / ((int64_t)Lo::bytes + 1024);
     constexpr int64_t by_threads = 2048 / Lo::THREADS;
     constexpr int64_t r = by_smem < by_threads ? by_smem : by_threads;
-    return 148 * (r < 32 ? r : 32);
+    return sm_count() * (r < 32 ? r : 32);
 }
 
 template <int NMAX>
@@ -1364,7 +1410,7 @@ int64_t split_segments_bound(int64_t batch, int64_t dim, int64_t L) {
 }
 
 void plan_segments(int64_t batch, int64_t dim, int64_t dstate, int64_t L, int64_t* nseg,
-                   int64_t* seg_len) {
+                   int64_t* seg_len, bool fp32_in) {
     // Each CTA of a split sweeps a whole segment, so a second, partial wave of CTAs costs a
     // whole segment's time again, while the split's extra pass costs about the same for
     // any number of segments: take no more segments than one wave of CTAs holds (and
@@ -1373,8 +1419,13 @@ void plan_segments(int64_t batch, int64_t dim, int64_t dstate, int64_t L, int64_
     if (n > 1) {
         const int64_t ch = dstate <= 4 ? tile_channels<4>() : dstate <= 8 ? tile_channels<8>()
                                                                            : tile_channels<16>();
-        const int64_t wave = dstate <= 4 ? wave_ctas<4>() : dstate <= 8 ? wave_ctas<8>()
-                                                                         : wave_ctas<16>();
+        int64_t wave;
+        if (fp32_in)
+            wave = dstate <= 4 ? wave_ctas<4, float>() : dstate <= 8 ? wave_ctas<8, float>()
+                                                                     : wave_ctas<16, float>();
+        else
+            wave = dstate <= 4 ? wave_ctas<4, __nv_bfloat16>()
+                   : dstate <= 8 ? wave_ctas<8, __nv_bfloat16>() : wave_ctas<16, __nv_bfloat16>();
         const int64_t per_seg = (dim + ch - 1) / ch * batch;
         n = std::max<int64_t>(1, std::min<int64_t>(n, wave / per_seg));
     }

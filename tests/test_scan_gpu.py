@@ -83,6 +83,18 @@ def test_m2p8b_workload_full(cuda_ok):
     assert stats["n"] == w.batch * w.dim * w.seqlen
 
 
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_single_wave_grid_with_producer_warps(cuda_ok, out_dtype):
+    """A grid of one wave at about three CTAs per SM takes the form in which producer warps
+    stage the chunks and form Delta and Delta u: here with a ragged channel tile (5000 =
+    104 x 48 + 8) and a ragged last chunk (1000 = 31 x 32 + 8), every output checked."""
+    b, d, n, L = 4, 5000, 16, 1000
+    p = inputs.scan_inputs(b, d, n, L, in_dtype=torch.bfloat16, seed=4242)
+    y, st = _gpu_scan(p, out_dtype=out_dtype)
+    y_ref, st_ref = _oracle_scan(p)
+    _check(y, st, y_ref, st_ref, torch.bfloat16, out_dtype)
+
+
 def test_m2p8b_fp32_output_literal_bound(cuda_ok):
     """The same layer with fp32 y: the literal max|y - y_ref| <= 2e-2 RMS bound on every
     element."""
