@@ -12,7 +12,8 @@
 //             then re-laid out per (4-step group, 4-state quad): fp32, or bf16 for bf16
 //             inputs (fewer shared-memory wavefronts for loads all 8 channels repeat);
 //   phase A   per (channel, t): Delta = softplus(delta + bias) and the gated output
-//             gradient dyt_t = dy_t silu(z_t);
+//             gradient dyt_t = dy_t silu(z_t) (16-step blocks also keep sigmoid(x) and
+//             sigmoid(z) for the gradients through softplus and the gate);
 //   forward   from the checkpoint, the chunk's states are recomputed; the state
 //             entering every group of 4 steps is kept in shared memory;
 //   reverse   per group of 4 steps, last group first: the group's states and Abar are
@@ -24,10 +25,12 @@
 //             dq, the state part of dDelta and C_t . h_t are summed over a channel's 4
 //             lanes once per group; C_t . h_t + D u_t gives dz_t = dy_t yt_t silu'(z_t).
 //             dB and dC, shared by all channels of a batch, are summed over the warp's
-//             8 channels every step (shuffles; for blocks of 16 steps) or every group
-//             (a per-warp exchange buffer, one lane per (step, quad), for longer
-//             blocks), added into the CTA's chunk accumulator (shared atomics), which is
-//             added to global memory once per (t, n) and CTA;
+//             8 channels through a per-warp exchange buffer every 2 steps (16-step
+//             blocks, bf16 inputs) or 4 steps (longer blocks), or with shuffles every
+//             step (16-step blocks, fp32 inputs); the sums land in the warp's own slice
+//             of the chunk accumulator (16-step blocks; the slices are added up once per
+//             chunk) or in one CTA-wide slice by shared atomics, and reach global memory
+//             once per (t, n) and CTA;
 //   store     du, dDelta_raw (= dDelta softplus'(x)), dz rows; dA, dD, dbias by atomics.
 //
 // State arithmetic runs on packed fp32 pairs (two states per instruction).  Gradients
@@ -73,11 +76,32 @@ struct BParams {
 #ifndef S6_BWD_WARPS
 #define S6_BWD_WARPS 4
 #endif
-// Steps per dB / dC exchange buffer.  16-step blocks sum each step's dB / dC over the
-// warp's 8 channels with shuffles (no buffer: the shared memory then holds five CTAs per
-// SM for either input type); longer blocks store them to a per-warp buffer and sum a
-// group of 4 steps at once (fewer instructions; measured faster there).
-template <int T> constexpr int exchange_steps() { return T == 16 ? 0 : 4; }
+// Steps per dB / dC exchange buffer: every channel stores its step's dB / dC to a per-warp
+// buffer, which the warp then sums over its 8 channels for that many steps at once.  16-step
+// blocks use 2 steps for bf16 inputs (measured 1.6% faster than summing each step with
+// shuffles, and five CTAs per SM still fit) and the shuffles (0) for fp32 inputs, whose
+// wider staging rows leave no room for the buffer at five CTAs per SM; longer blocks use 4.
+#ifndef S6_BWD_XS16
+#define S6_BWD_XS16 2
+#endif
+// dB / dC accumulators of a 16-step chunk: 1 = one [T][32] slice per warp, written with
+// plain stores and summed over the warps once per chunk (measured 3.5% faster on the
+// 2.8B-shaped layer); 0 = one slice per CTA that every warp adds into with shared-memory
+// atomics, which longer chunks keep (per-warp slices would cost them occupancy).
+#ifndef S6_BWD_WACC
+#define S6_BWD_WACC 1
+#endif
+template <int T> constexpr bool warp_acc() { return S6_BWD_WACC && T == 16; }
+// Phase A keeps softplus'(x) = sigmoid(x) and sigmoid(z) of every step in shared memory for
+// the gradient epilogue, which then does not evaluate them a second time (16-step blocks;
+// measured 1.9% faster there; longer blocks would lose occupancy to the two rows).
+#ifndef S6_BWD_SIG
+#define S6_BWD_SIG 1
+#endif
+template <int T> constexpr bool keep_sig() { return S6_BWD_SIG && T == 16; }
+template <int T, typename Tin> constexpr int exchange_steps() {
+    return T == 16 ? (sizeof(Tin) == 2 ? S6_BWD_XS16 : 0) : 4;
+}
 
 constexpr int kBW = S6_BWD_WARPS;  // warps per CTA
 constexpr int kBP = 4;             // lanes per channel, 4 states each
@@ -103,9 +127,12 @@ struct BLayout {
     static constexpr size_t off_dyt = off_del + f;               // dy * silu(z)
     static constexpr size_t off_h = off_dyt + f;                 // fp32 [T/4][CH][16]
     static constexpr size_t off_acc = off_h + (size_t)(T / 4) * kBCH * 16 * 4;  // fp32 [T][32]
-    static constexpr int XS = exchange_steps<T>();
-    static constexpr size_t off_red = off_acc + (size_t)T * 32 * 4;  // per warp fp32 [XS][8][32]
-    static constexpr size_t bytes = off_red + (size_t)kBW * XS * 8 * 32 * 4;
+    static constexpr int XS = exchange_steps<T, Tin>();
+    static constexpr size_t off_red =
+        off_acc + (size_t)(warp_acc<T>() ? kBW : 1) * T * 32 * 4;  // per warp fp32 [XS][8][32]
+    static constexpr size_t off_sg = off_red + (size_t)kBW * XS * 8 * 32 * 4;  // sigmoid(x) [CH][RS]
+    static constexpr size_t off_sz = off_sg + (keep_sig<T>() ? f : 0);          // sigmoid(z) [CH][RS]
+    static constexpr size_t bytes = off_sz + (keep_sig<T>() ? f : 0);
     static_assert(T % 8 == 0, "chunk length");
     static_assert((RR * sizeof(Tin)) % 16 == 0, "raw rows must stay 16-byte aligned");
 };
@@ -250,6 +277,8 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
     float* sDyt = reinterpret_cast<float*>(smem + Lo::off_dyt);
     float* sH = reinterpret_cast<float*>(smem + Lo::off_h);
     float* sAcc = reinterpret_cast<float*>(smem + Lo::off_acc);
+    float* sSg = reinterpret_cast<float*>(smem + Lo::off_sg);
+    float* sSz = reinterpret_cast<float*>(smem + Lo::off_sz);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int pp = lane & 3, cl = lane >> 2;
@@ -301,7 +330,8 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
                 sC[t * 16 + n] = io<Tin>::to_f(rC[n * RR + t]);
             }
         }
-        for (int i = tid; i < T * 32; i += kBW * 32) sAcc[i] = 0.f;
+        if constexpr (!warp_acc<T>())
+            for (int i = tid; i < T * 32; i += kBW * 32) sAcc[i] = 0.f;
 
         // phase A, per (channel, t) of this warp: Delta (zero on padded steps: Abar = 1, no
         // input) and the gated output gradient dyt = dy silu(z)
@@ -310,10 +340,25 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
             const int64_t d = d0 + c;
             const float bi = (d < p.dim && p.delta_bias) ? p.delta_bias[d] : 0.f;
             const float x = io<Tin>::to_f(rDr[c * RR + t]) + bi;
-            const float dt = p.softplus ? softplus(x) : x;
-            sDel[c * RS + t] = t < valid ? dt : 0.f;
             const float dyv = io<Tin>::to_f(rDy[c * RR + t]);
-            sDyt[c * RS + t] = has_z ? dyv * silu(io<Tin>::to_f(rZ[c * RR + t])) : dyv;
+            if constexpr (keep_sig<T>()) {
+                float dt = x, sg = 1.f;
+                if (p.softplus) softplus_sigmoid(x, dt, sg);
+                sDel[c * RS + t] = t < valid ? dt : 0.f;
+                sSg[c * RS + t] = sg;
+                if (has_z) {
+                    const float zz = io<Tin>::to_f(rZ[c * RR + t]);
+                    const float sz = rcp(1.f + ex2(-zz * kLog2e));
+                    sSz[c * RS + t] = sz;
+                    sDyt[c * RS + t] = dyv * (zz * sz);
+                } else {
+                    sDyt[c * RS + t] = dyv;
+                }
+            } else {
+                const float dt = p.softplus ? softplus(x) : x;
+                sDel[c * RS + t] = t < valid ? dt : 0.f;
+                sDyt[c * RS + t] = has_z ? dyv * silu(io<Tin>::to_f(rZ[c * RR + t])) : dyv;
+            }
         }
         __syncthreads();  // B, C converted, sAcc cleared
 
@@ -432,9 +477,12 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
                                      __shfl_xor_sync(0xffffffffu, b2 ? r2[0] : r2[1], 4);
                     const int idx = (lane >> 2) & 7;  // = 4 b4 + 2 b3 + b2
                     const int slot = (idx & 4) * 4 + pp * 4 + (idx & 3);
-                    atomicAdd(&sAcc[acc_idx(tg + s, slot)], r3);
+                    if constexpr (warp_acc<T>())
+                        sAcc[warp * T * 32 + acc_idx(tg + s, slot)] = r3;
+                    else
+                        atomicAdd(&sAcc[acc_idx(tg + s, slot)], r3);
                 } else {  // this channel's dB / dC of step t into the warp's exchange rows
-                    float* row = sRed + s * 256 + cl * 32;
+                    float* row = sRed + (s % (XS > 0 ? XS : 1)) * 256 + cl * 32;
                     float x0, x1, x2, x3;
                     unpack2(dB0, x0, x1);
                     unpack2(dB1, x2, x3);
@@ -442,6 +490,28 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
                     unpack2(dC0, x0, x1);
                     unpack2(dC1, x2, x3);
                     *reinterpret_cast<float4*>(row + red_quad(4 + pp, cl) * 4) = make_float4(x0, x1, x2, x3);
+                }
+                if (XS == 2 && s % 2 == 0) {
+                    // steps tg + s and tg + s + 1 are complete: lane (xs, xh) sums half xh & 1
+                    // of quad xh >> 1 of step tg + s + xs over the warp's 8 channels
+                    __syncwarp();
+                    const int xs = lane >> 4, xh = lane & 15, xq = xh >> 1, half = (xh & 1) * 2;
+                    f2 a = *reinterpret_cast<const f2*>(sRed + xs * 256 + red_quad(xq, 0) * 4 + half);
+#pragma unroll
+                    for (int ch = 1; ch < 8; ++ch)
+                        a = add2(a, *reinterpret_cast<const f2*>(sRed + xs * 256 + ch * 32 +
+                                                                 red_quad(xq, ch) * 4 + half));
+                    float v0, v1;
+                    unpack2(a, v0, v1);
+                    const int tt = tg + s + xs, slot = xq * 4 + half;
+                    if constexpr (warp_acc<T>()) {
+                        *reinterpret_cast<float2*>(sAcc + (warp * T + tt) * 32 + slot) =
+                            make_float2(v0, v1);
+                    } else {
+                        atomicAdd(&sAcc[acc_idx(tt, slot)], v0);
+                        atomicAdd(&sAcc[acc_idx(tt, slot + 1)], v1);
+                    }
+                    __syncwarp();
                 }
                 if (XS == 4 && s == 0) {
                     // the group is complete: lane (xs, xq) sums quad xq of step tg + xs over
@@ -460,10 +530,16 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
                     unpack2(a01, v0, v1);
                     unpack2(a23, v2, v3);
                     const int tt = tg + xs, slot = xq * 4;
-                    atomicAdd(&sAcc[acc_idx(tt, slot)], v0);
-                    atomicAdd(&sAcc[acc_idx(tt, slot + 1)], v1);
-                    atomicAdd(&sAcc[acc_idx(tt, slot + 2)], v2);
-                    atomicAdd(&sAcc[acc_idx(tt, slot + 3)], v3);
+                    if constexpr (warp_acc<T>()) {
+                        // unrotated rows: the 8 lanes of a step cover its 32 slots
+                        *reinterpret_cast<float4*>(sAcc + (warp * T + tt) * 32 + slot) =
+                            make_float4(v0, v1, v2, v3);
+                    } else {
+                        atomicAdd(&sAcc[acc_idx(tt, slot)], v0);
+                        atomicAdd(&sAcc[acc_idx(tt, slot + 1)], v1);
+                        atomicAdd(&sAcc[acc_idx(tt, slot + 2)], v2);
+                        atomicAdd(&sAcc[acc_idx(tt, slot + 3)], v3);
+                    }
                     __syncwarp();
                 }
             }
@@ -474,17 +550,20 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
             const float uu = io<Tin>::to_f(rU[cw * RR + t]);
             if (has_z) {  // dz = dy * (C . h + D u) * silu'(z), replacing z in its row
                 const float zz = io<Tin>::to_f(rZ[cw * RR + t]);
-                const float sz = rcp(1.f + ex2(-zz * kLog2e));
+                const float sz = keep_sig<T>() ? sSz[cw * RS + t] : rcp(1.f + ex2(-zz * kLog2e));
                 const float yt = fmaf(Dd, uu, cy);
                 rZ[cw * RR + t] = io<Tin>::from_f(io<Tin>::to_f(rDy[cw * RR + t]) * yt * sz *
                                                   (1.f + zz * (1.f - sz)));
             }
             const float dt = sDel[cw * RS + t], dyt = sDyt[cw * RS + t];
-            const float xr = io<Tin>::to_f(rDr[cw * RR + t]);
             float sg = 1.f;
             if (p.softplus) {
-                float sp;
-                softplus_sigmoid(xr + bias, sp, sg);
+                if constexpr (keep_sig<T>()) {
+                    sg = sSg[cw * RS + t];
+                } else {
+                    float sp;
+                    softplus_sigmoid(io<Tin>::to_f(rDr[cw * RR + t]) + bias, sp, sg);
+                }
             }
             const float ddelta = (ddl + dq * uu) * sg;
             rDy[cw * RR + t] = io<Tin>::from_f(fmaf(dyt, Dd, dq * dt));  // du replaces dy
@@ -521,7 +600,16 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
             const int t = i / 32, slot = i % 32, n = slot & 15;
             if (t >= valid || n >= p.N) continue;
             float* dst = slot < 16 ? p.dB : p.dC;
-            atomicAdd(dst + (b * p.N + n) * p.L + t0 + t, sAcc[acc_idx(t, slot)]);
+            float v;
+            if constexpr (warp_acc<T>()) {
+                const int idx = XS == 0 ? acc_idx(t, slot) : t * 32 + slot;
+                v = sAcc[idx];
+#pragma unroll
+                for (int w = 1; w < kBW; ++w) v += sAcc[w * T * 32 + idx];
+            } else {
+                v = sAcc[acc_idx(t, slot)];
+            }
+            atomicAdd(dst + (b * p.N + n) * p.L + t0 + t, v);
         }
     }
 

@@ -137,6 +137,12 @@ enum Mode : int { kFull = 0, kAggregate = 1, kCheckpoint = 2, kFullCkpt = 3, kFu
 #ifndef S6_WSP
 #define S6_WSP 2
 #endif
+// The checkpoint-recording forwards (the backward's own pass and the training forward)
+// with the same plan-based producer form: measured neutral on the 2.8B-shaped layer
+// (backward 3120 -> 3131 us, training step 3287 -> 3267 us), so off.
+#ifndef S6_WS_CKPT
+#define S6_WS_CKPT 0
+#endif
 // The exact-ZOH forward with the same plan-based producer form.
 #ifndef S6_ZOH_WS
 #define S6_ZOH_WS 0
@@ -254,7 +260,9 @@ template <int NMAX, int P, int WARPS, int T_, typename Tin, typename Tout, int M
           bool ZOH = false, int WS = 0, int CPL = 1>
 __global__ void __launch_bounds__(WARPS * 32 + 32 * (WS == 0 ? 0 : (WS == 1 ? 1 : S6_WSP)))
 scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
-    static_assert(!WS || (TMA && MODE == kFull), "producer warp: TMA full scans only");
+    // (modes without a CTA-wide barrier in the chunk loop: the producers do not join one)
+    static_assert(!WS || (TMA && (MODE == kFull || MODE == kCheckpoint || MODE == kFullCkpt)),
+                  "producer warps: TMA scans and checkpoint passes only");
     static_assert(!(WS && ZOH) || WS == 2, "exact ZOH with producers: form 2 only");
     constexpr int NPROD = WS == 0 ? 0 : (WS == 1 ? 1 : S6_WSP);  // producer warps
     static_assert(CPL == 1 || (MODE == kFull && !ZOH && !WS), "two channels per lane: plain scan");
@@ -1102,6 +1110,15 @@ bool tma_rows(const ScanArgs& a) {
     return fits && a.L > 0 && (a.L * (int64_t)sizeof(T)) % 16 == 0;
 }
 
+// The producer form pays off for a grid of one wave at 2.5 to 3 CTAs per SM (two producer
+// warps per CTA then fit beside the compute warps); elsewhere the plain form is faster.
+template <typename Lo>
+bool producer_plan(const ScanArgs& a, int64_t nz) {
+    const int64_t ctas = (a.dim + Lo::CH - 1) / Lo::CH * a.batch * nz;
+    const int64_t sms = sm_count();
+    return 2 * ctas >= 5 * sms && ctas <= 3 * sms;
+}
+
 // One launch of the scan kernel over (channel tiles, batch, segments); `nz` segments
 // (the grid's z extent).  TMA launches build their tensor maps from the kernel's layout.
 template <int NMAX, int P, int WARPS, int T, typename Tin, typename Tout, int MODE, bool TMA,
@@ -1177,9 +1194,15 @@ cudaError_t launch_typed(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
         if (e != cudaSuccess) return e;
     }
     if constexpr (!ZOH) {
-        if (a.ckpt)
+        if (a.ckpt) {
+            if constexpr (TMA && S6_WS_CKPT) {
+                if (producer_plan<Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout>>(a, a.nseg))
+                    return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFullCkpt, TMA,
+                                      false, 2>(a, kp, a.nseg, s);
+            }
             return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFullCkpt, TMA, false>(
                 a, kp, a.nseg, s);
+        }
         // the split's rescan keeps the tile its segment plan was made for
         if (a.nseg == 1) {
 #ifdef S6_WS
@@ -1187,10 +1210,7 @@ cudaError_t launch_typed(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
                               TMA ? S6_WS : 0, TF::CPL>(a, kp, 1, s);
 #else
             if constexpr (TMA && TF::CPL == 1) {
-                using LoF = Layout<NMAX, TF::P, TF::WARPS, TF::T, Tin, Tout, 1>;
-                const int64_t ctas = (a.dim + LoF::CH - 1) / LoF::CH * a.batch;
-                const int64_t sms = sm_count();
-                if (2 * ctas >= 5 * sms && ctas <= 3 * sms)
+                if (producer_plan<Layout<NMAX, TF::P, TF::WARPS, TF::T, Tin, Tout, 1>>(a, 1))
                     return launch_one<NMAX, TF::P, TF::WARPS, TF::T, Tin, Tout, kFull, TMA, false,
                                       2>(a, kp, 1, s);
             }
@@ -1207,13 +1227,8 @@ cudaError_t launch_typed(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
 #if S6_ZOH_WS
     // the exact-ZOH forward in one pass: the same plan as the Delta*B forward
     if constexpr (ZOH && TMA) {
-        if (a.nseg == 1) {
-            using LoZ = Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, 1>;
-            const int64_t ctas = (a.dim + LoZ::CH - 1) / LoZ::CH * a.batch;
-            const int64_t sms = sm_count();
-            if (2 * ctas >= 5 * sms && ctas <= 3 * sms)
-                return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA, ZOH, 2>(a, kp, 1, s);
-        }
+        if (a.nseg == 1 && producer_plan<Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, 1>>(a, 1))
+            return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA, ZOH, 2>(a, kp, 1, s);
     }
 #endif
     return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFull, TMA, ZOH, kWsSplit>(
@@ -1229,6 +1244,11 @@ cudaError_t launch_io(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
 template <int NMAX, typename Tin>
 cudaError_t launch_ckpt_io(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
     using TL = Tile<NMAX>;
+#if S6_WS_CKPT
+    if (tma_rows<Tin>(a) && producer_plan<Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin>>(a, 1))
+        return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kCheckpoint, true, false, 2>(
+            a, kp, 1, s);
+#endif
     return tma_rows<Tin>(a)
                ? launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kCheckpoint, true>(a, kp, 1, s)
                : launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kCheckpoint, false>(a, kp, 1, s);
