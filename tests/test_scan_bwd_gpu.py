@@ -145,24 +145,11 @@ def test_m130m_layer_backward_full(cuda_ok):
     _compare(_gpu_bwd(p, dy), _oracle_bwd(p, dy), p, w.in_dtype)
 
 
-def test_m2p8b_layer_backward_sampled_channels(cuda_ok):
-    """The 2.8B-shaped layer (4, 5120, 16, 4096) in bf16 at full size; the per-channel
-    gradients (du, ddelta, dz, dA, dD, ddelta_bias) of 48 sampled channels, every batch and
-    step, against the oracle run on those channels alone."""
+def test_m2p8b_layer_backward_full(cuda_ok):
+    """The 2.8B-shaped layer (4, 5120, 16, 4096) in bf16 at full size: every gradient of
+    every channel, batch and step against the oracle (about 25 s of single-thread fp64);
+    dB and dC are sums over all 5120 channels of a batch, built by the kernel across 160
+    CTAs with atomics."""
     w = inputs.SCAN_WORKLOADS["m2p8b"]
     p, dy = _grad_inputs(w.batch, w.dim, w.dstate, w.seqlen, w.in_dtype, w.seed)
-    g = _gpu_bwd(p, dy)
-    rng = np.random.default_rng(2812)
-    ch = np.sort(np.concatenate([[0, w.dim - 1], rng.choice(w.dim - 2, 46, replace=False) + 1]))
-    sub = dict(p)
-    for k in ("u", "delta", "z"):
-        sub[k] = p[k][:, ch]
-    for k in ("A",):
-        sub[k] = p[k][ch]
-    for k in ("D", "delta_bias"):
-        sub[k] = p[k][ch]
-    ref = _oracle_bwd(sub, dy[:, ch])
-    for gname, oname in (("du", "du"), ("ddelta", "ddelta"), ("dz", "dz")):
-        check_bf16_out(g[gname][:, ch], ref[oname], gname)
-    for gname, oname in (("dA", "dA"), ("dD", "dD"), ("ddelta_bias", "dbias")):
-        check_scaled(g[gname][ch], ref[oname], gname, 1e-3)
+    _compare(_gpu_bwd(p, dy), _oracle_bwd(p, dy), p, w.in_dtype)
