@@ -25,7 +25,8 @@ Abar in (0,1), small/large-Delta limits, the gated-RNN special case.  The ZOH
 variant (tests/test_oracle_zoh.py): the gated-RNN identity, the continuous-time
 steady state -B u / A, numerical integration of the continuous ODE, the
 small-Delta limit and A = 0.  The causal conv1d (tests/test_oracle_conv.py): numpy's
-convolution, the impulse response, causality, chunked prefill and decode steps.
+convolution, the impulse response, causality, chunked prefill and decode steps; its
+backward: central finite differences of the forward, the linear case in closed form.
 """
 from __future__ import annotations
 
@@ -85,6 +86,9 @@ def _load():
             lib.s6o_causal_conv1d_update.restype = ctypes.c_int
             lib.s6o_causal_conv1d_update.argtypes = [ctypes.c_long] * 2 + [_dp] * 4 + [
                 ctypes.c_int, _dp]
+            lib.s6o_causal_conv1d_backward.restype = ctypes.c_int
+            lib.s6o_causal_conv1d_backward.argtypes = [ctypes.c_long] * 3 + [_dp] * 4 + [
+                ctypes.c_int] + [_dp] * 5
             lib.s6o_num_threads.restype = ctypes.c_int
             lib.s6o_num_threads.argtypes = []
             lib.s6o_set_num_threads.restype = ctypes.c_int
@@ -345,3 +349,30 @@ def causal_conv1d_update(state, x, weight, bias=None, silu=True):
     if rc != 0:
         raise ValueError("s6o_causal_conv1d_update rejected its arguments")
     return st.reshape(b, d, K - 1), out.reshape(b, d)
+
+
+def causal_conv1d_backward(x, weight, dout, bias=None, initial_state=None, silu=True):
+    """Gradients of sum(out * dout) for ``causal_conv1d`` (same layouts).  Returns a dict:
+    dx (batch, dim, L), dweight (dim, K), dbias (dim), dinitial_state (batch, dim, K-1) or
+    None when no initial state was given."""
+    xx = _f64(x)
+    b, d, L = xx.shape
+    w = _f64(weight)
+    K = w.shape[1]
+    rows = b * d
+    wr = np.ascontiguousarray(np.tile(w, (b, 1)))
+    br = None if bias is None else np.ascontiguousarray(np.tile(_f64(bias), b))
+    init = None if initial_state is None else _f64(initial_state).reshape(rows, K - 1)
+    dx = np.empty((rows, L))
+    dw = np.empty((rows, K))
+    db = np.empty(rows)
+    dinit = None if init is None else np.zeros((rows, max(K - 1, 0)))
+    rc = _load().s6o_causal_conv1d_backward(
+        rows, L, K, _ptr(np.ascontiguousarray(xx.reshape(rows, L))), _ptr(wr), _ptr(br),
+        _ptr(init), int(bool(silu)), _ptr(np.ascontiguousarray(_f64(dout).reshape(rows, L))),
+        _ptr(dx), _ptr(dw), _ptr(db), _ptr(dinit) if (dinit is not None and K > 1) else None)
+    if rc != 0:
+        raise ValueError("s6o_causal_conv1d_backward rejected its arguments")
+    return dict(dx=dx.reshape(b, d, L), dweight=dw.reshape(b, d, K).sum(0),
+                dbias=db.reshape(b, d).sum(0),
+                dinitial_state=None if dinit is None else dinit.reshape(b, d, K - 1))

@@ -361,6 +361,80 @@ int s6o_causal_conv1d_update(long nrows, long K, double* state, const double* x,
     return S6O_OK;
 }
 
+/*
+ * Gradients of sum_t out[t] * dout[t] for the convolution above (the chain rule of its
+ * definition; the block trains end to end through it).  With pre[t] the value before
+ * the activation and g[t] = dout[t] * act'(pre[t]) (act' = 1 without SiLU, else
+ * sigmoid(p) * (1 + p * (1 - sigmoid(p)))):
+ *   dx[s]    = sum_k w[k] * g[s + (K-1) - k]        over the t = s + (K-1) - k in [0, L)
+ *   dw[k]    = sum_t g[t] * xe[t - (K-1) + k]       (xe = init ++ x, zero before init)
+ *   dbias    = sum_t g[t]
+ *   dinit[j] = dx at position j - (K-1) of xe, for the K-1 inputs before the sequence
+ *              (written only when init and dinit are given)
+ * Per row i: dx (nrows, L), dw (nrows, K), dbias (nrows).  dbias may be NULL.
+ */
+int s6o_causal_conv1d_backward(long nrows, long L, long K, const double* x, const double* w,
+                               const double* bias, const double* init, int silu_on,
+                               const double* dout, double* dx, double* dw, double* dbias,
+                               double* dinit) {
+    if (nrows < 0 || L < 0 || K < 1 || K > 64 || !w || !dw || (L > 0 && (!x || !dout || !dx)))
+        return S6O_ERR_ARG;
+    double* g = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    if (!g) return S6O_ERR_ARG;
+    for (long i = 0; i < nrows; ++i) {
+        const double* xi = x ? x + i * L : NULL;
+        const double* wi = w + i * K;
+        double sb = 0.0;
+        for (long t = 0; t < L; ++t) {
+            double pre = bias ? bias[i] : 0.0;
+            for (long k = 0; k < K; ++k) {
+                long s = t - (K - 1) + k;
+                double v;
+                if (s >= 0)
+                    v = xi[s];
+                else
+                    v = init ? init[i * (K - 1) + (K - 1) + s] : 0.0;
+                pre += wi[k] * v;
+            }
+            double d = 1.0;
+            if (silu_on) {
+                double sg = 1.0 / (1.0 + exp(-pre));
+                d = sg * (1.0 + pre * (1.0 - sg));
+            }
+            g[t] = dout[i * L + t] * d;
+            sb += g[t];
+        }
+        if (dbias) dbias[i] = sb;
+        for (long k = 0; k < K; ++k) {
+            double acc = 0.0;
+            for (long t = 0; t < L; ++t) {
+                long s = t - (K - 1) + k;
+                double v;
+                if (s >= 0)
+                    v = xi[s];
+                else
+                    v = init ? init[i * (K - 1) + (K - 1) + s] : 0.0;
+                acc += g[t] * v;
+            }
+            dw[i * K + k] = acc;
+        }
+        /* positions s of xe from -(K-1) to L-1: the outputs t = s + (K-1) - k that read it */
+        for (long s = -(K - 1); s < L; ++s) {
+            double acc = 0.0;
+            for (long k = 0; k < K; ++k) {
+                long t = s + (K - 1) - k;
+                if (t >= 0 && t < L) acc += wi[k] * g[t];
+            }
+            if (s >= 0)
+                dx[i * L + s] = acc;
+            else if (init && dinit)
+                dinit[i * (K - 1) + (K - 1) + s] = acc;
+        }
+    }
+    free(g);
+    return S6O_OK;
+}
+
 /* Threads the OpenMP runtime would use for the parallel loops above. */
 #ifdef _OPENMP
 #include <omp.h>

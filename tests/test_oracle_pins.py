@@ -316,7 +316,8 @@ def _mutated_oracle(src_text):
         real = oracle._load()
         lib = ctypes.CDLL(so)
         for name in ("s6o_softplus", "s6o_discretize", "s6o_scan", "s6o_state_update",
-                     "s6o_scan_backward", "s6o_causal_conv1d", "s6o_causal_conv1d_update"):
+                     "s6o_scan_backward", "s6o_causal_conv1d", "s6o_causal_conv1d_update",
+                     "s6o_causal_conv1d_backward"):
             getattr(lib, name).restype = getattr(real, name).restype
             getattr(lib, name).argtypes = getattr(real, name).argtypes
         lib.s6o_num_threads = real.s6o_num_threads
