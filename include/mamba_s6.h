@@ -8,6 +8,7 @@
  *   mamba_selective_scan_bwd      gradients of the forward scan, states recomputed
  *   mamba_causal_conv1d_fwd       the block's causal conv1d + SiLU producing the scan's u
  *   mamba_causal_conv1d_update    its one-token decode step on a rolling conv state
+ *   mamba_causal_conv1d_bwd       the gradients of that convolution (training)
  *
  * Definitions (Mamba: Linear-Time Sequence Modeling with Selective State Spaces,
  * page "xyznot.com/ar/paper/2312.00752", sections "Method", "Selection mechanism
@@ -365,6 +366,38 @@ int mamba_causal_conv1d_fwd(const void* x, const float* weight, const float* bia
 int mamba_causal_conv1d_update(void* conv_state, const void* x, const float* weight,
                                const float* bias, void* out, int64_t batch, int64_t dim,
                                int width, int silu, mamba_dtype dtype, void* stream);
+
+/*
+ * Gradients of sum_t out[b, d, t] * dout[b, d, t] for mamba_causal_conv1d_fwd with the same
+ * x, weight, bias, initial_state, width and silu (the training side of the Mamba block's
+ * convolution step; Mamba, section "Mamba Block", and the chain rule of the definition
+ * above).  With pre[t] the value before the activation and g[t] = dout[t] * act'(pre[t])
+ * (act' = 1 without SiLU, else sigmoid(p) (1 + p (1 - sigmoid(p)))):
+ *
+ *   dx[s]             = sum_k weight[d, k] * g[s + (width-1) - k]    (terms with t in [0, L))
+ *   dweight[d, k]     = sum_{b,t} g[t] * xe[t - (width-1) + k]       (xe = initial_state ++ x)
+ *   dbias[d]          = sum_{b,t} g[t]
+ *   dinitial_state[j] = sum_{k <= j} weight[d, k] * g[j - k]         (j < width-1)
+ *
+ *   x, dout, dx     : (batch, dim, seqlen) dtype       dx must not alias x or dout
+ *   weight          : (dim, width) float32             1 <= width <= 4
+ *   bias            : (dim) float32 or NULL
+ *   initial_state   : (batch, dim, width-1) dtype or NULL (zeros before the sequence)
+ *   dweight         : (dim, width) float32, overwritten (the library zeroes, then sums)
+ *   dbias           : (dim) float32 or NULL, overwritten likewise
+ *   dinitial_state  : (batch, dim, width-1) dtype or NULL; written only when initial_state
+ *                     is given (the zeros used without it have no gradient)
+ *   (with seqlen == 0, x, dout and dx may be NULL; dweight and dbias become zero)
+ *
+ * fp32 arithmetic; dx and dinitial_state rounded to dtype; dweight and dbias are sums
+ * formed with atomic adds, so their last bits may vary from call to call.
+ * Errors: NULL, DIMS, ALIGN, DTYPE, CUDA.
+ */
+int mamba_causal_conv1d_bwd(const void* x, const float* weight, const float* bias,
+                            const void* initial_state, const void* dout, void* dx,
+                            float* dweight, float* dbias, void* dinitial_state, int64_t batch,
+                            int64_t dim, int64_t seqlen, int width, int silu, mamba_dtype dtype,
+                            void* stream);
 
 /*
  * Reads the library's device error word on `stream`, synchronising that stream.

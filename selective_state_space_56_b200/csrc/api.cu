@@ -460,6 +460,39 @@ int mamba_causal_conv1d_update(void* conv_state, const void* x, const float* wei
     return cuda_status(s6::launch_conv1d_update(a, static_cast<cudaStream_t>(stream)));
 }
 
+int mamba_causal_conv1d_bwd(const void* x, const float* weight, const float* bias,
+                            const void* initial_state, const void* dout, void* dx,
+                            float* dweight, float* dbias, void* dinitial_state, int64_t batch,
+                            int64_t dim, int64_t seqlen, int width, int silu, mamba_dtype dtype,
+                            void* stream) {
+    if (!weight || !dweight || (seqlen > 0 && (!x || !dout || !dx))) return MAMBA_ERR_NULL;
+    if (!dtype_ok(dtype)) return MAMBA_ERR_DTYPE;
+    if (width < 1 || width > 4 || batch < 1 || dim < 1 || seqlen < 0) return MAMBA_ERR_DIMS;
+    if (!mul_ok(batch, dim) || !mul_ok(batch * dim, seqlen > 0 ? seqlen : 1) ||
+        !mul_ok(batch * dim * (seqlen > 0 ? seqlen : 1), 8))
+        return MAMBA_ERR_DIMS;
+    const void* ptrs[] = {x, weight, bias, initial_state, dout, dx, dweight, dbias, dinitial_state};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MAMBA_ERR_ALIGN;
+    s6::ConvBwdArgs a;
+    a.x = x;
+    a.weight = weight;
+    a.bias = bias;
+    a.initial_state = width > 1 ? initial_state : nullptr;
+    a.dout = dout;
+    a.dx = dx;
+    a.dweight = dweight;
+    a.dbias = dbias;
+    a.dinitial_state = width > 1 ? dinitial_state : nullptr;
+    a.batch = batch;
+    a.dim = dim;
+    a.L = seqlen;
+    a.width = width;
+    a.silu = silu;
+    a.dtype = to_dtype(dtype);
+    return cuda_status(s6::launch_conv1d_bwd(a, static_cast<cudaStream_t>(stream)));
+}
+
 int mamba_diag_wait_timeout(int64_t limit_cycles, void* stream) {
     if (limit_cycles < 1 || limit_cycles > 4000000000LL) return MAMBA_ERR_DIMS;
     return cuda_status(s6::launch_wait_timeout_probe((long long)limit_cycles,

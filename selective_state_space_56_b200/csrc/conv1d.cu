@@ -184,6 +184,231 @@ __global__ void __launch_bounds__(256) conv1d_update_kernel(T* state, const T* x
     for (int k = 0; k < K - 1; ++k) state[r * (K - 1) + k] = io<T>::from_f(win[k + 1]);
 }
 
+// ---- Backward ------------------------------------------------------------------------
+// Gradients of sum_t out[t] * dout[t] (the chain rule of the definition above): with
+// pre[t] the value before the activation and g[t] = dout[t] * act'(pre[t]),
+//   dx[s] = sum_k w[k] g[s + (K-1) - k],  dw[k] = sum_t g[t] xe[t - (K-1) + k],
+//   dbias = sum_t g[t],  dinit[j] = sum_{k <= j} w[k] g[j - k]  (xe = init ++ x).
+// Also a stream: x and dout read, dx written, 6 bytes per element in bf16.  A thread owns
+// kVPT consecutive 16-byte vectors of dx of one row: it loads the x vectors before, over
+// and after them and the dout vectors over and after them, recomputes pre and g over its
+// steps plus the K-1 after them, correlates, and stores.  dw and dbias are summed over the
+// CTA (one row per CTA) and added to global memory once per CTA.
+
+struct CBParams {
+    const void* x;
+    const float* w;
+    const float* bias;
+    const void* init;
+    const void* dout;
+    void* dx;
+    float* dw;
+    float* db;
+    void* dinit;
+    int64_t dim, batch, L;
+    int silu;
+};
+
+// act'(p) for SiLU: sigmoid(p) (1 + p (1 - sigmoid(p))).
+__device__ __forceinline__ float dsilu(float p) {
+    const float sg = rcp(1.f + ex2(-p * kLog2e));
+    return sg * fmaf(p, 1.f - sg, 1.f);
+}
+
+// Input at position s of row r of init ++ x (zero before init).
+template <typename T>
+__device__ __forceinline__ float xb_at(const CBParams& p, int64_t r, int64_t s, int K) {
+    if (s >= 0) return io<T>::to_f(static_cast<const T*>(p.x)[r * p.L + s]);
+    if (!p.init) return 0.f;
+    return io<T>::to_f(static_cast<const T*>(p.init)[r * (K - 1) + (K - 1) + s]);
+}
+
+// Sum of the K + 1 partial sums (dw[0..K-1], dbias) over the CTA, added to row d's entries.
+template <int K>
+__device__ __forceinline__ void cta_add(const CBParams& p, int64_t d, float (&part)[K + 1],
+                                        float* red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int k = 0; k <= K; ++k)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part[k] += __shfl_xor_sync(0xffffffffu, part[k], o);
+    if (lane == 0)
+#pragma unroll
+        for (int k = 0; k <= K; ++k) red[warp * (K + 1) + k] = part[k];
+    __syncthreads();
+    if ((int)threadIdx.x <= K) {
+        float v = 0.f;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) v += red[w * (K + 1) + threadIdx.x];
+        if ((int)threadIdx.x < K)
+            atomicAdd(p.dw + d * K + threadIdx.x, v);
+        else if (p.db)
+            atomicAdd(p.db + d, v);
+    }
+    __syncthreads();  // red is reused by the next row
+}
+
+// Rows of 16-byte multiples.  Grid (vector blocks, min(dim, 65535), min(batch, 65535));
+// each CTA walks rows (d, b) with strides gridDim.y, gridDim.z.
+template <typename T, int K>
+__global__ void __launch_bounds__(256) conv1d_bwd_vec_kernel(const CBParams p) {
+    constexpr int E = 16 / sizeof(T);
+    constexpr int NT = kVPT * E;  // steps of this thread
+    __shared__ float red[8 * (K + 1)];
+    const int64_t vpr = p.L / E;
+    const int64_t v0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * kVPT;
+    const bool active = v0 < vpr;
+    for (int64_t d = blockIdx.y; d < p.dim; d += gridDim.y) {
+        float w[K];
+#pragma unroll
+        for (int k = 0; k < K; ++k) w[k] = __ldg(p.w + d * K + k);
+        const float bias = p.bias ? __ldg(p.bias + d) : 0.f;
+        for (int64_t b = blockIdx.z; b < p.batch; b += gridDim.z) {
+            const int64_t r = b * p.dim + d;
+            float part[K + 1];
+#pragma unroll
+            for (int k = 0; k <= K; ++k) part[k] = 0.f;
+            if (active) {
+                const T* xr = static_cast<const T*>(p.x) + r * p.L;
+                const T* gr = static_cast<const T*>(p.dout) + r * p.L;
+                const int64_t s0 = v0 * E;
+                // x over [s0 - E, s0 + NT + E) and dout over [s0, s0 + NT + E): loads first
+                uint4 xv[kVPT + 2], gv[kVPT + 1];
+                const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int i = 0; i < kVPT; ++i) {
+                    const bool in = v0 + i < vpr;
+                    xv[i + 1] = in ? *reinterpret_cast<const uint4*>(xr + (v0 + i) * E) : zero;
+                    gv[i] = in ? *reinterpret_cast<const uint4*>(gr + (v0 + i) * E) : zero;
+                }
+                const bool nxt = v0 + kVPT < vpr;
+                xv[kVPT + 1] = (K > 1 && nxt) ? *reinterpret_cast<const uint4*>(xr + (v0 + kVPT) * E) : zero;
+                gv[kVPT] = (K > 1 && nxt) ? *reinterpret_cast<const uint4*>(gr + (v0 + kVPT) * E) : zero;
+                xv[0] = (K > 1 && v0 > 0) ? *reinterpret_cast<const uint4*>(xr + (v0 - 1) * E) : zero;
+                // xe[s0 - (K-1) + j] for j < NT + 2 (K-1), and dout[s0 + j] for j < NT + K - 1
+                float xs[NT + 2 * (K - 1)];
+                float gs[NT + K - 1];
+#pragma unroll
+                for (int j = 0; j < K - 1; ++j)
+                    xs[j] = v0 > 0 ? io<T>::to_f(reinterpret_cast<const T*>(&xv[0])[E - (K - 1) + j])
+                                   : xb_at<T>(p, r, j - (K - 1), K);
+#pragma unroll
+                for (int i = 0; i < kVPT; ++i)
+#pragma unroll
+                    for (int j = 0; j < E; ++j) {
+                        xs[K - 1 + i * E + j] = io<T>::to_f(reinterpret_cast<const T*>(&xv[i + 1])[j]);
+                        gs[i * E + j] = io<T>::to_f(reinterpret_cast<const T*>(&gv[i])[j]);
+                    }
+#pragma unroll
+                for (int j = 0; j < K - 1; ++j) {
+                    xs[K - 1 + NT + j] = io<T>::to_f(reinterpret_cast<const T*>(&xv[kVPT + 1])[j]);
+                    gs[NT + j] = io<T>::to_f(reinterpret_cast<const T*>(&gv[kVPT])[j]);
+                }
+                // g over steps s0 .. s0 + NT + K - 2 (zero past the row: those dout are zero)
+                float g[NT + K - 1];
+#pragma unroll
+                for (int j = 0; j < NT + K - 1; ++j) {
+                    float pre = bias;
+#pragma unroll
+                    for (int k = 0; k < K; ++k) pre = fmaf(w[k], xs[j + k], pre);
+                    g[j] = p.silu ? gs[j] * dsilu(pre) : gs[j];
+                }
+                // this thread's share of dw and dbias (its own steps only)
+#pragma unroll
+                for (int i = 0; i < kVPT; ++i) {
+                    if (v0 + i >= vpr) break;
+#pragma unroll
+                    for (int j = 0; j < E; ++j) {
+                        const int t = i * E + j;
+#pragma unroll
+                        for (int k = 0; k < K; ++k) part[k] = fmaf(g[t], xs[t + k], part[k]);
+                        part[K] += g[t];
+                    }
+                }
+                // dx[s0 + t] = sum_k w[k] g[t + K-1-k]
+#pragma unroll
+                for (int i = 0; i < kVPT; ++i) {
+                    if (v0 + i >= vpr) break;
+                    alignas(16) T o[E];
+#pragma unroll
+                    for (int j = 0; j < E; ++j) {
+                        const int t = i * E + j;
+                        float acc = 0.f;
+#pragma unroll
+                        for (int k = 0; k < K; ++k) acc = fmaf(w[k], g[t + K - 1 - k], acc);
+                        o[j] = io<T>::from_f(acc);
+                    }
+                    *reinterpret_cast<uint4*>(static_cast<T*>(p.dx) + r * p.L + (v0 + i) * E) =
+                        *reinterpret_cast<const uint4*>(o);
+                }
+                // the inputs before the sequence: dinit[j] = sum_{k <= j} w[k] g[j - k]
+                if (K > 1 && v0 == 0 && p.init && p.dinit) {
+#pragma unroll
+                    for (int j = 0; j < K - 1; ++j) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int k = 0; k <= j; ++k) acc = fmaf(w[k], g[j - k], acc);
+                        static_cast<T*>(p.dinit)[r * (K - 1) + j] = io<T>::from_f(acc);
+                    }
+                }
+            }
+            cta_add<K>(p, d, part, red);
+        }
+    }
+}
+
+// Any row length: one step per thread, the K values of g it needs formed from K x each.
+template <typename T, int K>
+__global__ void __launch_bounds__(256) conv1d_bwd_elem_kernel(const CBParams p) {
+    __shared__ float red[8 * (K + 1)];
+    const int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const bool active = s < p.L;
+    for (int64_t d = blockIdx.y; d < p.dim; d += gridDim.y) {
+        float w[K];
+#pragma unroll
+        for (int k = 0; k < K; ++k) w[k] = __ldg(p.w + d * K + k);
+        const float bias = p.bias ? __ldg(p.bias + d) : 0.f;
+        for (int64_t b = blockIdx.z; b < p.batch; b += gridDim.z) {
+            const int64_t r = b * p.dim + d;
+            float part[K + 1];
+#pragma unroll
+            for (int k = 0; k <= K; ++k) part[k] = 0.f;
+            if (active) {
+                // g at steps s .. s + K - 1 (zero past the row)
+                float g[K];
+#pragma unroll
+                for (int m = 0; m < K; ++m) {
+                    const int64_t t = s + m;
+                    g[m] = 0.f;
+                    if (t < p.L) {
+                        float pre = bias;
+#pragma unroll
+                        for (int k = 0; k < K; ++k) pre = fmaf(w[k], xb_at<T>(p, r, t - (K - 1) + k, K), pre);
+                        const float dv = io<T>::to_f(static_cast<const T*>(p.dout)[r * p.L + t]);
+                        g[m] = p.silu ? dv * dsilu(pre) : dv;
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < K; ++k) part[k] = fmaf(g[0], xb_at<T>(p, r, s - (K - 1) + k, K), part[k]);
+                part[K] = g[0];
+                float acc = 0.f;
+#pragma unroll
+                for (int k = 0; k < K; ++k) acc = fmaf(w[k], g[K - 1 - k], acc);
+                static_cast<T*>(p.dx)[r * p.L + s] = io<T>::from_f(acc);
+                if (K > 1 && s == 0 && p.init && p.dinit) {
+#pragma unroll
+                    for (int j = 0; j < K - 1; ++j) {
+                        float a = 0.f;
+#pragma unroll
+                        for (int k = 0; k <= j; ++k) a = fmaf(w[k], g[j - k], a);
+                        static_cast<T*>(p.dinit)[r * (K - 1) + j] = io<T>::from_f(a);
+                    }
+                }
+            }
+            cta_add<K>(p, d, part, red);
+        }
+    }
+}
+
 unsigned blocks_for(int64_t threads) { return (unsigned)((threads + 255) / 256); }
 
 template <typename T, int K>
@@ -263,6 +488,68 @@ cudaError_t launch_conv1d(const ConvArgs& a, cudaStream_t stream) {
 cudaError_t launch_conv1d_update(const ConvUpdateArgs& a, cudaStream_t stream) {
     if (a.dtype == DType::BF16) return launch_update_t<__nv_bfloat16>(a, stream);
     return launch_update_t<float>(a, stream);
+}
+
+namespace {
+
+template <typename T, int K>
+cudaError_t launch_conv_bwd_k(const CBParams& p, int64_t L, cudaStream_t s) {
+    constexpr int E = 16 / sizeof(T);
+    const unsigned gy = (unsigned)(p.dim < 65535 ? p.dim : 65535);
+    const unsigned gz = (unsigned)(p.batch < 65535 ? p.batch : 65535);
+    if (L % E == 0 && K - 1 <= E) {
+        const int64_t vpr = L / E;
+        const dim3 grid((unsigned)((vpr + 256 * kVPT - 1) / (256 * kVPT)), gy, gz);
+        conv1d_bwd_vec_kernel<T, K><<<grid, 256, 0, s>>>(p);
+    } else {
+        const dim3 grid((unsigned)((L + 255) / 256), gy, gz);
+        conv1d_bwd_elem_kernel<T, K><<<grid, 256, 0, s>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_conv_bwd_t(const CBParams& p, int K, cudaStream_t s) {
+    switch (K) {
+        case 1: return launch_conv_bwd_k<T, 1>(p, p.L, s);
+        case 2: return launch_conv_bwd_k<T, 2>(p, p.L, s);
+        case 3: return launch_conv_bwd_k<T, 3>(p, p.L, s);
+        case 4: return launch_conv_bwd_k<T, 4>(p, p.L, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_conv1d_bwd(const ConvBwdArgs& a, cudaStream_t stream) {
+    cudaError_t e = cudaMemsetAsync(a.dweight, 0, (size_t)a.dim * a.width * sizeof(float), stream);
+    if (e == cudaSuccess && a.dbias)
+        e = cudaMemsetAsync(a.dbias, 0, (size_t)a.dim * sizeof(float), stream);
+    if (e != cudaSuccess || a.L == 0) {
+        // an empty sequence: the gradients of the initial state are zero as well
+        if (e == cudaSuccess && a.L == 0 && a.initial_state && a.dinitial_state && a.width > 1)
+            e = cudaMemsetAsync(a.dinitial_state, 0,
+                                (size_t)a.batch * a.dim * (a.width - 1) *
+                                    (a.dtype == DType::BF16 ? 2 : 4), stream);
+        return e;
+    }
+    CBParams p;
+    memset(&p, 0, sizeof(p));
+    p.x = a.x;
+    p.w = a.weight;
+    p.bias = a.bias;
+    p.init = a.width > 1 ? a.initial_state : nullptr;
+    p.dout = a.dout;
+    p.dx = a.dx;
+    p.dw = a.dweight;
+    p.db = a.dbias;
+    p.dinit = a.width > 1 ? a.dinitial_state : nullptr;
+    p.dim = a.dim;
+    p.batch = a.batch;
+    p.L = a.L;
+    p.silu = a.silu ? 1 : 0;
+    if (a.dtype == DType::BF16) return launch_conv_bwd_t<__nv_bfloat16>(p, a.width, stream);
+    return launch_conv_bwd_t<float>(p, a.width, stream);
 }
 
 }  // namespace s6

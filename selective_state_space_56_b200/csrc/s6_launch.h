@@ -133,8 +133,26 @@ struct ConvUpdateArgs {
     DType dtype;
 };
 
+// Gradients of sum(out * dout) for the convolution above.
+struct ConvBwdArgs {
+    const void* x;
+    const float* weight;        // (dim, width)
+    const float* bias;          // (dim) or null
+    const void* initial_state;  // (batch, dim, width - 1) or null
+    const void* dout;           // (batch, dim, L)
+    void* dx;                   // (batch, dim, L)
+    float* dweight;             // (dim, width), zeroed here, then accumulated
+    float* dbias;               // (dim) or null, likewise
+    void* dinitial_state;       // (batch, dim, width - 1) or null (written with initial_state)
+    int64_t batch, dim, L;
+    int width;
+    int silu;
+    DType dtype;
+};
+
 cudaError_t launch_conv1d(const ConvArgs& a, cudaStream_t stream);
 cudaError_t launch_conv1d_update(const ConvUpdateArgs& a, cudaStream_t stream);
+cudaError_t launch_conv1d_bwd(const ConvBwdArgs& a, cudaStream_t stream);
 
 // One bounded device wait that nothing completes: sets bit 0 of the device error word
 // after limit_cycles SM clocks.

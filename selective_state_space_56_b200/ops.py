@@ -85,6 +85,8 @@ def load_library():
             lib.mamba_causal_conv1d_fwd.argtypes = [vp] * 6 + [i64, i64, i64, i32, i32, i32, vp]
             lib.mamba_causal_conv1d_update.restype = i32
             lib.mamba_causal_conv1d_update.argtypes = [vp] * 5 + [i64, i64, i32, i32, i32, vp]
+            lib.mamba_causal_conv1d_bwd.restype = i32
+            lib.mamba_causal_conv1d_bwd.argtypes = [vp] * 9 + [i64, i64, i64, i32, i32, i32, vp]
             lib.mamba_selective_state_update.restype = i32
             lib.mamba_selective_state_update.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
                                                          vp, i64, i64, i64, i32, vp]
@@ -431,6 +433,41 @@ def causal_conv1d_update(conv_state, x, weight, bias=None, silu=True, out=None):
     if rc != 0:
         raise MambaError(rc, "mamba_causal_conv1d_update")
     return out
+
+
+def causal_conv1d_bwd(x, weight, dout, bias=None, initial_state=None, silu=True):
+    """Gradients of sum(out * dout) for ``causal_conv1d_fwd`` with the same x, weight, bias,
+    initial_state and silu.  Returns a dict: dx (batch, dim, L) x.dtype, dweight (dim, K)
+    fp32, dbias (dim) fp32 (None without a bias), dinitial_state (batch, dim, K-1) x.dtype
+    (None without an initial state)."""
+    if not isinstance(x, torch.Tensor) or x.dim() != 3:
+        raise ValueError("x must be a (batch, dim, L) tensor")
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("causal_conv1d_bwd runs on CUDA tensors only")
+    b, d, L = x.shape
+    K = weight.shape[1] if weight.dim() == 2 else -1
+    dt = x.dtype
+    if dt not in _DTYPES:
+        raise ValueError("unsupported dtype %s" % dt)
+    _check(x, "x", dev, (b, d, L), (dt,))
+    _check(dout, "dout", dev, (b, d, L), (dt,))
+    _check(weight, "weight", dev, (d, K), (torch.float32,))
+    _check(bias, "bias", dev, (d,), (torch.float32,))
+    _check(initial_state, "initial_state", dev, (b, d, K - 1), (dt,))
+    g = dict(dx=torch.empty((b, d, L), dtype=dt, device=dev),
+             dweight=torch.empty((d, K), dtype=torch.float32, device=dev),
+             dbias=None if bias is None else torch.empty(d, dtype=torch.float32, device=dev),
+             dinitial_state=None if (initial_state is None or K < 2)
+             else torch.empty((b, d, K - 1), dtype=dt, device=dev))
+    with torch.cuda.device(dev):
+        rc = load_library().mamba_causal_conv1d_bwd(
+            _ptr(x), _ptr(weight), _ptr(bias), _ptr(initial_state), _ptr(dout), _ptr(g["dx"]),
+            _ptr(g["dweight"]), _ptr(g["dbias"]), _ptr(g["dinitial_state"]), b, d, L, K,
+            int(bool(silu)), _DTYPES[dt], _stream_handle(dev))
+    if rc != 0:
+        raise MambaError(rc, "mamba_causal_conv1d_bwd")
+    return g
 
 
 def selective_scan_summary(u, delta, A, B, C, delta_bias=None, delta_softplus=True,
