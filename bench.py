@@ -450,6 +450,8 @@ def compact_line(line):
                         "decode_us": _r(z["decode"]["ms_per_token_l2_flushed"] * 1e3, 4),
                         "decode_hbm_frac": _r(z["decode"]["roofline"]["frac"], 4)}
     out["conv1d"] = {"ms": _r(cv["ms_per_call"], 4), "hbm_frac": _r(cv["roofline"]["frac"], 4),
+                     "bwd_ms": _r(cv["backward"]["ms_per_call"], 4),
+                     "bwd_hbm_frac": _r(cv["backward"]["roofline"]["frac"], 4),
                      "decode_us": _r(cv["decode"]["ms_per_token_l2_flushed"] * 1e3, 4),
                      "decode_hbm_frac": _r(cv["decode"]["roofline"]["frac"], 4)}
     if line.get("lshard") is not None:
@@ -583,7 +585,8 @@ def run_zoh(g, dev, stream, world, w, steps=50):
 
 def run_conv(dev, stream, world, rank, steps=50):
     """The causal conv1d + SiLU producing the m2p8b layer's u (4, 5120, 4096, K = 4, bf16),
-    per launch, and its decode update on (256, 5120) after an L2 flush."""
+    per launch, its backward per call, and its decode update on (256, 5120) after an L2
+    flush."""
     from selective_state_space_56_b200 import inputs, ops
     b, d, L, K = 4, 5120, 4096, inputs.CONV_WIDTH
     p = inputs.conv_inputs(b, d, L, K, torch.bfloat16, seed=rank_seed(inputs.CONV_SEED, rank),
@@ -609,6 +612,28 @@ def run_conv(dev, stream, world, rank, steps=50):
     byts = 2 * elems * 2 + d * K * 4 + d * 4  # x read, out written (bf16), weights, bias
     peaks, kind = measured_peaks()
     del out, fin
+
+    # the backward: x and dout read, dx written (bf16); dweight, dbias summed in place
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(inputs.CONV_SEED + 2)
+    dout = torch.randn((b, d, L), generator=gen, device=dev).to(torch.bfloat16)
+
+    def conv_bwd():
+        return ops.causal_conv1d_bwd(p["x"], p["weight"], dout, p["bias"])
+
+    for _ in range(3):
+        conv_bwd()
+    torch.cuda.synchronize(dev)
+    bevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(steps)]
+    for a, b_ in bevs:
+        a.record(stream)
+        conv_bwd()
+        b_.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_bwd = max_over_ranks(med_ms(bevs), world)
+    bbytes = 3 * elems * 2 + d * K * 4 * 2 + d * 4 * 2  # x, dout, dx; weights in, gradients out
+    del dout
 
     db, dd = 256, 5120
     gen = torch.Generator(device=dev)
@@ -645,6 +670,18 @@ def run_conv(dev, stream, world, rank, steps=50):
                      "algorithmic_bytes": byts, "peak_kind": kind,
                      "traffic": profile_traffic("conv1d_m2p8b.txt",
                                                 "selective_state_space_56_b200/csrc/conv1d.cu")},
+        "backward": {"ms_per_call": ms_bwd, "value": world * elems / (ms_bwd * 1e-3),
+                     "unit": "elems/s",
+                     "workload": "gradients of the same conv for a fixed dout (4, 5120, 4096) "
+                                 "bf16: dx bf16, dweight and dbias fp32",
+                     "roofline": {"bound": "hbm", "unit": "GB/s",
+                                  "achieved": bbytes / (ms_bwd * 1e-3) / 1e9,
+                                  "peak": peaks["hbm_gbs"],
+                                  "frac": bbytes / (ms_bwd * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                  "algorithmic_bytes": bbytes, "peak_kind": kind,
+                                  "traffic": profile_traffic(
+                                      "conv1d_bwd_m2p8b.txt",
+                                      "selective_state_space_56_b200/csrc/conv1d.cu")}},
         "decode": {"ms_per_token_l2_flushed": ms_tok,
                    "workload": "conv state (256, 5120, 3) bf16 updated in place, x and out "
                                "(256, 5120) bf16",
@@ -653,7 +690,7 @@ def run_conv(dev, stream, world, rank, steps=50):
                                 "peak": peaks["hbm_gbs"],
                                 "frac": dbytes / (ms_tok * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                 "algorithmic_bytes": dbytes}},
-        "gpu_launches": 2 * steps + 6,
+        "gpu_launches": 3 * steps + 9,
     }
 
 
@@ -1040,7 +1077,8 @@ def run_reference(args, rank, world):
 def profile_target(which):
     """Three launches of the scan (m2p8b) or of its exact-ZOH variant, eight decode tokens
     (each after an L2 flush),
-    two backward calls of the m2p8b scan, or three conv1d launches, for ncu captures."""
+    two backward calls of the m2p8b scan, or three conv1d launches (forward or backward),
+    for ncu captures."""
     from selective_state_space_56_b200 import inputs, ops
     import selective_state_space_56_b200.build as s6build
     s6build.build()
@@ -1052,10 +1090,14 @@ def profile_target(which):
         for _ in range(3):
             ops.selective_scan_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"], z=p["z"],
                                    delta_bias=p["delta_bias"], y=y, exact_zoh=which == "zoh")
-    elif which == "conv":
+    elif which in ("conv", "conv_bwd"):
         p = inputs.conv_inputs(4, 5120, 4096, inputs.CONV_WIDTH, torch.bfloat16, device=dev)
+        dout = torch.randn((4, 5120, 4096), device=dev).to(torch.bfloat16)
         for _ in range(3):
-            ops.causal_conv1d_fwd(p["x"], p["weight"], p["bias"])
+            if which == "conv":
+                ops.causal_conv1d_fwd(p["x"], p["weight"], p["bias"])
+            else:
+                ops.causal_conv1d_bwd(p["x"], p["weight"], dout, p["bias"])
     elif which == "backward":
         w = inputs.SCAN_WORKLOADS[WORKLOAD]
         p = inputs.scan_inputs(w.batch, w.dim, w.dstate, w.seqlen, w.in_dtype, w.seed, device=dev)
@@ -1095,7 +1137,7 @@ def main(argv=None):
     ap.add_argument("--zoh-steps", type=int, default=50)
     ap.add_argument("--conv-steps", type=int, default=50)
     ap.add_argument("--lshard-steps", type=int, default=5)
-    ap.add_argument("--profile", choices=["scan", "zoh", "decode", "backward", "conv"],
+    ap.add_argument("--profile", choices=["scan", "zoh", "decode", "backward", "conv", "conv_bwd"],
                     help="run a few untimed launches of one workload (an ncu capture target) "
                          "and exit")
     args = ap.parse_args(argv)

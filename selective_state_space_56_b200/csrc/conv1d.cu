@@ -249,8 +249,14 @@ __device__ __forceinline__ void cta_add(const CBParams& p, int64_t d, float (&pa
 
 // Rows of 16-byte multiples.  Grid (vector blocks, min(dim, 65535), min(batch, 65535));
 // each CTA walks rows (d, b) with strides gridDim.y, gridDim.z.
-template <typename T, int K>
+#ifndef S6_CONVB_VPT
+#define S6_CONVB_VPT 2
+#endif
+constexpr int kVPTB = S6_CONVB_VPT;  // 16-byte dx vectors per thread in the backward
+
+template <typename T, int K, bool SILU>
 __global__ void __launch_bounds__(256) conv1d_bwd_vec_kernel(const CBParams p) {
+    constexpr int kVPT = kVPTB;
     constexpr int E = 16 / sizeof(T);
     constexpr int NT = kVPT * E;  // steps of this thread
     __shared__ float red[8 * (K + 1)];
@@ -310,7 +316,7 @@ __global__ void __launch_bounds__(256) conv1d_bwd_vec_kernel(const CBParams p) {
                     float pre = bias;
 #pragma unroll
                     for (int k = 0; k < K; ++k) pre = fmaf(w[k], xs[j + k], pre);
-                    g[j] = p.silu ? gs[j] * dsilu(pre) : gs[j];
+                    g[j] = SILU ? gs[j] * dsilu(pre) : gs[j];
                 }
                 // this thread's share of dw and dbias (its own steps only)
 #pragma unroll
@@ -357,7 +363,7 @@ __global__ void __launch_bounds__(256) conv1d_bwd_vec_kernel(const CBParams p) {
 }
 
 // Any row length: one step per thread, the K values of g it needs formed from K x each.
-template <typename T, int K>
+template <typename T, int K, bool SILU>
 __global__ void __launch_bounds__(256) conv1d_bwd_elem_kernel(const CBParams p) {
     __shared__ float red[8 * (K + 1)];
     const int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -384,7 +390,7 @@ __global__ void __launch_bounds__(256) conv1d_bwd_elem_kernel(const CBParams p) 
 #pragma unroll
                         for (int k = 0; k < K; ++k) pre = fmaf(w[k], xb_at<T>(p, r, t - (K - 1) + k, K), pre);
                         const float dv = io<T>::to_f(static_cast<const T*>(p.dout)[r * p.L + t]);
-                        g[m] = p.silu ? dv * dsilu(pre) : dv;
+                        g[m] = SILU ? dv * dsilu(pre) : dv;
                     }
                 }
 #pragma unroll
@@ -492,20 +498,25 @@ cudaError_t launch_conv1d_update(const ConvUpdateArgs& a, cudaStream_t stream) {
 
 namespace {
 
-template <typename T, int K>
-cudaError_t launch_conv_bwd_k(const CBParams& p, int64_t L, cudaStream_t s) {
+template <typename T, int K, bool SILU>
+cudaError_t launch_conv_bwd_ks(const CBParams& p, int64_t L, cudaStream_t s) {
     constexpr int E = 16 / sizeof(T);
     const unsigned gy = (unsigned)(p.dim < 65535 ? p.dim : 65535);
     const unsigned gz = (unsigned)(p.batch < 65535 ? p.batch : 65535);
     if (L % E == 0 && K - 1 <= E) {
         const int64_t vpr = L / E;
-        const dim3 grid((unsigned)((vpr + 256 * kVPT - 1) / (256 * kVPT)), gy, gz);
-        conv1d_bwd_vec_kernel<T, K><<<grid, 256, 0, s>>>(p);
+        const dim3 grid((unsigned)((vpr + 256 * kVPTB - 1) / (256 * kVPTB)), gy, gz);
+        conv1d_bwd_vec_kernel<T, K, SILU><<<grid, 256, 0, s>>>(p);
     } else {
         const dim3 grid((unsigned)((L + 255) / 256), gy, gz);
-        conv1d_bwd_elem_kernel<T, K><<<grid, 256, 0, s>>>(p);
+        conv1d_bwd_elem_kernel<T, K, SILU><<<grid, 256, 0, s>>>(p);
     }
     return cudaGetLastError();
+}
+
+template <typename T, int K>
+cudaError_t launch_conv_bwd_k(const CBParams& p, int64_t L, cudaStream_t s) {
+    return p.silu ? launch_conv_bwd_ks<T, K, true>(p, L, s) : launch_conv_bwd_ks<T, K, false>(p, L, s);
 }
 
 template <typename T>

@@ -47,6 +47,7 @@ def _full_record():
         "exact_zoh": {"ms_per_call": 0.962, "roofline": {"frac": 0.337},
                       "decode": {"ms_per_token_l2_flushed": 0.0412, "roofline": {"frac": 0.66}}},
         "conv1d": {"ms_per_call": 0.0575, "roofline": {"frac": 0.89},
+                   "backward": {"ms_per_call": 0.0912, "roofline": {"frac": 0.84}},
                    "decode": {"ms_per_token_l2_flushed": 0.0124, "roofline": {"frac": 0.26}}},
         "lshard": None,
         "workloads": {"m130m": {"ms": 0.218, "value": 1.156e11, "frac": 0.447},
