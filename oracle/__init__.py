@@ -24,7 +24,9 @@ associative-combine prefix of ``oracle.pscan``, the LTI convolution form,
 Abar in (0,1), small/large-Delta limits, the gated-RNN special case.  The ZOH
 variant (tests/test_oracle_zoh.py): the gated-RNN identity, the continuous-time
 steady state -B u / A, numerical integration of the continuous ODE, the
-small-Delta limit and A = 0.  The causal conv1d (tests/test_oracle_conv.py): numpy's
+small-Delta limit and A = 0; its backward (tests/test_oracle_backward.py): central
+differences of the ZOH forward, A = 0 and |A| = 1e-5 included.  The causal conv1d
+(tests/test_oracle_conv.py): numpy's
 convolution, the impulse response, causality, chunked prefill and decode steps; its
 backward: central finite differences of the forward, the linear case in closed form.
 """
@@ -78,8 +80,8 @@ def _load():
             lib.s6o_state_update.argtypes = ([ctypes.c_long] * 3 + [_dp] * 9 + [_lp, ctypes.c_int,
                                                                              ctypes.c_int, _dp])
             lib.s6o_scan_backward.restype = ctypes.c_int
-            lib.s6o_scan_backward.argtypes = ([ctypes.c_long] * 4 + [_dp] * 8 + [_lp, ctypes.c_int]
-                                              + [_dp] * 9)
+            lib.s6o_scan_backward.argtypes = ([ctypes.c_long] * 4 + [_dp] * 8 + [_lp, ctypes.c_int,
+                                               ctypes.c_int] + [_dp] * 9)
             lib.s6o_causal_conv1d.restype = ctypes.c_int
             lib.s6o_causal_conv1d.argtypes = [ctypes.c_long] * 3 + [_dp] * 4 + [ctypes.c_int,
                                                                                _dp, _dp]
@@ -264,7 +266,7 @@ def state_update_lanes(state, u, delta_raw, A, B, C, lane_batch, D=None, z=None,
 
 
 def scan_backward_lanes(u, delta_raw, A, B, C, lane_batch, dy, D=None, z=None, delta_bias=None,
-                        softplus=True):
+                        softplus=True, zoh=False):
     """Gradients of sum(y * dy) for lanes: returns dict du, ddelta, dz (nlanes, L),
     dA (nlanes, N), dD, dbias (nlanes), dB, dC (nbatch, N, L)."""
     u, dr, z, dy = _f64(u), _f64(delta_raw), _f64(z), _f64(dy)
@@ -279,7 +281,8 @@ def scan_backward_lanes(u, delta_raw, A, B, C, lane_batch, dy, D=None, z=None, d
                dB=np.empty((nb, N, L)), dC=np.empty((nb, N, L)))
     rc = _load().s6o_scan_backward(
         nl, N, L, nb, _ptr(u), _ptr(dr), _ptr(z), _ptr(Aa), _ptr(Dd), _ptr(bb), _ptr(Bm),
-        _ptr(Cm), lb.ctypes.data_as(_lp), int(bool(softplus)), _ptr(dy), _ptr(out["du"]),
+        _ptr(Cm), lb.ctypes.data_as(_lp), int(bool(softplus)), int(bool(zoh)), _ptr(dy),
+        _ptr(out["du"]),
         _ptr(out["ddelta"]), _ptr(out["dz"]), _ptr(out["dA"]), _ptr(out["dD"]),
         _ptr(out["dbias"]), _ptr(out["dB"]), _ptr(out["dC"]))
     if rc != 0:
@@ -288,7 +291,7 @@ def scan_backward_lanes(u, delta_raw, A, B, C, lane_batch, dy, D=None, z=None, d
 
 
 def selective_scan_backward(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
-                            softplus=True):
+                            softplus=True, zoh=False):
     """Backward in the library's layouts: u, delta, z, dy (b, d, L); A (d, N); B, C
     (b, N, L); D, delta_bias (d).  Returns du, ddelta, dz (b, d, L), dA (d, N), dD, dbias (d),
     dB, dC (b, N, L): the gradients of sum(y * dy)."""
@@ -301,7 +304,7 @@ def selective_scan_backward(u, delta, A, B, C, dy, D=None, z=None, delta_bias=No
                             np.tile(Aa, (b, 1)), B, C, np.repeat(np.arange(b), d),
                             _f64(dy).reshape(b * d, L), D=rep(D),
                             z=None if z is None else _f64(z).reshape(b * d, L),
-                            delta_bias=rep(delta_bias), softplus=softplus)
+                            delta_bias=rep(delta_bias), softplus=softplus, zoh=zoh)
     return dict(du=r["du"].reshape(b, d, L), ddelta=r["ddelta"].reshape(b, d, L),
                 dz=r["dz"].reshape(b, d, L), dA=r["dA"].reshape(b, d, N).sum(0),
                 dD=r["dD"].reshape(b, d).sum(0), dbias=r["dbias"].reshape(b, d).sum(0),

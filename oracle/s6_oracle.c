@@ -205,6 +205,14 @@ int s6o_state_update(long nlanes, long N, long nbatch, double* state,
  *   du_t = dyt_t D + dq_t Delta_t;  dx_t = dDelta_t softplus'(x_t) (= sigmoid(x_t))
  *   dbias += dx_t;  then g_n *= Abar_tn  (carried to step t-1)
  *
+ * With zoh nonzero the input weight q_t B_tn becomes w_tn u_t B_tn with the exact ZOH
+ * w_tn = expm1(Delta_t A_n) / A_n (Delta_t when A_n = 0), and the terms through it change
+ * to the derivatives of w: dB_tn += g_n w_tn u_t; du_t = dyt_t D + sum_n g_n w_tn B_tn;
+ * dDelta_t gains sum_n g_n B_tn u_t dw/dDelta with dw/dDelta = Abar_tn (instead of
+ * dq_t u_t); dA_n gains g_n B_tn u_t dw/dA with dw/dA = Delta_t^2 psi(Delta_t A_n),
+ * psi(y) = (y e^y - expm1(y)) / y^2 = 1/2 + y/3 + y^2/8 + y^3/30 + ... (the series for
+ * |y| < 1e-3, where the closed form cancels).
+ *
  * Shapes as in s6o_scan; dy (nlanes, L); outputs du, ddelta, dz (nlanes, L);
  * dA (nlanes, N); dD, dbias (nlanes); dB, dC (nbatch, N, L) accumulated over lanes
  * (zeroed here first).  Any output pointer may be NULL except du and ddelta.
@@ -216,11 +224,18 @@ static double sigmoid(double x) {
     return e / (1.0 + e);
 }
 
+/* psi(y) = (y e^y - expm1(y)) / y^2, the factor of Delta^2 in d(expm1(Delta A) / A) / dA */
+static double zoh_psi(double y) {
+    if (fabs(y) < 1e-3)
+        return 0.5 + y * (1.0 / 3.0 + y * (1.0 / 8.0 + y * (1.0 / 30.0 + y * (1.0 / 144.0))));
+    return (y * exp(y) - expm1(y)) / (y * y);
+}
+
 int s6o_scan_backward(long nlanes, long N, long L, long nbatch,
                       const double* u, const double* delta_raw, const double* z,
                       const double* A, const double* D, const double* delta_bias,
                       const double* Bm, const double* Cm, const long* lane_batch,
-                      int softplus, const double* dy,
+                      int softplus, int zoh, const double* dy,
                       double* du, double* ddelta, double* dz, double* dA, double* dD,
                       double* dbias, double* dB, double* dC) {
     if (nlanes < 0 || N < 1 || N > S6O_MAX_N || L < 0 || nbatch < 1) return S6O_ERR_ARG;
@@ -243,7 +258,8 @@ int s6o_scan_backward(long nlanes, long N, long L, long nbatch,
             const double dt = step_size(delta_raw[i * L + t], bias, softplus);
             for (long n = 0; n < N; ++n)
                 hs[(t + 1) * N + n] = exp(dt * A[i * N + n]) * hs[t * N + n] +
-                                      dt * u[i * L + t] * Bb[n * L + t];
+                                      input_weight(dt, A[i * N + n], zoh) * u[i * L + t] *
+                                          Bb[n * L + t];
         }
         double g[S6O_MAX_N], dAn[S6O_MAX_N];
         for (long n = 0; n < N; ++n) g[n] = 0.0, dAn[n] = 0.0;
@@ -262,21 +278,30 @@ int s6o_scan_backward(long nlanes, long N, long L, long nbatch,
             } else if (dz) {
                 dz[i * L + t] = 0.0;
             }
-            double dq = 0.0, ddt = 0.0;
+            double dq = 0.0, ddt = 0.0, duw = 0.0;
             for (long n = 0; n < N; ++n) {
-                const double abar = exp(dt * A[i * N + n]);
+                const double an = A[i * N + n];
+                const double abar = exp(dt * an);
+                const double w = input_weight(dt, an, zoh);
                 g[n] += dyt * Cb[n * L + t];
                 if (dC) dC[(lane_batch[i] * N + n) * L + t] += dyt * hs[(t + 1) * N + n];
-                if (dB) dB[(lane_batch[i] * N + n) * L + t] += g[n] * dt * ut;
-                dq += g[n] * Bb[n * L + t];
+                if (dB) dB[(lane_batch[i] * N + n) * L + t] += g[n] * w * ut;
+                if (zoh) {
+                    const double gb = g[n] * Bb[n * L + t];
+                    duw += gb * w;                        /* du through the weight */
+                    ddt += gb * ut * abar;                /* dw/dDelta = Abar */
+                    dAn[n] += gb * ut * dt * dt * zoh_psi(dt * an);  /* dw/dA */
+                } else {
+                    dq += g[n] * Bb[n * L + t];
+                }
                 const double gh = g[n] * hs[t * N + n] * abar;
-                ddt += gh * A[i * N + n];
+                ddt += gh * an;
                 dAn[n] += gh * dt;
                 g[n] *= abar;
             }
             ddt += dq * ut;
             dDi += dyt * ut;
-            du[i * L + t] = dyt * dskip + dq * dt;
+            du[i * L + t] = dyt * dskip + (zoh ? duw : dq * dt);
             const double dx = softplus ? ddt * sigmoid(x) : ddt;
             ddelta[i * L + t] = dx;
             dbi += dx;
