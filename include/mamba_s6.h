@@ -6,6 +6,7 @@
  *   mamba_selective_scan_fwd      the fused S6 forward scan over a whole sequence
  *   mamba_selective_state_update  one decode token, updating a carried state in place
  *   mamba_selective_scan_bwd      gradients of the forward scan, states recomputed
+ *                                 (_ex: also for the exact zero-order-hold forward)
  *   mamba_causal_conv1d_fwd       the block's causal conv1d + SiLU producing the scan's u
  *   mamba_causal_conv1d_update    its one-token decode step on a rolling conv state
  *   mamba_causal_conv1d_bwd       the gradients of that convolution (training)
@@ -282,7 +283,7 @@ size_t mamba_selective_scan_bwd_workspace_size(mamba_scan_dims dims);
  *                 contents on entry do not matter
  *
  * The backward is that of the Bbar = Delta * B discretisation (the forward without
- * flags).
+ * flags); mamba_selective_scan_bwd_ex below takes the flags word of the forward.
  * dA, dB, dC, dD and ddelta_bias are sums over many CTAs, formed with float32
  * atomics: their last bits may differ between runs.  With seqlen == 0 the
  * per-token arrays may be NULL and dA, dD, ddelta_bias are set to zero.
@@ -316,6 +317,25 @@ int mamba_selective_scan_fwd_train(const void* u, const void* delta, const float
                                    mamba_dtype out_dtype, void* workspace,
                                    size_t workspace_bytes, float* checkpoints,
                                    size_t checkpoint_bytes, void* stream);
+
+/*
+ * mamba_selective_scan_bwd with the flags word of the forward: with MAMBA_FLAG_EXACT_ZOH
+ * the gradients are those of the exact zero-order-hold forward (Mamba, section "Method":
+ * Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B, per state w = expm1(Delta A_n) / A_n
+ * times B_n, the weight Delta where A_n = 0), its states recomputed the same way.  The
+ * weight's own derivatives enter: dB gains g w u instead of g Delta u, du the sum over
+ * states of g w B, dDelta the sum of g B u dw/dDelta (dw/dDelta = exp(Delta A)), dA the sum
+ * of g B u dw/dA (dw/dA = Delta^2 psi(Delta A), psi(y) = (y e^y - expm1(y)) / y^2, taken
+ * from its series where |Delta A| < 1/16).  flags = 0 is exactly mamba_selective_scan_bwd.
+ * Errors: as mamba_selective_scan_bwd, and FLAGS for unknown flag bits.
+ */
+int mamba_selective_scan_bwd_ex(const void* u, const void* delta, const float* A, const void* B,
+                                const void* C, const float* D, const void* z,
+                                const float* delta_bias, int delta_softplus, const void* dy,
+                                void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC,
+                                float* dD, float* ddelta_bias, mamba_scan_dims dims,
+                                mamba_dtype in_dtype, void* workspace, size_t workspace_bytes,
+                                unsigned flags, void* stream);
 
 /*
  * mamba_selective_scan_bwd from the checkpoints a mamba_selective_scan_fwd_train call

@@ -48,7 +48,7 @@ int scan_bwd(const void* u, const void* delta, const float* A, const void* B, co
              const float* D, const void* z, const float* delta_bias, int delta_softplus,
              const void* dy, void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC,
              float* dD, float* ddelta_bias, mamba_scan_dims dims, mamba_dtype in_dtype,
-             void* ckpt, size_t ckpt_bytes, bool ckpt_ready, void* stream);
+             void* ckpt, size_t ckpt_bytes, bool ckpt_ready, unsigned flags, void* stream);
 
 int state_update(float* state, const void* u, const void* delta, const float* A, const void* B,
                  const void* C, const float* D, const void* z, const float* delta_bias,
@@ -307,8 +307,20 @@ int mamba_selective_scan_bwd(const void* u, const void* delta, const float* A, c
                              mamba_dtype in_dtype, void* workspace, size_t workspace_bytes,
                              void* stream) {
     return scan_bwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, dy, du, ddelta, dz, dA,
-                    dB, dC, dD, ddelta_bias, dims, in_dtype, workspace, workspace_bytes, false,
+                    dB, dC, dD, ddelta_bias, dims, in_dtype, workspace, workspace_bytes, false, 0u,
                     stream);
+}
+
+int mamba_selective_scan_bwd_ex(const void* u, const void* delta, const float* A, const void* B,
+                                const void* C, const float* D, const void* z,
+                                const float* delta_bias, int delta_softplus, const void* dy,
+                                void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC,
+                                float* dD, float* ddelta_bias, mamba_scan_dims dims,
+                                mamba_dtype in_dtype, void* workspace, size_t workspace_bytes,
+                                unsigned flags, void* stream) {
+    return scan_bwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, dy, du, ddelta, dz, dA,
+                    dB, dC, dD, ddelta_bias, dims, in_dtype, workspace, workspace_bytes, false,
+                    flags, stream);
 }
 
 int mamba_selective_scan_fwd_train(const void* u, const void* delta, const float* A,
@@ -332,7 +344,7 @@ int mamba_selective_scan_bwd_from_checkpoints(
     size_t checkpoint_bytes, void* stream) {
     return scan_bwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, dy, du, ddelta, dz, dA,
                     dB, dC, dD, ddelta_bias, dims, in_dtype, const_cast<float*>(checkpoints),
-                    checkpoint_bytes, true, stream);
+                    checkpoint_bytes, true, 0u, stream);
 }
 
 }  // extern "C"
@@ -343,7 +355,9 @@ int scan_bwd(const void* u, const void* delta, const float* A, const void* B, co
              const float* D, const void* z, const float* delta_bias, int delta_softplus,
              const void* dy, void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC,
              float* dD, float* ddelta_bias, mamba_scan_dims dims, mamba_dtype in_dtype,
-             void* workspace, size_t workspace_bytes, bool ckpt_ready, void* stream) {
+             void* workspace, size_t workspace_bytes, bool ckpt_ready, unsigned flags,
+             void* stream) {
+    if (flags & ~kKnownFlags) return MAMBA_ERR_FLAGS;
     const bool empty = dims.seqlen == 0;
     if (!A || !dA) return MAMBA_ERR_NULL;
     if (!empty && (!u || !delta || !B || !C || !dy || !du || !ddelta || !dB || !dC))
@@ -379,7 +393,7 @@ int scan_bwd(const void* u, const void* delta, const float* A, const void* B, co
     a.N = dims.dstate;
     a.L = dims.seqlen;
     a.softplus = delta_softplus;
-    a.zoh = 0;
+    a.zoh = (flags & MAMBA_FLAG_EXACT_ZOH) ? 1 : 0;
     a.in_dtype = to_dtype(in_dtype);
     a.out_dtype = a.in_dtype;
     a.nseg = 1;

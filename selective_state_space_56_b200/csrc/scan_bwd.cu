@@ -257,7 +257,26 @@ __device__ __forceinline__ void stage_chunk(const BParams& p, unsigned char* st,
     }
 }
 
-template <int T, typename Tin>
+// The exact ZOH weight w = expm1(Delta A) / A and its derivative in A,
+// dw/dA = Delta^2 psi(Delta A), psi(y) = (y e^y - expm1(y)) / y^2 = 1/2 + y/3 + y^2/8 +
+// y^3/30 + ..., on packed pairs from x = Delta A log2(e), e = 2^x (= Abar) and w: where
+// |Delta A| < 1/16 as the series (in x, coefficients ln2^k times those above; the first
+// dropped term, y^4/144, is below 1e-7 of psi there), elsewhere as (Delta e - w) / A.
+__device__ __forceinline__ f2 zoh_dw_da2(f2 x, f2 e, f2 w, f2 inv_a, f2 dd) {
+    f2 p = fma2(pack2(1.1100822e-2f, 1.1100822e-2f), x, pack2(6.0056627e-2f, 6.0056627e-2f));
+    p = fma2(p, x, pack2(2.3104906e-1f, 2.3104906e-1f));
+    p = fma2(p, x, pack2(0.5f, 0.5f));
+    const f2 small = mul2(mul2(dd, dd), p);
+    const f2 large = mul2(sub2(mul2(dd, e), w), inv_a);
+    float x0, x1, s0, s1, l0, l1;
+    unpack2(x, x0, x1);
+    unpack2(small, s0, s1);
+    unpack2(large, l0, l1);
+    constexpr float kTau = 0.09016844f;  // |Delta A| = 1/16 in log2 units
+    return pack2(fabsf(x0) < kTau ? s0 : l0, fabsf(x1) < kTau ? s1 : l1);
+}
+
+template <int T, typename Tin, bool ZOH>
 __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) {
     using Lo = BLayout<T, Tin>;
     constexpr int RS = Lo::RS, RR = Lo::RR;
@@ -298,6 +317,13 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
     }
     const f2 a2p[2] = {pack2(a2[0], a2[1]), pack2(a2[2], a2[3])};
     const f2 anp[2] = {pack2(an[0], an[1]), pack2(an[2], an[3])};
+    // 1 / A (infinite for A = 0, where the exact ZOH weight takes its series branch)
+    f2 invp[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};
+    if constexpr (ZOH) {
+        invp[0] = pack2(1.f / an[0], 1.f / an[1]);
+        invp[1] = pack2(1.f / an[2], 1.f / an[3]);
+    }
+    const f2 one2 = pack2(1.f, 1.f);
     const f2 zero2 = pack2(0.f, 0.f);
     f2 gp[2] = {zero2, zero2}, dAp[2] = {zero2, zero2};
     const float Dd = (chok && p.D) ? p.D[dch] : 0.f;
@@ -398,9 +424,16 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
                     const float q = dts[s] * uv[s];
                     const f2 qq = pack2(q, q);
                     const f2x2 bb = bq.at(s);
-                    const f2 e0 = ex2x2(mul2(dd, a2p[0])), e1 = ex2x2(mul2(dd, a2p[1]));
-                    hp[0] = fma2(e0, hp[0], mul2(qq, bb.lo));
-                    hp[1] = fma2(e1, hp[1], mul2(qq, bb.hi));
+                    const f2 x0 = mul2(dd, a2p[0]), x1 = mul2(dd, a2p[1]);
+                    const f2 e0 = ex2x2(x0), e1 = ex2x2(x1);
+                    if constexpr (ZOH) {  // input weight u w, w = expm1(Delta A) / A
+                        const f2 uu = pack2(uv[s], uv[s]);
+                        hp[0] = fma2(e0, hp[0], mul2(zoh_weight_u2(x0, e0, invp[0], uu, qq), bb.lo));
+                        hp[1] = fma2(e1, hp[1], mul2(zoh_weight_u2(x1, e1, invp[1], uu, qq), bb.hi));
+                    } else {
+                        hp[0] = fma2(e0, hp[0], mul2(qq, bb.lo));
+                        hp[1] = fma2(e1, hp[1], mul2(qq, bb.hi));
+                    }
                 }
             }
         }
@@ -424,10 +457,17 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
                 const float q = dts[s] * uv[s];
                 const f2 qq = pack2(q, q);
                 const f2x2 bb = bq.at(s);
-                ab[s][0] = ex2x2(mul2(dd, a2p[0]));
-                ab[s][1] = ex2x2(mul2(dd, a2p[1]));
-                hs[s][0] = fma2(ab[s][0], s ? hs[s - 1][0] : hin[0], mul2(qq, bb.lo));
-                hs[s][1] = fma2(ab[s][1], s ? hs[s - 1][1] : hin[1], mul2(qq, bb.hi));
+                const f2 x0 = mul2(dd, a2p[0]), x1 = mul2(dd, a2p[1]);
+                ab[s][0] = ex2x2(x0);
+                ab[s][1] = ex2x2(x1);
+                f2 w0 = qq, w1 = qq;
+                if constexpr (ZOH) {
+                    const f2 uu = pack2(uv[s], uv[s]);
+                    w0 = zoh_weight_u2(x0, ab[s][0], invp[0], uu, qq);
+                    w1 = zoh_weight_u2(x1, ab[s][1], invp[1], uu, qq);
+                }
+                hs[s][0] = fma2(ab[s][0], s ? hs[s - 1][0] : hin[0], mul2(w0, bb.lo));
+                hs[s][1] = fma2(ab[s][1], s ? hs[s - 1][1] : hin[1], mul2(w1, bb.hi));
             }
             cq.load(sC, tg, pp);
 
@@ -442,8 +482,27 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
                 gp[1] = fma2(yy, cc.hi, gp[1]);
                 ypv[s] = hsum(fma2(cc.lo, hs[s][0], mul2(cc.hi, hs[s][1])));  // C_t . h_t
                 const f2 dC0 = mul2(yy, hs[s][0]), dC1 = mul2(yy, hs[s][1]);
-                const f2 dB0 = mul2(gp[0], qq), dB1 = mul2(gp[1], qq);
-                dqv[s] = hsum(fma2(gp[0], bb.lo, mul2(gp[1], bb.hi)));
+                f2 dB0, dB1;
+                float dwu = 0.f;  // exact ZOH: sum_n g B dw/dDelta (= g B Abar), times u below
+                if constexpr (ZOH) {
+                    // the weight's terms: dB = g w u, du = sum g w B, dDelta += u sum g B Abar,
+                    // dA += g B u dw/dA
+                    const f2 uu = pack2(uv[s], uv[s]);
+                    const f2 x0 = mul2(dd, a2p[0]), x1 = mul2(dd, a2p[1]);
+                    const f2 w0 = zoh_weight_u2(x0, ab[s][0], invp[0], one2, dd);
+                    const f2 w1 = zoh_weight_u2(x1, ab[s][1], invp[1], one2, dd);
+                    dB0 = mul2(gp[0], mul2(w0, uu));
+                    dB1 = mul2(gp[1], mul2(w1, uu));
+                    const f2 gb0 = mul2(gp[0], bb.lo), gb1 = mul2(gp[1], bb.hi);
+                    dqv[s] = hsum(fma2(gb0, w0, mul2(gb1, w1)));
+                    dwu = hsum(fma2(gb0, ab[s][0], mul2(gb1, ab[s][1])));
+                    dAp[0] = fma2(mul2(gb0, uu), zoh_dw_da2(x0, ab[s][0], w0, invp[0], dd), dAp[0]);
+                    dAp[1] = fma2(mul2(gb1, uu), zoh_dw_da2(x1, ab[s][1], w1, invp[1], dd), dAp[1]);
+                } else {
+                    dB0 = mul2(gp[0], qq);
+                    dB1 = mul2(gp[1], qq);
+                    dqv[s] = hsum(fma2(gp[0], bb.lo, mul2(gp[1], bb.hi)));
+                }
                 // g Abar is the adjoint carried to step t - 1; times h_{t-1} it gives the
                 // terms of dA and of the state part of dDelta
                 gp[0] = mul2(gp[0], ab[s][0]);
@@ -451,6 +510,7 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
                 const f2 gh0 = mul2(gp[0], s ? hs[s - 1][0] : hin[0]);
                 const f2 gh1 = mul2(gp[1], s ? hs[s - 1][1] : hin[1]);
                 ddv[s] = hsum(fma2(gh0, anp[0], mul2(gh1, anp[1])));
+                if constexpr (ZOH) ddv[s] = fmaf(uv[s], dwu, ddv[s]);
                 dAp[0] = fma2(gh0, dd, dAp[0]);
                 dAp[1] = fma2(gh1, dd, dAp[1]);
                 if constexpr (XS == 0) {
@@ -565,8 +625,10 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
                     softplus_sigmoid(io<Tin>::to_f(rDr[cw * RR + t]) + bias, sp, sg);
                 }
             }
-            const float ddelta = (ddl + dq * uu) * sg;
-            rDy[cw * RR + t] = io<Tin>::from_f(fmaf(dyt, Dd, dq * dt));  // du replaces dy
+            // exact ZOH: dq is sum g w B (the weight's derivative in u) and ddl holds the
+            // weight's part of dDelta already; with Delta * B, dq = sum g B
+            const float ddelta = (ZOH ? ddl : fmaf(dq, uu, ddl)) * sg;
+            rDy[cw * RR + t] = io<Tin>::from_f(fmaf(dyt, Dd, ZOH ? dq : dq * dt));  // du replaces dy
             rDr[cw * RR + t] = io<Tin>::from_f(ddelta);                  // ddelta replaces delta
             if (t < valid) {
                 dbacc += ddelta;
@@ -632,10 +694,10 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
     }
 }
 
-template <int T, typename Tin>
+template <int T, typename Tin, bool ZOH>
 cudaError_t launch_bwd_typed(const BParams& bp, int64_t batch, int64_t dim, cudaStream_t s) {
     using Lo = BLayout<T, Tin>;
-    auto kern = scan_bwd_kernel<T, Tin>;
+    auto kern = scan_bwd_kernel<T, Tin, ZOH>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Lo::bytes);
     if (e != cudaSuccess) return e;
@@ -646,25 +708,26 @@ cudaError_t launch_bwd_typed(const BParams& bp, int64_t batch, int64_t dim, cuda
     return cudaGetLastError();
 }
 
-template <typename Tin>
+template <typename Tin, bool ZOH>
 cudaError_t launch_bwd_io(BParams bp, int T, int64_t batch, int64_t dim, cudaStream_t s) {
     // 16-byte staging needs every row start (a multiple of L elements) 16-byte aligned
     bp.vec = (bp.L * (int64_t)sizeof(Tin)) % 16 == 0 ? 1 : 0;
-    if (T == 16) return launch_bwd_typed<16, Tin>(bp, batch, dim, s);
-    if (T == 32) return launch_bwd_typed<32, Tin>(bp, batch, dim, s);
-    if (T == 64) return launch_bwd_typed<64, Tin>(bp, batch, dim, s);
+    if (T == 16) return launch_bwd_typed<16, Tin, ZOH>(bp, batch, dim, s);
+    if (T == 32) return launch_bwd_typed<32, Tin, ZOH>(bp, batch, dim, s);
+    if (T == 64) return launch_bwd_typed<64, Tin, ZOH>(bp, batch, dim, s);
     return cudaErrorInvalidConfiguration;
 }
 
 // Resident CTAs of the T-step backward kernel per SM on the current device.
-template <int T, typename Tin>
+template <int T, typename Tin, bool ZOH>
 int resident_ctas() {
     int n = 0;
-    if (cudaFuncSetAttribute(scan_bwd_kernel<T, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(scan_bwd_kernel<T, Tin, ZOH>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)BLayout<T, Tin>::bytes) != cudaSuccess ||
-        cudaFuncSetAttribute(scan_bwd_kernel<T, Tin>,
+        cudaFuncSetAttribute(scan_bwd_kernel<T, Tin, ZOH>,
                              cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, scan_bwd_kernel<T, Tin>, kBW * 32,
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, scan_bwd_kernel<T, Tin, ZOH>, kBW * 32,
                                                       BLayout<T, Tin>::bytes) != cudaSuccess)
         return 0;
     return n;
@@ -672,13 +735,13 @@ int resident_ctas() {
 
 // Block length for N > 8: 32 steps (half the per-block overhead) when every CTA of the
 // grid is resident at once with it, else 16 (less shared memory per CTA, so more fit).
-template <typename Tin>
+template <typename Tin, bool ZOH>
 int pick_block_steps(int64_t ctas) {
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return 16;
-    return ctas <= (int64_t)sms * resident_ctas<32, Tin>() ? 32 : 16;
+    return ctas <= (int64_t)sms * resident_ctas<32, Tin, ZOH>() ? 32 : 16;
 }
 
 }  // namespace
@@ -690,8 +753,10 @@ cudaError_t launch_scan_backward(const ScanArgs& a, const BackwardArgs& g, float
     const int64_t ctas = (a.dim + kBCH - 1) / kBCH * a.batch;
     int T = CK;
     if (a.N > 8 && CK == 16)
-        T = a.in_dtype == DType::BF16 ? pick_block_steps<__nv_bfloat16>(ctas)
-                                      : pick_block_steps<float>(ctas);
+        T = a.in_dtype == DType::BF16
+                ? (a.zoh ? pick_block_steps<__nv_bfloat16, true>(ctas)
+                         : pick_block_steps<__nv_bfloat16, false>(ctas))
+                : (a.zoh ? pick_block_steps<float, true>(ctas) : pick_block_steps<float, false>(ctas));
     const int64_t chunks = (a.L + T - 1) / T;
     cudaError_t e;
     // outputs accumulated with atomics start at zero
@@ -735,8 +800,11 @@ cudaError_t launch_scan_backward(const ScanArgs& a, const BackwardArgs& g, float
     bp.chunks = (int)chunks;
     bp.ck_blocks = (int)((a.L + CK - 1) / CK);
     bp.ck_stride = T / CK;
-    if (a.in_dtype == DType::BF16) return launch_bwd_io<__nv_bfloat16>(bp, T, a.batch, a.dim, stream);
-    return launch_bwd_io<float>(bp, T, a.batch, a.dim, stream);
+    if (a.in_dtype == DType::BF16)
+        return a.zoh ? launch_bwd_io<__nv_bfloat16, true>(bp, T, a.batch, a.dim, stream)
+                     : launch_bwd_io<__nv_bfloat16, false>(bp, T, a.batch, a.dim, stream);
+    return a.zoh ? launch_bwd_io<float, true>(bp, T, a.batch, a.dim, stream)
+                 : launch_bwd_io<float, false>(bp, T, a.batch, a.dim, stream);
 }
 
 }  // namespace s6

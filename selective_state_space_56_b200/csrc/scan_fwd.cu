@@ -1241,17 +1241,31 @@ cudaError_t launch_io(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
                             : launch_typed<NMAX, Tin, Tout, false, ZOH>(a, kp, s);
 }
 
-template <int NMAX, typename Tin>
+template <int NMAX, typename Tin, bool ZOH>
 cudaError_t launch_ckpt_io(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
     using TL = Tile<NMAX>;
 #if S6_WS_CKPT
-    if (tma_rows<Tin>(a) && producer_plan<Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin>>(a, 1))
+    if (!ZOH && tma_rows<Tin>(a) &&
+        producer_plan<Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin>>(a, 1))
         return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kCheckpoint, true, false, 2>(
             a, kp, 1, s);
 #endif
     return tma_rows<Tin>(a)
-               ? launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kCheckpoint, true>(a, kp, 1, s)
-               : launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kCheckpoint, false>(a, kp, 1, s);
+               ? launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kCheckpoint, true, ZOH>(a, kp, 1, s)
+               : launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kCheckpoint, false, ZOH>(a, kp, 1, s);
+}
+
+template <int NMAX, bool ZOH>
+cudaError_t launch_ckpt_n(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
+    return a.in_dtype == DType::BF16 ? launch_ckpt_io<NMAX, __nv_bfloat16, ZOH>(a, kp, s)
+                                     : launch_ckpt_io<NMAX, float, ZOH>(a, kp, s);
+}
+
+template <bool ZOH>
+cudaError_t launch_ckpt_z(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
+    if (a.N <= 4) return launch_ckpt_n<4, ZOH>(a, kp, s);
+    if (a.N <= 8) return launch_ckpt_n<8, ZOH>(a, kp, s);
+    return launch_ckpt_n<16, ZOH>(a, kp, s);
 }
 
 // Segment summaries: kAggregate over `nseg` segments (all of them) into seg_h / seg_sum.
@@ -1317,10 +1331,7 @@ cudaError_t launch_scan_checkpoints(const ScanArgs& a, float* ckpt, cudaStream_t
     kp.N = (int)a.N;
     kp.nseg = 1;
     kp.softplus = a.softplus ? 1 : 0;
-    const bool ib = a.in_dtype == DType::BF16;
-    if (a.N <= 4) return ib ? launch_ckpt_io<4, __nv_bfloat16>(a, kp, stream) : launch_ckpt_io<4, float>(a, kp, stream);
-    if (a.N <= 8) return ib ? launch_ckpt_io<8, __nv_bfloat16>(a, kp, stream) : launch_ckpt_io<8, float>(a, kp, stream);
-    return ib ? launch_ckpt_io<16, __nv_bfloat16>(a, kp, stream) : launch_ckpt_io<16, float>(a, kp, stream);
+    return a.zoh ? launch_ckpt_z<true>(a, kp, stream) : launch_ckpt_z<false>(a, kp, stream);
 }
 
 cudaError_t launch_fold(const float* hend, const float* dsum, const float* A, const float* h0,

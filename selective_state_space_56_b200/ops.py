@@ -58,6 +58,9 @@ def load_library():
             lib.mamba_selective_scan_bwd.restype = i32
             lib.mamba_selective_scan_bwd.argtypes = [vp] * 8 + [i32] + [vp] * 9 + [
                 ScanDims, i32, vp, ctypes.c_size_t, vp]
+            lib.mamba_selective_scan_bwd_ex.restype = i32
+            lib.mamba_selective_scan_bwd_ex.argtypes = [vp] * 8 + [i32] + [vp] * 9 + [
+                ScanDims, i32, vp, ctypes.c_size_t, ctypes.c_uint, vp]
             u32 = ctypes.c_uint
             lib.mamba_selective_scan_fwd_ex.restype = i32
             lib.mamba_selective_scan_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp,
@@ -263,13 +266,15 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
 
 
 def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
-                       delta_softplus=True, workspace=None, checkpoints=None):
+                       delta_softplus=True, workspace=None, checkpoints=None, exact_zoh=False):
     """Gradients of ``selective_scan_fwd`` for the upstream gradient dy (batch, dim, L),
     in the inputs' dtype.  Returns a dict with du, ddelta, dz (input dtype, dz None
     without a gate), dA (dim, N), dB, dC (batch, N, L), dD, ddelta_bias (dim) in fp32
     (None where the input is None).  checkpoints: the buffer a training forward
     (selective_scan_fwd(..., checkpoints=...)) filled for the same inputs; the backward
-    then skips its own checkpointing pass."""
+    then skips its own checkpointing pass.  exact_zoh: the gradients of the exact
+    zero-order-hold forward (``selective_scan_fwd(..., exact_zoh=True)``); not with
+    checkpoints (the training forward has no exact-ZOH form)."""
     if not isinstance(u, torch.Tensor) or u.dim() != 3:
         raise ValueError("u must be a (batch, dim, L) tensor")
     dev = u.device
@@ -298,6 +303,8 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
     lib = load_library()
     dims = ScanDims(b, d, N, L)
     if checkpoints is not None:
+        if exact_zoh:
+            raise ValueError("the training path has no exact-ZOH form")
         _check(checkpoints, "checkpoints", dev)
         with torch.cuda.device(dev):
             rc = lib.mamba_selective_scan_bwd_from_checkpoints(
@@ -314,13 +321,14 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(dev):
-        rc = lib.mamba_selective_scan_bwd(
+        rc = lib.mamba_selective_scan_bwd_ex(
             _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
             int(bool(delta_softplus)), _ptr(dy), _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dz"]),
             _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]), _ptr(g["ddelta_bias"]),
-            dims, _DTYPES[dt], _ptr(workspace), ws_bytes, _stream_handle(dev))
+            dims, _DTYPES[dt], _ptr(workspace), ws_bytes,
+            MAMBA_FLAG_EXACT_ZOH if exact_zoh else 0, _stream_handle(dev))
     if rc != 0:
-        raise MambaError(rc, "mamba_selective_scan_bwd")
+        raise MambaError(rc, "mamba_selective_scan_bwd_ex")
     return g
 
 
