@@ -447,6 +447,8 @@ def compact_line(line):
                        "train_ms": _r(bw["train_step"]["ms_per_step"], 4),
                        "train_frac": _r(bw["train_step"]["roofline"]["frac"], 4)}
     out["exact_zoh"] = {"ms": _r(z["ms_per_call"], 4), "frac": _r(z["roofline"]["frac"], 4),
+                        "bwd_ms": _r(z["backward"]["ms_per_call"], 4),
+                        "bwd_frac": _r(z["backward"]["roofline"]["frac"], 4),
                         "decode_us": _r(z["decode"]["ms_per_token_l2_flushed"] * 1e3, 4),
                         "decode_hbm_frac": _r(z["decode"]["roofline"]["frac"], 4)}
     out["conv1d"] = {"ms": _r(cv["ms_per_call"], 4), "hbm_frac": _r(cv["roofline"]["frac"], 4),
@@ -504,7 +506,8 @@ def run_probes(dev, stream, sms, fmax_mhz, reps=3):
 
 def run_zoh(g, dev, stream, world, w, steps=50):
     """The exact zero-order-hold variant (MAMBA_FLAG_EXACT_ZOH): the m2p8b scan per launch,
-    and decode tokens after an L2 flush, each timed with events on the launching stream."""
+    its backward per call, and decode tokens after an L2 flush, each timed with events on the
+    launching stream."""
     from selective_state_space_56_b200 import inputs, ops
     b, d, n, L = w.batch, w.dim, w.dstate, w.seqlen
     y = torch.empty((b, d, L), dtype=w.out_dtype, device=dev)
@@ -531,6 +534,32 @@ def run_zoh(g, dev, stream, world, w, steps=50):
     sfu_peak = sms * SFU_OPS_PER_CLK_PER_SM * fmax_mhz * 1e6
     exps = elems * (n + 2)
     del y
+
+    # its backward (checkpoint pass with the ZOH weight + sweep), for a fixed dy
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed + 7)
+    dy = torch.randn((b, d, L), generator=gen, device=dev).to(w.in_dtype)
+    ws = torch.empty(ops.selective_scan_bwd_workspace_size(b, d, n, L), dtype=torch.uint8,
+                     device=dev)
+
+    def bwd():
+        return ops.selective_scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], dy, D=g["D"],
+                                      z=g["z"], delta_bias=g["delta_bias"], workspace=ws,
+                                      exact_zoh=True)
+
+    for _ in range(3):
+        bwd()
+    torch.cuda.synchronize(dev)
+    bevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(max(3, steps // 5))]
+    for a, b_ in bevs:
+        a.record(stream)
+        bwd()
+        b_.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_bwd = max_over_ranks(med_ms(bevs), world)
+    sfu_bwd = elems * (2 * n + 4)  # as the Delta*B backward: the weight needs no SFU result
+    del dy, ws
 
     dw = inputs.DECODE_WORKLOAD
     prm = {k: v.to(dev) for k, v in inputs.decode_params(dw).items()}
@@ -572,6 +601,13 @@ def run_zoh(g, dev, stream, world, w, steps=50):
                          "selective_state_space_56_b200/csrc/s6_device.cuh"),
                      "note": "same N + 2 SFU exponentials per element as the Delta*B scan; the "
                              "exact weight adds FMA-pipe work (series + select), not SFU work"},
+        "backward": {"ms_per_call": ms_bwd, "value": world * elems / (ms_bwd * 1e-3),
+                     "unit": "elems/s",
+                     "roofline": {"bound": "alu", "unit": "Gop/s (SFU)",
+                                  "achieved": sfu_bwd / (ms_bwd * 1e-3) / 1e9,
+                                  "peak": sfu_peak / 1e9,
+                                  "frac": sfu_bwd / (ms_bwd * 1e-3) / sfu_peak,
+                                  "sfu_ops_per_elem": 2 * n + 4}},
         "decode": {"ms_per_token_l2_flushed": ms_tok,
                    "value": world * dw.batch * dw.dim / (ms_tok * 1e-3),
                    "unit": "(b,d) lane updates/s",
@@ -579,7 +615,7 @@ def run_zoh(g, dev, stream, world, w, steps=50):
                                 "achieved": byts / (ms_tok * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
                                 "frac": byts / (ms_tok * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                 "peak_kind": kind}},
-        "gpu_launches": 2 * steps + 6,
+        "gpu_launches": 2 * steps + 6 + 2 * (max(3, steps // 5) + 3),
     }
 
 

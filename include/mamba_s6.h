@@ -326,7 +326,7 @@ int mamba_selective_scan_fwd_train(const void* u, const void* delta, const float
  * weight's own derivatives enter: dB gains g w u instead of g Delta u, du the sum over
  * states of g w B, dDelta the sum of g B u dw/dDelta (dw/dDelta = exp(Delta A)), dA the sum
  * of g B u dw/dA (dw/dA = Delta^2 psi(Delta A), psi(y) = (y e^y - expm1(y)) / y^2, taken
- * from its series where |Delta A| < 1/16).  flags = 0 is exactly mamba_selective_scan_bwd.
+ * from its series where |Delta A| < 1/2).  flags = 0 is exactly mamba_selective_scan_bwd.
  * Errors: as mamba_selective_scan_bwd, and FLAGS for unknown flag bits.
  */
 int mamba_selective_scan_bwd_ex(const void* u, const void* delta, const float* A, const void* B,

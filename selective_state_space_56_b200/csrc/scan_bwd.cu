@@ -258,12 +258,19 @@ __device__ __forceinline__ void stage_chunk(const BParams& p, unsigned char* st,
 }
 
 // The exact ZOH weight w = expm1(Delta A) / A and its derivative in A,
-// dw/dA = Delta^2 psi(Delta A), psi(y) = (y e^y - expm1(y)) / y^2 = 1/2 + y/3 + y^2/8 +
-// y^3/30 + ..., on packed pairs from x = Delta A log2(e), e = 2^x (= Abar) and w: where
-// |Delta A| < 1/16 as the series (in x, coefficients ln2^k times those above; the first
-// dropped term, y^4/144, is below 1e-7 of psi there), elsewhere as (Delta e - w) / A.
+// dw/dA = Delta^2 psi(Delta A), psi(y) = (y e^y - expm1(y)) / y^2 = sum_j y^j (j+1) / (j+2)!
+// = 1/2 + y/3 + y^2/8 + y^3/30 + ..., on packed pairs from x = Delta A log2(e), e = 2^x
+// (= Abar) and w: where |Delta A| < 1/2 as the series through y^7 (Horner in x,
+// coefficients ln2^j times the above; the first dropped term is below 2e-8 of psi there),
+// elsewhere as (Delta e - w) / A, whose two terms then differ by at least a third of
+// themselves (next to 1/16, the weight's own switch, they would agree to 3%, and the SFU's
+// 2^x error would be magnified thirtyfold).
 __device__ __forceinline__ f2 zoh_dw_da2(f2 x, f2 e, f2 w, f2 inv_a, f2 dd) {
-    f2 p = fma2(pack2(1.1100822e-2f, 1.1100822e-2f), x, pack2(6.0056627e-2f, 6.0056627e-2f));
+    f2 p = fma2(pack2(1.6947482e-6f, 1.6947482e-6f), x, pack2(1.9254413e-5f, 1.9254413e-5f));
+    p = fma2(p, x, pack2(1.9047940e-4f, 1.9047940e-4f));
+    p = fma2(p, x, pack2(1.6030215e-3f, 1.6030215e-3f));
+    p = fma2(p, x, pack2(1.1100822e-2f, 1.1100822e-2f));
+    p = fma2(p, x, pack2(6.0056627e-2f, 6.0056627e-2f));
     p = fma2(p, x, pack2(2.3104906e-1f, 2.3104906e-1f));
     p = fma2(p, x, pack2(0.5f, 0.5f));
     const f2 small = mul2(mul2(dd, dd), p);
@@ -272,7 +279,7 @@ __device__ __forceinline__ f2 zoh_dw_da2(f2 x, f2 e, f2 w, f2 inv_a, f2 dd) {
     unpack2(x, x0, x1);
     unpack2(small, s0, s1);
     unpack2(large, l0, l1);
-    constexpr float kTau = 0.09016844f;  // |Delta A| = 1/16 in log2 units
+    constexpr float kTau = 0.72134752f;  // |Delta A| = 1/2 in log2 units
     return pack2(fabsf(x0) < kTau ? s0 : l0, fabsf(x1) < kTau ? s1 : l1);
 }
 

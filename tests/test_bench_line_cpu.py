@@ -45,6 +45,7 @@ def _full_record():
                      "train_step": {"ms_per_step": 3.54, "roofline": {"frac": 0.275}},
                      "cpu_baseline": {"sample": "s" * 90}},
         "exact_zoh": {"ms_per_call": 0.962, "roofline": {"frac": 0.337},
+                      "backward": {"ms_per_call": 4.1, "roofline": {"frac": 0.16}},
                       "decode": {"ms_per_token_l2_flushed": 0.0412, "roofline": {"frac": 0.66}}},
         "conv1d": {"ms_per_call": 0.0575, "roofline": {"frac": 0.89},
                    "backward": {"ms_per_call": 0.0912, "roofline": {"frac": 0.84}},
