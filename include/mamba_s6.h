@@ -253,9 +253,13 @@ int mamba_selective_scan_fwd_noalloc(const void* u, const void* delta, const flo
                                      mamba_dtype in_dtype, mamba_dtype out_dtype, void* stream);
 
 /*
- * Bytes of device workspace mamba_selective_scan_bwd needs for `dims`:
- * batch x dim x ceil(seqlen / T) x dstate x 4, T = 16 steps for dstate > 8 and 64
- * otherwise, rounded up to 256 bytes (0 when seqlen == 0).  Returns 0 for invalid dims.
+ * Bytes of device workspace mamba_selective_scan_bwd needs for `dims`: the checkpoints,
+ * batch x dim x ceil(seqlen / T) x dstate floats (T = 16 steps for dstate > 8 and 64
+ * otherwise), rounded up to 64 floats; plus, when a long sequence over few channels is
+ * swept in S segments side by side (seqlen >= 16384 and fewer CTAs of 32 channels than two
+ * per SM of the current device; S up to five CTAs per SM, segments of at least 4096 steps),
+ * S x batch x dim x (dstate + 1) floats for the segments' summaries.  Rounded up to 256
+ * bytes (0 when seqlen == 0).  Returns 0 for invalid dims.
  */
 size_t mamba_selective_scan_bwd_workspace_size(mamba_scan_dims dims);
 

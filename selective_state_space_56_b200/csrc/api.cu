@@ -295,7 +295,14 @@ size_t mamba_selective_scan_bwd_workspace_size(mamba_scan_dims dims) {
     const int64_t chunks = (dims.seqlen + T - 1) / T;
     if (!mul_ok(dims.batch * dims.dim, chunks) || !mul_ok(dims.batch * dims.dim * chunks, dims.dstate * 4))
         return 0;
-    const int64_t bytes = dims.batch * dims.dim * chunks * dims.dstate * 4;
+    int64_t floats = (dims.batch * dims.dim * chunks * dims.dstate + 63) / 64 * 64;
+    int64_t nseg = 1, seg_len = 0;
+    s6::backward_segments(dims.batch, dims.dim, dims.seqlen, &nseg, &seg_len);
+    if (nseg > 1) {  // the segments' adjoint summaries and summed steps
+        if (!mul_ok(nseg * dims.batch * dims.dim, dims.dstate + 1)) return 0;
+        floats += nseg * dims.batch * dims.dim * (dims.dstate + 1);
+    }
+    const int64_t bytes = floats * 4;
     return (size_t)((bytes + 255) / 256 * 256);
 }
 

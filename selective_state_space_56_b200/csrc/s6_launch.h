@@ -85,7 +85,15 @@ int checkpoint_steps(int64_t N);
 // Forward pass that writes the state entering every checkpoint block to
 // ckpt[((b * dim + d) * blocks + k) * N + n], blocks = ceil(L / checkpoint_steps(N)),
 // and no output.  Uses a.u, delta, A, B, C, delta_bias, softplus, dims and in_dtype.
+// With a.nseg > 1 (a.seg_len a multiple of 64) the segments run side by side from their
+// true starts, formed first in a.seg_h / a.seg_sum (nseg x batch x dim x N, and
+// nseg x batch x dim floats).
 cudaError_t launch_scan_checkpoints(const ScanArgs& a, float* ckpt, cudaStream_t stream);
+
+// The backward's split of a long sequence over few channels into nseg segments of seg_len
+// steps (a multiple of 64; nseg = 1 when it does not split).  Its workspace then holds,
+// after the checkpoints (rounded up to 64 floats), nseg x batch x dim x (N + 1) floats.
+void backward_segments(int64_t batch, int64_t dim, int64_t L, int64_t* nseg, int64_t* seg_len);
 
 // Gradients of the scan (outputs of the backward); dy is read, the rest written.
 struct BackwardArgs {

@@ -37,6 +37,7 @@
 // through softplus use softplus'(x) = sigmoid(x); through the gate
 // silu'(z) = sigmoid(z) (1 + z (1 - sigmoid(z))).  Per state and step the kernel
 // evaluates Abar twice (forward and group recompute), the checkpoint pass once.
+#include <algorithm>
 #include <cstring>
 
 #include "s6_device.cuh"
@@ -70,6 +71,15 @@ struct BParams {
     int chunks;     // blocks of T steps this kernel walks
     int ck_blocks;  // checkpoints per channel (blocks of checkpoint_steps(N))
     int ck_stride;  // checkpoints per block of T steps
+    // a sequence split into nseg segments of seg_chunks blocks (grid z = segment): g_carry
+    // [nseg][batch][dim][N] holds, per segment, the adjoint its first step carries backwards
+    // from the segment alone (the summary pass), then, after the fold, in slot s + 1 the
+    // adjoint entering segment s from all later steps; g_dsum [nseg][batch][dim] the summed
+    // steps of each segment
+    int nseg;
+    int seg_chunks;
+    float* g_carry;
+    float* g_dsum;
     int vec;  // rows start on 16-byte boundaries: stage them with 16-byte copies
 };
 
@@ -336,8 +346,20 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
     const float Dd = (chok && p.D) ? p.D[dch] : 0.f;
     const float bias = (chok && p.delta_bias) ? p.delta_bias[dch] : 0.f;
     float dDacc = 0.f, dbacc = 0.f;
+    // this CTA's segment of a split sequence (all of it otherwise) and the adjoint that
+    // enters its last step from the later segments (zero for the last segment)
+    const int seg = (int)blockIdx.z;
+    const int kbeg = seg * p.seg_chunks, kend = min(p.chunks, kbeg + p.seg_chunks);
+    if (p.nseg > 1 && seg + 1 < p.nseg && chok) {
+        const float* gc = p.g_carry + (((int64_t)(seg + 1) * p.batch + b) * p.dim + dch) * p.N;
+        float g4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) g4[j] = pp * 4 + j < p.N ? gc[pp * 4 + j] : 0.f;
+        gp[0] = pack2(g4[0], g4[1]);
+        gp[1] = pack2(g4[2], g4[3]);
+    }
 
-    for (int k = p.chunks - 1; k >= 0; --k) {
+    for (int k = kend - 1; k >= kbeg; --k) {
         const int64_t t0 = (int64_t)k * T;
         const int valid = (int)min((int64_t)T, p.L - t0);
         __syncthreads();  // the previous chunk's outputs have left the staging rows
@@ -701,6 +723,120 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
     }
 }
 
+// Summary pass of a split sequence's backward, for segments 1 .. nseg-1 (grid z + 1): the
+// adjoint the segment's first step carries backwards when the segment alone is swept from
+// a zero adjoint (last step first: g += dyt C, then g *= Abar), and the segment's summed
+// steps.  The adjoint recurrence involves no state, so nothing is recomputed and no
+// gradient is formed; the input weight does not enter it either (Delta * B or exact ZOH).
+template <int T, typename Tin>
+__global__ void __launch_bounds__(kBW * 32) adjoint_summary_kernel(const BParams p) {
+    using Lo = BLayout<T, Tin>;
+    constexpr int RS = Lo::RS, RR = Lo::RR;
+    extern __shared__ __align__(16) unsigned char smem[];
+    unsigned char* st = smem + Lo::off_stage;
+    const Tin* rDr = reinterpret_cast<const Tin*>(st + Lo::rows);
+    const Tin* rZ = reinterpret_cast<const Tin*>(st + 2 * Lo::rows);
+    const Tin* rDy = reinterpret_cast<const Tin*>(st + 3 * Lo::rows);
+    const Tin* rC = reinterpret_cast<const Tin*>(st + 4 * Lo::rows + Lo::coef);
+    float* sC = reinterpret_cast<float*>(smem + Lo::off_C);
+    float* sDel = reinterpret_cast<float*>(smem + Lo::off_del);
+    float* sDyt = reinterpret_cast<float*>(smem + Lo::off_dyt);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int pp = lane & 3, cl = lane >> 2;
+    const int cw = warp * kBG + cl;
+    const int64_t b = blockIdx.y, d0 = (int64_t)blockIdx.x * kBCH, dch = d0 + cw;
+    const bool chok = dch < p.dim;
+    const bool has_z = p.z != nullptr;
+    float a2[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int n = pp * 4 + j;
+        a2[j] = (chok && n < p.N) ? p.A[dch * p.N + n] * kLog2e : 0.f;
+    }
+    const f2 a2p[2] = {pack2(a2[0], a2[1]), pack2(a2[2], a2[3])};
+    f2 gp[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};
+    float dsum = 0.f;
+    const int seg = (int)blockIdx.z + 1;
+    const int kbeg = seg * p.seg_chunks, kend = min(p.chunks, kbeg + p.seg_chunks);
+    for (int k = kend - 1; k >= kbeg; --k) {
+        const int64_t t0 = (int64_t)k * T;
+        const int valid = (int)min((int64_t)T, p.L - t0);
+        __syncthreads();  // the previous chunk's rows are no longer read
+        stage_chunk<T, Tin>(p, st, b, d0, k, tid);
+        __syncthreads();
+        if constexpr (sizeof(Tin) == 2) {  // C to the bf16 blocks the sweep's loads read
+            for (int i = tid; i < 4 * T; i += kBW * 32) {
+                const int t = i / 4, pq = i % 4;
+                const unsigned short* src = reinterpret_cast<const unsigned short*>(rC) + pq * 4 * RR + t;
+                uint2 w;
+                w.x = (uint32_t)src[0] | ((uint32_t)src[RR] << 16);
+                w.y = (uint32_t)src[2 * RR] | ((uint32_t)src[3 * RR] << 16);
+                reinterpret_cast<uint2*>(sC)[((t / 4) * 4 + pq) * 4 + t % 4] = w;
+            }
+        } else {
+            for (int i = tid; i < 16 * T; i += kBW * 32) {
+                const int n = i & 15, t = i >> 4;
+                sC[t * 16 + n] = io<Tin>::to_f(rC[n * RR + t]);
+            }
+        }
+        for (int i = lane; i < kBG * T; i += 32) {  // Delta and dyt, as in the sweep
+            const int c = warp * kBG + i / T, t = i % T;
+            const int64_t d = d0 + c;
+            const float bi = (d < p.dim && p.delta_bias) ? p.delta_bias[d] : 0.f;
+            const float x = io<Tin>::to_f(rDr[c * RR + t]) + bi;
+            const float dt = p.softplus ? softplus(x) : x;
+            sDel[c * RS + t] = t < valid ? dt : 0.f;
+            const float dyv = io<Tin>::to_f(rDy[c * RR + t]);
+            sDyt[c * RS + t] = has_z ? dyv * silu(io<Tin>::to_f(rZ[c * RR + t])) : dyv;
+        }
+        __syncthreads();
+        for (int tg = T - 4; tg >= 0; tg -= 4) {
+            const float4 d4 = lds4(sDel + cw * RS + tg), y4 = lds4(sDyt + cw * RS + tg);
+            const float dts[4] = {d4.x, d4.y, d4.z, d4.w}, dyts[4] = {y4.x, y4.y, y4.z, y4.w};
+            Coef<Tin> cq;
+            cq.load(sC, tg, pp);
+#pragma unroll
+            for (int s = 3; s >= 0; --s) {
+                const f2x2 cc = cq.at(s);
+                const f2 yy = pack2(dyts[s], dyts[s]), dd = pack2(dts[s], dts[s]);
+                gp[0] = mul2(fma2(yy, cc.lo, gp[0]), ex2x2(mul2(dd, a2p[0])));
+                gp[1] = mul2(fma2(yy, cc.hi, gp[1]), ex2x2(mul2(dd, a2p[1])));
+            }
+            dsum += (d4.x + d4.y) + (d4.z + d4.w);
+        }
+    }
+    if (chok) {
+        const int64_t row = ((int64_t)seg * p.batch + b) * p.dim + dch;
+        float g4[4];
+        unpack2(gp[0], g4[0], g4[1]);
+        unpack2(gp[1], g4[2], g4[3]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (pp * 4 + j < p.N) p.g_carry[row * p.N + pp * 4 + j] = g4[j];
+        if (pp == 0) p.g_dsum[row] = dsum;
+    }
+}
+
+// The fold of the summaries, last segment first.  Thread per (batch, channel, state): the
+// adjoint entering segment s - 1 from every later step is segment s's own carry plus what
+// enters segment s, decayed through it: G_{s-1} = carry_s + exp(A sum_s Delta) G_s, G_{nseg-1}
+// = 0.  G_{s-1} replaces carry_s in place (slot s), which the sweep of segment s - 1 reads.
+__global__ void adjoint_fold_kernel(float* g_carry, const float* g_dsum, const float* A,
+                                    int64_t batch, int64_t dim, int N, int nseg) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= batch * dim * N) return;
+    const int n = (int)(i % N);
+    const int64_t bd = i / N;
+    const int64_t d = bd % dim;
+    const float a2 = A[d * N + n] * kLog2e;
+    float G = 0.f;
+    for (int s = nseg - 1; s >= 1; --s) {
+        const int64_t row = (int64_t)s * batch * dim + bd;
+        G = fmaf(ex2(a2 * g_dsum[row]), G, g_carry[row * N + n]);
+        g_carry[row * N + n] = G;
+    }
+}
+
 template <int T, typename Tin, bool ZOH>
 cudaError_t launch_bwd_typed(const BParams& bp, int64_t batch, int64_t dim, cudaStream_t s) {
     using Lo = BLayout<T, Tin>;
@@ -710,7 +846,20 @@ cudaError_t launch_bwd_typed(const BParams& bp, int64_t batch, int64_t dim, cuda
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)((dim + kBCH - 1) / kBCH), (unsigned)batch, 1);
+    if (bp.nseg > 1) {  // the summaries of segments 1.., then their fold
+        auto sk = adjoint_summary_kernel<T, Tin>;
+        e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lo::bytes);
+        if (e != cudaSuccess) return e;
+        const dim3 sgrid((unsigned)((dim + kBCH - 1) / kBCH), (unsigned)batch,
+                         (unsigned)(bp.nseg - 1));
+        sk<<<sgrid, kBW * 32, Lo::bytes, s>>>(bp);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        const int64_t lanes = batch * dim * bp.N;
+        adjoint_fold_kernel<<<(unsigned)((lanes + 255) / 256), 256, 0, s>>>(
+            bp.g_carry, bp.g_dsum, bp.A, batch, dim, bp.N, bp.nseg);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    const dim3 grid((unsigned)((dim + kBCH - 1) / kBCH), (unsigned)batch, (unsigned)bp.nseg);
     kern<<<grid, kBW * 32, Lo::bytes, s>>>(bp);
     return cudaGetLastError();
 }
@@ -753,11 +902,45 @@ int pick_block_steps(int64_t ctas) {
 
 }  // namespace
 
-cudaError_t launch_scan_backward(const ScanArgs& a, const BackwardArgs& g, float* ckpt,
+void backward_segments(int64_t batch, int64_t dim, int64_t L, int64_t* nseg, int64_t* seg_len) {
+    // Split the sequence only when the channels alone leave most of the GPU idle (fewer
+    // CTAs than two per SM) and it is long: then as many segments as five CTAs per SM hold,
+    // none shorter than 4096 steps, each a multiple of 64 steps (whole checkpoint blocks
+    // and sweep blocks).
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        sms = 148;
+    const int64_t ctas = (dim + kBCH - 1) / kBCH * batch;
+    int64_t n = 1;
+    if (L >= 16384 && ctas < 2 * (int64_t)sms)
+        n = std::max<int64_t>(1, std::min<int64_t>(5 * (int64_t)sms / ctas, L / 4096));
+    int64_t len = (L + n - 1) / n;
+    len = (len + 63) / 64 * 64;
+    if (len == 0) len = 64;
+    *seg_len = len;
+    *nseg = std::max<int64_t>(1, (L + len - 1) / len);
+}
+
+cudaError_t launch_scan_backward(const ScanArgs& a_in, const BackwardArgs& g, float* ckpt,
                                  cudaStream_t stream, bool ckpt_ready) {
     // checkpoints every CK steps; the kernel walks blocks of T = CK (or 2 CK) steps
-    const int CK = checkpoint_steps(a.N);
-    const int64_t ctas = (a.dim + kBCH - 1) / kBCH * a.batch;
+    const int CK = checkpoint_steps(a_in.N);
+    // a long sequence over few channels is swept in segments (the workspace holds their
+    // summaries after the checkpoints)
+    ScanArgs a = a_in;
+    int64_t nseg = 1, seg_len = a.L;
+    backward_segments(a.batch, a.dim, a.L, &nseg, &seg_len);
+    const size_t ck_floats = (size_t)a.batch * a.dim * ((a.L + CK - 1) / CK) * a.N;
+    float* seg_h = ckpt + (ck_floats + 63) / 64 * 64;
+    float* seg_sum = seg_h + (size_t)nseg * a.batch * a.dim * a.N;
+    if (nseg > 1) {
+        a.nseg = nseg;
+        a.seg_len = seg_len;
+        a.seg_h = seg_h;
+        a.seg_sum = seg_sum;
+    }
+    const int64_t ctas = (a.dim + kBCH - 1) / kBCH * a.batch * nseg;
     int T = CK;
     if (a.N > 8 && CK == 16)
         T = a.in_dtype == DType::BF16
@@ -807,6 +990,10 @@ cudaError_t launch_scan_backward(const ScanArgs& a, const BackwardArgs& g, float
     bp.chunks = (int)chunks;
     bp.ck_blocks = (int)((a.L + CK - 1) / CK);
     bp.ck_stride = T / CK;
+    bp.nseg = (int)nseg;
+    bp.seg_chunks = nseg > 1 ? (int)(seg_len / T) : (int)chunks;
+    bp.g_carry = seg_h;
+    bp.g_dsum = seg_sum;
     if (a.in_dtype == DType::BF16)
         return a.zoh ? launch_bwd_io<__nv_bfloat16, true>(bp, T, a.batch, a.dim, stream)
                      : launch_bwd_io<__nv_bfloat16, false>(bp, T, a.batch, a.dim, stream);

@@ -340,7 +340,7 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
                 const bool ok = dchk[k] < p.dim && nn < p.N;
                 a[q] = ok ? p.A[dchk[k] * p.N + nn] * kLog2e : 0.f;  // padded states: Abar = 1, b = 0
                 // initial state: the segment's start (split sequences) or the caller's h0
-                h[q] = ((kOut && MODE != kFullAgg) && p.seg_h != nullptr && ok)
+                h[q] = ((kOut || MODE == kCheckpoint) && MODE != kFullAgg && p.seg_h != nullptr && ok)
                            ? p.seg_h[(((int64_t)seg * p.batch + b) * p.dim + dchk[k]) * p.N + nn]
                            : 0.f;
             }
@@ -1244,6 +1244,22 @@ cudaError_t launch_io(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
 template <int NMAX, typename Tin, bool ZOH>
 cudaError_t launch_ckpt_io(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
     using TL = Tile<NMAX>;
+    if (a.nseg > 1) {
+        // a split sequence: every segment's true start first (the summaries of all but the
+        // last segment from zero, then the fold), so each segment records true states
+        const bool tr = tma_rows<Tin>(a);
+        cudaError_t e =
+            tr ? launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kAggregate, true, ZOH>(a, kp, a.nseg - 1, s)
+               : launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kAggregate, false, ZOH>(a, kp, a.nseg - 1, s);
+        if (e != cudaSuccess) return e;
+        const int64_t lanes = a.batch * a.dim * a.N;
+        carry_kernel<<<(unsigned)((lanes + 255) / 256), 256, 0, s>>>(
+            a.seg_h, a.seg_sum, a.A, a.batch, a.dim, (int)a.N, (int)a.nseg, nullptr);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        return tr ? launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kCheckpoint, true, ZOH>(a, kp, a.nseg, s)
+                  : launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin, kCheckpoint, false, ZOH>(a, kp, a.nseg, s);
+    }
 #if S6_WS_CKPT
     if (!ZOH && tma_rows<Tin>(a) &&
         producer_plan<Layout<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tin>>(a, 1))
@@ -1331,6 +1347,12 @@ cudaError_t launch_scan_checkpoints(const ScanArgs& a, float* ckpt, cudaStream_t
     kp.N = (int)a.N;
     kp.nseg = 1;
     kp.softplus = a.softplus ? 1 : 0;
+    if (a.nseg > 1) {  // segments of a split sequence, each from its true start
+        kp.seg_len = a.seg_len;
+        kp.nseg = (int)a.nseg;
+        kp.seg_h = a.seg_h;
+        kp.seg_sum = a.seg_sum;
+    }
     return a.zoh ? launch_ckpt_z<true>(a, kp, stream) : launch_ckpt_z<false>(a, kp, stream);
 }
 

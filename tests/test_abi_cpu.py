@@ -193,6 +193,21 @@ def test_bwd_workspace_is_one_checkpoint_per_chunk(lib):
     assert ws(2, 64, 17, 8) == 0
 
 
+def test_bwd_workspace_of_a_split_sequence(lib):
+    """A long sequence over few channels is swept in segments: after the checkpoints
+    (rounded up to 64 floats) the workspace holds each segment's adjoint summary and summed
+    step, S x batch x dim x (N + 1) floats.  Without a GPU the plan assumes 148 SMs: the
+    million-length layer (1, 2048, 16, 2^20) has 64 CTAs of 32 channels, so S = 740 // 64 = 11
+    segments of 95,360 steps."""
+    ws = lambda *d: lib.mamba_selective_scan_bwd_workspace_size(_dims(*d))  # noqa: E731
+    b, d, N, L = 1, 2048, 16, 1 << 20
+    ck = (b * d * (L // 16) * N + 63) // 64 * 64
+    assert ws(b, d, N, L) == ((ck + 11 * b * d * (N + 1)) * 4 + 255) // 256 * 256
+    # enough channels (640 CTAs for the 2.8B-shaped layer), or a short sequence: no split
+    assert ws(4, 5120, 16, 1 << 15) == 4 * 5120 * (1 << 11) * 16 * 4
+    assert ws(1, 64, 16, 8192) == 64 * 512 * 16 * 4
+
+
 ERR_FLAGS = -8
 
 

@@ -104,3 +104,10 @@ def test_zoh_backward_flag_zero_is_the_plain_backward(cuda_ok):
     for name, _ in GRADS:
         if g0[name] is not None and name in ("du", "ddelta", "dz"):
             assert torch.equal(g0[name], g1[name]), name
+
+
+def test_zoh_backward_of_a_split_sequence(cuda_ok):
+    """The exact-ZOH backward of a sequence swept in segments (checkpoint pass with the ZOH
+    weight from each segment's true start, adjoint summaries and their fold)."""
+    p, dy = _grad_inputs(1, 40, 16, 20000, torch.float32, seed=9)
+    _compare(_gpu_bwd_zoh(p, dy), _oracle_bwd_zoh(p, dy), p, torch.float32)
