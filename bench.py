@@ -853,7 +853,8 @@ def run_workloads(dev, stream, world, steps=20):
     """The forward scan on the other scan workloads of the metric: the Mamba-130M-shaped
     layer (8, 1536, 16, 2048) and the million-length layer (1, 2048, 16, 2^20, split along
     L inside the call), each call timed with events (median), against the same SFU
-    roofline of N + 2 exponentials per element."""
+    roofline of N + 2 exponentials per element; and the million-length layer's backward
+    (swept in segments inside the call) against its 2N + 4."""
     from selective_state_space_56_b200 import inputs, ops
     peaks, _ = measured_peaks()
     fmax_mhz = peaks.get("sm_max_mhz", 1965.0)
@@ -887,7 +888,34 @@ def run_workloads(dev, stream, world, steps=20):
         out[name] = {"ms": ms, "value": world * elems / (ms * 1e-3),
                      "frac": elems * (w.dstate + 2) / (ms * 1e-3) / sfu_peak}
         launches += (reps + 3) * (3 if nws else 1)
-        del p, y, ws
+        del y, ws
+        if name == "million":
+            gen = torch.Generator(device=dev)
+            gen.manual_seed(w.seed + 7)
+            dy = torch.randn((w.batch, w.dim, w.seqlen), generator=gen, device=dev).to(w.in_dtype)
+            wsb = torch.empty(ops.selective_scan_bwd_workspace_size(w.batch, w.dim, w.dstate,
+                                                                    w.seqlen),
+                              dtype=torch.uint8, device=dev)
+
+            def bwd():
+                ops.selective_scan_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, D=p["D"],
+                                       z=p["z"], delta_bias=p["delta_bias"], workspace=wsb)
+
+            bwd()
+            torch.cuda.synchronize(dev)
+            bevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(3)]
+            for a, b_ in bevs:
+                a.record(stream)
+                bwd()
+                b_.record(stream)
+            torch.cuda.synchronize(dev)
+            mb = max_over_ranks(med_ms(bevs), world)
+            out["million_bwd"] = {"ms": mb, "value": world * elems / (mb * 1e-3),
+                                  "frac": elems * (2 * w.dstate + 4) / (mb * 1e-3) / sfu_peak}
+            launches += 4 * 6  # checkpoint split (2 + fold), summary, fold, sweep
+            del dy, wsb
+        del p
         torch.cuda.empty_cache()
     out["gpu_launches"] = launches
     return out
