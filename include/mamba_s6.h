@@ -270,7 +270,11 @@ size_t mamba_selective_scan_bwd_workspace_size(mamba_scan_dims dims);
  * recomputed: a forward pass records the state entering every T-step block in the
  * workspace, and a reverse sweep rebuilds each chunk's states from its record
  * before propagating the adjoint state backwards through it (Mamba, section
- * "Hardware-aware state expansion").
+ * "Hardware-aware state expansion").  A long sequence over few channels (see the
+ * workspace size above) is swept in segments side by side: the checkpoints from each
+ * segment's true start, then each segment's adjoint summary and their fold (the
+ * adjoint obeys a linear recurrence backwards in time, so segments combine as the
+ * forward's do), then every segment's sweep from the adjoint entering it.
  *
  *   u, delta, A, B, C, D, z, delta_bias, delta_softplus, dims, in_dtype
  *               : exactly the forward's inputs (same layouts and rules)
