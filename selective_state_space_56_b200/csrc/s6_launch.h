@@ -78,11 +78,12 @@ cudaError_t launch_fold(const float* hend, const float* dsum, const float* A, co
 // Steps per chunk of the forward kernel for state width N.
 int scan_chunk_steps(int64_t N);
 
-// Steps between the backward's checkpoints (a divisor of scan_chunk_steps(N)); the
-// backward recomputes states block by block from them.
+// Steps between the backward's checkpoints: the state entering every group of 4 steps,
+// the unit the reverse sweep recomputes from (so it runs no forward pass of its own).
+constexpr int kCkptSteps = 4;
 int checkpoint_steps(int64_t N);
 
-// Forward pass that writes the state entering every checkpoint block to
+// Forward pass that writes the state entering every checkpoint group to
 // ckpt[((b * dim + d) * blocks + k) * N + n], blocks = ceil(L / checkpoint_steps(N)),
 // and no output.  Uses a.u, delta, A, B, C, delta_bias, softplus, dims and in_dtype.
 // With a.nseg > 1 (a.seg_len a multiple of 64) the segments run side by side from their

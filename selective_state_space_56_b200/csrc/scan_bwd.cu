@@ -2,20 +2,20 @@
 //
 // Mamba ("Hardware-aware state expansion"): the intermediate states are not stored for
 // the backward pass; they are recomputed on chip.  The forward kernel first records
-// only the state entering every 16 steps (checkpoints, one N-vector per channel; every 64
-// steps for N <= 8).  This kernel then walks blocks of T steps of a channel tile in
-// reverse -- T = 16, or 32 (every other checkpoint) when the whole grid is resident at
-// once with the larger shared-memory footprint of 32-step blocks:
+// only the state entering every group of 4 steps (checkpoints, one N-vector per channel
+// and group: N / 4 floats per element, against the N floats of every state).  This kernel
+// then walks blocks of T steps of a channel tile in reverse -- T = 16 for N > 8, or 32
+// when the whole grid is resident at once with the larger shared-memory footprint of
+// 32-step blocks; 64 for N <= 8:
 //
-//   stage     u, delta, z, dy rows and the batch's B, C for the chunk -> shared memory
-//             (16-byte cp.async copies into rows padded against bank conflicts); B, C
-//             then re-laid out per (4-step group, 4-state quad): fp32, or bf16 for bf16
-//             inputs (fewer shared-memory wavefronts for loads all 8 channels repeat);
+//   stage     u, delta, z, dy rows, the batch's B, C and the block's group entry states
+//             for the chunk -> shared memory (16-byte cp.async copies into rows padded
+//             against bank conflicts); B, C then re-laid out per (4-step group, 4-state
+//             quad): fp32, or bf16 for bf16 inputs (fewer shared-memory wavefronts for
+//             loads all 8 channels repeat);
 //   phase A   per (channel, t): Delta = softplus(delta + bias) and the gated output
 //             gradient dyt_t = dy_t silu(z_t) (16-step blocks also keep sigmoid(x) and
 //             sigmoid(z) for the gradients through softplus and the gate);
-//   forward   from the checkpoint, the chunk's states are recomputed; the state
-//             entering every group of 4 steps is kept in shared memory;
 //   reverse   per group of 4 steps, last group first: the group's states and Abar are
 //             recomputed into registers from the group's entry state; then the adjoint
 //             state g (registers) is swept from the group's last step to its first:
@@ -36,7 +36,7 @@
 // State arithmetic runs on packed fp32 pairs (two states per instruction).  Gradients
 // through softplus use softplus'(x) = sigmoid(x); through the gate
 // silu'(z) = sigmoid(z) (1 + z (1 - sigmoid(z))).  Per state and step the kernel
-// evaluates Abar twice (forward and group recompute), the checkpoint pass once.
+// evaluates Abar once (the group recompute), the checkpoint pass once.
 #include <algorithm>
 #include <cstring>
 
@@ -56,7 +56,7 @@ struct BParams {
     const void* C;
     const float* D;
     const float* delta_bias;
-    const float* ckpt;
+    const float* ckpt;  // the state entering every 4-step group: [batch][dim][ck_blocks][N]
     void* du;
     void* ddelta;
     void* dz;
@@ -69,8 +69,8 @@ struct BParams {
     int N;
     int softplus;
     int chunks;     // blocks of T steps this kernel walks
-    int ck_blocks;  // checkpoints per channel (blocks of checkpoint_steps(N))
-    int ck_stride;  // checkpoints per block of T steps
+    int ck_blocks;  // checkpoints per channel, ceil(L / 4)
+    int ck_vec;     // N = 16 and ckpt 16-byte aligned: group states staged by 16-byte copies
     // a sequence split into nseg segments of seg_chunks blocks (grid z = segment): g_carry
     // [nseg][batch][dim][N] holds, per segment, the adjoint its first step carries backwards
     // from the segment alone (the summary pass), then, after the fold, in slot s + 1 the
@@ -210,17 +210,39 @@ __device__ __forceinline__ int red_quad(int q, int ch) { return q ^ (((ch ^ (ch 
 // 4 steps x 8 quads at a time, fall in distinct banks.
 __device__ __forceinline__ int acc_idx(int t, int slot) { return t * 32 + ((slot + (t & 3)) & 31); }
 
-// Stage chunk k's rows into the raw buffer.  Rows past dim, steps past L and a missing z
-// become zeros.  16-byte cp.async copies when rows are 16-byte aligned (then every
-// 16-byte piece is either wholly inside the sequence or wholly past it); plain loads
-// otherwise.
-template <int T, typename Tin>
-__device__ __forceinline__ void stage_chunk(const BParams& p, unsigned char* st, int64_t b,
-                                            int64_t d0, int k, int tid) {
+// Stage chunk k's rows into the raw buffer and, with kStates, the state entering each of
+// its T / 4 groups into sH [T/4][CH][16].  Rows past dim, steps past L, groups past the
+// sequence, states past N and a missing z become zeros.  16-byte cp.async copies when rows
+// are 16-byte aligned (then every 16-byte piece is either wholly inside the sequence or
+// wholly past it), and for the states when N = 16 and the checkpoints are 16-byte aligned;
+// plain loads otherwise.
+template <int T, typename Tin, bool kStates>
+__device__ __forceinline__ void stage_chunk(const BParams& p, unsigned char* st, float* sH,
+                                            int64_t b, int64_t d0, int k, int tid) {
     using Lo = BLayout<T, Tin>;
     constexpr int RR = Lo::RR;
+    constexpr int GT = T / 4;  // groups per block
     const int64_t t0 = (int64_t)k * T;
     const int valid = (int)min((int64_t)T, p.L - t0);
+    if constexpr (kStates) {
+        const int64_t kb0 = (int64_t)k * GT;
+        if (p.ck_vec) {
+            for (int i = tid; i < kBCH * GT * 4; i += kBW * 32) {
+                const int q = i & 3, g = (i >> 2) % GT, c = i / (4 * GT);
+                const bool ok = d0 + c < p.dim && kb0 + g < p.ck_blocks;
+                const float* src = p.ckpt + ((b * p.dim + d0 + c) * p.ck_blocks + kb0 + g) * 16 + 4 * q;
+                cp_async16(sH + (g * kBCH + c) * 16 + 4 * q, ok ? static_cast<const void*>(src) : p.A,
+                           ok ? 16 : 0);
+            }
+        } else {
+            for (int i = tid; i < kBCH * GT * 16; i += kBW * 32) {
+                const int n = i & 15, g = (i >> 4) % GT, c = i / (16 * GT);
+                const bool ok = d0 + c < p.dim && kb0 + g < p.ck_blocks && n < p.N;
+                sH[(g * kBCH + c) * 16 + n] =
+                    ok ? p.ckpt[((b * p.dim + d0 + c) * p.ck_blocks + kb0 + g) * p.N + n] : 0.f;
+            }
+        }
+    }
     if (p.vec) {
         constexpr int E = 16 / sizeof(Tin);  // elements per copy
         constexpr int VPR = T / E;           // copies per row
@@ -263,6 +285,10 @@ __device__ __forceinline__ void stage_chunk(const BParams& p, unsigned char* st,
             Tin v = Tin(0.f);
             if (n < p.N && t < valid) v = src[(b * p.N + n) * p.L + t0 + t];
             reinterpret_cast<Tin*>(st + 4 * Lo::rows + which * Lo::coef)[n * RR + t] = v;
+        }
+        if (kStates && p.ck_vec) {
+            cp_async_commit();
+            cp_async_wait<0>();
         }
     }
 }
@@ -363,7 +389,7 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
         const int64_t t0 = (int64_t)k * T;
         const int valid = (int)min((int64_t)T, p.L - t0);
         __syncthreads();  // the previous chunk's outputs have left the staging rows
-        stage_chunk<T, Tin>(p, st, b, d0, k, tid);
+        stage_chunk<T, Tin, true>(p, st, sH, b, d0, k, tid);
         __syncthreads();  // chunk k staged
 
         if constexpr (sizeof(Tin) == 2) {
@@ -416,57 +442,6 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
             }
         }
         __syncthreads();  // B, C converted, sAcc cleared
-
-        // forward: the state entering every group of four steps
-        {
-            f2 hp[2];
-            {
-                float h[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int n = pp * 4 + j;
-                    h[j] = (chok && n < p.N)
-                               ? p.ckpt[((b * p.dim + dch) * p.ck_blocks +
-                                         (int64_t)k * p.ck_stride) * p.N + n]
-                               : 0.f;
-                }
-                hp[0] = pack2(h[0], h[1]);
-                hp[1] = pack2(h[2], h[3]);
-            }
-                        for (int t = 0; t < T; t += 4) {
-                {
-                    float h0, h1, h2, h3;
-                    unpack2(hp[0], h0, h1);
-                    unpack2(hp[1], h2, h3);
-                    *reinterpret_cast<float4*>(sH + ((t / 4) * kBCH + cw) * 16 + pp * 4) =
-                        make_float4(h0, h1, h2, h3);
-                }
-                const float4 d4 = lds4(sDel + cw * RS + t);
-                float uv[4];
-                V4::to_f(*reinterpret_cast<const VT*>(rU + cw * RR + t), uv);
-                const float dts[4] = {d4.x, d4.y, d4.z, d4.w};
-                Coef<Tin> bq;
-                bq.load(sB, t, pp);
-#pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    const f2 dd = pack2(dts[s], dts[s]);
-                    const float q = dts[s] * uv[s];
-                    const f2 qq = pack2(q, q);
-                    const f2x2 bb = bq.at(s);
-                    const f2 x0 = mul2(dd, a2p[0]), x1 = mul2(dd, a2p[1]);
-                    const f2 e0 = ex2x2(x0), e1 = ex2x2(x1);
-                    if constexpr (ZOH) {  // input weight u w, w = expm1(Delta A) / A
-                        const f2 uu = pack2(uv[s], uv[s]);
-                        hp[0] = fma2(e0, hp[0], mul2(zoh_weight_u2(x0, e0, invp[0], uu, qq), bb.lo));
-                        hp[1] = fma2(e1, hp[1], mul2(zoh_weight_u2(x1, e1, invp[1], uu, qq), bb.hi));
-                    } else {
-                        hp[0] = fma2(e0, hp[0], mul2(qq, bb.lo));
-                        hp[1] = fma2(e1, hp[1], mul2(qq, bb.hi));
-                    }
-                }
-            }
-        }
-        __syncwarp();
 
         // reverse sweep, one group of four steps at a time (last group first)
                 for (int tg = T - 4; tg >= 0; tg -= 4) {
@@ -762,7 +737,7 @@ __global__ void __launch_bounds__(kBW * 32) adjoint_summary_kernel(const BParams
         const int64_t t0 = (int64_t)k * T;
         const int valid = (int)min((int64_t)T, p.L - t0);
         __syncthreads();  // the previous chunk's rows are no longer read
-        stage_chunk<T, Tin>(p, st, b, d0, k, tid);
+        stage_chunk<T, Tin, false>(p, st, nullptr, b, d0, k, tid);
         __syncthreads();
         if constexpr (sizeof(Tin) == 2) {  // C to the bf16 blocks the sweep's loads read
             for (int i = tid; i < 4 * T; i += kBW * 32) {
@@ -924,7 +899,8 @@ void backward_segments(int64_t batch, int64_t dim, int64_t L, int64_t* nseg, int
 
 cudaError_t launch_scan_backward(const ScanArgs& a_in, const BackwardArgs& g, float* ckpt,
                                  cudaStream_t stream, bool ckpt_ready) {
-    // checkpoints every CK steps; the kernel walks blocks of T = CK (or 2 CK) steps
+    // checkpoints every CK = 4 steps; the kernel walks blocks of T = 16 or 32 steps (N > 8)
+    // or 64 (N <= 8)
     const int CK = checkpoint_steps(a_in.N);
     // a long sequence over few channels is swept in segments (the workspace holds their
     // summaries after the checkpoints)
@@ -941,8 +917,8 @@ cudaError_t launch_scan_backward(const ScanArgs& a_in, const BackwardArgs& g, fl
         a.seg_sum = seg_sum;
     }
     const int64_t ctas = (a.dim + kBCH - 1) / kBCH * a.batch * nseg;
-    int T = CK;
-    if (a.N > 8 && CK == 16)
+    int T = 64;
+    if (a.N > 8)
         T = a.in_dtype == DType::BF16
                 ? (a.zoh ? pick_block_steps<__nv_bfloat16, true>(ctas)
                          : pick_block_steps<__nv_bfloat16, false>(ctas))
@@ -989,7 +965,7 @@ cudaError_t launch_scan_backward(const ScanArgs& a_in, const BackwardArgs& g, fl
     bp.softplus = a.softplus ? 1 : 0;
     bp.chunks = (int)chunks;
     bp.ck_blocks = (int)((a.L + CK - 1) / CK);
-    bp.ck_stride = T / CK;
+    bp.ck_vec = (a.N == 16 && reinterpret_cast<uintptr_t>(ckpt) % 16 == 0) ? 1 : 0;
     bp.nseg = (int)nseg;
     bp.seg_chunks = nseg > 1 ? (int)(seg_len / T) : (int)chunks;
     bp.g_carry = seg_h;

@@ -622,30 +622,39 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         float* sDuK = sDu + (WS == 2 ? (k & 1) * Lo::dq_stride : 0);
         if constexpr (WS != 2) phase_a(k, warp * CW, CW * (T / 4), lane, 32, sDelK, sDuK);
 
-        // checkpoint mode: the state entering every CKPT-step block of the sequence,
-        // ckpt[((b * dim + d) * blocks + kb) * N + n], blocks = ceil(L / CKPT)
-        constexpr int CKPT = NMAX == 16 ? 16 : T;
+        // checkpoint modes: the state entering every 4-step group of the sequence,
+        // ckpt[((b * dim + d) * blocks + kb) * N + n], blocks = ceil(L / 4) -- what the
+        // backward's reverse sweep starts each group from, so it recomputes no other state
         auto write_ckpt = [&](int t) {
-            const int64_t blocks = (p.L + CKPT - 1) / CKPT;
-            const int64_t kb = (t0 + t) / CKPT;
+            const int64_t blocks = (p.L + kCkptSteps - 1) / kCkptSteps;
+            const int64_t kb = (t0 + t) / kCkptSteps;
             if (dch >= p.dim || t0 + t >= p.L) return;
-            float* ck = p.ckpt + ((b * p.dim + dch) * blocks + kb) * p.N;
+            float* ck = p.ckpt + ((b * p.dim + dch) * blocks + kb) * p.N + pp * NS;
+            if (NS % 4 == 0 && p.N == NMAX && (reinterpret_cast<uintptr_t>(ck) & 15) == 0) {
+#pragma unroll
+                for (int j = 0; j < NS / 2; j += 2) {
+                    float h0, h1, h2, h3;
+                    unpack2(hp[0][j], h0, h1);
+                    unpack2(hp[0][j + 1], h2, h3);
+                    *reinterpret_cast<float4*>(ck + 2 * j) = make_float4(h0, h1, h2, h3);
+                }
+                return;
+            }
 #pragma unroll
             for (int j = 0; j < NS / 2; ++j) {
                 float h0, h1;
                 unpack2(hp[0][j], h0, h1);
-                if (pp * NS + 2 * j < p.N) ck[pp * NS + 2 * j] = h0;
-                if (pp * NS + 2 * j + 1 < p.N) ck[pp * NS + 2 * j + 1] = h1;
+                if (pp * NS + 2 * j < p.N) ck[2 * j] = h0;
+                if (pp * NS + 2 * j + 1 < p.N) ck[2 * j + 1] = h1;
             }
         };
-        if (kCk) write_ckpt(0);
 
         // Phase B: the recurrence, four steps per iteration, states in packed pairs.
         f2 ee_next[4][NS / 2];  // the lookahead's Abar of the next group (S6_PIPE)
         float yp8[CPL][8];      // P = 8: partial outputs of two groups for one transpose-reduce
 #pragma unroll
         for (int t = 0; t < T; t += 4) {
-            if (kCk && t > 0 && t % CKPT == 0) write_ckpt(t);
+            if (kCk) write_ckpt(t);
             float4 d4[CPL], q4[CPL];
 #pragma unroll
             for (int k = 0; k < CPL; ++k) {
@@ -1328,7 +1337,7 @@ int scan_chunk_steps(int64_t N) {
     return Tile<16>::T;
 }
 
-int checkpoint_steps(int64_t N) { return N <= 8 ? scan_chunk_steps(N) : 16; }
+int checkpoint_steps(int64_t) { return kCkptSteps; }
 
 cudaError_t launch_scan_checkpoints(const ScanArgs& a, float* ckpt, cudaStream_t stream) {
     KParams kp;

@@ -182,13 +182,13 @@ def test_bwd_dims_dtype_align_workspace(lib):
     assert _bwd(lib, ws=A16 + 8, wsb=need) == ERR_ALIGN
 
 
-def test_bwd_workspace_is_one_checkpoint_per_chunk(lib):
+def test_bwd_workspace_is_one_checkpoint_per_group(lib):
     ws = lambda *d: lib.mamba_selective_scan_bwd_workspace_size(_dims(*d))  # noqa: E731
-    # 16-step blocks for dstate > 8, 64-step blocks otherwise; fp32 states
-    assert ws(4, 5120, 16, 4096) == 4 * 5120 * 256 * 16 * 4
-    assert ws(2, 64, 16, 33) == 2 * 64 * 3 * 16 * 4
-    assert ws(2, 64, 8, 64) == 2 * 64 * 1 * 8 * 4
-    assert ws(1, 3, 5, 65) == (1 * 3 * 2 * 5 * 4 + 255) // 256 * 256
+    # the state entering every group of 4 steps, fp32, for every dstate
+    assert ws(4, 5120, 16, 4096) == 4 * 5120 * 1024 * 16 * 4
+    assert ws(2, 64, 16, 33) == 2 * 64 * 9 * 16 * 4
+    assert ws(2, 64, 8, 64) == 2 * 64 * 16 * 8 * 4
+    assert ws(1, 3, 5, 65) == (1 * 3 * 17 * 5 * 4 + 255) // 256 * 256
     assert ws(2, 64, 16, 0) == 0
     assert ws(2, 64, 17, 8) == 0
 
@@ -201,11 +201,11 @@ def test_bwd_workspace_of_a_split_sequence(lib):
     segments of 95,360 steps."""
     ws = lambda *d: lib.mamba_selective_scan_bwd_workspace_size(_dims(*d))  # noqa: E731
     b, d, N, L = 1, 2048, 16, 1 << 20
-    ck = (b * d * (L // 16) * N + 63) // 64 * 64
+    ck = (b * d * (L // 4) * N + 63) // 64 * 64
     assert ws(b, d, N, L) == ((ck + 11 * b * d * (N + 1)) * 4 + 255) // 256 * 256
     # enough channels (640 CTAs for the 2.8B-shaped layer), or a short sequence: no split
-    assert ws(4, 5120, 16, 1 << 15) == 4 * 5120 * (1 << 11) * 16 * 4
-    assert ws(1, 64, 16, 8192) == 64 * 512 * 16 * 4
+    assert ws(4, 5120, 16, 1 << 15) == 4 * 5120 * (1 << 13) * 16 * 4
+    assert ws(1, 64, 16, 8192) == 64 * 2048 * 16 * 4
 
 
 ERR_FLAGS = -8
