@@ -11,8 +11,8 @@
 //   stage     u, delta, z, dy rows, the batch's B, C and the block's group entry states
 //             for the chunk -> shared memory (16-byte cp.async copies into rows padded
 //             against bank conflicts); B, C then re-laid out per (4-step group, 4-state
-//             quad): fp32, or bf16 for bf16 inputs (fewer shared-memory wavefronts for
-//             loads all 8 channels repeat);
+//             quad): fp32, or bf16 for bf16 inputs of the Delta * B sweep (fewer
+//             shared-memory wavefronts for loads all 8 channels repeat);
 //   phase A   per (channel, t): Delta = softplus(delta + bias) and the gated output
 //             gradient dyt_t = dy_t silu(z_t) (16-step blocks also keep sigmoid(x) and
 //             sigmoid(z) for the gradients through softplus and the gate);
@@ -39,6 +39,7 @@
 // evaluates Abar once (the group recompute), the checkpoint pass once.
 #include <algorithm>
 #include <cstring>
+#include <type_traits>
 
 #include "s6_device.cuh"
 #include "s6_launch.h"
@@ -319,8 +320,17 @@ __device__ __forceinline__ f2 zoh_dw_da2(f2 x, f2 e, f2 w, f2 inv_a, f2 dd) {
     return pack2(fabsf(x0) < kTau ? s0 : l0, fabsf(x1) < kTau ? s1 : l1);
 }
 
+// The exact-ZOH sweep keeps more per-state values live (the weight and its derivatives):
+// held to 96 registers (five CTAs per SM) it spills, at 128 (four CTAs) it does not, and
+// there it reads B and C from fp32 tiles, which need no widening.  Measured on the
+// 2.8B-shaped layer: exact-ZOH backward 5276 -> 4846 us; the Delta * B sweep is fastest
+// with bf16 blocks at five CTAs per SM (2940 us, against 3027 with fp32 tiles and 3505 at
+// four CTAs per SM).
+template <bool ZOH> constexpr int bwd_min_blocks() { return ZOH ? 4 : 5; }
+template <typename Tin, bool ZOH> constexpr bool bwd_bf16_coef() { return sizeof(Tin) == 2 && !ZOH; }
+
 template <int T, typename Tin, bool ZOH>
-__global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) {
+__global__ void __launch_bounds__(kBW * 32, bwd_min_blocks<ZOH>()) scan_bwd_kernel(const BParams p) {
     using Lo = BLayout<T, Tin>;
     constexpr int RS = Lo::RS, RR = Lo::RR;
     using V4 = vec4<Tin>;
@@ -392,7 +402,7 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
         stage_chunk<T, Tin, true>(p, st, sH, b, d0, k, tid);
         __syncthreads();  // chunk k staged
 
-        if constexpr (sizeof(Tin) == 2) {
+        if constexpr (bwd_bf16_coef<Tin, ZOH>()) {
             // B and C to bf16 blocks [t / 4][quad][t % 4][4 states], one (step, quad) per item
             for (int i = tid; i < 2 * 4 * T; i += kBW * 32) {
                 const int which = i / (4 * T), t = (i / 4) % T, pq = i % 4;
@@ -453,7 +463,7 @@ __global__ void __launch_bounds__(kBW * 32, 5) scan_bwd_kernel(const BParams p) 
             const f2 hin[2] = {lo2(h4), hi2(h4)};
             // the group's Abar and states, recomputed into registers
             f2 ab[4][2], hs[4][2];
-            Coef<Tin> bq, cq;
+            Coef<typename std::conditional<bwd_bf16_coef<Tin, ZOH>(), __nv_bfloat16, float>::type> bq, cq;
             bq.load(sB, tg, pp);
 #pragma unroll
             for (int s = 0; s < 4; ++s) {

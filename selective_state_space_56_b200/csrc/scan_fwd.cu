@@ -385,16 +385,18 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
     auto issue_chunk = [&](int64_t k) {  // TMA: called by one thread
         unsigned char* st = smem + (k & 1) * Lo::stage_bytes;
         const int tt = (int)(t_begin + k * T);
-        // the correction has no input: neither u nor B is needed
+        // the correction has no input: neither u nor B is needed; the passes without
+        // output (checkpoints, segment summaries) need no C
         const uint32_t bytes = kCorrM ? (uint32_t)((has_z ? 2 : 1) * Lo::rows_bytes + Lo::coef_bytes)
-                                      : (uint32_t)((has_z ? 3 : 2) * Lo::rows_bytes + 2 * Lo::coef_bytes);
+                                      : (uint32_t)((has_z ? 3 : 2) * Lo::rows_bytes +
+                                                   (kOut ? 2 : 1) * Lo::coef_bytes);
         uint64_t* bk = &bar[k & 1];
         mbar_arrive_expect_tx(bk, bytes);
         if (!kCorrM) tma_load_3d(st, &tm.u, tt, (int)d0, (int)b, bk);
         tma_load_3d(st + Lo::off_dr, &tm.dr, tt, (int)d0, (int)b, bk);
         if (has_z) tma_load_3d(st + Lo::off_z, &tm.z, tt, (int)d0, (int)b, bk);
         if (!kCorrM) tma_load_3d(st + Lo::off_B, &tm.B, tt, 0, (int)b, bk);
-        tma_load_3d(st + Lo::off_C, &tm.C, tt, 0, (int)b, bk);
+        if (kOut) tma_load_3d(st + Lo::off_C, &tm.C, tt, 0, (int)b, bk);
     };
     auto load_chunk_elementwise = [&](int64_t k) {  // rows not 16-byte multiples
         unsigned char* st = smem + (k & 1) * Lo::stage_bytes;
@@ -434,7 +436,7 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         // B, C of the chunk, time-major: every lane then reads the coefficients of its four
         // states for step t with one 16-byte load (bf16: B[4] and C[4] as pairs; fp32: a
         // 16-byte vector from each of two tiles, transposed through 4x4 register blocks).
-        if constexpr (Lo::kBC == 1 || Lo::kBC == 2) {
+        if constexpr (Lo::kBC == 1 || (Lo::kBC == 2 && kOut)) {
             // bf16 pairs.  Format 1: per (step, 4-state group) [B0|B1][B2|B3][C0|C1][C2|C3];
             // format 2: the C half only, [C0|C1][C2|C3] per (step, group), after the B tile.
             // Work item: (4-state group, step pair, B or C) -> two 8-byte half-groups.
@@ -463,8 +465,9 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
             }
         }
         if constexpr (Lo::kBC == 0 || Lo::kBC == 2) {
-            // fp32 tiles [T][NMAX], transposed through 4x4 register blocks
-            constexpr int kTiles = Lo::kBC == 0 ? 2 : 1;
+            // fp32 tiles [T][NMAX], transposed through 4x4 register blocks (C only for the
+            // passes with output)
+            constexpr int kTiles = Lo::kBC == 0 && kOut ? 2 : 1;
             for (int i = first; i < (NMAX / 4) * (T / 4) * kTiles; i += stride) {
                 const int which = kTiles == 2 ? (i & 1) : 0;
                 const int i2 = kTiles == 2 ? (i >> 1) : i;
