@@ -15,6 +15,7 @@
 // the halo of the second vector in registers, computes in fp32 and stores 16 bytes per
 // vector.  The grid is (vector blocks, dim, batch), so no thread divides to find its row.
 // Rows whose length is not a multiple of the vector take an element-wise path.
+#include <algorithm>
 #include <cstring>
 
 #include "s6_device.cuh"
@@ -214,6 +215,14 @@ __device__ __forceinline__ float dsilu(float p) {
     const float sg = rcp(1.f + ex2(-p * kLog2e));
     return sg * fmaf(p, 1.f - sg, 1.f);
 }
+// The same on a packed pair (each half rounded exactly as dsilu rounds it).
+__device__ __forceinline__ f2 dsilu2(f2 p) {
+    const f2 e = ex2x2(mul2(p, pack2(-kLog2e, -kLog2e)));
+    float d0, d1;
+    unpack2(add2(e, pack2(1.f, 1.f)), d0, d1);
+    const f2 sg = pack2(rcp(d0), rcp(d1));
+    return mul2(sg, fma2(p, sub2(pack2(1.f, 1.f), sg), pack2(1.f, 1.f)));
+}
 
 // Input at position s of row r of init ++ x (zero before init).
 template <typename T>
@@ -247,15 +256,31 @@ __device__ __forceinline__ void cta_add(const CBParams& p, int64_t d, float (&pa
     __syncthreads();  // red is reused by the next row
 }
 
-// Rows of 16-byte multiples.  Grid (vector blocks, min(dim, 65535), min(batch, 65535));
-// each CTA walks rows (d, b) with strides gridDim.y, gridDim.z.
+// Rows of 16-byte multiples.  Grid (vector blocks, min(dim, 65535), batch slices); each CTA
+// walks channels d with stride gridDim.y and, for each, the batch rows b with stride
+// gridDim.z, carrying its dweight / dbias partial sums across those rows and reducing them
+// once per channel.  Steps go in packed pairs (two independent fp32 lanes per instruction,
+// so every element is rounded as in the scalar form; only the order in which a thread's
+// partial sums are added differs).
 #ifndef S6_CONVB_VPT
 #define S6_CONVB_VPT 2
 #endif
 constexpr int kVPTB = S6_CONVB_VPT;  // 16-byte dx vectors per thread in the backward
 
+// Register budget of the vector kernel: four CTAs of 256 threads per SM (64 registers, a
+// 24-byte spill) measured faster than the compiler's own choice (76 registers, three CTAs):
+// 125.3 against 129.4 us for the 2.8B-shaped layer's conv (149.9 us before the packed
+// pairs and the per-channel reduction).  0 leaves the choice to the compiler.
+#ifndef S6_CONVB_MINB
+#define S6_CONVB_MINB 4
+#endif
+#if S6_CONVB_MINB > 0
+#define S6_CONVB_BOUNDS __launch_bounds__(256, S6_CONVB_MINB)
+#else
+#define S6_CONVB_BOUNDS __launch_bounds__(256)
+#endif
 template <typename T, int K, bool SILU>
-__global__ void __launch_bounds__(256) conv1d_bwd_vec_kernel(const CBParams p) {
+__global__ void S6_CONVB_BOUNDS conv1d_bwd_vec_kernel(const CBParams p) {
     constexpr int kVPT = kVPTB;
     constexpr int E = 16 / sizeof(T);
     constexpr int NT = kVPT * E;  // steps of this thread
@@ -265,14 +290,19 @@ __global__ void __launch_bounds__(256) conv1d_bwd_vec_kernel(const CBParams p) {
     const bool active = v0 < vpr;
     for (int64_t d = blockIdx.y; d < p.dim; d += gridDim.y) {
         float w[K];
+        f2 w2[K];
 #pragma unroll
-        for (int k = 0; k < K; ++k) w[k] = __ldg(p.w + d * K + k);
+        for (int k = 0; k < K; ++k) {
+            w[k] = __ldg(p.w + d * K + k);
+            w2[k] = pack2(w[k], w[k]);
+        }
         const float bias = p.bias ? __ldg(p.bias + d) : 0.f;
+        const f2 bias2 = pack2(bias, bias);
+        f2 part2[K + 1];  // even and odd steps of every batch row of this channel
+#pragma unroll
+        for (int k = 0; k <= K; ++k) part2[k] = pack2(0.f, 0.f);
         for (int64_t b = blockIdx.z; b < p.batch; b += gridDim.z) {
             const int64_t r = b * p.dim + d;
-            float part[K + 1];
-#pragma unroll
-            for (int k = 0; k <= K; ++k) part[k] = 0.f;
             if (active) {
                 const T* xr = static_cast<const T*>(p.x) + r * p.L;
                 const T* gr = static_cast<const T*>(p.dout) + r * p.L;
@@ -309,26 +339,33 @@ __global__ void __launch_bounds__(256) conv1d_bwd_vec_kernel(const CBParams p) {
                     xs[K - 1 + NT + j] = io<T>::to_f(reinterpret_cast<const T*>(&xv[kVPT + 1])[j]);
                     gs[NT + j] = io<T>::to_f(reinterpret_cast<const T*>(&gv[kVPT])[j]);
                 }
-                // g over steps s0 .. s0 + NT + K - 2 (zero past the row: those dout are zero)
-                float g[NT + K - 1];
+                // g over steps s0 .. s0 + NT + K - 2 (zero past the row: those dout are zero),
+                // two steps per packed pair
+                constexpr int NG = NT + K - 1;
+                float g[NG];
 #pragma unroll
-                for (int j = 0; j < NT + K - 1; ++j) {
+                for (int j = 0; j + 1 < NG; j += 2) {
+                    f2 pre = bias2;
+#pragma unroll
+                    for (int k = 0; k < K; ++k) pre = fma2(w2[k], pack2(xs[j + k], xs[j + k + 1]), pre);
+                    f2 gg = pack2(gs[j], gs[j + 1]);
+                    if (SILU) gg = mul2(gg, dsilu2(pre));
+                    unpack2(gg, g[j], g[j + 1]);
+                }
+                if constexpr (NG % 2 == 1) {
                     float pre = bias;
 #pragma unroll
-                    for (int k = 0; k < K; ++k) pre = fmaf(w[k], xs[j + k], pre);
-                    g[j] = SILU ? gs[j] * dsilu(pre) : gs[j];
+                    for (int k = 0; k < K; ++k) pre = fmaf(w[k], xs[NG - 1 + k], pre);
+                    g[NG - 1] = SILU ? gs[NG - 1] * dsilu(pre) : gs[NG - 1];
                 }
-                // this thread's share of dw and dbias (its own steps only)
+                // this thread's share of dw and dbias (its own steps; past the row g and x
+                // are zero and add nothing)
 #pragma unroll
-                for (int i = 0; i < kVPT; ++i) {
-                    if (v0 + i >= vpr) break;
+                for (int t = 0; t < NT; t += 2) {
+                    const f2 gg = pack2(g[t], g[t + 1]);
 #pragma unroll
-                    for (int j = 0; j < E; ++j) {
-                        const int t = i * E + j;
-#pragma unroll
-                        for (int k = 0; k < K; ++k) part[k] = fmaf(g[t], xs[t + k], part[k]);
-                        part[K] += g[t];
-                    }
+                    for (int k = 0; k < K; ++k) part2[k] = fma2(gg, pack2(xs[t + k], xs[t + k + 1]), part2[k]);
+                    part2[K] = add2(part2[K], gg);
                 }
                 // dx[s0 + t] = sum_k w[k] g[t + K-1-k]
 #pragma unroll
@@ -336,12 +373,16 @@ __global__ void __launch_bounds__(256) conv1d_bwd_vec_kernel(const CBParams p) {
                     if (v0 + i >= vpr) break;
                     alignas(16) T o[E];
 #pragma unroll
-                    for (int j = 0; j < E; ++j) {
+                    for (int j = 0; j < E; j += 2) {
                         const int t = i * E + j;
-                        float acc = 0.f;
+                        f2 acc = pack2(0.f, 0.f);
 #pragma unroll
-                        for (int k = 0; k < K; ++k) acc = fmaf(w[k], g[t + K - 1 - k], acc);
-                        o[j] = io<T>::from_f(acc);
+                        for (int k = 0; k < K; ++k)
+                            acc = fma2(w2[k], pack2(g[t + K - 1 - k], g[t + K - k]), acc);
+                        float a0, a1;
+                        unpack2(acc, a0, a1);
+                        o[j] = io<T>::from_f(a0);
+                        o[j + 1] = io<T>::from_f(a1);
                     }
                     *reinterpret_cast<uint4*>(static_cast<T*>(p.dx) + r * p.L + (v0 + i) * E) =
                         *reinterpret_cast<const uint4*>(o);
@@ -357,12 +398,20 @@ __global__ void __launch_bounds__(256) conv1d_bwd_vec_kernel(const CBParams p) {
                     }
                 }
             }
-            cta_add<K>(p, d, part, red);
         }
+        float part[K + 1];
+#pragma unroll
+        for (int k = 0; k <= K; ++k) {
+            float lo, hi;
+            unpack2(part2[k], lo, hi);
+            part[k] = lo + hi;
+        }
+        cta_add<K>(p, d, part, red);
     }
 }
 
-// Any row length: one step per thread, the K values of g it needs formed from K x each.
+// Any row length: one step per thread, the K values of g it needs formed from K x each;
+// dweight / dbias partial sums carried across the batch rows of a channel as above.
 template <typename T, int K, bool SILU>
 __global__ void __launch_bounds__(256) conv1d_bwd_elem_kernel(const CBParams p) {
     __shared__ float red[8 * (K + 1)];
@@ -373,11 +422,11 @@ __global__ void __launch_bounds__(256) conv1d_bwd_elem_kernel(const CBParams p) 
 #pragma unroll
         for (int k = 0; k < K; ++k) w[k] = __ldg(p.w + d * K + k);
         const float bias = p.bias ? __ldg(p.bias + d) : 0.f;
+        float part[K + 1];
+#pragma unroll
+        for (int k = 0; k <= K; ++k) part[k] = 0.f;
         for (int64_t b = blockIdx.z; b < p.batch; b += gridDim.z) {
             const int64_t r = b * p.dim + d;
-            float part[K + 1];
-#pragma unroll
-            for (int k = 0; k <= K; ++k) part[k] = 0.f;
             if (active) {
                 // g at steps s .. s + K - 1 (zero past the row)
                 float g[K];
@@ -395,7 +444,7 @@ __global__ void __launch_bounds__(256) conv1d_bwd_elem_kernel(const CBParams p) 
                 }
 #pragma unroll
                 for (int k = 0; k < K; ++k) part[k] = fmaf(g[0], xb_at<T>(p, r, s - (K - 1) + k, K), part[k]);
-                part[K] = g[0];
+                part[K] += g[0];
                 float acc = 0.f;
 #pragma unroll
                 for (int k = 0; k < K; ++k) acc = fmaf(w[k], g[K - 1 - k], acc);
@@ -410,8 +459,8 @@ __global__ void __launch_bounds__(256) conv1d_bwd_elem_kernel(const CBParams p) 
                     }
                 }
             }
-            cta_add<K>(p, d, part, red);
         }
+        cta_add<K>(p, d, part, red);
     }
 }
 
@@ -498,17 +547,32 @@ cudaError_t launch_conv1d_update(const ConvUpdateArgs& a, cudaStream_t stream) {
 
 namespace {
 
+// Batch slices of the grid: one (each CTA walks every batch row of its channels, reducing
+// dweight / dbias once per channel) unless the channels and row blocks alone give fewer
+// than 8 CTAs per SM.
+unsigned batch_slices(int64_t xy_ctas, int64_t batch) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        sms = 148;
+    const int64_t want = 8 * (int64_t)sms;
+    int64_t gz = xy_ctas >= want ? 1 : (want + xy_ctas - 1) / xy_ctas;
+    gz = std::min<int64_t>(std::min<int64_t>(gz, batch), 65535);
+    return (unsigned)std::max<int64_t>(gz, 1);
+}
+
 template <typename T, int K, bool SILU>
 cudaError_t launch_conv_bwd_ks(const CBParams& p, int64_t L, cudaStream_t s) {
     constexpr int E = 16 / sizeof(T);
     const unsigned gy = (unsigned)(p.dim < 65535 ? p.dim : 65535);
-    const unsigned gz = (unsigned)(p.batch < 65535 ? p.batch : 65535);
     if (L % E == 0 && K - 1 <= E) {
         const int64_t vpr = L / E;
-        const dim3 grid((unsigned)((vpr + 256 * kVPTB - 1) / (256 * kVPTB)), gy, gz);
+        const unsigned gx = (unsigned)((vpr + 256 * kVPTB - 1) / (256 * kVPTB));
+        const dim3 grid(gx, gy, batch_slices((int64_t)gx * gy, p.batch));
         conv1d_bwd_vec_kernel<T, K, SILU><<<grid, 256, 0, s>>>(p);
     } else {
-        const dim3 grid((unsigned)((L + 255) / 256), gy, gz);
+        const unsigned gx = (unsigned)((L + 255) / 256);
+        const dim3 grid(gx, gy, batch_slices((int64_t)gx * gy, p.batch));
         conv1d_bwd_elem_kernel<T, K, SILU><<<grid, 256, 0, s>>>(p);
     }
     return cudaGetLastError();
