@@ -254,8 +254,9 @@ int mamba_selective_scan_fwd_noalloc(const void* u, const void* delta, const flo
 
 /*
  * Bytes of device workspace mamba_selective_scan_bwd needs for `dims`: the checkpoints,
- * batch x dim x ceil(seqlen / T) x dstate floats (T = 16 steps for dstate > 8 and 64
- * otherwise), rounded up to 64 floats; plus, when a long sequence over few channels is
+ * the state entering every group of 4 steps, batch x dim x ceil(seqlen / 4) x dstate
+ * floats (16 bytes per (batch, channel, step) at dstate = 16), rounded up to 64 floats;
+ * plus, when a long sequence over few channels is
  * swept in S segments side by side (seqlen >= 16384 and fewer CTAs of 32 channels than two
  * per SM of the current device; S up to five CTAs per SM, segments of at least 4096 steps),
  * S x batch x dim x (dstate + 1) floats for the segments' summaries.  Rounded up to 256
@@ -308,8 +309,8 @@ int mamba_selective_scan_bwd(const void* u, const void* delta, const float* A, c
 
 /*
  * Training forward: mamba_selective_scan_fwd that also records the backward's checkpoints
- * (the state entering every 16 steps for dstate > 8, every 64 otherwise -- the layout the
- * backward's own recomputing pass writes), so that a following
+ * (the state entering every group of 4 steps -- the layout the backward's own
+ * recomputing pass writes), so that a following
  * mamba_selective_scan_bwd_from_checkpoints needs no forward pass of its own.
  *
  *   checkpoints      : device buffer of at least mamba_selective_scan_bwd_workspace_size(dims)
