@@ -12,10 +12,13 @@ compared to 1e-5 relative.  A sequence long enough to be split has its segment s
 folded from segment summaries in the training forward but recomputed straight through by
 the backward's own pass, so the states -- and the gradients that depend on them -- agree
 to rounding there (du, which depends on no state, still bit for bit)."""
+import numpy as np
 import pytest
 import torch
 
+import oracle
 from selective_state_space_56_b200 import inputs, ops
+from tests.s6_compare import check_fp32, check_rms
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -81,3 +84,33 @@ def test_training_forward_rejects_zoh_and_initial_state(cuda_ok):
     with pytest.raises(ValueError):
         ops.selective_scan_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], checkpoints=ck,
                                exact_zoh=True)
+
+
+@pytest.mark.parametrize("shape,dtype", [((2, 40, 16, 200), torch.float32),
+                                         ((2, 24, 16, 77), torch.bfloat16),
+                                         ((1, 16, 5, 130), torch.float32)],
+                         ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
+def test_checkpoints_are_the_group_entry_states(cuda_ok, shape, dtype):
+    """The recorded checkpoints are the layout the header documents: per (batch, channel)
+    the state entering every group of 4 steps, ckpt[b, d, g, n] = h_{4g-1} (zero for g = 0),
+    fp32, batch x dim x ceil(L / 4) x N.  Compared with the oracle's states under the
+    last_state tolerances (fp32 inputs per element, bf16 inputs against the RMS)."""
+    b, d, N, L = shape
+    p = inputs.scan_inputs(b, d, N, L, dtype, seed=4 * L + N)
+    g = {k: (None if v is None else v.to(DEV)) for k, v in p.items()}
+    ck = torch.zeros(ops.selective_scan_bwd_workspace_size(b, d, N, L), dtype=torch.uint8,
+                     device=DEV)
+    ops.selective_scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D=g["D"], z=g["z"],
+                           delta_bias=g["delta_bias"], checkpoints=ck)
+    torch.cuda.synchronize()
+    G = (L + 3) // 4
+    got = ck[: b * d * G * N * 4].view(torch.float32).reshape(b, d, G, N)
+    _, _, hs = oracle.selective_scan(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"],
+                                     z=p["z"], delta_bias=p["delta_bias"], return_states=True)
+    ref = np.zeros((b, d, G, N))
+    ref[:, :, 1:, :] = hs[:, :, 3:4 * (G - 1):4, :]
+    assert float(got[:, :, 0].abs().max()) == 0.0
+    if dtype == torch.float32:
+        check_fp32(got, ref, "checkpoints")
+    else:
+        check_rms(got, ref, "checkpoints")
