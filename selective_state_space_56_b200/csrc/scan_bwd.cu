@@ -713,19 +713,82 @@ __global__ void __launch_bounds__(kBW * 32, bwd_min_blocks<ZOH>()) scan_bwd_kern
 // a zero adjoint (last step first: g += dyt C, then g *= Abar), and the segment's summed
 // steps.  The adjoint recurrence involves no state, so nothing is recomputed and no
 // gradient is formed; the input weight does not enter it either (Delta * B or exact ZOH).
+// It reads only delta, z, dy and C, through a ring of kSumBufs staging buffers: the copies
+// of the next kSumBufs - 1 blocks are in flight while a block is swept (its work per step
+// is small next to a copy's latency).
+constexpr int kSumBufs = 3;
+template <int T, typename Tin>
+struct SLayout {
+    static constexpr int RR = BLayout<T, Tin>::RR;  // raw row stride, as the sweep's
+    static constexpr int RS = BLayout<T, Tin>::RS;
+    static constexpr size_t rows = (size_t)kBCH * RR * sizeof(Tin);  // one [CH][RR] set
+    static constexpr size_t coef = (size_t)16 * RR * sizeof(Tin);    // C rows
+    static constexpr size_t stage = a16(3 * rows + coef);            // delta, z, dy, C
+    static constexpr size_t off_C = kSumBufs * stage;                // C, as the sweep's tile
+    static constexpr size_t off_del = off_C + (size_t)T * 16 * 4;
+    static constexpr size_t off_dyt = off_del + (size_t)kBCH * RS * 4;
+    static constexpr size_t bytes = off_dyt + (size_t)kBCH * RS * 4;
+};
+
+// Issue block k's delta, z, dy rows and C into one staging buffer (16-byte cp.async, one
+// commit group) when rows are 16-byte aligned; plain loads and stores otherwise.
+template <int T, typename Tin>
+__device__ __forceinline__ void stage_summary(const BParams& p, unsigned char* st, int64_t b,
+                                              int64_t d0, int k, int tid) {
+    using SL = SLayout<T, Tin>;
+    constexpr int RR = SL::RR;
+    const int64_t t0 = (int64_t)k * T;
+    const int valid = (int)min((int64_t)T, p.L - t0);
+    if (p.vec) {
+        constexpr int E = 16 / sizeof(Tin);
+        constexpr int VPR = T / E;
+        constexpr int NROW = 3 * kBCH + 16;
+        for (int i = tid; i < NROW * VPR; i += kBW * 32) {
+            const int row = i / VPR, col = (i % VPR) * E;
+            const Tin* src;
+            Tin* dst;
+            bool ok;
+            if (row < 3 * kBCH) {
+                const int which = row / kBCH, r = row % kBCH;
+                src = static_cast<const Tin*>(which == 0 ? p.delta : which == 1 ? p.z : p.dy);
+                ok = src != nullptr && d0 + r < p.dim && col < valid;
+                if (ok) src += (b * p.dim + d0 + r) * p.L + t0 + col;
+                dst = reinterpret_cast<Tin*>(st + which * SL::rows) + r * RR + col;
+            } else {
+                const int n = row - 3 * kBCH;
+                src = static_cast<const Tin*>(p.C);
+                ok = n < p.N && col < valid;
+                if (ok) src += (b * p.N + n) * p.L + t0 + col;
+                dst = reinterpret_cast<Tin*>(st + 3 * SL::rows) + n * RR + col;
+            }
+            cp_async16(dst, ok ? static_cast<const void*>(src) : p.A, ok ? 16 : 0);
+        }
+        cp_async_commit();
+    } else {
+        for (int i = tid; i < 3 * kBCH * T; i += kBW * 32) {
+            const int which = i / (kBCH * T), r = (i / T) % kBCH, t = i % T;
+            const Tin* src = static_cast<const Tin*>(which == 0 ? p.delta : which == 1 ? p.z : p.dy);
+            Tin v = Tin(0.f);
+            if (src && d0 + r < p.dim && t < valid) v = src[(b * p.dim + d0 + r) * p.L + t0 + t];
+            reinterpret_cast<Tin*>(st + which * SL::rows)[r * RR + t] = v;
+        }
+        for (int i = tid; i < 16 * T; i += kBW * 32) {
+            const int n = i / T, t = i % T;
+            Tin v = Tin(0.f);
+            if (n < p.N && t < valid) v = static_cast<const Tin*>(p.C)[(b * p.N + n) * p.L + t0 + t];
+            reinterpret_cast<Tin*>(st + 3 * SL::rows)[n * RR + t] = v;
+        }
+    }
+}
+
 template <int T, typename Tin>
 __global__ void __launch_bounds__(kBW * 32) adjoint_summary_kernel(const BParams p) {
-    using Lo = BLayout<T, Tin>;
-    constexpr int RS = Lo::RS, RR = Lo::RR;
+    using SL = SLayout<T, Tin>;
+    constexpr int RS = SL::RS, RR = SL::RR;
     extern __shared__ __align__(16) unsigned char smem[];
-    unsigned char* st = smem + Lo::off_stage;
-    const Tin* rDr = reinterpret_cast<const Tin*>(st + Lo::rows);
-    const Tin* rZ = reinterpret_cast<const Tin*>(st + 2 * Lo::rows);
-    const Tin* rDy = reinterpret_cast<const Tin*>(st + 3 * Lo::rows);
-    const Tin* rC = reinterpret_cast<const Tin*>(st + 4 * Lo::rows + Lo::coef);
-    float* sC = reinterpret_cast<float*>(smem + Lo::off_C);
-    float* sDel = reinterpret_cast<float*>(smem + Lo::off_del);
-    float* sDyt = reinterpret_cast<float*>(smem + Lo::off_dyt);
+    float* sC = reinterpret_cast<float*>(smem + SL::off_C);
+    float* sDel = reinterpret_cast<float*>(smem + SL::off_del);
+    float* sDyt = reinterpret_cast<float*>(smem + SL::off_dyt);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int pp = lane & 3, cl = lane >> 2;
     const int cw = warp * kBG + cl;
@@ -743,12 +806,31 @@ __global__ void __launch_bounds__(kBW * 32) adjoint_summary_kernel(const BParams
     float dsum = 0.f;
     const int seg = (int)blockIdx.z + 1;
     const int kbeg = seg * p.seg_chunks, kend = min(p.chunks, kbeg + p.seg_chunks);
+    auto buf = [&](int k) { return smem + (k % kSumBufs) * SL::stage; };
+    // the first kSumBufs - 1 blocks (last first) in flight before the loop
+#pragma unroll
+    for (int j = 0; j < kSumBufs - 1; ++j)
+        if (kend - 1 - j >= kbeg) stage_summary<T, Tin>(p, buf(kend - 1 - j), b, d0, kend - 1 - j, tid);
     for (int k = kend - 1; k >= kbeg; --k) {
         const int64_t t0 = (int64_t)k * T;
         const int valid = (int)min((int64_t)T, p.L - t0);
-        __syncthreads();  // the previous chunk's rows are no longer read
-        stage_chunk<T, Tin, false>(p, st, nullptr, b, d0, k, tid);
-        __syncthreads();
+        // block k - (kBufs - 1) into the buffer block k + 1 used (its readers finished at the
+        // barrier that ended the previous iteration); then wait for block k's copies, which
+        // were committed before every group issued after them
+        const int kn = k - (kSumBufs - 1);
+        if (kn >= kbeg) stage_summary<T, Tin>(p, buf(kn), b, d0, kn, tid);
+        if (p.vec) {
+            const int later = min(kSumBufs - 1, k - kbeg);  // groups committed after block k's
+            if (later >= 2) cp_async_wait<2>();
+            else if (later == 1) cp_async_wait<1>();
+            else cp_async_wait<0>();
+        }
+        __syncthreads();  // block k staged for every thread
+        const unsigned char* st = buf(k);
+        const Tin* rDr = reinterpret_cast<const Tin*>(st);
+        const Tin* rZ = reinterpret_cast<const Tin*>(st + SL::rows);
+        const Tin* rDy = reinterpret_cast<const Tin*>(st + 2 * SL::rows);
+        const Tin* rC = reinterpret_cast<const Tin*>(st + 3 * SL::rows);
         if constexpr (sizeof(Tin) == 2) {  // C to the bf16 blocks the sweep's loads read
             for (int i = tid; i < 4 * T; i += kBW * 32) {
                 const int t = i / 4, pq = i % 4;
@@ -789,6 +871,7 @@ __global__ void __launch_bounds__(kBW * 32) adjoint_summary_kernel(const BParams
             }
             dsum += (d4.x + d4.y) + (d4.z + d4.w);
         }
+        __syncthreads();  // sC, sDel, sDyt and this block's buffer are free again
     }
     if (chok) {
         const int64_t row = ((int64_t)seg * p.batch + b) * p.dim + dch;
@@ -833,11 +916,12 @@ cudaError_t launch_bwd_typed(const BParams& bp, int64_t batch, int64_t dim, cuda
     if (e != cudaSuccess) return e;
     if (bp.nseg > 1) {  // the summaries of segments 1.., then their fold
         auto sk = adjoint_summary_kernel<T, Tin>;
-        e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lo::bytes);
+        e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)SLayout<T, Tin>::bytes);
         if (e != cudaSuccess) return e;
         const dim3 sgrid((unsigned)((dim + kBCH - 1) / kBCH), (unsigned)batch,
                          (unsigned)(bp.nseg - 1));
-        sk<<<sgrid, kBW * 32, Lo::bytes, s>>>(bp);
+        sk<<<sgrid, kBW * 32, SLayout<T, Tin>::bytes, s>>>(bp);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t lanes = batch * dim * bp.N;
         adjoint_fold_kernel<<<(unsigned)((lanes + 255) / 256), 256, 0, s>>>(
