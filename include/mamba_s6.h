@@ -254,9 +254,11 @@ int mamba_selective_scan_fwd_noalloc(const void* u, const void* delta, const flo
 
 /*
  * Bytes of device workspace mamba_selective_scan_bwd needs for `dims`: the checkpoints,
- * the state entering every group of 4 steps, batch x dim x ceil(seqlen / 4) x dstate
- * floats (16 bytes per (batch, channel, step) at dstate = 16), rounded up to 64 floats;
- * plus, when a long sequence over few channels is
+ * the state entering every group of 4 steps, batch x dim' x ceil(seqlen / 4) x dstate
+ * floats with dim' = dim rounded up to a multiple of 32 (16 bytes per (batch, channel,
+ * step) at dstate = 16; stored [batch][dim][group][dstate] while seqlen * dstate < 2^20,
+ * tile-major [batch][dim' / 32][group][32][dstate] beyond), rounded up to 64 floats; plus,
+ * when a long sequence over few channels is
  * swept in S segments side by side (seqlen >= 16384 and fewer CTAs of 32 channels than two
  * per SM of the current device; S up to five CTAs per SM, segments of at least 4096 steps),
  * S x batch x dim x (dstate + 1) floats for the segments' summaries.  Rounded up to 256

@@ -291,11 +291,13 @@ int mamba_selective_state_update_ex(float* state, const void* u, const void* del
 
 size_t mamba_selective_scan_bwd_workspace_size(mamba_scan_dims dims) {
     if (!dims_ok(dims.batch, dims.dim, dims.dstate, dims.seqlen)) return 0;
+    // checkpoints: tile-major, the channel count padded to whole tiles
+    const int64_t dpad = (dims.dim + s6::kCkptTile - 1) / s6::kCkptTile * s6::kCkptTile;
     const int64_t T = s6::checkpoint_steps(dims.dstate);
     const int64_t chunks = (dims.seqlen + T - 1) / T;
-    if (!mul_ok(dims.batch * dims.dim, chunks) || !mul_ok(dims.batch * dims.dim * chunks, dims.dstate * 4))
+    if (!mul_ok(dims.batch * dpad, chunks) || !mul_ok(dims.batch * dpad * chunks, dims.dstate * 4))
         return 0;
-    int64_t floats = (dims.batch * dims.dim * chunks * dims.dstate + 63) / 64 * 64;
+    int64_t floats = (s6::ckpt_floats(dims.batch, dims.dim, dims.seqlen, dims.dstate) + 63) / 64 * 64;
     int64_t nseg = 1, seg_len = 0;
     s6::backward_segments(dims.batch, dims.dim, dims.seqlen, &nseg, &seg_len);
     if (nseg > 1) {  // the segments' adjoint summaries and summed steps

@@ -57,7 +57,7 @@ struct BParams {
     const void* C;
     const float* D;
     const float* delta_bias;
-    const float* ckpt;  // the state entering every 4-step group: [batch][dim][ck_blocks][N]
+    const float* ckpt;  // the state entering every 4-step group, at ckpt_index(b, d, group)
     void* du;
     void* ddelta;
     void* dz;
@@ -72,6 +72,7 @@ struct BParams {
     int chunks;     // blocks of T steps this kernel walks
     int ck_blocks;  // checkpoints per channel, ceil(L / 4)
     int ck_vec;     // N = 16 and ckpt 16-byte aligned: group states staged by 16-byte copies
+    int ck_tiled;   // ckpt_tiled(L, N): the checkpoints' layout
     // a sequence split into nseg segments of seg_chunks blocks (grid z = segment): g_carry
     // [nseg][batch][dim][N] holds, per segment, the adjoint its first step carries backwards
     // from the segment alone (the summary pass), then, after the fold, in slot s + 1 the
@@ -118,6 +119,7 @@ constexpr int kBW = S6_BWD_WARPS;  // warps per CTA
 constexpr int kBP = 4;             // lanes per channel, 4 states each
 constexpr int kBG = 32 / kBP;      // channels per warp
 constexpr int kBCH = kBW * kBG;    // channels per CTA
+static_assert(kBCH == kCkptTile, "a CTA's checkpoints of one group are one contiguous tile row");
 
 constexpr size_t a16(size_t x) { return (x + 15) / 16 * 16; }
 
@@ -217,7 +219,7 @@ __device__ __forceinline__ int acc_idx(int t, int slot) { return t * 32 + ((slot
 // are 16-byte aligned (then every 16-byte piece is either wholly inside the sequence or
 // wholly past it), and for the states when N = 16 and the checkpoints are 16-byte aligned;
 // plain loads otherwise.
-template <int T, typename Tin, bool kStates>
+template <int T, typename Tin, bool kStates, bool kTiled = false>
 __device__ __forceinline__ void stage_chunk(const BParams& p, unsigned char* st, float* sH,
                                             int64_t b, int64_t d0, int k, int tid) {
     using Lo = BLayout<T, Tin>;
@@ -227,7 +229,18 @@ __device__ __forceinline__ void stage_chunk(const BParams& p, unsigned char* st,
     const int valid = (int)min((int64_t)T, p.L - t0);
     if constexpr (kStates) {
         const int64_t kb0 = (int64_t)k * GT;
-        if (p.ck_vec) {
+        // (one loop per layout, each walking its source contiguously: the copies are issued
+        // at the start of every block, on the sweep's critical path)
+        if (kTiled && p.ck_vec) {
+            const float* tile = p.ckpt + ckpt_index(b, d0, kb0, p.dim, p.ck_blocks, 16, true);
+            for (int i = tid; i < kBCH * GT * 4; i += kBW * 32) {
+                const int q = i & 3, c = (i >> 2) % kBCH, g = i / (4 * kBCH);
+                const bool ok = d0 + c < p.dim && kb0 + g < p.ck_blocks;
+                cp_async16(sH + (g * kBCH + c) * 16 + 4 * q,
+                           ok ? static_cast<const void*>(tile + (g * kBCH + c) * 16 + 4 * q) : p.A,
+                           ok ? 16 : 0);
+            }
+        } else if (!kTiled && p.ck_vec) {
             for (int i = tid; i < kBCH * GT * 4; i += kBW * 32) {
                 const int q = i & 3, g = (i >> 2) % GT, c = i / (4 * GT);
                 const bool ok = d0 + c < p.dim && kb0 + g < p.ck_blocks;
@@ -237,10 +250,13 @@ __device__ __forceinline__ void stage_chunk(const BParams& p, unsigned char* st,
             }
         } else {
             for (int i = tid; i < kBCH * GT * 16; i += kBW * 32) {
-                const int n = i & 15, g = (i >> 4) % GT, c = i / (16 * GT);
+                const int n = i & 15;
+                const int g = kTiled ? i / (16 * kBCH) : (i >> 4) % GT;
+                const int c = kTiled ? (i >> 4) % kBCH : i / (16 * GT);
                 const bool ok = d0 + c < p.dim && kb0 + g < p.ck_blocks && n < p.N;
                 sH[(g * kBCH + c) * 16 + n] =
-                    ok ? p.ckpt[((b * p.dim + d0 + c) * p.ck_blocks + kb0 + g) * p.N + n] : 0.f;
+                    ok ? p.ckpt[ckpt_index(b, d0 + c, kb0 + g, p.dim, p.ck_blocks, p.N, kTiled) + n]
+                       : 0.f;
             }
         }
     }
@@ -329,7 +345,7 @@ __device__ __forceinline__ f2 zoh_dw_da2(f2 x, f2 e, f2 w, f2 inv_a, f2 dd) {
 template <bool ZOH> constexpr int bwd_min_blocks() { return ZOH ? 4 : 5; }
 template <typename Tin, bool ZOH> constexpr bool bwd_bf16_coef() { return sizeof(Tin) == 2 && !ZOH; }
 
-template <int T, typename Tin, bool ZOH>
+template <int T, typename Tin, bool ZOH, bool kTiled = false>
 __global__ void __launch_bounds__(kBW * 32, bwd_min_blocks<ZOH>()) scan_bwd_kernel(const BParams p) {
     using Lo = BLayout<T, Tin>;
     constexpr int RS = Lo::RS, RR = Lo::RR;
@@ -399,7 +415,7 @@ __global__ void __launch_bounds__(kBW * 32, bwd_min_blocks<ZOH>()) scan_bwd_kern
         const int64_t t0 = (int64_t)k * T;
         const int valid = (int)min((int64_t)T, p.L - t0);
         __syncthreads();  // the previous chunk's outputs have left the staging rows
-        stage_chunk<T, Tin, true>(p, st, sH, b, d0, k, tid);
+        stage_chunk<T, Tin, true, kTiled>(p, st, sH, b, d0, k, tid);
         __syncthreads();  // chunk k staged
 
         if constexpr (bwd_bf16_coef<Tin, ZOH>()) {
@@ -908,7 +924,8 @@ __global__ void adjoint_fold_kernel(float* g_carry, const float* g_dsum, const f
 template <int T, typename Tin, bool ZOH>
 cudaError_t launch_bwd_typed(const BParams& bp, int64_t batch, int64_t dim, cudaStream_t s) {
     using Lo = BLayout<T, Tin>;
-    auto kern = scan_bwd_kernel<T, Tin, ZOH>;
+    // the checkpoints' layout is a template choice: each instantiation stages its own way
+    auto kern = bp.ck_tiled ? scan_bwd_kernel<T, Tin, ZOH, true> : scan_bwd_kernel<T, Tin, ZOH, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Lo::bytes);
     if (e != cudaSuccess) return e;
@@ -1001,7 +1018,7 @@ cudaError_t launch_scan_backward(const ScanArgs& a_in, const BackwardArgs& g, fl
     ScanArgs a = a_in;
     int64_t nseg = 1, seg_len = a.L;
     backward_segments(a.batch, a.dim, a.L, &nseg, &seg_len);
-    const size_t ck_floats = (size_t)a.batch * a.dim * ((a.L + CK - 1) / CK) * a.N;
+    const size_t ck_floats = (size_t)ckpt_floats(a.batch, a.dim, a.L, a.N);
     float* seg_h = ckpt + (ck_floats + 63) / 64 * 64;
     float* seg_sum = seg_h + (size_t)nseg * a.batch * a.dim * a.N;
     if (nseg > 1) {
@@ -1060,6 +1077,7 @@ cudaError_t launch_scan_backward(const ScanArgs& a_in, const BackwardArgs& g, fl
     bp.chunks = (int)chunks;
     bp.ck_blocks = (int)((a.L + CK - 1) / CK);
     bp.ck_vec = (a.N == 16 && reinterpret_cast<uintptr_t>(ckpt) % 16 == 0) ? 1 : 0;
+    bp.ck_tiled = ckpt_tiled(a.L, a.N) ? 1 : 0;
     bp.nseg = (int)nseg;
     bp.seg_chunks = nseg > 1 ? (int)(seg_len / T) : (int)chunks;
     bp.g_carry = seg_h;

@@ -67,7 +67,8 @@ struct KParams {
     float* last_state;
     float* seg_h;
     float* seg_sum;
-    float* ckpt;  // checkpoint modes: (batch, dim, blocks, N)
+    float* ckpt;  // checkpoint modes: the state entering every 4-step group (ckpt_index)
+    int ck_tiled;  // ckpt_tiled(L, N): the checkpoints' layout
     int64_t batch, dim, L, seg_len;
     int N;
     int nseg;
@@ -357,6 +358,14 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
             }
         }
     }
+    // checkpoint modes: this lane's states of group 0 and the distance between groups
+    float* ck_lane = nullptr;
+    int64_t ck_gstride = 0;
+    if constexpr (MODE == kCheckpoint || MODE == kFullCkpt) {
+        const int64_t blocks = (p.L + kCkptSteps - 1) / kCkptSteps;
+        ck_lane = p.ckpt + ckpt_index(b, dch < p.dim ? dch : 0, 0, p.dim, blocks, p.N, p.ck_tiled) + pp * NS;
+        ck_gstride = (p.ck_tiled ? kCkptTile : 1) * (int64_t)p.N;
+    }
     float dsum = 0.f;
     // Correction pass: the state it carries decays monotonically when every A of the lane
     // is <= 0 and Delta >= 0 (softplus); then it may stop once every state is below
@@ -625,14 +634,12 @@ scan_kernel(const KParams p, const __grid_constant__ TMaps tm) {
         float* sDuK = sDu + (WS == 2 ? (k & 1) * Lo::dq_stride : 0);
         if constexpr (WS != 2) phase_a(k, warp * CW, CW * (T / 4), lane, 32, sDelK, sDuK);
 
-        // checkpoint modes: the state entering every 4-step group of the sequence,
-        // ckpt[((b * dim + d) * blocks + kb) * N + n], blocks = ceil(L / 4) -- what the
-        // backward's reverse sweep starts each group from, so it recomputes no other state
+        // checkpoint modes: the state entering every 4-step group of the sequence, at
+        // ckpt_index(b, d, group) -- what the backward's reverse sweep starts each group
+        // from, so it recomputes no other state
         auto write_ckpt = [&](int t) {
-            const int64_t blocks = (p.L + kCkptSteps - 1) / kCkptSteps;
-            const int64_t kb = (t0 + t) / kCkptSteps;
             if (dch >= p.dim || t0 + t >= p.L) return;
-            float* ck = p.ckpt + ((b * p.dim + dch) * blocks + kb) * p.N + pp * NS;
+            float* ck = ck_lane + ((t0 + t) / kCkptSteps) * ck_gstride;
             if (NS % 4 == 0 && p.N == NMAX && (reinterpret_cast<uintptr_t>(ck) & 15) == 0) {
 #pragma unroll
                 for (int j = 0; j < NS / 2; j += 2) {
@@ -1352,6 +1359,7 @@ cudaError_t launch_scan_checkpoints(const ScanArgs& a, float* ckpt, cudaStream_t
     kp.C = a.C;
     kp.delta_bias = a.delta_bias;
     kp.ckpt = ckpt;
+    kp.ck_tiled = ckpt_tiled(a.L, a.N) ? 1 : 0;
     kp.batch = a.batch;
     kp.dim = a.dim;
     kp.L = a.L;
@@ -1512,6 +1520,7 @@ cudaError_t launch_scan(const ScanArgs& a, cudaStream_t stream) {
     // with one segment the kernel reads its initial state through seg_h (read only)
     kp.seg_h = a.nseg > 1 ? a.seg_h : const_cast<float*>(a.h0);
     kp.ckpt = a.ckpt;
+    kp.ck_tiled = ckpt_tiled(a.L, a.N) ? 1 : 0;
     kp.seg_sum = a.seg_sum;
     kp.batch = a.batch;
     kp.dim = a.dim;

@@ -184,11 +184,13 @@ def test_bwd_dims_dtype_align_workspace(lib):
 
 def test_bwd_workspace_is_one_checkpoint_per_group(lib):
     ws = lambda *d: lib.mamba_selective_scan_bwd_workspace_size(_dims(*d))  # noqa: E731
-    # the state entering every group of 4 steps, fp32, for every dstate
+    # the state entering every group of 4 steps, fp32, for every dstate; channels in tiles
+    # of 32 (3 channels take one whole tile)
     assert ws(4, 5120, 16, 4096) == 4 * 5120 * 1024 * 16 * 4
     assert ws(2, 64, 16, 33) == 2 * 64 * 9 * 16 * 4
     assert ws(2, 64, 8, 64) == 2 * 64 * 16 * 8 * 4
-    assert ws(1, 3, 5, 65) == (1 * 3 * 17 * 5 * 4 + 255) // 256 * 256
+    assert ws(1, 3, 5, 65) == (1 * 32 * 17 * 5 * 4 + 255) // 256 * 256
+    assert ws(2, 40, 16, 8) == 2 * 64 * 2 * 16 * 4
     assert ws(2, 64, 16, 0) == 0
     assert ws(2, 64, 17, 8) == 0
 

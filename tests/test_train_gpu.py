@@ -88,13 +88,16 @@ def test_training_forward_rejects_zoh_and_initial_state(cuda_ok):
 
 @pytest.mark.parametrize("shape,dtype", [((2, 40, 16, 200), torch.float32),
                                          ((2, 24, 16, 77), torch.bfloat16),
-                                         ((1, 16, 5, 130), torch.float32)],
+                                         ((1, 70, 5, 130), torch.float32),
+                                         ((1, 40, 16, 65536), torch.float32)],
                          ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
 def test_checkpoints_are_the_group_entry_states(cuda_ok, shape, dtype):
-    """The recorded checkpoints are the layout the header documents: per (batch, channel)
-    the state entering every group of 4 steps, ckpt[b, d, g, n] = h_{4g-1} (zero for g = 0),
-    fp32, batch x dim x ceil(L / 4) x N.  Compared with the oracle's states under the
-    last_state tolerances (fp32 inputs per element, bf16 inputs against the RMS)."""
+    """The recorded checkpoints are the layout the header documents: the state entering
+    every group of 4 steps, h_{4g-1} (zero for g = 0), fp32, per channel
+    ([batch][dim][group][N]) while L * N < 2^20 and tile-major beyond ([batch][tile of 32
+    channels][group][channel in tile][N]; the last shape, a split sequence).  Compared with
+    the oracle's states under the last_state tolerances (fp32 inputs per element, bf16
+    inputs against the RMS)."""
     b, d, N, L = shape
     p = inputs.scan_inputs(b, d, N, L, dtype, seed=4 * L + N)
     g = {k: (None if v is None else v.to(DEV)) for k, v in p.items()}
@@ -104,7 +107,12 @@ def test_checkpoints_are_the_group_entry_states(cuda_ok, shape, dtype):
                            delta_bias=g["delta_bias"], checkpoints=ck)
     torch.cuda.synchronize()
     G = (L + 3) // 4
-    got = ck[: b * d * G * N * 4].view(torch.float32).reshape(b, d, G, N)
+    if L * N >= 1 << 20:
+        nt = (d + 31) // 32
+        tiled = ck[: b * nt * G * 32 * N * 4].view(torch.float32).reshape(b, nt, G, 32, N)
+        got = tiled.permute(0, 1, 3, 2, 4).reshape(b, nt * 32, G, N)[:, :d]
+    else:
+        got = ck[: b * d * G * N * 4].view(torch.float32).reshape(b, d, G, N)
     _, _, hs = oracle.selective_scan(p["u"], p["delta"], p["A"], p["B"], p["C"], D=p["D"],
                                      z=p["z"], delta_bias=p["delta_bias"], return_states=True)
     ref = np.zeros((b, d, G, N))
