@@ -140,7 +140,8 @@ enum Mode : int { kFull = 0, kAggregate = 1, kCheckpoint = 2, kFullCkpt = 3, kFu
 #endif
 // The checkpoint-recording forwards (the backward's own pass and the training forward)
 // with the same plan-based producer form: measured neutral on the 2.8B-shaped layer
-// (backward 3120 -> 3131 us, training step 3287 -> 3267 us), so off.
+// (backward 3120 -> 3131 us, training step 3287 -> 3267 us with 16-step checkpoints;
+// 2908 -> 2900 us and 3096 -> 3087 us with 4-step groups), so off.
 #ifndef S6_WS_CKPT
 #define S6_WS_CKPT 0
 #endif
