@@ -157,13 +157,15 @@ def test_m2p8b_layer_backward_full(cuda_ok):
 
 @pytest.mark.parametrize("shape,dtype", [((1, 64, 16, 40000), torch.bfloat16),
                                          ((2, 33, 5, 20000), torch.float32),
-                                         ((1, 40, 16, 65536), torch.bfloat16)],
+                                         ((1, 40, 16, 65536), torch.bfloat16),
+                                         ((1, 24, 8, 131072), torch.float32)],
                          ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
 def test_backward_of_a_split_sequence(cuda_ok, shape, dtype):
     """Long sequences over few channels are swept in segments side by side: checkpoints
     from each segment's true start, the adjoint entering each segment from a summary pass
     and its fold (the last segment ragged here); every gradient against the oracle.  The
-    last shape (L * N = 2^20) keeps its checkpoints tile-major, with a partly filled tile."""
+    last two shapes (L * N = 2^20) keep their checkpoints tile-major, with a partly filled
+    tile (N = 8: element-wise staging of the states, 64-step blocks)."""
     b, d, N, L = shape
     ws = ops.selective_scan_bwd_workspace_size(b, d, N, L)
     ck = (b * -(-d // 32) * 32 * -(-L // 4) * N + 63) // 64 * 64 * 4  # the checkpoints alone

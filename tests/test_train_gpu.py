@@ -89,7 +89,8 @@ def test_training_forward_rejects_zoh_and_initial_state(cuda_ok):
 @pytest.mark.parametrize("shape,dtype", [((2, 40, 16, 200), torch.float32),
                                          ((2, 24, 16, 77), torch.bfloat16),
                                          ((1, 70, 5, 130), torch.float32),
-                                         ((1, 40, 16, 65536), torch.float32)],
+                                         ((1, 40, 16, 65536), torch.float32),
+                                         ((1, 24, 8, 131072), torch.bfloat16)],
                          ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
 def test_checkpoints_are_the_group_entry_states(cuda_ok, shape, dtype):
     """The recorded checkpoints are the layout the header documents: the state entering
