@@ -291,7 +291,8 @@ int mamba_selective_state_update_ex(float* state, const void* u, const void* del
 
 size_t mamba_selective_scan_bwd_workspace_size(mamba_scan_dims dims) {
     if (!dims_ok(dims.batch, dims.dim, dims.dstate, dims.seqlen)) return 0;
-    // checkpoints: tile-major, the channel count padded to whole tiles
+    // checkpoints: sized for the tile-major layout (the channel count padded to whole
+    // tiles), which also holds the per-channel one used for shorter sequences
     const int64_t dpad = (dims.dim + s6::kCkptTile - 1) / s6::kCkptTile * s6::kCkptTile;
     const int64_t T = s6::checkpoint_steps(dims.dstate);
     const int64_t chunks = (dims.seqlen + T - 1) / T;
