@@ -99,13 +99,15 @@ def test_conv1d_m2p8b_layer(cuda_ok):
     np.testing.assert_array_equal(to64(fin), fref)
 
 
+@pytest.mark.parametrize("b", [3, 6])
 @pytest.mark.parametrize("d", [48, 45])
 @pytest.mark.parametrize("K,dt", [(4, torch.bfloat16), (3, torch.float32), (2, torch.bfloat16),
                                   (1, torch.float32)])
-def test_conv1d_decode_continues_the_prefill(cuda_ok, K, dt, d):
+def test_conv1d_decode_continues_the_prefill(cuda_ok, K, dt, d, b):
     """Decode steps after a prefill equal the prefill of the longer sequence (channel
-    counts with and without a multiple-of-8 tail)."""
-    b, L, steps = 3, 20, 6
+    counts with and without a multiple-of-8 tail; 3 batch rows take one row per thread, 6
+    take four rows per thread with the last slice ragged)."""
+    L, steps = 20, 6
     p = inputs.conv_inputs(b, d, L + steps, K, dt, seed=77 + K, with_initial_state=True)
     full_ref, _ = _ref(p)
     pre = dict(p)
