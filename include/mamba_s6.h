@@ -317,7 +317,8 @@ int mamba_selective_scan_bwd(const void* u, const void* delta, const float* A, c
  *
  *   checkpoints      : device buffer of at least mamba_selective_scan_bwd_workspace_size(dims)
  *                      bytes, written (may be NULL when seqlen == 0)
- *   everything else  : as mamba_selective_scan_fwd (no flags: the Delta * B form)
+ *   everything else  : as mamba_selective_scan_fwd (no flags: the Delta * B form; the _ex
+ *                      form below takes the flags word)
  *
  * Errors: as mamba_selective_scan_fwd, plus WORKSPACE when checkpoint_bytes is too small.
  */
@@ -360,6 +361,30 @@ int mamba_selective_scan_bwd_from_checkpoints(
     void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC, float* dD,
     float* ddelta_bias, mamba_scan_dims dims, mamba_dtype in_dtype, const float* checkpoints,
     size_t checkpoint_bytes, void* stream);
+
+/*
+ * The training pair with the flags word: mamba_selective_scan_fwd_train_ex records the
+ * checkpoints of the forward the flags select (MAMBA_FLAG_EXACT_ZOH: the exact zero-order
+ * hold of mamba_selective_scan_fwd_ex, states and checkpoints with the weight
+ * w = expm1(Delta A) / A), and mamba_selective_scan_bwd_from_checkpoints_ex returns the
+ * gradients of mamba_selective_scan_bwd_ex with the same flags from them.  Both calls of a
+ * pair take the same flags; flags = 0 is exactly the plain pair.
+ * Errors: as mamba_selective_scan_fwd_train / mamba_selective_scan_bwd_from_checkpoints,
+ * and FLAGS for unknown flag bits.
+ */
+int mamba_selective_scan_fwd_train_ex(const void* u, const void* delta, const float* A,
+                                      const void* B, const void* C, const float* D, const void* z,
+                                      const float* delta_bias, int delta_softplus, void* y,
+                                      float* last_state, mamba_scan_dims dims, mamba_dtype in_dtype,
+                                      mamba_dtype out_dtype, void* workspace,
+                                      size_t workspace_bytes, float* checkpoints,
+                                      size_t checkpoint_bytes, unsigned flags, void* stream);
+int mamba_selective_scan_bwd_from_checkpoints_ex(
+    const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int delta_softplus, const void* dy,
+    void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC, float* dD,
+    float* ddelta_bias, mamba_scan_dims dims, mamba_dtype in_dtype, const float* checkpoints,
+    size_t checkpoint_bytes, unsigned flags, void* stream);
 
 /*
  * Causal depthwise conv1d with an optional SiLU: the Mamba block's step between the input

@@ -357,6 +357,30 @@ int mamba_selective_scan_bwd_from_checkpoints(
                     checkpoint_bytes, true, 0u, stream);
 }
 
+int mamba_selective_scan_fwd_train_ex(const void* u, const void* delta, const float* A,
+                                      const void* B, const void* C, const float* D, const void* z,
+                                      const float* delta_bias, int delta_softplus, void* y,
+                                      float* last_state, mamba_scan_dims dims, mamba_dtype in_dtype,
+                                      mamba_dtype out_dtype, void* workspace,
+                                      size_t workspace_bytes, float* checkpoints,
+                                      size_t checkpoint_bytes, unsigned flags, void* stream) {
+    if (!checkpoints && dims.seqlen > 0) return MAMBA_ERR_NULL;
+    return scan_fwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, y, last_state,
+                    dims, in_dtype, out_dtype, workspace, workspace_bytes, flags, stream,
+                    dims.seqlen > 0 ? checkpoints : nullptr, checkpoint_bytes);
+}
+
+int mamba_selective_scan_bwd_from_checkpoints_ex(
+    const void* u, const void* delta, const float* A, const void* B, const void* C,
+    const float* D, const void* z, const float* delta_bias, int delta_softplus, const void* dy,
+    void* du, void* ddelta, void* dz, float* dA, float* dB, float* dC, float* dD,
+    float* ddelta_bias, mamba_scan_dims dims, mamba_dtype in_dtype, const float* checkpoints,
+    size_t checkpoint_bytes, unsigned flags, void* stream) {
+    return scan_bwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, dy, du, ddelta, dz, dA,
+                    dB, dC, dD, ddelta_bias, dims, in_dtype, const_cast<float*>(checkpoints),
+                    checkpoint_bytes, true, flags, stream);
+}
+
 }  // extern "C"
 
 namespace {

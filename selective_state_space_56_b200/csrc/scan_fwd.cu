@@ -1213,6 +1213,11 @@ cudaError_t launch_typed(const ScanArgs& a, const KParams& kp, cudaStream_t s) {
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
+    if constexpr (ZOH) {
+        if (a.ckpt)  // the training forward of the exact-ZOH scan: barrier form
+            return launch_one<NMAX, TL::P, TL::WARPS, TL::T, Tin, Tout, kFullCkpt, TMA, true>(
+                a, kp, a.nseg, s);
+    }
     if constexpr (!ZOH) {
         if (a.ckpt) {
             if constexpr (TMA && S6_WS_CKPT) {

@@ -73,6 +73,12 @@ def load_library():
             lib.mamba_selective_scan_bwd_from_checkpoints.restype = i32
             lib.mamba_selective_scan_bwd_from_checkpoints.argtypes = [vp] * 8 + [i32] + [vp] * 9 + [
                 ScanDims, i32, vp, ctypes.c_size_t, vp]
+            lib.mamba_selective_scan_fwd_train_ex.restype = i32
+            lib.mamba_selective_scan_fwd_train_ex.argtypes = [vp] * 8 + [
+                i32, vp, vp, ScanDims, i32, i32, vp, ctypes.c_size_t, vp, ctypes.c_size_t, u32, vp]
+            lib.mamba_selective_scan_bwd_from_checkpoints_ex.restype = i32
+            lib.mamba_selective_scan_bwd_from_checkpoints_ex.argtypes = [vp] * 8 + [i32] + [vp] * 9 + [
+                ScanDims, i32, vp, ctypes.c_size_t, u32, vp]
             lib.mamba_selective_scan_fwd_init.restype = i32
             lib.mamba_selective_scan_fwd_init.argtypes = [vp] * 8 + [i32] + [vp] * 3 + [
                 ScanDims, i32, i32, vp, ctypes.c_size_t, u32, vp]
@@ -204,7 +210,7 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
     instead of Delta * B.  initial_state: (batch, dim, N) fp32 state before the sequence
     (zero when None).  checkpoints: a uint8 CUDA tensor of at least
     selective_scan_bwd_workspace_size(...) bytes to record the backward's checkpoints in
-    (a training forward; not with exact_zoh or initial_state)."""
+    (a training forward, also with exact_zoh; not with initial_state)."""
     if not isinstance(u, torch.Tensor) or u.dim() != 3:
         raise ValueError("u must be a (batch, dim, L) tensor")
     dev = u.device
@@ -243,14 +249,14 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta
             int(bool(delta_softplus)), _ptr(y), _ptr(last_state), dims, _DTYPES[in_dt],
             _DTYPES[out_dt], _ptr(workspace), ws_bytes)
     flags = MAMBA_FLAG_EXACT_ZOH if exact_zoh else 0
-    if checkpoints is not None and (exact_zoh or initial_state is not None):
-        raise ValueError("checkpoints are recorded by the plain forward only")
+    if checkpoints is not None and initial_state is not None:
+        raise ValueError("checkpoints are recorded by a forward from h = 0 only")
     with torch.cuda.device(dev):
         if checkpoints is not None:
             _check(checkpoints, "checkpoints", dev)
-            rc = lib.mamba_selective_scan_fwd_train(
+            rc = lib.mamba_selective_scan_fwd_train_ex(
                 *args, _ptr(checkpoints), checkpoints.numel() * checkpoints.element_size(),
-                _stream_handle(dev))
+                flags, _stream_handle(dev))
         elif initial_state is not None:
             rc = lib.mamba_selective_scan_fwd_init(*args[:9], _ptr(initial_state), *args[9:], flags,
                                                    _stream_handle(dev))
@@ -272,9 +278,9 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
     without a gate), dA (dim, N), dB, dC (batch, N, L), dD, ddelta_bias (dim) in fp32
     (None where the input is None).  checkpoints: the buffer a training forward
     (selective_scan_fwd(..., checkpoints=...)) filled for the same inputs; the backward
-    then skips its own checkpointing pass.  exact_zoh: the gradients of the exact
-    zero-order-hold forward (``selective_scan_fwd(..., exact_zoh=True)``); not with
-    checkpoints (the training forward has no exact-ZOH form)."""
+    then skips its own checkpointing pass (with the exact_zoh the forward used).
+    exact_zoh: the gradients of the exact zero-order-hold forward
+    (``selective_scan_fwd(..., exact_zoh=True)``)."""
     if not isinstance(u, torch.Tensor) or u.dim() != 3:
         raise ValueError("u must be a (batch, dim, L) tensor")
     dev = u.device
@@ -303,16 +309,15 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None,
     lib = load_library()
     dims = ScanDims(b, d, N, L)
     if checkpoints is not None:
-        if exact_zoh:
-            raise ValueError("the training path has no exact-ZOH form")
         _check(checkpoints, "checkpoints", dev)
         with torch.cuda.device(dev):
-            rc = lib.mamba_selective_scan_bwd_from_checkpoints(
+            rc = lib.mamba_selective_scan_bwd_from_checkpoints_ex(
                 _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
                 _ptr(delta_bias), int(bool(delta_softplus)), _ptr(dy), _ptr(g["du"]),
                 _ptr(g["ddelta"]), _ptr(g["dz"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]),
                 _ptr(g["dD"]), _ptr(g["ddelta_bias"]), dims, _DTYPES[dt], _ptr(checkpoints),
-                checkpoints.numel() * checkpoints.element_size(), _stream_handle(dev))
+                checkpoints.numel() * checkpoints.element_size(),
+                MAMBA_FLAG_EXACT_ZOH if exact_zoh else 0, _stream_handle(dev))
         if rc != 0:
             raise MambaError(rc, "mamba_selective_scan_bwd_from_checkpoints")
         return g

@@ -222,6 +222,20 @@ def test_ex_entry_points_reject_unknown_flags(lib):
     assert lib.mamba_selective_scan_fwd_ex(*([None] + scan_args[1:]), 1, None) == ERR_NULL
     assert lib.mamba_selective_scan_fwd_ex(*scan_args[:11], _dims(2, 64, 17, 8), 0, 0, None, 0,
                                            1, None) == ERR_DIMS
+    # the training pair's flags forms: unknown bits refused, known ones reach the usual checks
+    need = lib.mamba_selective_scan_bwd_workspace_size(_dims())
+    for flags in (2, 0x80000000):
+        assert lib.mamba_selective_scan_fwd_train_ex(*scan_args, vp(A16), need, flags,
+                                                     None) == ERR_FLAGS
+    assert lib.mamba_selective_scan_fwd_train_ex(*scan_args, None, need, 1, None) == ERR_NULL
+    assert lib.mamba_selective_scan_fwd_train_ex(*scan_args, vp(A16), need - 1, 1,
+                                                 None) == ERR_WORKSPACE
+    bw = [vp(A16)] * 5 + [None, None, None, 1] + [vp(A16)] * 3 + [None] + [vp(A16)] * 3 + \
+        [None, None, _dims(), 1]
+    assert lib.mamba_selective_scan_bwd_from_checkpoints_ex(*bw, vp(A16), need, 2,
+                                                            None) == ERR_FLAGS
+    assert lib.mamba_selective_scan_bwd_from_checkpoints_ex(*bw, vp(A16), need - 1, 1,
+                                                            None) == ERR_WORKSPACE
     upd = [vp(A16)] * 6 + [None, None, None, 1, vp(A16), 4, 64, 16, 1]
     assert lib.mamba_selective_state_update_ex(*upd, 4, None) == ERR_FLAGS
     assert lib.mamba_selective_state_update_ex(*([None] + upd[1:]), 1, None) == ERR_NULL

@@ -77,13 +77,64 @@ def test_training_forward_and_backward_match(cuda_ok, shape, dtype):
     ops.check_device_error()
 
 
-def test_training_forward_rejects_zoh_and_initial_state(cuda_ok):
+def test_training_forward_rejects_an_initial_state(cuda_ok):
     p = inputs.scan_inputs(1, 8, 16, 16, torch.float32, seed=1, device=DEV)
     ck = torch.empty(ops.selective_scan_bwd_workspace_size(1, 8, 16, 16), dtype=torch.uint8,
                      device=DEV)
+    h0 = torch.zeros(1, 8, 16, device=DEV)
     with pytest.raises(ValueError):
         ops.selective_scan_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"], checkpoints=ck,
-                               exact_zoh=True)
+                               initial_state=h0)
+
+
+@pytest.mark.parametrize("shape,dtype", [((2, 40, 16, 200), torch.float32),
+                                         ((2, 24, 16, 77), torch.bfloat16),
+                                         ((1, 64, 16, 40000), torch.bfloat16),  # split plan
+                                         ((2, 33, 5, 130), torch.float32)],
+                         ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
+def test_exact_zoh_training_pair(cuda_ok, shape, dtype):
+    """The training pair with the exact-ZOH weight: the forward's outputs equal the exact-ZOH
+    forward's (bit for bit in one pass; a split sequence's to the bf16-output bound, as for
+    the Delta * B pair), and the gradients from its checkpoints equal the recomputing
+    exact-ZOH backward's (du, ddelta, dz bit for bit in one pass; sums to 1e-5)."""
+    b, d, N, L = shape
+    p = inputs.scan_inputs(b, d, N, L, dtype, seed=L + d + 1, device=DEV)
+    gen = torch.Generator(device=DEV).manual_seed(4)
+    dy = torch.randn(b, d, L, generator=gen, device=DEV).to(dtype)
+    ck = torch.empty(ops.selective_scan_bwd_workspace_size(b, d, N, L), dtype=torch.uint8,
+                     device=DEV)
+    kw = dict(D=p["D"], z=p["z"], delta_bias=p["delta_bias"], exact_zoh=True)
+    y_t, st_t = ops.selective_scan_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"],
+                                       return_last_state=True, checkpoints=ck, **kw)
+    y_p, st_p = ops.selective_scan_fwd(p["u"], p["delta"], p["A"], p["B"], p["C"],
+                                       return_last_state=True, **kw)
+    torch.cuda.synchronize()
+    split = ops.selective_scan_workspace_size(b, d, N, L) > 0
+    if not split:
+        assert torch.equal(y_t, y_p) and torch.equal(st_t, st_p)
+    else:
+        yt, yp = y_t.double(), y_p.double()
+        mag = torch.maximum(yt.abs(), yp.abs()).clamp_min(2.0 ** -126)
+        ulp = torch.exp2(torch.floor(torch.log2(mag)) - (7 if dtype == torch.bfloat16 else 23))
+        tol = 2 * ulp + 2 * 2e-2 * yp.pow(2).mean().sqrt()
+        assert bool(((yt - yp).abs() <= tol).all())
+        torch.testing.assert_close(st_t, st_p, rtol=1e-4, atol=1e-6 * st_p.abs().max().item())
+    g_c = ops.selective_scan_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, checkpoints=ck,
+                                 **kw)
+    g_r = ops.selective_scan_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], dy, **kw)
+    torch.cuda.synchronize()
+    for k in ("du", "ddelta", "dz"):
+        if not split:
+            assert torch.equal(g_c[k], g_r[k]), k
+        else:
+            diff = (g_c[k].float() - g_r[k].float()).abs()
+            tol = (g_r[k].float().abs() * (2.0 ** -7 if dtype == torch.bfloat16 else 1e-5) +
+                   1e-6 * g_r[k].float().abs().max())
+            assert bool((diff <= tol).all()), k
+    for k in ("dA", "dB", "dC", "dD", "ddelta_bias"):
+        torch.testing.assert_close(g_c[k], g_r[k], rtol=1e-4 if split else 1e-5,
+                                   atol=1e-6 * g_r[k].abs().max().item())
+    ops.check_device_error()
 
 
 @pytest.mark.parametrize("shape,dtype", [((2, 40, 16, 200), torch.float32),
